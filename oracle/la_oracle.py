@@ -1,0 +1,214 @@
+"""fp64 CPU oracle for the gated ReLU linear-attention token mixer.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import or call this
+module: only the tests, the smoke check and the CPU-baseline leg of the
+benchmark use it.  It shares no code with the CUDA library.
+
+What it computes, per (batch, head), written out as plainly as possible:
+
+* Feature map and RoPE placement -- "SANA-Video: Efficient Video Generation
+  with Block Linear Diffusion Transformer", Sec. 3.2 (the RoPE-after-ReLU
+  formula and its pseudocode): RoPE is applied to ReLU(x), and only in the
+  numerator; the denominator uses the un-rotated ReLU features.
+* State, normaliser, gate -- "SANA-Video 2.0: Hybrid Linear Attention with
+  Attention Residuals for Efficient Video Generation", Sec. 2, Eq. (1):
+  S = sum_n k_n^r v_n^T, o_j = (q_j^r S) / (sum_n phi(k_n).phi(q_j) + eps)
+  * sigmoid(g_j), with the write gate beta fixed to 1 and RMSNorm / W_o left
+  out (they sit outside this operator).
+* Block-causal mode -- "SANA-Video" Sec. 3.4 (causal linear attention with a
+  constant-memory cache, and Algorithm 1's per-block cache update): a token
+  in block b reads the sum of the states of blocks 0..b, its own block
+  included.
+
+Readings where the pages are silent (each one is listed in the design notes):
+3D RoPE splits d into consecutive t / h / w bands; pair i of a band of width D
+rotates channels (2i, 2i+1) of that band by angle pos * base**(-2i/D),
+counter-clockwise; positions are the integer latent indices starting at 0;
+token n sits at grid position (t, h, w) with n = (t*Hh + h)*W + w; eps is added
+after the dot product.
+
+Every input is converted to float64 exactly before use, and all arithmetic is
+float64.  A matrix product (numpy ``@``) is the only library primitive used.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "band_frequencies", "grid_positions", "relu", "sigmoid", "rope3d",
+    "head_state", "head_apply", "forward_positions", "forward_bidir",
+    "block_of_tokens", "block_states", "forward_blockcausal", "forward_brute",
+]
+
+
+def band_frequencies(D: int, base: float) -> np.ndarray:
+    """theta_i = base ** (-2 i / D) for the D/2 pairs of one RoPE band."""
+    i = np.arange(D // 2, dtype=np.float64)
+    return np.power(float(base), -2.0 * i / float(D))
+
+
+def grid_positions(T: int, Hh: int, W: int) -> np.ndarray:
+    """(N, 3) integer positions (t, h, w) of the tokens, n = (t*Hh + h)*W + w."""
+    t, h, w = np.meshgrid(np.arange(T), np.arange(Hh), np.arange(W), indexing="ij")
+    return np.stack([t.reshape(-1), h.reshape(-1), w.reshape(-1)], axis=1).astype(np.int64)
+
+
+def relu(x: np.ndarray) -> np.ndarray:
+    """phi = ReLU ("SANA-Video 2.0", Sec. 2)."""
+    return np.maximum(x, 0.0)
+
+
+def sigmoid(x: np.ndarray) -> np.ndarray:
+    """The logistic output gate sigma(g) of Eq. (1)."""
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-x))
+
+
+def rope3d(x: np.ndarray, pos: np.ndarray, bands, base: float) -> np.ndarray:
+    """Rotate each channel pair of each band by its position along that band's axis.
+
+    x: (N, d) float64; pos: (N, 3) positions (t, h, w); bands = (dt, dh, dw).
+    Channel block [0, dt) follows t, [dt, dt+dh) follows h, [dt+dh, d) follows w.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    y = x.copy()
+    off = 0
+    for axis, D in enumerate(bands):
+        theta = band_frequencies(D, base)
+        p = pos[:, axis].astype(np.float64)
+        for i in range(D // 2):
+            angle = p * theta[i]
+            c, s = np.cos(angle), np.sin(angle)
+            x0 = x[:, off + 2 * i]
+            x1 = x[:, off + 2 * i + 1]
+            y[:, off + 2 * i] = x0 * c - x1 * s
+            y[:, off + 2 * i + 1] = x0 * s + x1 * c
+        off += D
+    assert off == x.shape[1], "bands must add up to d"
+    return y
+
+
+def head_state(k: np.ndarray, v: np.ndarray, pos: np.ndarray, bands, base: float):
+    """S = sum_n RoPE(ReLU(k_n))^T v_n (d x d) and z = sum_n ReLU(k_n) (d) over the given tokens."""
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    kp = relu(k)
+    kr = rope3d(kp, pos, bands, base)
+    S = kr.T @ v
+    z = kp.sum(axis=0)
+    return S, z
+
+
+def head_apply(q: np.ndarray, g: np.ndarray, S: np.ndarray, z: np.ndarray, pos: np.ndarray,
+               bands, base: float, eps: float) -> np.ndarray:
+    """o_n = (RoPE(ReLU(q_n)) S) / (ReLU(q_n) . z + eps) * sigmoid(g_n)."""
+    q = np.asarray(q, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    qp = relu(q)
+    qr = rope3d(qp, pos, bands, base)
+    num = qr @ S
+    den = qp @ z + float(eps)
+    return num / den[:, None] * sigmoid(g)
+
+
+def forward_positions(q, k, v, g, pos, bands, base, eps):
+    """Bidirectional output of one head whose tokens sit at explicit positions ``pos``."""
+    S, z = head_state(k, v, pos, bands, base)
+    return head_apply(q, g, S, z, pos, bands, base, eps)
+
+
+def _heads(x):
+    x = np.asarray(x, dtype=np.float64)
+    B, H, N, d = x.shape
+    return x.reshape(B * H, N, d)
+
+
+def forward_bidir(Q, K, V, G, grid, bands, base=10000.0, eps=1e-6, return_state=False):
+    """Bidirectional mixer over [B, H, N, d] inputs on a (T, Hh, W) latent grid."""
+    T, Hh, W = grid
+    pos = grid_positions(T, Hh, W)
+    B, H, N, d = np.shape(Q)
+    assert N == T * Hh * W
+    q, k, v, g = _heads(Q), _heads(K), _heads(V), _heads(G)
+    O = np.empty((B * H, N, d))
+    Ss = np.empty((B * H, d, d))
+    zs = np.empty((B * H, d))
+    for u in range(B * H):
+        Ss[u], zs[u] = head_state(k[u], v[u], pos, bands, base)
+        O[u] = head_apply(q[u], g[u], Ss[u], zs[u], pos, bands, base, eps)
+    O = O.reshape(B, H, N, d)
+    if return_state:
+        return O, Ss.reshape(B, H, d, d), zs.reshape(B, H, d)
+    return O
+
+
+def block_of_tokens(pos: np.ndarray, block_frames: int) -> np.ndarray:
+    """Block index of each token: floor(t / block_frames)."""
+    return pos[:, 0] // int(block_frames)
+
+
+def block_states(k, v, pos, bands, base, block_frames):
+    """Per-block states (not prefixed) of one head: S_b, z_b for b = 0..nblk-1."""
+    blk = block_of_tokens(pos, block_frames)
+    nblk = int(blk.max()) + 1 if len(blk) else 0
+    d = k.shape[1]
+    Sb = np.zeros((nblk, d, d))
+    zb = np.zeros((nblk, d))
+    for b in range(nblk):
+        sel = blk == b
+        Sb[b], zb[b] = head_state(k[sel], v[sel], pos[sel], bands, base)
+    return Sb, zb
+
+
+def forward_blockcausal(Q, K, V, G, grid, bands, base=10000.0, eps=1e-6, block_frames=1,
+                        return_state=False):
+    """Block-causal mixer: a token of block b reads sum_{b' <= b} (S_b', z_b').
+
+    Returns O and, if asked, the inclusive per-block states [B, H, nblk, d, d] and
+    [B, H, nblk, d] (the constant-memory cache after each block).
+    """
+    T, Hh, W = grid
+    pos = grid_positions(T, Hh, W)
+    B, H, N, d = np.shape(Q)
+    q, k, v, g = _heads(Q), _heads(K), _heads(V), _heads(G)
+    blk = block_of_tokens(pos, block_frames)
+    nblk = -(-T // block_frames)
+    O = np.empty((B * H, N, d))
+    Sinc = np.empty((B * H, nblk, d, d))
+    zinc = np.empty((B * H, nblk, d))
+    for u in range(B * H):
+        Sb, zb = block_states(k[u], v[u], pos, bands, base, block_frames)
+        S_run = np.zeros((d, d))
+        z_run = np.zeros(d)
+        for b in range(nblk):
+            S_run = S_run + Sb[b]
+            z_run = z_run + zb[b]
+            Sinc[u, b], zinc[u, b] = S_run, z_run
+            sel = blk == b
+            O[u][sel] = head_apply(q[u][sel], g[u][sel], S_run, z_run, pos[sel], bands, base, eps)
+    O = O.reshape(B, H, N, d)
+    if return_state:
+        return O, Sinc.reshape(B, H, nblk, d, d), zinc.reshape(B, H, nblk, d)
+    return O
+
+
+def forward_brute(q, k, v, g, pos, bands, base, eps, visible=None):
+    """O(N^2) form of one head: o_n = sum_m (q_n^r . k_m^r) v_m / (sum_m q_n^+ . k_m^+ + eps) * sigmoid(g_n).
+
+    ``visible[n, m]`` (bool) restricts which keys token n reads; None means all.
+    This is the pair-wise form the linear one is the associative rewrite of.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    qp, kp = relu(q), relu(k)
+    qr, kr = rope3d(qp, pos, bands, base), rope3d(kp, pos, bands, base)
+    N = q.shape[0]
+    out = np.empty_like(q)
+    for n in range(N):
+        m = np.arange(N) if visible is None else np.nonzero(visible[n])[0]
+        a = kr[m] @ qr[n]  # rotated similarities
+        b = kp[m] @ qp[n]  # un-rotated similarities
+        out[n] = (a @ v[m]) / (b.sum() + float(eps)) * sigmoid(g[n])
+    return out

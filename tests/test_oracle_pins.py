@@ -1,0 +1,340 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+The pages print no worked numeric example for this operator, so the oracle is
+pinned by closed forms, textbook special cases, brute force on tiny inputs and
+invariants that the mathematics fixes.  Each pin is chosen so that a plausible
+mistake (a swapped band, a wrong rotation sign, RoPE in the denominator, eps
+inside the dot product, a transposed state, a block that cannot see itself)
+makes at least one of them fail.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle as orc
+from gated_linear_attention_relu_b200 import workloads as wl
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+# --------------------------------------------------------------------------
+# RoPE: closed forms and the properties of a rotation
+# --------------------------------------------------------------------------
+
+def test_band_frequencies_decimal_closed_form():
+    # base 10000, band width 8: base**(-2i/8) = 10**(-i).
+    th = orc.band_frequencies(8, 10000.0)
+    assert np.allclose(th, [1.0, 0.1, 0.01, 0.001], rtol=1e-15, atol=0)
+
+
+def test_grid_positions_row_major_time_slowest():
+    pos = orc.grid_positions(2, 3, 5)
+    assert pos.shape == (30, 3)
+    for n, expect in [(0, (0, 0, 0)), (4, (0, 0, 4)), (5, (0, 1, 0)), (14, (0, 2, 4)),
+                      (15, (1, 0, 0)), (29, (1, 2, 4))]:
+        assert tuple(pos[n]) == expect
+
+
+@pytest.mark.parametrize("channel,angle,pair", [
+    (0, 3.0, (0, 1)),      # t band, pair 0, theta 1, t = 3
+    (2, 0.3, (2, 3)),      # t band, pair 1, theta 0.1, t = 3
+    (10, 0.5, (10, 11)),   # h band (offset 8), pair 1, theta 0.1, h = 5
+    (22, 0.007, (22, 23)), # w band (offset 16), pair 3, theta 0.001, w = 7
+])
+def test_rope_unit_vectors_closed_form(channel, angle, pair):
+    # bands (8, 8, 8), base 10000 -> theta = 1, 0.1, 0.01, 0.001 in every band.
+    pos = np.array([[3, 5, 7]])
+    x = np.zeros((1, 24))
+    x[0, channel] = 1.0
+    y = orc.rope3d(x, pos, (8, 8, 8), 10000.0)[0]
+    expect = np.zeros(24)
+    # The first channel of a pair goes to (cos a, sin a): counter-clockwise rotation.
+    expect[pair[0]] = math.cos(angle)
+    expect[pair[1]] = math.sin(angle)
+    assert np.allclose(y, expect, atol=1e-15)
+    # The second channel of the pair goes to (-sin a, cos a).
+    x2 = np.zeros((1, 24))
+    x2[0, pair[1]] = 1.0
+    y2 = orc.rope3d(x2, pos, (8, 8, 8), 10000.0)[0]
+    expect2 = np.zeros(24)
+    expect2[pair[0]] = -math.sin(angle)
+    expect2[pair[1]] = math.cos(angle)
+    assert np.allclose(y2, expect2, atol=1e-15)
+
+
+def test_rope_matches_complex_multiplication():
+    # RoFormer's complex form: pair (x0, x1) as x0 + i x1, multiplied by exp(i * pos * theta).
+    rng = np.random.default_rng(1)
+    bands = (4, 6, 6)
+    x = _rand(rng, 20, 16)
+    pos = rng.integers(0, 50, size=(20, 3))
+    y = orc.rope3d(x, pos, bands, 100.0)
+    off = 0
+    for axis, D in enumerate(bands):
+        for i in range(D // 2):
+            theta = 100.0 ** (-2.0 * i / D)
+            zc = (x[:, off + 2 * i] + 1j * x[:, off + 2 * i + 1]) * np.exp(1j * pos[:, axis] * theta)
+            assert np.allclose(y[:, off + 2 * i], zc.real, atol=1e-12)
+            assert np.allclose(y[:, off + 2 * i + 1], zc.imag, atol=1e-12)
+        off += D
+
+
+def test_rope_norm_identity_relative_composition():
+    rng = np.random.default_rng(2)
+    bands = (8, 12, 12)
+    x = _rand(rng, 64, 32)
+    y = _rand(rng, 64, 32)
+    p = rng.integers(0, 300, size=(64, 3))
+    p2 = rng.integers(0, 300, size=(64, 3))
+    rx = orc.rope3d(x, p, bands, 10000.0)
+    # norm preservation
+    assert np.allclose(np.linalg.norm(rx, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+    # identity at position 0
+    assert np.array_equal(orc.rope3d(x, np.zeros_like(p), bands, 10000.0), x)
+    # relative property: R(p)x . R(p')y = x . R(p'-p)y
+    lhs = np.sum(rx * orc.rope3d(y, p2, bands, 10000.0), axis=1)
+    rhs = np.sum(x * orc.rope3d(y, p2 - p, bands, 10000.0), axis=1)
+    assert np.allclose(lhs, rhs, rtol=1e-10, atol=1e-10)
+    # composition: R(p') R(p) = R(p + p')
+    assert np.allclose(orc.rope3d(rx, p2, bands, 10000.0), orc.rope3d(x, p + p2, bands, 10000.0),
+                       atol=1e-11)
+
+
+# --------------------------------------------------------------------------
+# The operator: brute force, closed forms, special cases, invariants
+# --------------------------------------------------------------------------
+
+def test_linear_form_equals_brute_form_on_tiny_workload():
+    import torch
+
+    w = wl.WORKLOADS["tiny_f32"]
+    Q, K, V, G = (t.double().numpy() for t in wl.generate(w, "cpu"))
+    O = orc.forward_bidir(Q, K, V, G, (w.T, w.Hh, w.W), w.bands, w.rope_base, w.eps)
+    pos = orc.grid_positions(w.T, w.Hh, w.W)
+    for h in range(w.H):
+        ob = orc.forward_brute(Q[0, h], K[0, h], V[0, h], G[0, h], pos, w.bands, w.rope_base, w.eps)
+        assert np.max(np.abs(ob - O[0, h])) <= 1e-12 * np.max(np.abs(ob))
+    del torch
+
+
+@pytest.mark.parametrize("grid,d,bands", [((3, 5, 7), 16, (4, 6, 6)), ((4, 4, 32), 32, (8, 12, 12)),
+                                          ((1, 1, 1), 8, (2, 2, 4)), ((7, 1, 3), 32, (0, 16, 16))])
+def test_linear_form_equals_brute_form_random_grids(grid, d, bands):
+    rng = np.random.default_rng(sum(grid) + d)
+    N = grid[0] * grid[1] * grid[2]
+    q, k, v, g = (_rand(rng, 1, 1, N, d) for _ in range(4))
+    O = orc.forward_bidir(q, k, v, g, grid, bands, 500.0, 1e-6)[0, 0]
+    ob = orc.forward_brute(q[0, 0], k[0, 0], v[0, 0], g[0, 0], orc.grid_positions(*grid), bands,
+                           500.0, 1e-6)
+    assert np.max(np.abs(ob - O)) <= 1e-11 * np.max(np.abs(ob))
+
+
+def test_single_token_closed_form_and_eps_placement():
+    # N = 1: the rotation cancels (same position), so o = (q+.k+)/(q+.k+ + eps) v sigmoid(g).
+    d = 8
+    q = np.zeros((1, 1, 1, d)); k = np.zeros((1, 1, 1, d))
+    q[..., 3] = 1e-3; q[..., 5] = -2.0  # the negative entry is cut by ReLU
+    k[..., 3] = 1e-3; k[..., 5] = 7.0
+    v = np.arange(1.0, d + 1).reshape(1, 1, 1, d)
+    g = np.full((1, 1, 1, d), 0.3)
+    eps = 1e-6
+    O = orc.forward_bidir(q, k, v, g, (1, 1, 1), (2, 2, 4), 10000.0, eps)[0, 0, 0]
+    dot = 1e-6  # q+ . k+ = 1e-3 * 1e-3
+    expect = dot / (dot + eps) * np.arange(1.0, d + 1) / (1.0 + math.exp(-0.3))
+    assert np.allclose(O, expect, rtol=1e-14)
+    assert np.allclose(O, 0.5 * np.arange(1.0, d + 1) / (1.0 + math.exp(-0.3)), rtol=1e-14)
+
+
+def test_two_token_numerator_rotated_denominator_not():
+    # q = k_m = e0 (t band pair 0, theta 1) at t = 0 and t = 1.
+    d = 8
+    bands = (2, 2, 4)
+    q = np.zeros((1, 1, 2, d)); k = np.zeros((1, 1, 2, d))
+    q[..., 0] = 1.0; k[..., 0] = 1.0
+    a = np.array([1.0, -2.0, 3.0, 0.5, 0.0, 4.0, -1.0, 2.0])
+    b = np.array([0.0, 1.0, -1.0, 2.0, 5.0, -3.0, 1.0, 1.0])
+    v = np.stack([a, b]).reshape(1, 1, 2, d)
+    g = np.full((1, 1, 2, d), 50.0)  # sigmoid = 1 - 2e-22
+    eps = 1e-6
+    O = orc.forward_bidir(q, k, v, g, (2, 1, 1), bands, 10000.0, eps)[0, 0]
+    c1 = math.cos(1.0)
+    assert np.allclose(O[0], (a + c1 * b) / (2.0 + eps), rtol=1e-13)
+    assert np.allclose(O[1], (c1 * a + b) / (2.0 + eps), rtol=1e-13)
+
+
+def test_zero_angles_reduce_to_relu_linear_attention_convex_combination():
+    # All positions 0: no rotation; o / sigmoid(g) is a convex combination of the
+    # value rows up to eps (Katharopoulos-style ReLU linear attention).
+    rng = np.random.default_rng(5)
+    N, d = 50, 16
+    q, k, v, g = (_rand(rng, N, d) for _ in range(4))
+    pos0 = np.zeros((N, 3), dtype=np.int64)
+    O = orc.forward_positions(q, k, v, g, pos0, (4, 6, 6), 10000.0, 0.0)
+    r = O / orc.sigmoid(g)
+    assert np.all(r <= v.max(axis=0) + 1e-12)
+    assert np.all(r >= v.min(axis=0) - 1e-12)
+    # and with V = 1 everywhere, o = sigmoid(g) exactly (eps = 0)
+    O1 = orc.forward_positions(q, k, np.ones_like(v), g, pos0, (4, 6, 6), 10000.0, 0.0)
+    assert np.allclose(O1, orc.sigmoid(g), rtol=1e-13)
+
+
+def test_joint_permutation_equivariance_and_state_invariance():
+    rng = np.random.default_rng(6)
+    N, d, bands = 60, 16, (4, 6, 6)
+    q, k, v, g = (_rand(rng, N, d) for _ in range(4))
+    pos = rng.integers(0, 20, size=(N, 3))
+    perm = rng.permutation(N)
+    O = orc.forward_positions(q, k, v, g, pos, bands, 10000.0, 1e-6)
+    Op = orc.forward_positions(q[perm], k[perm], v[perm], g[perm], pos[perm], bands, 10000.0, 1e-6)
+    assert np.allclose(Op, O[perm], rtol=1e-12, atol=1e-14)
+    S, z = orc.head_state(k, v, pos, bands, 10000.0)
+    Sp, zp = orc.head_state(k[perm], v[perm], pos[perm], bands, 10000.0)
+    assert np.allclose(S, Sp, atol=1e-12) and np.allclose(z, zp, atol=1e-12)
+
+
+@pytest.mark.parametrize("axis", [0, 1, 2])
+def test_translation_invariance(axis):
+    rng = np.random.default_rng(7 + axis)
+    w = wl.custom("t", 1, 1, 3, 4, 5, d=16, bands=(4, 6, 6), dtype="f32")
+    N = w.N
+    q, k, v, g = (_rand(rng, N, 16) for _ in range(4))
+    pos = orc.grid_positions(3, 4, 5)
+    O = orc.forward_positions(q, k, v, g, pos, w.bands, 10000.0, 1e-6)
+    shift = np.zeros(3, dtype=np.int64)
+    shift[axis] = 37
+    O2 = orc.forward_positions(q, k, v, g, pos + shift, w.bands, 10000.0, 1e-6)
+    assert np.allclose(O, O2, rtol=1e-11, atol=1e-13)
+
+
+def test_scale_invariance_in_q_and_k_and_linearity_in_v():
+    rng = np.random.default_rng(8)
+    N, d, bands = 40, 16, (4, 6, 6)
+    q, k, v, v2, g = (_rand(rng, N, d) for _ in range(5))
+    pos = rng.integers(0, 9, size=(N, 3))
+    f = lambda q_, k_, v_: orc.forward_positions(q_, k_, v_, g, pos, bands, 10000.0, 0.0)
+    O = f(q, k, v)
+    assert np.allclose(f(3.5 * q, k, v), O, rtol=1e-12)
+    assert np.allclose(f(q, 0.25 * k, v), O, rtol=1e-12)
+    assert np.allclose(f(q, k, 2.0 * v - 3.0 * v2), 2.0 * O - 3.0 * f(q, k, v2), rtol=1e-10, atol=1e-12)
+
+
+def test_gate_limits():
+    rng = np.random.default_rng(9)
+    N, d, bands = 30, 16, (4, 6, 6)
+    q, k, v = (_rand(rng, N, d) for _ in range(3))
+    pos = rng.integers(0, 9, size=(N, 3))
+    ungated = orc.forward_positions(q, k, v, np.full((N, d), 60.0), pos, bands, 10000.0, 1e-6)
+    half = orc.forward_positions(q, k, v, np.zeros((N, d)), pos, bands, 10000.0, 1e-6)
+    off = orc.forward_positions(q, k, v, np.full((N, d), -800.0), pos, bands, 10000.0, 1e-6)
+    assert np.allclose(half, 0.5 * ungated, rtol=1e-14)
+    assert np.all(off == 0.0)
+
+
+def test_denominator_positive_with_sparse_keys():
+    # K shifted by -0.5 (about 69% of ReLU(K) is zero): the un-rotated denominator stays >= eps.
+    rng = np.random.default_rng(10)
+    N, d = 400, 32
+    q = _rand(rng, N, d)
+    k = _rand(rng, N, d) - 0.5
+    qp, kp = orc.relu(q), orc.relu(k)
+    den = qp @ kp.sum(axis=0) + 1e-6
+    assert np.all(den >= 1e-6)
+    assert 0.6 < np.mean(kp == 0.0) < 0.75
+
+
+# --------------------------------------------------------------------------
+# Block-causal mode
+# --------------------------------------------------------------------------
+
+def _small_blockcausal(rng, grid=(7, 3, 4), d=16, bands=(4, 6, 6), H=2):
+    N = grid[0] * grid[1] * grid[2]
+    return [_rand(rng, 1, H, N, d) for _ in range(4)], grid, d, bands
+
+
+@pytest.mark.parametrize("bf", [1, 2, 3])
+def test_blockcausal_equals_masked_brute_form(bf):
+    rng = np.random.default_rng(11 + bf)
+    (q, k, v, g), grid, d, bands = _small_blockcausal(rng)
+    O = orc.forward_blockcausal(q, k, v, g, grid, bands, 10000.0, 1e-6, block_frames=bf)
+    pos = orc.grid_positions(*grid)
+    blk = pos[:, 0] // bf
+    visible = blk[None, :] <= blk[:, None]  # token n reads every key of blocks <= its own
+    for h in range(q.shape[1]):
+        ob = orc.forward_brute(q[0, h], k[0, h], v[0, h], g[0, h], pos, bands, 10000.0, 1e-6, visible)
+        assert np.max(np.abs(ob - O[0, h])) <= 1e-11 * np.max(np.abs(ob))
+
+
+def test_blockcausal_last_block_equals_bidirectional():
+    rng = np.random.default_rng(20)
+    (q, k, v, g), grid, d, bands = _small_blockcausal(rng)
+    Ob, Sb, zb = orc.forward_bidir(q, k, v, g, grid, bands, 10000.0, 1e-6, return_state=True)
+    Oc, Sc, zc = orc.forward_blockcausal(q, k, v, g, grid, bands, 10000.0, 1e-6, block_frames=2,
+                                         return_state=True)
+    assert np.allclose(Sc[:, :, -1], Sb, atol=1e-12)
+    assert np.allclose(zc[:, :, -1], zb, atol=1e-12)
+    last = orc.grid_positions(*grid)[:, 0] // 2 == Sc.shape[2] - 1
+    assert np.allclose(Oc[:, :, last], Ob[:, :, last], rtol=1e-12, atol=1e-14)
+
+
+def test_blockcausal_one_block_is_bidirectional_and_first_block_is_local():
+    rng = np.random.default_rng(21)
+    (q, k, v, g), grid, d, bands = _small_blockcausal(rng)
+    Ob = orc.forward_bidir(q, k, v, g, grid, bands, 10000.0, 1e-6)
+    for bf in (grid[0], grid[0] + 5):
+        Oc = orc.forward_blockcausal(q, k, v, g, grid, bands, 10000.0, 1e-6, block_frames=bf)
+        assert np.allclose(Oc, Ob, rtol=1e-12, atol=1e-14)
+    # Block 0 (2 frames) equals a bidirectional run on those frames alone.
+    n0 = 2 * grid[1] * grid[2]
+    Oc = orc.forward_blockcausal(q, k, v, g, grid, bands, 10000.0, 1e-6, block_frames=2)
+    O0 = orc.forward_bidir(q[:, :, :n0], k[:, :, :n0], v[:, :, :n0], g[:, :, :n0],
+                           (2, grid[1], grid[2]), bands, 10000.0, 1e-6)
+    assert np.allclose(Oc[:, :, :n0], O0, rtol=1e-12, atol=1e-14)
+
+
+def test_blockcausal_inclusive_states_are_prefix_sums_of_block_states():
+    rng = np.random.default_rng(22)
+    (q, k, v, g), grid, d, bands = _small_blockcausal(rng, H=1)
+    _, Sc, zc = orc.forward_blockcausal(q, k, v, g, grid, bands, 10000.0, 1e-6, block_frames=3,
+                                        return_state=True)
+    pos = orc.grid_positions(*grid)
+    Sb, zb = orc.block_states(k[0, 0], v[0, 0], pos, bands, 10000.0, 3)
+    assert Sb.shape[0] == 3  # 7 frames in blocks of 3: 3, 3, 1
+    assert np.allclose(np.cumsum(Sb, axis=0), Sc[0, 0], atol=1e-12)
+    assert np.allclose(np.cumsum(zb, axis=0), zc[0, 0], atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Planted mistakes: each must be caught by one of the pins above
+# --------------------------------------------------------------------------
+
+def _rotated_denominator_forward(q, k, v, g, pos, bands, base, eps):
+    qp, kp = orc.relu(q), orc.relu(k)
+    qr, kr = orc.rope3d(qp, pos, bands, base), orc.rope3d(kp, pos, bands, base)
+    return (qr @ (kr.T @ v)) / ((qr @ kr.sum(0)) + eps)[:, None] * orc.sigmoid(g)
+
+
+def test_planted_rotated_denominator_is_caught():
+    d = 8
+    q = np.zeros((2, d)); k = np.zeros((2, d)); q[:, 0] = 1.0; k[:, 0] = 1.0
+    v = np.eye(2, d)
+    g = np.full((2, d), 50.0)
+    pos = orc.grid_positions(2, 1, 1)
+    good = orc.forward_positions(q, k, v, g, pos, (2, 2, 4), 10000.0, 1e-6)
+    bad = _rotated_denominator_forward(q, k, v, g, pos, (2, 2, 4), 10000.0, 1e-6)
+    expect0 = (v[0] + math.cos(1.0) * v[1]) / (2.0 + 1e-6)
+    assert np.allclose(good[0], expect0, rtol=1e-13)
+    assert not np.allclose(bad[0], expect0, rtol=1e-3)
+
+
+def test_planted_transposed_state_is_caught_by_brute_form():
+    rng = np.random.default_rng(30)
+    N, d, bands = 24, 8, (2, 2, 4)
+    q, k, v, g = (_rand(rng, N, d) for _ in range(4))
+    pos = orc.grid_positions(2, 3, 4)
+    S, z = orc.head_state(k, v, pos, bands, 10000.0)
+    bad = orc.head_apply(q, g, S.T, z, pos, bands, 10000.0, 1e-6)
+    ob = orc.forward_brute(q, k, v, g, pos, bands, 10000.0, 1e-6)
+    assert np.max(np.abs(bad - ob)) > 1e-3 * np.max(np.abs(ob))
