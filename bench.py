@@ -1,0 +1,348 @@
+#!/usr/bin/env python
+"""Throughput of the gated ReLU linear-attention token mixer on B200.
+
+One step = the whole operator (state reduction, combine, apply) over one synthetic
+720p/5s-shaped problem (B=1, H=32, d=128, 21 x 45 x 80 latent grid, N = 75,600) already
+resident in HBM.  Prints one JSON line.  Multi-GPU runs (torchrun) give every rank its own
+problem (weak scaling, no collective on the data path); the time is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gated linear-attn tokens·heads/s at 720p shapes; % of B200 HBM roofline"
+UNIT = "tokens*heads/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = {
+    "apply_tc_kernel": "gated_linear_attention_relu_b200/csrc/apply_tc.cuh",
+    "state_tc_kernel": "gated_linear_attention_relu_b200/csrc/state_tc.cuh",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="720p_5s")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--simt", action="store_true", help="force the CUDA-core kernels")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work of the oracle baseline")
+    return ap.parse_args()
+
+
+def measured_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_traffic(name):
+    """DRAM bytes per launch of `name` from the committed ncu summary, if the kernel source is
+    unchanged since the capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[name]
+        src = os.path.join(ROOT, KERNEL_SOURCES[name])
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if rec.get("source_sha") != sha:
+            return None, rec
+        return rec, rec
+    except Exception:
+        return None, None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clocks"}
+
+    def __init__(self, index, period=0.005):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period, self._stop = period, threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # clocks are reported as unavailable
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = get_r(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+def oracle_sample(w, seconds, steps=None, warmup=0):
+    """Time the fp64 oracle on one head of the workload (all its tokens): token*heads/s."""
+    import numpy as np
+
+    import oracle as orc
+    from gated_linear_attention_relu_b200 import workloads as wl
+
+    one = w.with_(B=1, H=1)
+    Q, K, V, G = (t.float().numpy().astype(np.float64)[0, 0] for t in wl.generate(one, "cpu"))
+    pos = orc.grid_positions(w.T, w.Hh, w.W)
+
+    def run():
+        if w.block_frames > 0:
+            Sb, zb = orc.block_states(K, V, pos, w.bands, w.rope_base, w.block_frames)
+            Si, zi = np.cumsum(Sb, 0), np.cumsum(zb, 0)
+            blk = orc.block_of_tokens(pos, w.block_frames)
+            for b in range(Si.shape[0]):
+                sel = blk == b
+                orc.head_apply(Q[sel], G[sel], Si[b], zi[b], pos[sel], w.bands, w.rope_base, w.eps)
+        else:
+            S, z = orc.head_state(K, V, pos, w.bands, w.rope_base)
+            orc.head_apply(Q, G, S, z, pos, w.bands, w.rope_base, w.eps)
+
+    for _ in range(warmup):
+        run()
+    times = []
+    t_all = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t0)
+        if steps is not None and len(times) >= steps:
+            break
+        if steps is None and time.perf_counter() - t_all >= seconds:
+            break
+    threads = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        pass
+    value = w.N * len(times) / sum(times)
+    return value, threads, times
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from gated_linear_attention_relu_b200 import workloads as wl
+
+    w = wl.WORKLOADS[args.workload]
+    value, cores, times = oracle_sample(w, 0, steps=max(1, args.steps), warmup=max(0, args.warmup))
+    sample = f"one head of {w.name} (all {w.N} tokens), fp64 numpy oracle, per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": len(times), "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, n):
+    return {"workload": w.name, "B": w.B, "H": w.H, "grid_T_Hh_W": [w.T, w.Hh, w.W], "N": w.N, "d": w.d,
+            "rope_bands": list(w.bands), "block_frames": w.block_frames, "global_batch": w.B * n,
+            "seq_len": w.N, "parallelism": f"dp{n}" if n > 1 else "single",
+            "l2": f"inputs {w.min_bytes * 4 / 5 / 1e9:.2f} GB > 126 MB L2 (no flush)"}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+
+    import gated_linear_attention_relu_b200 as la
+    from gated_linear_attention_relu_b200 import dist as ldist
+    from gated_linear_attention_relu_b200 import workloads as wl
+
+    rank, local, world = ldist.env_rank()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ldist.init("nccl")
+    w = wl.WORKLOADS[args.workload]
+    p = la.Problem.from_workload(w, force_simt=args.simt)
+    la.load()
+
+    Q, K, V, G = wl.generate(w, dev, seed=w.seed + 1000 * rank)
+    O = torch.empty_like(Q)
+    ws, _ = la.workspace(p, dev)
+    stream = torch.cuda.current_stream()
+    S_incl = z_incl = None
+    if w.block_frames > 0:
+        S_incl = torch.empty((w.B, w.H, w.nblk, w.d, w.d), dtype=torch.float32, device=dev)
+        z_incl = torch.empty((w.B, w.H, w.nblk, w.d), dtype=torch.float32, device=dev)
+
+    # Marker events around each kernel of each timed step; recorded once here so their CUDA
+    # handles exist before the timed region.
+    nmark = 4
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nmark)] for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    for _ in range(max(3, args.warmup)):
+        la.forward_marked(p, Q, K, V, G, O, ws, evs[0], S_incl, z_incl)
+    launches_per_step = la.last_launch_count()
+    torch.cuda.synchronize()
+    assert la.device_error() == 0, "device-side error during warm-up"
+
+    # Timed region: K steps bracketed by a barrier and a synchronize on both sides.
+    ldist.barrier(dev)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            la.forward_marked(p, Q, K, V, G, O, ws, evs[k], S_incl, z_incl)
+        end.record(stream)
+        torch.cuda.synchronize()
+    ldist.barrier(dev)
+    t_ms = start.elapsed_time(end)
+    t_max = ldist.max_over_ranks(t_ms, dev)
+    assert la.device_error() == 0, "device-side error in the timed region"
+
+    # Per-kernel durations inside the timed steps.
+    names = ["state_tc_kernel", "combine_kernel", "apply_tc_kernel"] if not args.simt and w.d == 128 \
+        and w.dtype == "bf16" else ["state_simt_kernel", "combine_kernel", "apply_simt_kernel"]
+    names = names[:launches_per_step]
+    per = {n: [] for n in names}
+    for k in range(args.steps):
+        for i, n in enumerate(names):
+            per[n].append(evs[k][i].elapsed_time(evs[k][i + 1]))
+    kern_ms = {n: sum(v) / len(v) for n, v in per.items()}
+    tot = sum(kern_ms.values())
+    elem = w.elem_bytes
+    th = w.B * w.H * w.N
+    alg_bytes = {names[0]: 2 * th * w.d * elem, names[-1]: 3 * th * w.d * elem}
+    dominant = max((n for n in names if n in alg_bytes), key=lambda n: kern_ms[n])
+    peak, peak_kind = measured_hbm()
+    achieved = alg_bytes[dominant] / (kern_ms[dominant] * 1e-3) / 1e9
+    traffic_rec, _ = kernel_traffic(dominant)
+    traffic = None
+    if traffic_rec is not None and traffic_rec.get("workload") == w.name:
+        traffic = traffic_rec.get("bytes_per_launch")
+
+    value = world * th * args.steps / (t_max * 1e-3)
+    ms_per_step = t_max / args.steps
+    roof_all = w.min_bytes / (ms_per_step * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
+        "config": config_of(w, world),
+        "hbm_roofline_frac_8tbs": roof_all / NOMINAL_HBM_GBS,
+        "hbm_roofline_frac_measured": roof_all / peak,
+        "achieved_gbs_whole_step": roof_all,
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": alg_bytes[dominant]},
+        "kernels": {n: {"ms": kern_ms[n], "share": kern_ms[n] / tot if tot else None} for n in names},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, times = oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"one head of {w.name} (all {w.N} tokens), {len(times)} runs, "
+                                          f"fp64 numpy oracle"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ldist.finalize()
+    return 0
+
+
+def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world):
+    """Same metric through the public API with the inputs in pinned host memory: every step
+    copies Q, K, V, G host->device, runs the operator and copies O device->host."""
+    import torch
+
+    hosts = [t.cpu().pin_memory() for t in (Q, K, V, G)]
+    Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    steps = max(3, min(args.steps, 10))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for hsrc, dst in zip(hosts, (Q, K, V, G)):
+            dst.copy_(hsrc, non_blocking=True)
+        la.forward(p, Q, K, V, G, O=O, ws=ws)
+        Oh.copy_(O, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    ldist.barrier(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    t = ldist.max_over_ranks(s.elapsed_time(e), dev)
+    th = w.B * w.H * w.N
+    nbytes = Q.numel() * Q.element_size()
+    return {"value": world * th * steps / (t * 1e-3), "unit": UNIT, "h2d_bytes_per_step": 4 * nbytes,
+            "d2h_bytes_per_step": nbytes, "steps": steps}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

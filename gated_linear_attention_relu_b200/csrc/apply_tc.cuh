@@ -1,0 +1,311 @@
+// apply_tc.cuh -- apply step on the 5th-generation tensor cores (bf16, d = 128).
+//
+//   O_n = (RoPE(ReLU(Q_n)) S) / (ReLU(Q_n) . z + eps) * sigmoid(G_n)
+// (SANA-Video 2.0, Eq. (1); SANA-Video Sec. 3.2: rotated numerator, un-rotated denominator).
+//
+// Per 128-token tile one tcgen05 MMA chain computes the numerator D[128 tok x 128] =
+// A[128 tok x 128 ch] * S[128 x 128], with A = RoPE(ReLU(Q)) written in place over the staged
+// Q tile (K-major, 128B swizzle) and S the unit's state as a bf16 operand (N-major).  The
+// denominator, the divide and the gate run on the CUDA cores around it: the thread that
+// transforms row n of Q also owns TMEM lane n, so the denominator never leaves its register.
+//
+// Warps (one CTA per SM, persistent over a contiguous range of tiles):
+//   warp 0      TMA producer: Q and G tiles, plus the state operand once per unit (bulk copy)
+//   warp 1      MMA issuer
+//   warps 2-5   math group 0 (even local tiles), warps 6-9 math group 1 (odd local tiles):
+//               transform Q, then epilogue: TMEM -> registers, divide, gate, bf16, written in
+//               place over the staged G tile
+//   warp 10     TMA store of the finished O tile, then releases the G stage
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace la {
+namespace ap {
+
+constexpr int TILE = 128;
+constexpr int D = 128;
+constexpr int QST = 3;   // Q stages
+constexpr int GST = 2;   // G / O stages
+constexpr int NSB = 2;   // state operand buffers
+constexpr int THREADS = 352;
+constexpr uint32_t HALF = 128 * 128;
+constexpr uint32_t BUF = 2 * HALF;  // 32 KB: a 128 x 128 bf16 tile
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_G = OFF_Q + QST * BUF;
+constexpr uint32_t OFF_S = OFF_G + GST * BUF;
+constexpr uint32_t OFF_Z = OFF_S + NSB * BUF;
+constexpr uint32_t OFF_BAR = OFF_Z + NSB * 512;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
+constexpr uint32_t TMEM_COLS = 256;                    // one 128-column accumulator per math group
+constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/true);
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+struct Bars {
+  uint64_t qfull[QST], aready[QST], qempty[QST];
+  uint64_t gfull[GST], gempty[GST], ostaged[GST];
+  uint64_t sfull[NSB], sfree[NSB];
+  uint64_t accfull[2], accempty[2];
+  uint64_t final_;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block too large");
+
+__device__ __forceinline__ float sigmoidf_fast(float g) { return __frcp_rn(1.0f + __expf(-g)); }
+
+__global__ void __launch_bounds__(THREADS, 1)
+apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
+                const __grid_constant__ CUtensorMap tmO, const Plan p, const __grid_constant__ Rope rope,
+                const uint8_t* __restrict__ simg, const float* __restrict__ zimg,
+                __nv_bfloat16* __restrict__ O) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
+  const uint32_t sbase = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t c = blockIdx.x;
+  const int64_t g0 = cta_start(p, c);
+  const int64_t g1 = cta_start(p, c + 1);
+  const int64_t u_first = unit_of_tile(p, g0);
+  volatile int* abort_flag = &bars->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < QST; ++s) {
+      mbar_init(&bars->qfull[s], 1);
+      mbar_init(&bars->aready[s], 4);
+      mbar_init(&bars->qempty[s], 1);
+    }
+    for (int s = 0; s < GST; ++s) {
+      mbar_init(&bars->gfull[s], 1);
+      mbar_init(&bars->gempty[s], 1);
+      mbar_init(&bars->ostaged[s], 4);
+    }
+    for (int s = 0; s < NSB; ++s) {
+      mbar_init(&bars->sfull[s], 1);
+      mbar_init(&bars->sfree[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bars->accfull[a], 1);
+      mbar_init(&bars->accempty[a], 4);
+    }
+    mbar_init(&bars->final_, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmG);
+    tma_prefetch_desc(&tmO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int64_t issued_q = 0, issued_g = 0, issued_s = 0;
+      int64_t prev_unit = -1;
+      for (int64_t g = g0; g < g1; ++g) {
+        const int64_t i = g - g0;
+        const TileInfo ti = tile_info(p, g);
+        if (ti.unit != prev_unit) {
+          const int64_t ku = ti.unit - u_first;
+          const int b = static_cast<int>(ku % NSB);
+          if (!mbar_wait(&bars->sfree[b], static_cast<uint32_t>(((ku / NSB) & 1) ^ 1), abort_flag)) break;
+          mbar_arrive_expect_tx(&bars->sfull[b], BUF + 512);
+          bulk_load(smem + OFF_S + b * BUF, simg + ti.unit * static_cast<int64_t>(BUF), BUF, &bars->sfull[b]);
+          bulk_load(smem + OFF_Z + b * 512, zimg + ti.unit * D, 512, &bars->sfull[b]);
+          prev_unit = ti.unit;
+          ++issued_s;
+        }
+        const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
+        const int qs = static_cast<int>(i % QST);
+        if (!mbar_wait(&bars->qempty[qs], static_cast<uint32_t>(((i / QST) & 1) ^ 1), abort_flag)) break;
+        mbar_arrive_expect_tx(&bars->qfull[qs], BUF);
+        tma_load_3d(smem + OFF_Q + qs * BUF, &tmQ, 0, n0, bh, &bars->qfull[qs]);
+        tma_load_3d(smem + OFF_Q + qs * BUF + HALF, &tmQ, 64, n0, bh, &bars->qfull[qs]);
+        ++issued_q;
+        const int gs = static_cast<int>(i % GST);
+        if (!mbar_wait(&bars->gempty[gs], static_cast<uint32_t>(((i / GST) & 1) ^ 1), abort_flag)) break;
+        mbar_arrive_expect_tx(&bars->gfull[gs], BUF);
+        tma_load_3d(smem + OFF_G + gs * BUF, &tmG, 0, n0, bh, &bars->gfull[gs]);
+        tma_load_3d(smem + OFF_G + gs * BUF + HALF, &tmG, 64, n0, bh, &bars->gfull[gs]);
+        ++issued_g;
+      }
+      if (*abort_flag) {
+        // Let every copy still in flight land before the CTA's shared memory goes away.
+        for (int64_t j = (issued_q > QST ? issued_q - QST : 0); j < issued_q; ++j)
+          mbar_wait_drain(&bars->qfull[j % QST], static_cast<uint32_t>((j / QST) & 1));
+        for (int64_t j = (issued_g > GST ? issued_g - GST : 0); j < issued_g; ++j)
+          mbar_wait_drain(&bars->gfull[j % GST], static_cast<uint32_t>((j / GST) & 1));
+        for (int64_t j = (issued_s > NSB ? issued_s - NSB : 0); j < issued_s; ++j)
+          mbar_wait_drain(&bars->sfull[j % NSB], static_cast<uint32_t>((j / NSB) & 1));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      for (int64_t g = g0; g < g1; ++g) {
+        const int64_t i = g - g0;
+        const int64_t u = unit_of_tile(p, g);
+        const int64_t ku = u - u_first;
+        const int b = static_cast<int>(ku % NSB);
+        const int wg = static_cast<int>(i & 1);
+        const int qs = static_cast<int>(i % QST);
+        const uint32_t qph = static_cast<uint32_t>((i / QST) & 1);
+        if (!mbar_wait(&bars->accempty[wg], static_cast<uint32_t>(((i >> 1) & 1) ^ 1), abort_flag)) break;
+        if (!mbar_wait(&bars->sfull[b], static_cast<uint32_t>((ku / NSB) & 1), abort_flag)) break;
+        if (!mbar_wait(&bars->qfull[qs], qph, abort_flag)) break;
+        if (!mbar_wait(&bars->aready[qs], qph, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + static_cast<uint32_t>(wg) * 128u;
+        const uint32_t qa = sbase + OFF_Q + qs * BUF;
+        const uint32_t sa = sbase + OFF_S + b * BUF;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(qa + (kk >> 2) * HALF + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sa + kk * 2048, HALF, 1024);
+          mma_bf16(acc, ad, bd, IDESC, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->accfull[wg]);
+        mma_commit(&bars->qempty[qs]);
+        const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != u);
+        if (last) mma_commit(&bars->sfree[b]);
+      }
+      mma_commit(&bars->final_);
+      mbar_wait_drain(&bars->final_, 0);
+    }
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ math groups
+    const int wg = (warp - 2) >> 2;
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;
+    const uint32_t swz = static_cast<uint32_t>(row & 7);
+    const uint32_t row_off = static_cast<uint32_t>(row) * 128u;
+    for (int64_t g = g0 + wg; g < g1; g += 2) {
+      const int64_t i = g - g0;
+      const TileInfo ti = tile_info(p, g);
+      const int64_t ku = ti.unit - u_first;
+      const int b = static_cast<int>(ku % NSB);
+      const int qs = static_cast<int>(i % QST);
+      const int gs = static_cast<int>(i % GST);
+      if (!warp_wait(&bars->sfull[b], static_cast<uint32_t>((ku / NSB) & 1), abort_flag)) break;
+      if (!warp_wait(&bars->qfull[qs], static_cast<uint32_t>((i / QST) & 1), abort_flag)) break;
+
+      // -- transform: A = RoPE(ReLU(q)) in place, den = ReLU(q) . z
+      const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
+      uint32_t pt, ph, pw;
+      token_pos(p, n, pt, ph, pw);
+      const uint32_t qrow = sbase + OFF_Q + qs * BUF + row_off;
+      const uint32_t zb = sbase + OFF_Z + b * 512;
+      float den = 0.f;
+#pragma unroll
+      for (int ck = 0; ck < 16; ++ck) {
+        const uint32_t addr = qrow + (ck >> 3) * HALF + (((static_cast<uint32_t>(ck) & 7u) ^ swz) << 4);
+        const uint4 raw = lds128(addr);
+        const float4 za = lds128f(zb + ck * 32);
+        const float4 zc = lds128f(zb + ck * 32 + 16);
+        const float zz[8] = {za.x, za.y, za.z, za.w, zc.x, zc.y, zc.z, zc.w};
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float x0 = fmaxf(bf16lo(w[q]), 0.f);
+          const float x1 = fmaxf(bf16hi(w[q]), 0.f);
+          den = fmaf(x0, zz[2 * q], den);
+          den = fmaf(x1, zz[2 * q + 1], den);
+          const int pi = 4 * ck + q;
+          const int bnd = rope.band[pi];
+          const uint32_t pos = bnd == 0 ? pt : (bnd == 1 ? ph : pw);
+          float sn, cs;
+          __sincosf(static_cast<float>(pos) * rope.theta[pi], &sn, &cs);
+          o[q] = pack_bf16(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+        }
+        sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->aready[qs]);
+      const float inv = 1.0f / (den + p.eps);
+
+      // -- epilogue: O = acc * inv * sigmoid(g), bf16, in place over the G tile
+      if (!warp_wait(&bars->accfull[wg], static_cast<uint32_t>((i >> 1) & 1), abort_flag)) break;
+      if (!warp_wait(&bars->gfull[gs], static_cast<uint32_t>((i / GST) & 1), abort_flag)) break;
+      tc_fence_after();
+      const bool tma_out = (ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N);
+      const bool valid = static_cast<int64_t>(n) < ti.n_end;
+      const uint32_t grow = sbase + OFF_G + gs * BUF + row_off;
+      __nv_bfloat16* orow = O + (ti.bh * p.N + static_cast<int64_t>(n)) * D;
+      const uint32_t taddr = tmem + static_cast<uint32_t>(wg) * 128u + (static_cast<uint32_t>(quarter * 32) << 16);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t r[32];
+        tmem_ld_x32(taddr + ch * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int ck = ch * 4 + cc;
+          const uint32_t addr = grow + (ck >> 3) * HALF + (((static_cast<uint32_t>(ck) & 7u) ^ swz) << 4);
+          const uint4 graw = lds128(addr);
+          const uint32_t gw[4] = {graw.x, graw.y, graw.z, graw.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float a0 = __uint_as_float(r[cc * 8 + 2 * q]) * inv;
+            const float a1 = __uint_as_float(r[cc * 8 + 2 * q + 1]) * inv;
+            o[q] = pack_bf16(a0 * sigmoidf_fast(bf16lo(gw[q])), a1 * sigmoidf_fast(bf16hi(gw[q])));
+          }
+          const uint4 ov = make_uint4(o[0], o[1], o[2], o[3]);
+          if (tma_out) {
+            sts128(addr, ov);
+          } else if (valid) {
+            *reinterpret_cast<uint4*>(orow + ck * 8) = ov;
+          }
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars->accempty[wg]);
+        mbar_arrive(&bars->ostaged[gs]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ TMA store of O
+    if (lane == 0) {
+      for (int64_t g = g0; g < g1; ++g) {
+        const int64_t i = g - g0;
+        const int gs = static_cast<int>(i % GST);
+        if (!mbar_wait(&bars->ostaged[gs], static_cast<uint32_t>((i / GST) & 1), abort_flag)) break;
+        const TileInfo ti = tile_info(p, g);
+        if ((ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N)) {
+          const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
+          tma_store_3d(&tmO, smem + OFF_G + gs * BUF, 0, n0, bh);
+          tma_store_3d(&tmO, smem + OFF_G + gs * BUF + HALF, 64, n0, bh);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        mbar_arrive(&bars->gempty[gs]);
+      }
+      bulk_wait_group0();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace ap
+}  // namespace la

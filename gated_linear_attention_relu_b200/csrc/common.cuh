@@ -1,0 +1,111 @@
+// common.cuh -- work decomposition shared by the kernels.
+//
+// Tokens are grouped in "units": one unit is the token range one state is reduced over
+// (a whole head in bidirectional mode, one block of latent frames of a head in block-causal
+// mode).  Each unit is cut into tiles of `tile` tokens; the last tile of a unit may be
+// ragged.  Tiles are numbered globally, head-major then block then tile, and a persistent
+// grid of `grid` CTAs splits that sequence into contiguous, nearly equal ranges:
+// CTA c owns tiles [c*total/grid, (c+1)*total/grid).  A CTA whose range crosses a unit
+// boundary emits one partial state per unit it touches ("segment" k = 0, 1, ...), into slot
+// c*maxseg + k.  The combine kernel sums the slots of a unit in increasing c, so the result
+// is the same bit for bit on every run.
+#pragma once
+#include <cstdint>
+
+namespace la {
+
+struct Plan {
+  int64_t BH;              // B * H
+  int64_t N;               // tokens per head
+  int64_t T, Hh, W, HW;    // latent grid
+  int64_t nblk;            // units per head (1 when bidirectional)
+  int64_t blk_tokens;      // tokens of a full unit
+  int64_t tile;            // tokens per tile
+  int64_t tiles_full;      // tiles of a full unit
+  int64_t tiles_last;      // tiles of the last unit of a head
+  int64_t tiles_per_head;
+  int64_t total;           // total tiles
+  int32_t grid;            // persistent CTAs (each owns >= 1 tile when total > 0)
+  int32_t maxseg;          // partial slots per CTA
+  int32_t d;
+  int32_t zparts;          // partial z rows per slot (summed in order by the combine kernel)
+  float eps;
+};
+
+// Rotation parameters of the d/2 channel pairs (at most 64 for d = 128).
+struct Rope {
+  float theta[64];      // base^(-2i/D) of the pair's band, fp32
+  double theta_d[64];   // same in fp64
+  int32_t band[64];     // 0: t, 1: h, 2: w
+};
+
+struct TileInfo {
+  int64_t bh;      // flat head index b*H + h
+  int64_t unit;    // bh * nblk + blk
+  int64_t n0;      // first token of the tile (within the head)
+  int64_t n_end;   // one past the last token of the tile's unit
+};
+
+__host__ __device__ inline TileInfo tile_info(const Plan& p, int64_t g) {
+  TileInfo t;
+  t.bh = g / p.tiles_per_head;
+  int64_t r = g - t.bh * p.tiles_per_head;
+  int64_t blk = r / p.tiles_full;
+  if (blk > p.nblk - 1) blk = p.nblk - 1;
+  int64_t tib = r - blk * p.tiles_full;
+  int64_t start = blk * p.blk_tokens;
+  int64_t end = start + p.blk_tokens;
+  if (end > p.N) end = p.N;
+  t.unit = t.bh * p.nblk + blk;
+  t.n0 = start + tib * p.tile;
+  t.n_end = end;
+  return t;
+}
+
+__host__ __device__ inline int64_t unit_of_tile(const Plan& p, int64_t g) {
+  int64_t bh = g / p.tiles_per_head;
+  int64_t blk = (g - bh * p.tiles_per_head) / p.tiles_full;
+  if (blk > p.nblk - 1) blk = p.nblk - 1;
+  return bh * p.nblk + blk;
+}
+
+__host__ __device__ inline int64_t cta_start(const Plan& p, int64_t c) { return c * p.total / p.grid; }
+
+// The CTA whose range holds tile g.
+__host__ __device__ inline int64_t cta_of(const Plan& p, int64_t g) {
+  return ((g + 1) * static_cast<int64_t>(p.grid) - 1) / p.total;
+}
+
+// Global tile range [first, first + count) of unit u.
+__host__ __device__ inline void unit_tiles(const Plan& p, int64_t u, int64_t* first, int64_t* count) {
+  int64_t bh = u / p.nblk;
+  int64_t blk = u - bh * p.nblk;
+  *first = bh * p.tiles_per_head + blk * p.tiles_full;
+  *count = (blk == p.nblk - 1) ? p.tiles_last : p.tiles_full;
+}
+
+// Grid position of token n, row-major over (T, Hh, W) with t slowest.
+__device__ __forceinline__ void token_pos(const Plan& p, uint32_t n, uint32_t& t, uint32_t& h, uint32_t& w) {
+  uint32_t hw = static_cast<uint32_t>(p.HW);
+  uint32_t W = static_cast<uint32_t>(p.W);
+  t = n / hw;
+  uint32_t rem = n - t * hw;
+  h = rem / W;
+  w = rem - h * W;
+}
+
+// Advance a grid position by `step` tokens.
+__device__ __forceinline__ void token_pos_advance(const Plan& p, uint32_t step, uint32_t& t, uint32_t& h,
+                                                  uint32_t& w) {
+  uint32_t W = static_cast<uint32_t>(p.W), Hh = static_cast<uint32_t>(p.Hh);
+  w += step;
+  while (w >= W) {
+    w -= W;
+    if (++h >= Hh) {
+      h = 0;
+      ++t;
+    }
+  }
+}
+
+}  // namespace la

@@ -1,0 +1,496 @@
+// la_api.cu -- the C ABI declared in include/la.h: argument checks, work planning, TMA
+// descriptors and kernel launches.  Single translation unit: the kernels are included here.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "la.h"
+#include "common.cuh"
+#include "sm100.cuh"
+#include "state_tc.cuh"
+#include "apply_tc.cuh"
+#include "simt.cuh"
+
+namespace {
+
+using la::Plan;
+using la::Rope;
+
+thread_local int g_last_launches = 0;
+
+constexpr int64_t kMaxTokens = (int64_t(1) << 31) - 1024;  // token indices stay in 32 bits
+
+// ------------------------------------------------------------------------------- validation
+bool is_pow2_dim(int32_t d) { return d == 32 || d == 64 || d == 128; }
+
+int validate(const la_problem* p) {
+  if (!p) return LA_ERR_NULL;
+  if (p->B < 0 || p->H < 0 || p->T < 0 || p->Hh < 0 || p->W < 0 || p->block_frames < 0) return LA_ERR_SHAPE;
+  if (p->dtype != LA_BF16 && p->dtype != LA_F32) return LA_ERR_UNSUPPORTED;
+  if ((p->flags & ~LA_FLAG_FORCE_SIMT) != 0u) return LA_ERR_UNSUPPORTED;
+  if (!is_pow2_dim(p->d)) return LA_ERR_UNSUPPORTED;
+  if (p->dt < 0 || p->dh < 0 || p->dw < 0 || (p->dt & 1) || (p->dh & 1) || (p->dw & 1) ||
+      p->dt + p->dh + p->dw != p->d)
+    return LA_ERR_BANDS;
+  if (!(p->rope_base > 0.0) || !std::isfinite(p->rope_base)) return LA_ERR_SHAPE;
+  if (!std::isfinite(p->eps) || p->eps < 0.f) return LA_ERR_SHAPE;
+  // Overflow-safe size checks.
+  const int64_t lim = int64_t(1) << 31;
+  if (p->T >= lim || p->Hh >= lim || p->W >= lim || p->B >= lim || p->H >= lim) return LA_ERR_SHAPE;
+  const double n = double(p->T) * double(p->Hh) * double(p->W);
+  if (n > double(kMaxTokens)) return LA_ERR_SHAPE;
+  if (double(p->B) * double(p->H) > double(lim - 1)) return LA_ERR_SHAPE;
+  if (double(p->B) * double(p->H) * n * double(p->d) > 4.0e18) return LA_ERR_SHAPE;
+  return LA_OK;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+// Checks a tensor pointer that must be present whenever the problem has elements.
+int check_ptr(const void* ptr, bool needed) {
+  if (!needed) return LA_OK;
+  if (!ptr) return LA_ERR_NULL;
+  if (!aligned16(ptr)) return LA_ERR_ALIGN;
+  return LA_OK;
+}
+
+// ------------------------------------------------------------------------------- planning
+Plan build_plan(const la_problem& q, int64_t tile, int64_t grid_cap, int zparts) {
+  Plan p;
+  std::memset(&p, 0, sizeof p);
+  p.BH = q.B * q.H;
+  p.T = q.T;
+  p.Hh = q.Hh;
+  p.W = q.W;
+  p.HW = q.Hh * q.W;
+  p.N = q.T * p.HW;
+  p.d = q.d;
+  p.zparts = zparts;
+  p.eps = q.eps;
+  p.tile = tile;
+  if (q.block_frames > 0) {
+    p.nblk = (q.T + q.block_frames - 1) / q.block_frames;
+    p.blk_tokens = int64_t(q.block_frames) * p.HW;
+  } else {
+    p.nblk = 1;
+    p.blk_tokens = p.N;
+  }
+  if (p.N == 0 || p.BH == 0 || p.nblk == 0) {
+    p.total = 0;
+    p.grid = 0;
+    p.maxseg = 0;
+    p.tiles_full = p.tiles_last = p.tiles_per_head = 0;
+    return p;
+  }
+  const int64_t full_len = p.blk_tokens < p.N ? p.blk_tokens : p.N;
+  const int64_t last_len = p.N - (p.nblk - 1) * p.blk_tokens;
+  p.tiles_full = (full_len + tile - 1) / tile;
+  p.tiles_last = (last_len + tile - 1) / tile;
+  p.tiles_per_head = (p.nblk - 1) * p.tiles_full + p.tiles_last;
+  p.total = p.BH * p.tiles_per_head;
+  p.grid = static_cast<int32_t>(p.total < grid_cap ? p.total : grid_cap);
+  int64_t maxseg = 0;
+  for (int64_t c = 0; c < p.grid; ++c) {
+    const int64_t a = la::cta_start(p, c), b = la::cta_start(p, c + 1);
+    const int64_t segs = la::unit_of_tile(p, b - 1) - la::unit_of_tile(p, a) + 1;
+    if (segs > maxseg) maxseg = segs;
+  }
+  p.maxseg = static_cast<int32_t>(maxseg);
+  return p;
+}
+
+struct PlanSet {
+  bool tc;            // tensor-core kernels (bf16, d = 128)
+  Plan ps;            // state reduction
+  Plan pa;            // apply
+  int64_t units;      // B*H*nblk
+  size_t off_partial, off_states, off_img, off_zimg, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+PlanSet make_plans(const la_problem& q, int sm_count) {
+  PlanSet s;
+  s.tc = q.dtype == LA_BF16 && q.d == 128 && !(q.flags & LA_FLAG_FORCE_SIMT);
+  if (s.tc) {
+    s.ps = build_plan(q, la::st::TILE, sm_count, la::st::ZPARTS);
+    s.pa = build_plan(q, la::ap::TILE, sm_count, 1);
+  } else {
+    s.ps = build_plan(q, la::simt::TS, int64_t(sm_count) * 2, 1);
+    s.pa = build_plan(q, la::simt::TS, sm_count, 1);
+  }
+  const int64_t D = q.d;
+  s.units = s.ps.BH * s.ps.nblk;
+  const size_t slot_bytes = size_t(D * D + int64_t(s.ps.zparts) * D) * 4;
+  size_t off = 0;
+  s.off_partial = off;
+  off = align256(off + size_t(s.ps.grid) * size_t(s.ps.maxseg) * slot_bytes);
+  s.off_states = off;
+  off = align256(off + size_t(s.units) * size_t(D * D + D) * 4);
+  s.off_img = off;
+  off = align256(off + (s.tc ? size_t(s.units) * 32768 : 0));
+  s.off_zimg = off;
+  off = align256(off + (s.tc ? size_t(s.units) * 512 : 0));
+  s.total = off;
+  return s;
+}
+
+Rope make_rope(const la_problem& q) {
+  Rope r;
+  std::memset(&r, 0, sizeof r);
+  const int bands[3] = {q.dt, q.dh, q.dw};
+  int pi = 0;
+  for (int axis = 0; axis < 3; ++axis) {
+    for (int i = 0; i < bands[axis] / 2; ++i, ++pi) {
+      const double th = std::pow(q.rope_base, -2.0 * double(i) / double(bands[axis]));
+      r.theta_d[pi] = th;
+      r.theta[pi] = static_cast<float>(th);
+      r.band[pi] = axis;
+    }
+  }
+  return r;
+}
+
+// ------------------------------------------------------------------------------- CUDA helpers
+int current_sm_count(int* sm) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LA_ERR_CUDA;
+  return LA_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [BH, N, 128] bf16 viewed as a 3D tensor {128, N, BH}; boxes of 64 channels x 128 tokens,
+// 128-byte swizzle (the canonical UMMA operand layout).
+bool make_tmap(CUtensorMap* m, const void* base, int64_t BH, int64_t N) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {128 * 2, cuuint64_t(N) * 128 * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int launched_ok() { return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
+
+// ------------------------------------------------------------------------------- launchers
+int launch_state(const PlanSet& s, const la_problem& q, const void* K, const void* V, void* ws,
+                 cudaStream_t st, int* nl) {
+  if (s.ps.total == 0) return LA_OK;
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + s.off_partial);
+  const Rope rope = make_rope(q);
+  if (s.tc) {
+    CUtensorMap tk, tv;
+    if (!make_tmap(&tk, K, s.ps.BH, s.ps.N) || !make_tmap(&tv, V, s.ps.BH, s.ps.N)) return LA_ERR_CUDA;
+    if (cudaFuncSetAttribute(la::st::state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             la::st::SMEM_BYTES) != cudaSuccess)
+      return LA_ERR_CUDA;
+    la::st::state_tc_kernel<<<s.ps.grid, la::st::THREADS, la::st::SMEM_BYTES, st>>>(tk, tv, s.ps, rope, partial);
+  } else {
+#define LA_STATE_SIMT(DD, TT)                                                                         \
+  la::simt::state_simt_kernel<DD, TT><<<s.ps.grid, la::simt::THREADS, 0, st>>>(                      \
+      static_cast<const TT*>(K), static_cast<const TT*>(V), s.ps, rope, partial)
+    if (q.dtype == LA_BF16) {
+      if (q.d == 32) LA_STATE_SIMT(32, __nv_bfloat16);
+      else if (q.d == 64) LA_STATE_SIMT(64, __nv_bfloat16);
+      else LA_STATE_SIMT(128, __nv_bfloat16);
+    } else {
+      if (q.d == 32) LA_STATE_SIMT(32, float);
+      else if (q.d == 64) LA_STATE_SIMT(64, float);
+      else LA_STATE_SIMT(128, float);
+    }
+#undef LA_STATE_SIMT
+  }
+  ++*nl;
+  return launched_ok();
+}
+
+int launch_combine(const PlanSet& s, void* ws, float* S_blk, float* z_blk, float* S_inc, float* z_inc, bool img,
+                   cudaStream_t st, int* nl) {
+  const int64_t groups = (int64_t(s.ps.d) * s.ps.d + s.ps.d) / 8;
+  const int64_t threads = s.ps.BH * groups;
+  if (threads == 0 || s.ps.nblk == 0) return LA_OK;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const float* partial = reinterpret_cast<const float*>(w + s.off_partial);
+  uint8_t* im = img ? w + s.off_img : nullptr;
+  float* zim = img ? reinterpret_cast<float*>(w + s.off_zimg) : nullptr;
+  const unsigned blocks = unsigned((threads + la::cmb::THREADS - 1) / la::cmb::THREADS);
+  la::cmb::combine_kernel<<<blocks, la::cmb::THREADS, 0, st>>>(s.ps, partial, S_blk, z_blk, S_inc, z_inc, im, zim);
+  ++*nl;
+  return launched_ok();
+}
+
+size_t apply_simt_smem(int d) {
+  const size_t D = size_t(d), TS = la::simt::TS;
+  return (D * D + D + 3 * TS * (D + 1) + TS) * sizeof(float);
+}
+
+int launch_apply(const PlanSet& s, const la_problem& q, const void* Q, const void* G, const float* S,
+                 const float* z, void* O, void* ws, cudaStream_t st, int* nl) {
+  if (s.pa.total == 0) return LA_OK;
+  const Rope rope = make_rope(q);
+  if (s.tc) {
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    CUtensorMap tq, tg, to;
+    if (!make_tmap(&tq, Q, s.pa.BH, s.pa.N) || !make_tmap(&tg, G, s.pa.BH, s.pa.N) ||
+        !make_tmap(&to, O, s.pa.BH, s.pa.N))
+      return LA_ERR_CUDA;
+    if (cudaFuncSetAttribute(la::ap::apply_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             la::ap::SMEM_BYTES) != cudaSuccess)
+      return LA_ERR_CUDA;
+    la::ap::apply_tc_kernel<<<s.pa.grid, la::ap::THREADS, la::ap::SMEM_BYTES, st>>>(
+        tq, tg, to, s.pa, rope, w + s.off_img, reinterpret_cast<const float*>(w + s.off_zimg),
+        static_cast<__nv_bfloat16*>(O));
+  } else {
+    const size_t smem = apply_simt_smem(q.d);
+#define LA_APPLY_SIMT(DD, TT)                                                                              \
+  do {                                                                                                     \
+    if (cudaFuncSetAttribute(la::simt::apply_simt_kernel<DD, TT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             int(smem)) != cudaSuccess)                                                    \
+      return LA_ERR_CUDA;                                                                                  \
+    la::simt::apply_simt_kernel<DD, TT><<<s.pa.grid, la::simt::THREADS, smem, st>>>(                       \
+        static_cast<const TT*>(Q), static_cast<const TT*>(G), S, z, static_cast<TT*>(O), s.pa, rope);      \
+  } while (0)
+    if (q.dtype == LA_BF16) {
+      if (q.d == 32) LA_APPLY_SIMT(32, __nv_bfloat16);
+      else if (q.d == 64) LA_APPLY_SIMT(64, __nv_bfloat16);
+      else LA_APPLY_SIMT(128, __nv_bfloat16);
+    } else {
+      if (q.d == 32) LA_APPLY_SIMT(32, float);
+      else if (q.d == 64) LA_APPLY_SIMT(64, float);
+      else LA_APPLY_SIMT(128, float);
+    }
+#undef LA_APPLY_SIMT
+  }
+  ++*nl;
+  return launched_ok();
+}
+
+int check_ws(const PlanSet& s, const void* ws, size_t ws_bytes) {
+  if (s.total == 0) return LA_OK;
+  if (!ws || ws_bytes < s.total) return LA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return LA_ERR_ALIGN;
+  return LA_OK;
+}
+
+int64_t elems(const la_problem& q) { return q.B * q.H * q.T * q.Hh * q.W * int64_t(q.d); }
+int64_t state_units(const la_problem& q) {
+  const int64_t nblk = q.block_frames > 0 ? (q.T + q.block_frames - 1) / q.block_frames : 1;
+  return q.B * q.H * nblk;
+}
+
+}  // namespace
+
+// ================================================================================= C ABI
+extern "C" {
+
+size_t la_workspace_bytes_for(const la_problem* p, int sm_count) {
+  if (validate(p) != LA_OK || sm_count <= 0) return 0;
+  return make_plans(*p, sm_count).total;
+}
+
+size_t la_workspace_bytes(const la_problem* p) {
+  if (validate(p) != LA_OK) return 0;
+  int sm = 0;
+  if (current_sm_count(&sm) != LA_OK) return 0;
+  return make_plans(*p, sm).total;
+}
+
+int la_state_reduce(const la_problem* p, const void* K, const void* V, float* S, float* z, void* ws,
+                    size_t ws_bytes, cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  const bool has_tok = elems(*p) > 0;
+  const bool has_state = state_units(*p) > 0;
+  if ((rc = check_ptr(K, has_tok)) || (rc = check_ptr(V, has_tok)) || (rc = check_ptr(S, has_state)) ||
+      (rc = check_ptr(z, has_state)))
+    return rc;
+  int sm = 0;
+  if ((rc = current_sm_count(&sm))) return rc;
+  const PlanSet s = make_plans(*p, sm);
+  if ((rc = check_ws(s, ws, ws_bytes))) return rc;
+  int nl = 0;
+  if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
+  if ((rc = launch_combine(s, ws, S, z, nullptr, nullptr, false, stream, &nl))) return rc;
+  g_last_launches = nl;
+  return LA_OK;
+}
+
+int la_state_scan(const la_problem* p, float* S, float* z, cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  if (p->block_frames == 0) {
+    g_last_launches = 0;
+    return LA_OK;
+  }
+  const int64_t BH = p->B * p->H;
+  const int64_t nblk = (p->T + p->block_frames - 1) / p->block_frames;
+  const bool has_state = BH * nblk > 0;
+  if ((rc = check_ptr(S, has_state)) || (rc = check_ptr(z, has_state))) return rc;
+  if (!has_state) {
+    g_last_launches = 0;
+    return LA_OK;
+  }
+  const int64_t threads = BH * ((int64_t(p->d) * p->d + p->d) / 8);
+  const unsigned blocks = unsigned((threads + la::cmb::THREADS - 1) / la::cmb::THREADS);
+  la::cmb::scan_kernel<<<blocks, la::cmb::THREADS, 0, stream>>>(BH, nblk, p->d, S, z);
+  if ((rc = launched_ok())) return rc;
+  g_last_launches = 1;
+  return LA_OK;
+}
+
+int la_apply(const la_problem* p, const void* Q, const void* G, const float* S, const float* z, void* O,
+             void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  const bool has_tok = elems(*p) > 0;
+  if ((rc = check_ptr(Q, has_tok)) || (rc = check_ptr(G, has_tok)) || (rc = check_ptr(O, has_tok)) ||
+      (rc = check_ptr(S, has_tok)) || (rc = check_ptr(z, has_tok)))
+    return rc;
+  if (!has_tok) {
+    g_last_launches = 0;
+    return LA_OK;
+  }
+  int sm = 0;
+  if ((rc = current_sm_count(&sm))) return rc;
+  const PlanSet s = make_plans(*p, sm);
+  int nl = 0;
+  if (s.tc) {
+    if ((rc = check_ws(s, ws, ws_bytes))) return rc;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    const int64_t threads = s.units * ((128 * 128 + 128) / 8);
+    const unsigned blocks = unsigned((threads + la::cmb::THREADS - 1) / la::cmb::THREADS);
+    la::cmb::pack_kernel<<<blocks, la::cmb::THREADS, 0, stream>>>(s.units, 128, S, z, w + s.off_img,
+                                                                   reinterpret_cast<float*>(w + s.off_zimg));
+    ++nl;
+    if ((rc = launched_ok())) return rc;
+  }
+  if ((rc = launch_apply(s, *p, Q, G, S, z, O, ws, stream, &nl))) return rc;
+  g_last_launches = nl;
+  return LA_OK;
+}
+
+static int forward_common(const la_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                          void* O, float* S_incl, float* z_incl, void* ws, size_t ws_bytes, cudaStream_t stream,
+                          cudaEvent_t* marks = nullptr, int nmarks = 0) {
+  int rc;
+  const bool has_tok = elems(*p) > 0;
+  if ((rc = check_ptr(Q, has_tok)) || (rc = check_ptr(K, has_tok)) || (rc = check_ptr(V, has_tok)) ||
+      (rc = check_ptr(G, has_tok)) || (rc = check_ptr(O, has_tok)))
+    return rc;
+  if (S_incl && !aligned16(S_incl)) return LA_ERR_ALIGN;
+  if (z_incl && !aligned16(z_incl)) return LA_ERR_ALIGN;
+  if ((S_incl == nullptr) != (z_incl == nullptr)) return LA_ERR_NULL;
+  const bool want_states = S_incl != nullptr && state_units(*p) > 0;
+  if (!has_tok && !want_states) {
+    g_last_launches = 0;
+    return LA_OK;
+  }
+  int sm = 0;
+  if ((rc = current_sm_count(&sm))) return rc;
+  const PlanSet s = make_plans(*p, sm);
+  if ((rc = check_ws(s, ws, ws_bytes))) return rc;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* st_S = S_incl ? S_incl : reinterpret_cast<float*>(w + s.off_states);
+  float* st_z = z_incl ? z_incl : reinterpret_cast<float*>(w + s.off_states) + s.units * p->d * p->d;
+  // The tensor-core apply reads the bf16 operand image; the CUDA-core apply reads fp32 states.
+  const bool need_fp32 = !s.tc || S_incl != nullptr;
+  int nl = 0;
+  auto mark = [&](int i) {
+    if (i < nmarks && marks && marks[i]) cudaEventRecord(marks[i], stream);
+  };
+  mark(0);
+  if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
+  mark(nl);
+  const int before = nl;
+  if ((rc = launch_combine(s, ws, nullptr, nullptr, need_fp32 ? st_S : nullptr, need_fp32 ? st_z : nullptr,
+                           s.tc, stream, &nl)))
+    return rc;
+  if (nl != before) mark(nl);
+  if (has_tok) {
+    const int b2 = nl;
+    if ((rc = launch_apply(s, *p, Q, G, st_S, st_z, O, ws, stream, &nl))) return rc;
+    if (nl != b2) mark(nl);
+  }
+  g_last_launches = nl;
+  return LA_OK;
+}
+
+int la_forward_bidir(const la_problem* p, const void* Q, const void* K, const void* V, const void* G, void* O,
+                     void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  if (p->block_frames != 0) return LA_ERR_SHAPE;
+  return forward_common(p, Q, K, V, G, O, nullptr, nullptr, ws, ws_bytes, stream);
+}
+
+int la_forward_blockcausal(const la_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                           void* O, float* S_incl, float* z_incl, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  if (p->block_frames <= 0) return LA_ERR_SHAPE;
+  return forward_common(p, Q, K, V, G, O, S_incl, z_incl, ws, ws_bytes, stream);
+}
+
+int la_forward_marked(const la_problem* p, const void* Q, const void* K, const void* V, const void* G, void* O,
+                      float* S_incl, float* z_incl, void* ws, size_t ws_bytes, cudaStream_t stream, cudaEvent_t* marks,
+                      int nmarks) {
+  int rc = validate(p);
+  if (rc) return rc;
+  if (nmarks < 0 || (nmarks > 0 && !marks)) return LA_ERR_NULL;
+  if (p->block_frames == 0 && (S_incl || z_incl)) return LA_ERR_SHAPE;
+  return forward_common(p, Q, K, V, G, O, S_incl, z_incl, ws, ws_bytes, stream, marks, nmarks);
+}
+
+const char* la_status_string(int status) {
+  switch (status) {
+    case LA_OK: return "ok";
+    case LA_ERR_NULL: return "a required pointer is NULL";
+    case LA_ERR_SHAPE: return "invalid or inconsistent sizes";
+    case LA_ERR_BANDS: return "RoPE bands must be even, non-negative and add up to d";
+    case LA_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+    case LA_ERR_UNSUPPORTED: return "unsupported head dimension, dtype or flag";
+    case LA_ERR_WORKSPACE: return "workspace missing or smaller than la_workspace_bytes()";
+    case LA_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case LA_ERR_DEVICE: return "a kernel reported a device-side failure (a bounded wait ran out)";
+    default: return "unknown status";
+  }
+}
+
+int la_device_error(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return LA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, la::g_la_error, sizeof v) != cudaSuccess) return LA_ERR_CUDA;
+  if (v == 0) return LA_OK;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(la::g_la_error, &zero, sizeof zero) != cudaSuccess) return LA_ERR_CUDA;
+  return LA_ERR_DEVICE;
+}
+
+int la_last_launch_count(void) { return g_last_launches; }
+
+}  // extern "C"

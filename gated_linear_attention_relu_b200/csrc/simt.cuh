@@ -1,0 +1,330 @@
+// simt.cuh -- CUDA-core kernels: the fp32 dtype path, head dimensions 32 and 64, and the
+// reference point the tensor-core kernels are measured against (LA_FLAG_FORCE_SIMT).
+//
+// Same operator and the same work decomposition as the tensor-core kernels (common.cuh), with
+// fp32 FFMA accumulation.  RoPE angles are formed and reduced modulo 2*pi in fp64 before the
+// fp32 sincos, so the rotation is accurate to a few ulp even at large grid positions.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace la {
+namespace simt {
+
+constexpr int THREADS = 256;
+constexpr int TS = 32;  // tokens per tile (state and apply)
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ void rope_cs(double pos, double theta, float& c, float& s) {
+  const double two_pi = 6.283185307179586476925286766559;
+  double a = pos * theta;
+  a -= two_pi * rint(a / two_pi);
+  sincosf(static_cast<float>(a), &s, &c);
+}
+
+__device__ __forceinline__ uint32_t axis_pos(int band, uint32_t t, uint32_t h, uint32_t w) {
+  return band == 0 ? t : (band == 1 ? h : w);
+}
+
+// ---------------------------------------------------------------------------------------------
+// State: per CTA, partial S (D x D) and z (D) for every unit it touches, into partial slots.
+template <int D, typename T>
+__global__ void __launch_bounds__(THREADS)
+state_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const Plan p,
+                  const __grid_constant__ Rope rope, float* __restrict__ partial) {
+  constexpr int R = D / 16;  // each thread owns an R x R block of S
+  __shared__ float kr[TS][D];
+  __shared__ float vs[TS][D];
+  __shared__ float kp[TS][D];
+  const int tid = threadIdx.x;
+  const int ty = tid / 16, tx = tid % 16;
+  const int64_t c = blockIdx.x;
+  const int64_t g0 = cta_start(p, c), g1 = cta_start(p, c + 1);
+  const int64_t u_first = unit_of_tile(p, g0);
+  const int64_t slot_floats = static_cast<int64_t>(D) * D + static_cast<int64_t>(p.zparts) * D;
+  float acc[R][R];
+  float zacc = 0.f;
+#pragma unroll
+  for (int a = 0; a < R; ++a)
+#pragma unroll
+    for (int b = 0; b < R; ++b) acc[a][b] = 0.f;
+
+  for (int64_t g = g0; g < g1; ++g) {
+    const TileInfo ti = tile_info(p, g);
+    const T* kb = K + (ti.bh * p.N) * D;
+    const T* vb = V + (ti.bh * p.N) * D;
+    __syncthreads();
+    for (int e = tid; e < TS * D / 2; e += THREADS) {
+      const int r = e / (D / 2), pi = e % (D / 2);
+      const int64_t n = ti.n0 + r;
+      float x0 = 0.f, x1 = 0.f, v0 = 0.f, v1 = 0.f;
+      uint32_t pt = 0, ph = 0, pw = 0;
+      if (n < ti.n_end) {
+        x0 = fmaxf(to_f(kb[n * D + 2 * pi]), 0.f);
+        x1 = fmaxf(to_f(kb[n * D + 2 * pi + 1]), 0.f);
+        v0 = to_f(vb[n * D + 2 * pi]);
+        v1 = to_f(vb[n * D + 2 * pi + 1]);
+        token_pos(p, static_cast<uint32_t>(n), pt, ph, pw);
+      }
+      float cs, sn;
+      rope_cs(static_cast<double>(axis_pos(rope.band[pi], pt, ph, pw)), rope.theta_d[pi], cs, sn);
+      kp[r][2 * pi] = x0;
+      kp[r][2 * pi + 1] = x1;
+      kr[r][2 * pi] = x0 * cs - x1 * sn;
+      kr[r][2 * pi + 1] = x0 * sn + x1 * cs;
+      vs[r][2 * pi] = v0;
+      vs[r][2 * pi + 1] = v1;
+    }
+    __syncthreads();
+    for (int r = 0; r < TS; ++r) {
+      float a[R], b[R];
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        a[i] = kr[r][ty * R + i];
+        b[i] = vs[r][tx * R + i];
+      }
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int j = 0; j < R; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    if (tid < D)
+      for (int r = 0; r < TS; ++r) zacc += kp[r][tid];
+
+    const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != ti.unit);
+    if (last) {
+      float* dst = partial + (c * p.maxseg + (ti.unit - u_first)) * slot_floats;
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+          dst[(ty * R + i) * D + tx * R + j] = acc[i][j];
+          acc[i][j] = 0.f;
+        }
+      if (tid < D) {
+        dst[D * D + tid] = zacc;
+        zacc = 0.f;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Apply: O_n = (RoPE(ReLU(q_n)) S) / (ReLU(q_n) . z + eps) * sigmoid(g_n), state fp32 in smem.
+template <int D, typename T>
+__global__ void __launch_bounds__(THREADS)
+apply_simt_kernel(const T* __restrict__ Q, const T* __restrict__ G, const float* __restrict__ S,
+                  const float* __restrict__ z, T* __restrict__ O, const Plan p,
+                  const __grid_constant__ Rope rope) {
+  extern __shared__ float sm[];
+  float* Ss = sm;                   // [D][D]
+  float* zs = Ss + D * D;           // [D]
+  float* qr = zs + D;               // [TS][D+1] rotated features
+  float* qp = qr + TS * (D + 1);    // [TS][D+1] un-rotated ReLU features
+  float* inv = qp + TS * (D + 1);   // [TS]
+  float* ot = inv + TS;             // [TS][D+1] numerators
+  constexpr int CW = D / 8;         // columns per thread
+  const int tid = threadIdx.x;
+  const int r_own = tid % TS, cg = tid / TS;
+  const int64_t c = blockIdx.x;
+  const int64_t g0 = cta_start(p, c), g1 = cta_start(p, c + 1);
+  int64_t cur_unit = -1;
+  for (int64_t g = g0; g < g1; ++g) {
+    const TileInfo ti = tile_info(p, g);
+    __syncthreads();
+    if (ti.unit != cur_unit) {
+      cur_unit = ti.unit;
+      const float* Su = S + ti.unit * D * D;
+      for (int e = tid; e < D * D; e += THREADS) Ss[e] = Su[e];
+      for (int e = tid; e < D; e += THREADS) zs[e] = z[ti.unit * D + e];
+    }
+    const T* qb = Q + (ti.bh * p.N) * D;
+    for (int e = tid; e < TS * D / 2; e += THREADS) {
+      const int r = e / (D / 2), pi = e % (D / 2);
+      const int64_t n = ti.n0 + r;
+      float x0 = 0.f, x1 = 0.f;
+      uint32_t pt = 0, ph = 0, pw = 0;
+      if (n < ti.n_end) {
+        x0 = fmaxf(to_f(qb[n * D + 2 * pi]), 0.f);
+        x1 = fmaxf(to_f(qb[n * D + 2 * pi + 1]), 0.f);
+        token_pos(p, static_cast<uint32_t>(n), pt, ph, pw);
+      }
+      float cs, sn;
+      rope_cs(static_cast<double>(axis_pos(rope.band[pi], pt, ph, pw)), rope.theta_d[pi], cs, sn);
+      qp[r * (D + 1) + 2 * pi] = x0;
+      qp[r * (D + 1) + 2 * pi + 1] = x1;
+      qr[r * (D + 1) + 2 * pi] = x0 * cs - x1 * sn;
+      qr[r * (D + 1) + 2 * pi + 1] = x0 * sn + x1 * cs;
+    }
+    __syncthreads();
+    if (tid < TS) {
+      float den = 0.f;
+      for (int k = 0; k < D; ++k) den = fmaf(qp[tid * (D + 1) + k], zs[k], den);
+      inv[tid] = 1.0f / (den + p.eps);
+    }
+    {
+      float acc[CW];
+#pragma unroll
+      for (int j = 0; j < CW; ++j) acc[j] = 0.f;
+      for (int k = 0; k < D; ++k) {
+        const float a = qr[r_own * (D + 1) + k];
+#pragma unroll
+        for (int j = 0; j < CW; ++j) acc[j] = fmaf(a, Ss[k * D + cg * CW + j], acc[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < CW; ++j) ot[r_own * (D + 1) + cg * CW + j] = acc[j];
+    }
+    __syncthreads();
+    const T* gb = G + (ti.bh * p.N) * D;
+    T* ob = O + (ti.bh * p.N) * D;
+    for (int e = tid; e < TS * D; e += THREADS) {
+      const int r = e / D, v = e % D;
+      const int64_t n = ti.n0 + r;
+      if (n < ti.n_end) {
+        const float gv = to_f(gb[n * D + v]);
+        const float sig = 1.0f / (1.0f + expf(-gv));
+        ob[n * D + v] = from_f<T>(ot[r * (D + 1) + v] * inv[r] * sig);
+      }
+    }
+  }
+}
+
+}  // namespace simt
+
+// ---------------------------------------------------------------------------------------------
+// Combine: sum the partial slots of every unit in a fixed order; optionally the per-block states,
+// the inclusive prefix over blocks, and the bf16 operand image the tensor-core apply reads.
+// One thread per (head, group of 8 consecutive elements of [S | z]).
+namespace cmb {
+
+constexpr int THREADS = 256;
+
+// Byte offset of S[k][v] (bf16) in the 128B-swizzled, N-major operand image of a 128 x 128 state:
+// two 64-column halves of 128 rows x 128 B; 16-byte chunk j of row k sits at chunk j ^ (k % 8).
+__device__ __forceinline__ uint32_t img_offset(int k, int v) {
+  const int half = v >> 6, chunk = (v & 63) >> 3;
+  return static_cast<uint32_t>(half * 16384 + k * 128 + ((chunk ^ (k & 7)) << 4) + (v & 7) * 2);
+}
+
+__device__ __forceinline__ void write_image(uint8_t* img, float* zimg, int64_t unit, int D, int e0,
+                                            const float (&x)[8]) {
+  if (e0 < D * D) {
+    const int k = e0 / D, v = e0 % D;
+    uint4 pk = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                          pack_bf16(x[6], x[7]));
+    *reinterpret_cast<uint4*>(img + unit * 32768 + img_offset(k, v)) = pk;
+  } else {
+    float4* zd = reinterpret_cast<float4*>(zimg + unit * D + (e0 - D * D));
+    zd[0] = make_float4(x[0], x[1], x[2], x[3]);
+    zd[1] = make_float4(x[4], x[5], x[6], x[7]);
+  }
+}
+
+__device__ __forceinline__ void store8(float* S, float* z, int64_t unit, int D, int e0, const float (&x)[8]) {
+  float* dst = (e0 < D * D) ? S + unit * D * D + e0 : z + unit * D + (e0 - D * D);
+  float4* d4 = reinterpret_cast<float4*>(dst);
+  d4[0] = make_float4(x[0], x[1], x[2], x[3]);
+  d4[1] = make_float4(x[4], x[5], x[6], x[7]);
+}
+
+__global__ void __launch_bounds__(THREADS)
+combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, float* z_blk, float* S_inc,
+               float* z_inc, uint8_t* img, float* zimg) {
+  const int D = p.d;
+  const int groups = (D * D + D) / 8;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
+  const int64_t bh = idx / groups;
+  if (bh >= p.BH) return;
+  const int e0 = static_cast<int>(idx - bh * groups) * 8;
+  const int64_t slot_floats = static_cast<int64_t>(D) * D + static_cast<int64_t>(p.zparts) * D;
+  float run[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) run[e] = 0.f;
+  for (int64_t blk = 0; blk < p.nblk; ++blk) {
+    const int64_t u = bh * p.nblk + blk;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    int64_t first = 0, count = 0;
+    if (p.total > 0) unit_tiles(p, u, &first, &count);
+    if (count > 0) {
+      const int64_t c0 = cta_of(p, first), c1 = cta_of(p, first + count - 1);
+      for (int64_t cc = c0; cc <= c1; ++cc) {
+        const int64_t k = u - unit_of_tile(p, cta_start(p, cc));
+        const float* src = partial + (cc * p.maxseg + k) * slot_floats;
+        if (e0 < D * D) {
+          const float4* s4 = reinterpret_cast<const float4*>(src + e0);
+          const float4 a = s4[0], b = s4[1];
+          acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+          acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+        } else {
+          for (int zp = 0; zp < p.zparts; ++zp) {
+            const float4* s4 = reinterpret_cast<const float4*>(src + D * D + zp * D + (e0 - D * D));
+            const float4 a = s4[0], b = s4[1];
+            acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+            acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+          }
+        }
+      }
+    }
+    if (S_blk) store8(S_blk, z_blk, u, D, e0, acc);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) run[e] += acc[e];
+    if (S_inc) store8(S_inc, z_inc, u, D, e0, run);
+    if (img) write_image(img, zimg, u, D, e0, run);
+  }
+}
+
+// In-place inclusive prefix over blocks of [B*H][nblk][D*D] and [B*H][nblk][D].
+__global__ void __launch_bounds__(THREADS)
+scan_kernel(int64_t BH, int64_t nblk, int D, float* S, float* z) {
+  const int groups = (D * D + D) / 8;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
+  const int64_t bh = idx / groups;
+  if (bh >= BH) return;
+  const int e0 = static_cast<int>(idx - bh * groups) * 8;
+  float run[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) run[e] = 0.f;
+  for (int64_t blk = 0; blk < nblk; ++blk) {
+    const int64_t u = bh * nblk + blk;
+    float* src = (e0 < D * D) ? S + u * D * D + e0 : z + u * D + (e0 - D * D);
+    float4* s4 = reinterpret_cast<float4*>(src);
+    const float4 a = s4[0], b = s4[1];
+    run[0] += a.x; run[1] += a.y; run[2] += a.z; run[3] += a.w;
+    run[4] += b.x; run[5] += b.y; run[6] += b.z; run[7] += b.w;
+    s4[0] = make_float4(run[0], run[1], run[2], run[3]);
+    s4[1] = make_float4(run[4], run[5], run[6], run[7]);
+  }
+}
+
+// bf16 operand image of given fp32 states (for the tensor-core apply called on its own).
+__global__ void __launch_bounds__(THREADS)
+pack_kernel(int64_t units, int D, const float* __restrict__ S, const float* __restrict__ z, uint8_t* img,
+            float* zimg) {
+  const int groups = (D * D + D) / 8;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
+  const int64_t u = idx / groups;
+  if (u >= units) return;
+  const int e0 = static_cast<int>(idx - u * groups) * 8;
+  const float* src = (e0 < D * D) ? S + u * D * D + e0 : z + u * D + (e0 - D * D);
+  const float4 a = reinterpret_cast<const float4*>(src)[0], b = reinterpret_cast<const float4*>(src)[1];
+  const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  write_image(img, zimg, u, D, e0, x);
+}
+
+}  // namespace cmb
+}  // namespace la

@@ -1,0 +1,256 @@
+// state_tc.cuh -- state reduction on the 5th-generation tensor cores (bf16, d = 128).
+//
+// Computes, per unit (a head, or one block of a head), the partial sums over the tiles a CTA
+// owns of
+//   S[k][v] = sum_n RoPE(ReLU(K_n))[k] V_n[v]     (SANA-Video 2.0, Eq. (1), the state)
+//   z[k]    = sum_n ReLU(K_n)[k]                  (the un-rotated normaliser, SANA-Video Sec. 3.2)
+// as one tcgen05 MMA per 16 tokens: D[128 x 128] += A[128 x 16] * B[16 x 128], where
+// A = RoPE(ReLU(K))^T (channels x tokens, M-major) and B = V (tokens x channels, N-major).
+//
+// Pipeline (one CTA per SM, persistent over a contiguous range of 128-token tiles):
+//   warp 0      TMA producer: K and V tiles (two 64-channel, 128-row, 128B-swizzled boxes each)
+//   warp 1      MMA issuer: 8 x tcgen05.mma per tile into one of two TMEM accumulators
+//   warps 2-5   transform: ReLU + RoPE of K in place (bf16), z accumulated in registers
+//   warps 6-9   drain: TMEM accumulator -> fp32 partial S in global memory, once per unit
+// The staged K tile is already in the canonical 128B-swizzled MN-major operand layout, so the
+// transform rewrites it in place.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace la {
+namespace st {
+
+constexpr int TILE = 128;
+constexpr int D = 128;
+constexpr int STAGES = 3;
+constexpr int THREADS = 320;
+constexpr uint32_t HALF = 128 * 128;          // one 64-channel box of 128 rows x 128 B
+constexpr uint32_t BUF = 2 * HALF;            // 128 tokens x 128 channels bf16
+constexpr uint32_t STAGE = 2 * BUF;           // K + V
+constexpr uint32_t OFF_BAR = STAGES * STAGE;  // barriers after the stages
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
+constexpr int ZPARTS = 8;                     // z is written as 8 row-group partial sums
+constexpr int64_t SLOT = D * D + ZPARTS * D;  // floats per partial slot: S, then ZPARTS x z
+constexpr uint32_t TMEM_COLS = 256;           // two 128-column fp32 accumulators
+constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, /*a_mn=*/true, /*b_mn=*/true);
+
+struct Bars {
+  uint64_t full[STAGES];     // TMA landed K and V            (1 arrival + tx bytes)
+  uint64_t aready[STAGES];   // transform wrote the A operand  (4 warps)
+  uint64_t empty[STAGES];    // MMAs of the stage completed    (tcgen05.commit)
+  uint64_t accfull[2];       // accumulator holds a finished unit (tcgen05.commit)
+  uint64_t accempty[2];      // drain finished reading it     (4 warps)
+  uint64_t final_;           // all MMAs completed (teardown)
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block too large");
+
+__global__ void __launch_bounds__(THREADS, 1)
+state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                const Plan p, const __grid_constant__ Rope rope, float* __restrict__ partial) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
+  const uint32_t sbase = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t c = blockIdx.x;
+  const int64_t g0 = cta_start(p, c);
+  const int64_t g1 = cta_start(p, c + 1);
+  const int64_t u_first = unit_of_tile(p, g0);
+  volatile int* abort_flag = &bars->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->aready[s], 4);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bars->accfull[a], 1);
+      mbar_init(&bars->accempty[a], 4);
+    }
+    mbar_init(&bars->final_, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int64_t issued = 0;
+      for (int64_t g = g0; g < g1; ++g, ++issued) {
+        const int64_t i = g - g0;
+        const int s = static_cast<int>(i % STAGES);
+        const uint32_t ph = static_cast<uint32_t>((i / STAGES) & 1);
+        if (!mbar_wait(&bars->empty[s], ph ^ 1u, abort_flag)) break;
+        const TileInfo ti = tile_info(p, g);
+        uint8_t* kb = smem + s * STAGE;
+        uint8_t* vb = kb + BUF;
+        mbar_arrive_expect_tx(&bars->full[s], STAGE);
+        const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
+        tma_load_3d(kb, &tmK, 0, n0, bh, &bars->full[s]);
+        tma_load_3d(kb + HALF, &tmK, 64, n0, bh, &bars->full[s]);
+        tma_load_3d(vb, &tmV, 0, n0, bh, &bars->full[s]);
+        tma_load_3d(vb + HALF, &tmV, 64, n0, bh, &bars->full[s]);
+      }
+      if (*abort_flag) {
+        // Let every copy still in flight land before the CTA's shared memory goes away.
+        for (int64_t j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+          mbar_wait_drain(&bars->full[j % STAGES], static_cast<uint32_t>((j / STAGES) & 1));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int64_t seg = -1;
+      int64_t prev_unit = -1;
+      for (int64_t g = g0; g < g1; ++g) {
+        const int64_t i = g - g0;
+        const int s = static_cast<int>(i % STAGES);
+        const uint32_t ph = static_cast<uint32_t>((i / STAGES) & 1);
+        const int64_t u = unit_of_tile(p, g);
+        const bool first = (u != prev_unit);
+        const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != u);
+        prev_unit = u;
+        if (first) {
+          ++seg;
+          if (!mbar_wait(&bars->accempty[seg & 1], static_cast<uint32_t>(((seg >> 1) & 1) ^ 1), abort_flag)) break;
+        }
+        if (!mbar_wait(&bars->full[s], ph, abort_flag)) break;
+        if (!mbar_wait(&bars->aready[s], ph, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + static_cast<uint32_t>(seg & 1) * 128u;
+        const uint32_t ka = sbase + s * STAGE;
+        const uint32_t va = ka + BUF;
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(ka + kk * 2048, HALF, 1024);
+          const uint64_t bd = smem_desc_sw128(va + kk * 2048, HALF, 1024);
+          mma_bf16(acc, ad, bd, IDESC, (kk > 0 || !first) ? 1u : 0u);
+        }
+        mma_commit(&bars->empty[s]);
+        if (last) mma_commit(&bars->accfull[seg & 1]);
+      }
+      mma_commit(&bars->final_);
+      mbar_wait_drain(&bars->final_, 0);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ transform: ReLU + RoPE of K
+    const int tt = threadIdx.x - 64;  // 0..127
+    const int ck = tt & 15;           // 8-channel chunk: channels 8ck .. 8ck+7
+    const int rg = tt >> 4;           // rows rg, rg+8, ..., rg+120 (so row % 8 == rg)
+    const uint32_t chunk_off = static_cast<uint32_t>((ck >> 3) * HALF + (((ck & 7) ^ rg) << 4));
+    float th[4];
+    int bd[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      th[q] = rope.theta[4 * ck + q];
+      bd[q] = rope.band[4 * ck + q];
+    }
+    float zacc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
+    int64_t seg = -1;
+    int64_t prev_unit = -1;
+    for (int64_t g = g0; g < g1; ++g) {
+      const int64_t i = g - g0;
+      const int s = static_cast<int>(i % STAGES);
+      const uint32_t ph = static_cast<uint32_t>((i / STAGES) & 1);
+      const TileInfo ti = tile_info(p, g);
+      if (ti.unit != prev_unit) {
+        ++seg;
+        prev_unit = ti.unit;
+      }
+      const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != ti.unit);
+      if (!warp_wait(&bars->full[s], ph, abort_flag)) break;
+      const uint32_t base = sbase + s * STAGE + chunk_off;
+      uint32_t n = static_cast<uint32_t>(ti.n0) + rg;
+      const uint32_t n_end = static_cast<uint32_t>(ti.n_end);
+      uint32_t pt, ph_, pw;
+      token_pos(p, n, pt, ph_, pw);
+#pragma unroll 2
+      for (int j = 0; j < TILE / 8; ++j) {
+        const uint32_t addr = base + static_cast<uint32_t>((rg + 8 * j) * 128);
+        uint4 raw = lds128(addr);
+        const bool valid = n < n_end;
+        uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float x0 = valid ? fmaxf(bf16lo(w[q]), 0.f) : 0.f;
+          float x1 = valid ? fmaxf(bf16hi(w[q]), 0.f) : 0.f;
+          zacc[2 * q] += x0;
+          zacc[2 * q + 1] += x1;
+          const uint32_t pos = bd[q] == 0 ? pt : (bd[q] == 1 ? ph_ : pw);
+          float sn, cs;
+          __sincosf(static_cast<float>(pos) * th[q], &sn, &cs);
+          o[q] = pack_bf16(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+        }
+        sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
+        n += 8;
+        token_pos_advance(p, 8, pt, ph_, pw);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->aready[s]);
+      if (last) {
+        // z of this unit, one partial per row group rg; the combine kernel adds the 8 in order.
+        const int64_t slot = c * p.maxseg + (ti.unit - u_first);
+        float4* zd = reinterpret_cast<float4*>(partial + slot * SLOT + D * D + rg * D + 8 * ck);
+        zd[0] = make_float4(zacc[0], zacc[1], zacc[2], zacc[3]);
+        zd[1] = make_float4(zacc[4], zacc[5], zacc[6], zacc[7]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ drain TMEM -> partial S
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;
+    const int64_t nseg = (g1 > g0) ? unit_of_tile(p, g1 - 1) - u_first + 1 : 0;
+    for (int64_t k = 0; k < nseg; ++k) {
+      if (!warp_wait(&bars->accfull[k & 1], static_cast<uint32_t>((k >> 1) & 1), abort_flag)) break;
+      tc_fence_after();
+      float* dst = partial + (c * p.maxseg + k) * SLOT + static_cast<int64_t>(row) * D;
+      const uint32_t taddr = tmem + static_cast<uint32_t>(k & 1) * 128u + (static_cast<uint32_t>(quarter * 32) << 16);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t r[32];
+        tmem_ld_x32(taddr + ch * 32, r);
+        tmem_ld_wait();
+        float4* d4 = reinterpret_cast<float4*>(dst + ch * 32);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          d4[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                              __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->accempty[k & 1]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace st
+}  // namespace la

@@ -1,0 +1,145 @@
+/*
+ * la.h -- C ABI of the gated ReLU linear-attention token mixer for NVIDIA B200 (sm_100a).
+ *
+ * The operator, per (batch b, head h), on tokens n of a (T, Hh, W) latent grid:
+ *
+ *   phi(x) = RoPE3D(ReLU(x))                        (RoPE applied after ReLU)
+ *   S      = sum_n phi(K_n)^T V_n                   (d x d state)
+ *   z      = sum_n ReLU(K_n)                        (d normaliser, NOT rotated)
+ *   O_n    = (phi(Q_n) S) / (ReLU(Q_n) . z + eps) * sigmoid(G_n)
+ *
+ * Sources: "SANA-Video 2.0: Hybrid Linear Attention with Attention Residuals for
+ * Efficient Video Generation", Sec. 2, Eq. (1) (state, normaliser, sigmoid output
+ * gate; the write gate beta is 1 and RMSNorm / W_o are outside this operator), and
+ * "SANA-Video: Efficient Video Generation with Block Linear Diffusion Transformer",
+ * Sec. 3.2 (RoPE after ReLU, un-rotated denominator) and Sec. 3.4 (block-causal
+ * constant-memory cache: a block reads the summed states of all earlier blocks plus
+ * its own; Algorithm 1 updates the cache once per block).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Q, K, V, G, O are dense, contiguous [B, H, N, d] tensors in device memory, of
+ *    the dtype given in la_problem.dtype (bf16 or fp32).  N = T * Hh * W.  Token n of a
+ *    head sits at grid position (t, h, w) with n = (t * Hh + h) * W + w.
+ *  - 3D RoPE: channels [0, dt) rotate with t, [dt, dt+dh) with h, [dt+dh, d) with w.
+ *    Pair i of a band of width D rotates channels (2i, 2i+1) of the band by the angle
+ *    pos * rope_base^(-2i/D), counter-clockwise: (x0, x1) -> (x0 c - x1 s, x0 s + x1 c).
+ *  - States are fp32: S is [B, H, nblk, d, d] with S[k][v] = sum_n phi(K_n)[k] V_n[v],
+ *    z is [B, H, nblk, d].  nblk = 1 in bidirectional mode, ceil(T / block_frames) in
+ *    block-causal mode; block j holds latent frames [j*block_frames, (j+1)*block_frames)
+ *    (the last block may be shorter).
+ *  - Every device pointer must be 16-byte aligned.  Inputs must be finite.
+ *  - Ownership: the caller allocates and frees every buffer, including the workspace.
+ *    The library never allocates, frees or synchronises; all work is queued on the
+ *    given stream, in stream order, and the call returns before it finishes.
+ *  - Errors: every entry point returns an la_status.  Invalid arguments are detected
+ *    on the host before anything is launched; LA_ERR_CUDA reports a launch failure.
+ *    No exception crosses the ABI.  A device-side failure (a bounded wait that ran
+ *    out) sets a per-device error word that la_device_error() reads and clears.
+ *  - Results are deterministic: the same problem, inputs and device give bitwise the
+ *    same outputs (no floating-point atomics; every reduction has a fixed order).
+ *  - Concurrent calls on different streams must use different workspaces.
+ */
+#ifndef LA_H_
+#define LA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LA_OK = 0,
+  LA_ERR_NULL = 1,        /* a required pointer is NULL */
+  LA_ERR_SHAPE = 2,       /* negative / inconsistent sizes, or sizes beyond the limits */
+  LA_ERR_BANDS = 3,       /* dt + dh + dw != d, or a band width is odd or negative */
+  LA_ERR_ALIGN = 4,       /* a device pointer is not 16-byte aligned */
+  LA_ERR_UNSUPPORTED = 5, /* d not in {32, 64, 128}, unknown dtype or flag */
+  LA_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than la_workspace_bytes() */
+  LA_ERR_CUDA = 7,        /* a CUDA runtime call or kernel launch failed */
+  LA_ERR_DEVICE = 8       /* la_device_error(): a kernel reported a device-side failure */
+} la_status;
+
+typedef enum { LA_BF16 = 0, LA_F32 = 1 } la_dtype;
+
+/* la_problem.flags */
+#define LA_FLAG_FORCE_SIMT 1u /* use the CUDA-core kernels even where tcgen05 kernels exist */
+
+typedef struct {
+  int64_t B, H;          /* batch and heads */
+  int64_t T, Hh, W;      /* latent grid; N = T * Hh * W tokens per head */
+  int32_t d;             /* head dimension: 32, 64 or 128 */
+  int32_t dt, dh, dw;    /* RoPE band widths along t, h, w; even, dt + dh + dw == d */
+  double rope_base;      /* RoPE base (> 0), e.g. 10000 */
+  float eps;             /* added to the denominator after the dot product, e.g. 1e-6 */
+  int32_t block_frames;  /* 0: bidirectional; > 0: latent frames per causal block */
+  int32_t dtype;         /* la_dtype of Q, K, V, G and O */
+  uint32_t flags;        /* LA_FLAG_* */
+} la_problem;
+
+/* Bytes of device workspace the calls below need for this problem on the CURRENT
+ * device (the split of the token range over SMs depends on the device's SM count).
+ * Returns 0 for an invalid problem.  One workspace serves every entry point. */
+size_t la_workspace_bytes(const la_problem* p);
+
+/* The same for an explicit SM count (pure host computation, no CUDA call). */
+size_t la_workspace_bytes_for(const la_problem* p, int sm_count);
+
+/* State reduction (SANA-Video 2.0, Eq. (1), the sum defining S; SANA-Video Sec. 3.4,
+ * per-block states): writes S [B,H,nblk,d,d] and z [B,H,nblk,d], fp32.  In block-causal
+ * mode these are the states of each block alone (not prefixed).  K, V: [B,H,N,d]. */
+int la_state_reduce(const la_problem* p, const void* K, const void* V, float* S, float* z,
+                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* In-place inclusive prefix over blocks (SANA-Video Sec. 3.4: the cache after block j
+ * is the sum of the states of blocks 0..j).  S: [B,H,nblk,d,d], z: [B,H,nblk,d].
+ * A no-op in bidirectional mode. */
+int la_state_scan(const la_problem* p, float* S, float* z, cudaStream_t stream);
+
+/* Apply (SANA-Video 2.0, Eq. (1) output; SANA-Video Sec. 3.2 numerator/denominator):
+ * O_n = (phi(Q_n) S_j) / (ReLU(Q_n) . z_j + eps) * sigmoid(G_n), where j is the block of
+ * token n (j = 0 in bidirectional mode) and S, z are the states each block READS, i.e.
+ * the inclusive prefixes in block-causal mode.  Q, G, O: [B,H,N,d]. */
+int la_apply(const la_problem* p, const void* Q, const void* G, const float* S, const float* z,
+             void* O, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Whole bidirectional operator: state reduction then apply.  p->block_frames must be 0. */
+int la_forward_bidir(const la_problem* p, const void* Q, const void* K, const void* V,
+                     const void* G, void* O, void* workspace, size_t workspace_bytes,
+                     cudaStream_t stream);
+
+/* Whole block-causal operator: per-block states, inclusive scan over blocks, apply.
+ * p->block_frames must be > 0.  S_incl [B,H,nblk,d,d] and z_incl [B,H,nblk,d] receive the
+ * inclusive states (the constant-memory cache after each block) when non-NULL. */
+int la_forward_blockcausal(const la_problem* p, const void* Q, const void* K, const void* V,
+                           const void* G, void* O, float* S_incl, float* z_incl,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* The whole operator (bidirectional if p->block_frames == 0, else block-causal, with the
+ * same arguments as la_forward_bidir / la_forward_blockcausal) with timing marks: records
+ * marks[0] on `stream` before the first kernel and marks[i] right after the i-th kernel it
+ * queues, for every i < nmarks.  The events are created and owned by the caller.  Used to time
+ * the individual kernels of one forward pass with CUDA events. */
+int la_forward_marked(const la_problem* p, const void* Q, const void* K, const void* V,
+                      const void* G, void* O, float* S_incl, float* z_incl, void* workspace,
+                      size_t workspace_bytes, cudaStream_t stream, cudaEvent_t* marks, int nmarks);
+
+/* Static description of a status code. */
+const char* la_status_string(int status);
+
+/* Synchronises `stream`, then reads and clears the current device's error word.
+ * Returns LA_OK, LA_ERR_DEVICE if a kernel gave up on a bounded wait since the last
+ * call, or LA_ERR_CUDA if the synchronisation itself failed. */
+int la_device_error(cudaStream_t stream);
+
+/* Number of kernels the last successful entry point on this host thread queued. */
+int la_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_H_ */

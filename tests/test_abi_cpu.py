@@ -1,0 +1,89 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every entry point
+the header declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_linear_attention_relu_b200 as la
+from gated_linear_attention_relu_b200 import binding as bnd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "la.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(la_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_entry_point():
+    lib = la.load()
+    names = _declared()
+    assert "la_forward_bidir" in names and "la_state_reduce" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(bnd.EXPORTS)
+
+
+def test_status_strings():
+    for code in range(9):
+        assert la.status_string(code) and la.status_string(code) != "unknown status"
+    assert la.status_string(99) == "unknown status"
+
+
+def _call_bidir(p, ptrs=(16, 16, 16, 16, 16)):
+    lib = la.load()
+    cp = p.c()
+    return lib.la_forward_bidir(ctypes.byref(cp), *ptrs, 16, 1 << 30, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=48, bands=(16, 16, 16)), 5),
+    (dict(bands=(32, 48, 40)), 3),
+    (dict(bands=(31, 49, 48)), 3),
+    (dict(T=-1), 2),
+    (dict(eps=float("nan")), 2),
+    (dict(rope_base=0.0), 2),
+    (dict(block_frames=2), 2),          # la_forward_bidir wants block_frames == 0
+    (dict(T=100000, Hh=1000, W=1000), 2),  # N beyond 2^31 tokens
+])
+def test_invalid_problems_rejected_before_cuda(kw, status):
+    args = dict(B=1, H=2, T=3, Hh=4, W=5)
+    args.update(kw)
+    assert _call_bidir(la.Problem(**args)) == status
+
+
+def test_null_and_misaligned_pointers_rejected_before_cuda():
+    p = la.Problem(B=1, H=2, T=3, Hh=4, W=5)
+    assert _call_bidir(p, (None, 16, 16, 16, 16)) == 1
+    assert _call_bidir(p, (16, 16, 16, 16, 18)) == 4
+    lib = la.load()
+    cp = p.c()
+    assert lib.la_state_reduce(ctypes.byref(cp), 16, 16, None, 16, 16, 1 << 20, None) == 1
+
+
+def test_invalid_flags_and_dtype():
+    lib = la.load()
+    cp = la.Problem(B=1, H=1, T=1, Hh=1, W=8).c()
+    cp.flags = 8
+    assert lib.la_forward_bidir(ctypes.byref(cp), 16, 16, 16, 16, 16, 16, 1, None) == 5
+    cp.flags = 0
+    cp.dtype = 7
+    assert lib.la_forward_bidir(ctypes.byref(cp), 16, 16, 16, 16, 16, 16, 1, None) == 5
+
+
+def test_workspace_sizes_are_consistent():
+    base = la.Problem(B=1, H=32, T=21, Hh=45, W=80)
+    ws1 = la.workspace_bytes(base, sm_count=148)
+    ws2 = la.workspace_bytes(la.Problem(B=2, H=32, T=21, Hh=45, W=80), sm_count=148)
+    assert ws1 > 0 and ws2 > ws1
+    # bf16 d=128 uses the tensor-core kernels: partial slots of 128x128 + 8x128 floats, the fp32
+    # states and the bf16 operand images.
+    units = 32
+    assert ws1 >= units * (128 * 128 + 128) * 4 + units * (32768 + 512)
+    bc = la.Problem(B=1, H=32, T=81, Hh=45, W=80, block_frames=3)
+    assert la.workspace_bytes(bc, sm_count=148) >= 32 * 27 * (32768 + 512)
+    assert la.workspace_bytes(la.Problem(B=1, H=1, T=1, Hh=1, W=1, d=40, bands=(8, 16, 16)), 148) == 0
+    assert la.workspace_bytes(la.Problem(B=0, H=4, T=2, Hh=2, W=2), sm_count=148) >= 0
