@@ -8,6 +8,8 @@
 // Q tile (K-major, 128B swizzle) and S the unit's state as a bf16 operand (N-major).  The
 // denominator, the divide and the gate run on the CUDA cores around it: the thread that
 // transforms row n of Q also owns TMEM lane n, so the denominator never leaves its register.
+// The rotation reads cos/sin from a per-band table (fp64-accurate, built by the combine
+// kernel), indexed [pair][position] so the 32 rows of a warp read consecutive entries.
 //
 // Warps (one CTA per SM, persistent over a contiguous range of tiles):
 //   warp 0      TMA producer: Q and G tiles, plus the state operand once per unit (bulk copy)
@@ -25,8 +27,8 @@ namespace ap {
 
 constexpr int TILE = 128;
 constexpr int D = 128;
-constexpr int QST = 3;   // Q stages
-constexpr int GST = 2;   // G / O stages
+constexpr int QST = 2;   // Q stages (freed when the MMA has read them)
+constexpr int GST = 3;   // G / O stages (freed when the O tile has been stored)
 constexpr int NSB = 2;   // state operand buffers
 constexpr int THREADS = 352;
 constexpr uint32_t HALF = 128 * 128;
@@ -52,13 +54,18 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 256, "barrier block too large");
 
-__device__ __forceinline__ float sigmoidf_fast(float g) { return __frcp_rn(1.0f + __expf(-g)); }
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
+template <int DT, int DH>
 __global__ void __launch_bounds__(THREADS, 1)
 apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
                 const __grid_constant__ CUtensorMap tmO, const Plan p, const __grid_constant__ Rope rope,
                 const uint8_t* __restrict__ simg, const float* __restrict__ zimg,
-                __nv_bfloat16* __restrict__ O) {
+                const float2* __restrict__ tab, __nv_bfloat16* __restrict__ O) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
@@ -191,6 +198,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int row = quarter * 32 + lane;
     const uint32_t swz = static_cast<uint32_t>(row & 7);
     const uint32_t row_off = static_cast<uint32_t>(row) * 128u;
+    const int ext_t = static_cast<int>(p.T), ext_h = static_cast<int>(p.Hh), ext_w = static_cast<int>(p.W);
     for (int64_t g = g0 + wg; g < g1; g += 2) {
       const int64_t i = g - g0;
       const TileInfo ti = tile_info(p, g);
@@ -203,11 +211,15 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
       // -- transform: A = RoPE(ReLU(q)) in place, den = ReLU(q) . z
       const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
-      uint32_t pt, ph, pw;
-      token_pos(p, n, pt, ph, pw);
+      uint32_t pt = 0, ph = 0, pw = 0;
+      // Rows past the end of the head keep position 0 (their output is dropped).
+      if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph, pw);
+      const int it = static_cast<int>(pt);
+      const int ih = static_cast<int>(rope.tab_off_h + ph);
+      const int iw = static_cast<int>(rope.tab_off_w + pw);
       const uint32_t qrow = sbase + OFF_Q + qs * BUF + row_off;
       const uint32_t zb = sbase + OFF_Z + b * 512;
-      float den = 0.f;
+      float den4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int ck = 0; ck < 16; ++ck) {
         const uint32_t addr = qrow + (ck >> 3) * HALF + (((static_cast<uint32_t>(ck) & 7u) ^ swz) << 4);
@@ -219,25 +231,26 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
+          const int pi = 4 * ck + q;
+          const int bnd = band_of<DT, DH>(pi, rope);
+          const int loc = pair_in_band<DT, DH>(pi, rope);
+          const int idx = bnd == 0 ? it + loc * ext_t : (bnd == 1 ? ih + loc * ext_h : iw + loc * ext_w);
+          const float2 cs = __ldg(tab + idx);
           const float x0 = fmaxf(bf16lo(w[q]), 0.f);
           const float x1 = fmaxf(bf16hi(w[q]), 0.f);
-          den = fmaf(x0, zz[2 * q], den);
-          den = fmaf(x1, zz[2 * q + 1], den);
-          const int pi = 4 * ck + q;
-          const int bnd = rope.band[pi];
-          const uint32_t pos = bnd == 0 ? pt : (bnd == 1 ? ph : pw);
-          float sn, cs;
-          __sincosf(static_cast<float>(pos) * rope.theta[pi], &sn, &cs);
-          o[q] = pack_bf16(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+          den4[q] = fmaf(x0, zz[2 * q], den4[q]);
+          den4[q] = fmaf(x1, zz[2 * q + 1], den4[q]);
+          o[q] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
         }
         sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->aready[qs]);
-      const float inv = 1.0f / (den + p.eps);
+      // o = acc / den * sigmoid(g) = a + a * tanh(g / 2) with a = acc * 0.5 / den.
+      const float hinv = 0.5f / ((den4[0] + den4[1]) + (den4[2] + den4[3]) + p.eps);
 
-      // -- epilogue: O = acc * inv * sigmoid(g), bf16, in place over the G tile
+      // -- epilogue, in place over the G tile
       if (!warp_wait(&bars->accfull[wg], static_cast<uint32_t>((i >> 1) & 1), abort_flag)) break;
       if (!warp_wait(&bars->gfull[gs], static_cast<uint32_t>((i / GST) & 1), abort_flag)) break;
       tc_fence_after();
@@ -247,22 +260,27 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       __nv_bfloat16* orow = O + (ti.bh * p.N + static_cast<int64_t>(n)) * D;
       const uint32_t taddr = tmem + static_cast<uint32_t>(wg) * 128u + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t r[32];
-        tmem_ld_x32(taddr + ch * 32, r);
+      for (int hv = 0; hv < 2; ++hv) {
+        uint32_t r0[32], r1[32];
+        tmem_ld_x32(taddr + hv * 64, r0);
+        tmem_ld_x32(taddr + hv * 64 + 32, r1);
         tmem_ld_wait();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int ck = ch * 4 + cc;
+        for (int cc = 0; cc < 8; ++cc) {
+          const int ck = hv * 8 + cc;
           const uint32_t addr = grow + (ck >> 3) * HALF + (((static_cast<uint32_t>(ck) & 7u) ^ swz) << 4);
           const uint4 graw = lds128(addr);
           const uint32_t gw[4] = {graw.x, graw.y, graw.z, graw.w};
           uint32_t o[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float a0 = __uint_as_float(r[cc * 8 + 2 * q]) * inv;
-            const float a1 = __uint_as_float(r[cc * 8 + 2 * q + 1]) * inv;
-            o[q] = pack_bf16(a0 * sigmoidf_fast(bf16lo(gw[q])), a1 * sigmoidf_fast(bf16hi(gw[q])));
+            const int col = (cc & 3) * 8 + 2 * q;
+            const float acc0 = __uint_as_float(cc < 4 ? r0[col] : r1[col]);
+            const float acc1 = __uint_as_float(cc < 4 ? r0[col + 1] : r1[col + 1]);
+            const float a0 = acc0 * hinv, a1 = acc1 * hinv;
+            const float t0 = tanh_approx(0.5f * bf16lo(gw[q]));
+            const float t1 = tanh_approx(0.5f * bf16hi(gw[q]));
+            o[q] = pack_bf16(fmaf(a0, t0, a0), fmaf(a1, t1, a1));
           }
           const uint4 ov = make_uint4(o[0], o[1], o[2], o[3]);
           if (tma_out) {

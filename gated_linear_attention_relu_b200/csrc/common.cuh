@@ -37,7 +37,27 @@ struct Rope {
   float theta[64];      // base^(-2i/D) of the pair's band, fp32
   double theta_d[64];   // same in fp64
   int32_t band[64];     // 0: t, 1: h, 2: w
+  int32_t dt, dh, dw;   // band widths in channels
+  // cos/sin table (float2 entries), band-major then pair then position:
+  //   t band: [dt/2][T] at 0, h band: [dh/2][Hh] at off_h, w band: [dw/2][W] at off_w.
+  int64_t tab_off_h, tab_off_w, tab_entries;
 };
+
+// Band (0: t, 1: h, 2: w) of channel pair `pair`.  DT/DH >= 0 fix the split at compile time.
+template <int DT, int DH>
+__host__ __device__ __forceinline__ int band_of(int pair, const Rope& r) {
+  const int dt = DT >= 0 ? DT : r.dt;
+  const int dh = DH >= 0 ? DH : r.dh;
+  return (2 * pair < dt) ? 0 : (2 * pair < dt + dh ? 1 : 2);
+}
+// Index of `pair` within its band.
+template <int DT, int DH>
+__host__ __device__ __forceinline__ int pair_in_band(int pair, const Rope& r) {
+  const int dt = DT >= 0 ? DT : r.dt;
+  const int dh = DH >= 0 ? DH : r.dh;
+  const int b = band_of<DT, DH>(pair, r);
+  return b == 0 ? pair : (b == 1 ? pair - dt / 2 : pair - (dt + dh) / 2);
+}
 
 struct TileInfo {
   int64_t bh;      // flat head index b*H + h

@@ -108,7 +108,8 @@ struct PlanSet {
   Plan ps;            // state reduction
   Plan pa;            // apply
   int64_t units;      // B*H*nblk
-  size_t off_partial, off_states, off_img, off_zimg, total;
+  size_t off_partial, off_states, off_img, off_zimg, off_tab, total;
+  int64_t tab_entries;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -135,6 +136,9 @@ PlanSet make_plans(const la_problem& q, int sm_count) {
   off = align256(off + (s.tc ? size_t(s.units) * 32768 : 0));
   s.off_zimg = off;
   off = align256(off + (s.tc ? size_t(s.units) * 512 : 0));
+  s.tab_entries = (s.tc && s.pa.total > 0) ? (q.dt / 2) * q.T + (q.dh / 2) * q.Hh + (q.dw / 2) * q.W : 0;
+  s.off_tab = off;
+  off = align256(off + size_t(s.tab_entries) * 8);
   s.total = off;
   return s;
 }
@@ -152,8 +156,18 @@ Rope make_rope(const la_problem& q) {
       r.band[pi] = axis;
     }
   }
+  r.dt = q.dt;
+  r.dh = q.dh;
+  r.dw = q.dw;
+  r.tab_off_h = int64_t(q.dt / 2) * q.T;
+  r.tab_off_w = r.tab_off_h + int64_t(q.dh / 2) * q.Hh;
+  r.tab_entries = r.tab_off_w + int64_t(q.dw / 2) * q.W;
   return r;
 }
+
+// The band split of the production head (d = 128: t/h/w = 32/48/48) gets kernels with the split
+// fixed at compile time; any other split uses the run-time variant.
+bool standard_bands(const la_problem& q) { return q.d == 128 && q.dt == 32 && q.dh == 48 && q.dw == 48; }
 
 // ------------------------------------------------------------------------------- CUDA helpers
 int current_sm_count(int* sm) {
@@ -206,10 +220,10 @@ int launch_state(const PlanSet& s, const la_problem& q, const void* K, const voi
   if (s.tc) {
     CUtensorMap tk, tv;
     if (!make_tmap(&tk, K, s.ps.BH, s.ps.N) || !make_tmap(&tv, V, s.ps.BH, s.ps.N)) return LA_ERR_CUDA;
-    if (cudaFuncSetAttribute(la::st::state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             la::st::SMEM_BYTES) != cudaSuccess)
+    auto kern = standard_bands(q) ? la::st::state_tc_kernel<32, 48> : la::st::state_tc_kernel<-1, -1>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::st::SMEM_BYTES) != cudaSuccess)
       return LA_ERR_CUDA;
-    la::st::state_tc_kernel<<<s.ps.grid, la::st::THREADS, la::st::SMEM_BYTES, st>>>(tk, tv, s.ps, rope, partial);
+    kern<<<s.ps.grid, la::st::THREADS, la::st::SMEM_BYTES, st>>>(tk, tv, s.ps, rope, partial);
   } else {
 #define LA_STATE_SIMT(DD, TT)                                                                         \
   la::simt::state_simt_kernel<DD, TT><<<s.ps.grid, la::simt::THREADS, 0, st>>>(                      \
@@ -229,8 +243,8 @@ int launch_state(const PlanSet& s, const la_problem& q, const void* K, const voi
   return launched_ok();
 }
 
-int launch_combine(const PlanSet& s, void* ws, float* S_blk, float* z_blk, float* S_inc, float* z_inc, bool img,
-                   cudaStream_t st, int* nl) {
+int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk, float* z_blk, float* S_inc,
+                   float* z_inc, bool img, cudaStream_t st, int* nl) {
   const int64_t groups = (int64_t(s.ps.d) * s.ps.d + s.ps.d) / 8;
   const int64_t threads = s.ps.BH * groups;
   if (threads == 0 || s.ps.nblk == 0) return LA_OK;
@@ -238,8 +252,14 @@ int launch_combine(const PlanSet& s, void* ws, float* S_blk, float* z_blk, float
   const float* partial = reinterpret_cast<const float*>(w + s.off_partial);
   uint8_t* im = img ? w + s.off_img : nullptr;
   float* zim = img ? reinterpret_cast<float*>(w + s.off_zimg) : nullptr;
-  const unsigned blocks = unsigned((threads + la::cmb::THREADS - 1) / la::cmb::THREADS);
-  la::cmb::combine_kernel<<<blocks, la::cmb::THREADS, 0, st>>>(s.ps, partial, S_blk, z_blk, S_inc, z_inc, im, zim);
+  // The apply's cos/sin table is filled by extra blocks of the same launch.
+  const int64_t tab_n = img ? s.tab_entries : 0;
+  float2* tab = tab_n ? reinterpret_cast<float2*>(w + s.off_tab) : nullptr;
+  const int64_t cblocks = (threads + la::cmb::THREADS - 1) / la::cmb::THREADS;
+  const int64_t tblocks = (tab_n + la::cmb::THREADS - 1) / la::cmb::THREADS;
+  const Rope rope = make_rope(q);
+  la::cmb::combine_kernel<<<unsigned(cblocks + tblocks), la::cmb::THREADS, 0, st>>>(
+      s.ps, partial, S_blk, z_blk, S_inc, z_inc, im, zim, rope, tab, cblocks);
   ++*nl;
   return launched_ok();
 }
@@ -259,12 +279,12 @@ int launch_apply(const PlanSet& s, const la_problem& q, const void* Q, const voi
     if (!make_tmap(&tq, Q, s.pa.BH, s.pa.N) || !make_tmap(&tg, G, s.pa.BH, s.pa.N) ||
         !make_tmap(&to, O, s.pa.BH, s.pa.N))
       return LA_ERR_CUDA;
-    if (cudaFuncSetAttribute(la::ap::apply_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             la::ap::SMEM_BYTES) != cudaSuccess)
+    auto kern = standard_bands(q) ? la::ap::apply_tc_kernel<32, 48> : la::ap::apply_tc_kernel<-1, -1>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::ap::SMEM_BYTES) != cudaSuccess)
       return LA_ERR_CUDA;
-    la::ap::apply_tc_kernel<<<s.pa.grid, la::ap::THREADS, la::ap::SMEM_BYTES, st>>>(
+    kern<<<s.pa.grid, la::ap::THREADS, la::ap::SMEM_BYTES, st>>>(
         tq, tg, to, s.pa, rope, w + s.off_img, reinterpret_cast<const float*>(w + s.off_zimg),
-        static_cast<__nv_bfloat16*>(O));
+        reinterpret_cast<const float2*>(w + s.off_tab), static_cast<__nv_bfloat16*>(O));
   } else {
     const size_t smem = apply_simt_smem(q.d);
 #define LA_APPLY_SIMT(DD, TT)                                                                              \
@@ -335,7 +355,7 @@ int la_state_reduce(const la_problem* p, const void* K, const void* V, float* S,
   if ((rc = check_ws(s, ws, ws_bytes))) return rc;
   int nl = 0;
   if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
-  if ((rc = launch_combine(s, ws, S, z, nullptr, nullptr, false, stream, &nl))) return rc;
+  if ((rc = launch_combine(s, *p, ws, S, z, nullptr, nullptr, false, stream, &nl))) return rc;
   g_last_launches = nl;
   return LA_OK;
 }
@@ -383,9 +403,12 @@ int la_apply(const la_problem* p, const void* Q, const void* G, const float* S, 
     if ((rc = check_ws(s, ws, ws_bytes))) return rc;
     uint8_t* w = static_cast<uint8_t*>(ws);
     const int64_t threads = s.units * ((128 * 128 + 128) / 8);
-    const unsigned blocks = unsigned((threads + la::cmb::THREADS - 1) / la::cmb::THREADS);
-    la::cmb::pack_kernel<<<blocks, la::cmb::THREADS, 0, stream>>>(s.units, 128, S, z, w + s.off_img,
-                                                                   reinterpret_cast<float*>(w + s.off_zimg));
+    const int64_t pblocks = (threads + la::cmb::THREADS - 1) / la::cmb::THREADS;
+    const int64_t tblocks = (s.tab_entries + la::cmb::THREADS - 1) / la::cmb::THREADS;
+    const Rope rope = make_rope(*p);
+    la::cmb::pack_kernel<<<unsigned(pblocks + tblocks), la::cmb::THREADS, 0, stream>>>(
+        s.units, 128, S, z, w + s.off_img, reinterpret_cast<float*>(w + s.off_zimg), s.pa, rope,
+        reinterpret_cast<float2*>(w + s.off_tab), pblocks);
     ++nl;
     if ((rc = launched_ok())) return rc;
   }
@@ -427,7 +450,7 @@ static int forward_common(const la_problem* p, const void* Q, const void* K, con
   if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
   mark(nl);
   const int before = nl;
-  if ((rc = launch_combine(s, ws, nullptr, nullptr, need_fp32 ? st_S : nullptr, need_fp32 ? st_z : nullptr,
+  if ((rc = launch_combine(s, *p, ws, nullptr, nullptr, need_fp32 ? st_S : nullptr, need_fp32 ? st_z : nullptr,
                            s.tc, stream, &nl)))
     return rc;
   if (nl != before) mark(nl);

@@ -240,9 +240,34 @@ __device__ __forceinline__ void store8(float* S, float* z, int64_t unit, int D, 
   d4[1] = make_float4(x[4], x[5], x[6], x[7]);
 }
 
+// cos/sin of every (band, pair, position) the tensor-core apply reads, computed in fp64:
+// entry e of band b holds (cos, sin)(x * theta) for pair i = (e - off_b) / extent_b and
+// position x = (e - off_b) % extent_b.
+__device__ __forceinline__ void rope_table_entry(const Plan& p, const Rope& r, int64_t e, float2* tab) {
+  int64_t i, x;
+  int pair;
+  if (e < r.tab_off_h) {
+    i = e / p.T; x = e - i * p.T; pair = static_cast<int>(i);
+  } else if (e < r.tab_off_w) {
+    i = (e - r.tab_off_h) / p.Hh; x = (e - r.tab_off_h) - i * p.Hh; pair = r.dt / 2 + static_cast<int>(i);
+  } else {
+    i = (e - r.tab_off_w) / p.W; x = (e - r.tab_off_w) - i * p.W; pair = (r.dt + r.dh) / 2 + static_cast<int>(i);
+  }
+  double s, c;
+  sincos(static_cast<double>(x) * r.theta_d[pair], &s, &c);
+  tab[e] = make_float2(static_cast<float>(c), static_cast<float>(s));
+}
+
+// Blocks [0, comb_blocks) combine states; blocks past them (if any) fill the cos/sin table.
 __global__ void __launch_bounds__(THREADS)
 combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, float* z_blk, float* S_inc,
-               float* z_inc, uint8_t* img, float* zimg) {
+               float* z_inc, uint8_t* img, float* zimg, const __grid_constant__ Rope rope, float2* tab,
+               int64_t comb_blocks) {
+  if (static_cast<int64_t>(blockIdx.x) >= comb_blocks) {
+    const int64_t e = (static_cast<int64_t>(blockIdx.x) - comb_blocks) * THREADS + threadIdx.x;
+    if (tab && e < rope.tab_entries) rope_table_entry(p, rope, e, tab);
+    return;
+  }
   const int D = p.d;
   const int groups = (D * D + D) / 8;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
@@ -314,7 +339,12 @@ scan_kernel(int64_t BH, int64_t nblk, int D, float* S, float* z) {
 // bf16 operand image of given fp32 states (for the tensor-core apply called on its own).
 __global__ void __launch_bounds__(THREADS)
 pack_kernel(int64_t units, int D, const float* __restrict__ S, const float* __restrict__ z, uint8_t* img,
-            float* zimg) {
+            float* zimg, const Plan p, const __grid_constant__ Rope rope, float2* tab, int64_t pack_blocks) {
+  if (static_cast<int64_t>(blockIdx.x) >= pack_blocks) {
+    const int64_t e = (static_cast<int64_t>(blockIdx.x) - pack_blocks) * THREADS + threadIdx.x;
+    if (tab && e < rope.tab_entries) rope_table_entry(p, rope, e, tab);
+    return;
+  }
   const int groups = (D * D + D) / 8;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
   const int64_t u = idx / groups;

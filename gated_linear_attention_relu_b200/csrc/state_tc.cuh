@@ -8,10 +8,11 @@
 // A = RoPE(ReLU(K))^T (channels x tokens, M-major) and B = V (tokens x channels, N-major).
 //
 // Pipeline (one CTA per SM, persistent over a contiguous range of 128-token tiles):
-//   warp 0      TMA producer: K and V tiles (two 64-channel, 128-row, 128B-swizzled boxes each)
-//   warp 1      MMA issuer: 8 x tcgen05.mma per tile into one of two TMEM accumulators
-//   warps 2-5   transform: ReLU + RoPE of K in place (bf16), z accumulated in registers
-//   warps 6-9   drain: TMEM accumulator -> fp32 partial S in global memory, once per unit
+//   warp 0       TMA producer: K and V tiles (two 64-channel, 128-row, 128B-swizzled boxes each)
+//   warp 1       MMA issuer: 8 x tcgen05.mma per tile into one of two TMEM accumulators
+//   warps 2-9    transform, two groups of four warps splitting each tile's rows: ReLU + RoPE of
+//                K in place (bf16), z accumulated in registers
+//   warps 10-13  drain: TMEM accumulator -> fp32 partial S in global memory, once per unit
 // The staged K tile is already in the canonical 128B-swizzled MN-major operand layout, so the
 // transform rewrites it in place.
 #pragma once
@@ -24,20 +25,22 @@ namespace st {
 constexpr int TILE = 128;
 constexpr int D = 128;
 constexpr int STAGES = 3;
-constexpr int THREADS = 320;
+constexpr int TGROUPS = 2;                    // transform warpgroups
+constexpr int THREADS = 32 * (2 + 4 * TGROUPS + 4);
 constexpr uint32_t HALF = 128 * 128;          // one 64-channel box of 128 rows x 128 B
 constexpr uint32_t BUF = 2 * HALF;            // 128 tokens x 128 channels bf16
 constexpr uint32_t STAGE = 2 * BUF;           // K + V
 constexpr uint32_t OFF_BAR = STAGES * STAGE;  // barriers after the stages
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
-constexpr int ZPARTS = 8;                     // z is written as 8 row-group partial sums
+constexpr int ZPARTS = 8 * TGROUPS;           // z is written as one partial sum per row group
 constexpr int64_t SLOT = D * D + ZPARTS * D;  // floats per partial slot: S, then ZPARTS x z
 constexpr uint32_t TMEM_COLS = 256;           // two 128-column fp32 accumulators
 constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, /*a_mn=*/true, /*b_mn=*/true);
+constexpr int DRAIN_WARP0 = 2 + 4 * TGROUPS;
 
 struct Bars {
   uint64_t full[STAGES];     // TMA landed K and V            (1 arrival + tx bytes)
-  uint64_t aready[STAGES];   // transform wrote the A operand  (4 warps)
+  uint64_t aready[STAGES];   // transform wrote the A operand  (one arrival per transform warp)
   uint64_t empty[STAGES];    // MMAs of the stage completed    (tcgen05.commit)
   uint64_t accfull[2];       // accumulator holds a finished unit (tcgen05.commit)
   uint64_t accempty[2];      // drain finished reading it     (4 warps)
@@ -47,6 +50,7 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 256, "barrier block too large");
 
+template <int DT, int DH>
 __global__ void __launch_bounds__(THREADS, 1)
 state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const Plan p, const __grid_constant__ Rope rope, float* __restrict__ partial) {
@@ -66,7 +70,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&bars->full[s], 1);
-      mbar_init(&bars->aready[s], 4);
+      mbar_init(&bars->aready[s], 4 * TGROUPS);
       mbar_init(&bars->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -150,51 +154,47 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       mma_commit(&bars->final_);
       mbar_wait_drain(&bars->final_, 0);
     }
-  } else if (warp < 6) {
+  } else if (warp < DRAIN_WARP0) {
     // ------------------------------------------------------------ transform: ReLU + RoPE of K
-    const int tt = threadIdx.x - 64;  // 0..127
-    const int ck = tt & 15;           // 8-channel chunk: channels 8ck .. 8ck+7
-    const int rg = tt >> 4;           // rows rg, rg+8, ..., rg+120 (so row % 8 == rg)
+    const int tg = (warp - 2) >> 2;               // transform group: rows 64*tg .. 64*tg+63
+    const int tt = threadIdx.x - 64 - 128 * tg;   // 0..127 within the group
+    const int ck = tt & 15;                       // 8-channel chunk: channels 8ck .. 8ck+7
+    const int rg = tt >> 4;                       // rows 64tg + rg + 8j, j < 8 (row % 8 == rg)
     const uint32_t chunk_off = static_cast<uint32_t>((ck >> 3) * HALF + (((ck & 7) ^ rg) << 4));
     float th[4];
     int bd[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       th[q] = rope.theta[4 * ck + q];
-      bd[q] = rope.band[4 * ck + q];
+      bd[q] = band_of<DT, DH>(4 * ck + q, rope);
     }
     float zacc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
-    int64_t seg = -1;
-    int64_t prev_unit = -1;
     for (int64_t g = g0; g < g1; ++g) {
       const int64_t i = g - g0;
       const int s = static_cast<int>(i % STAGES);
       const uint32_t ph = static_cast<uint32_t>((i / STAGES) & 1);
       const TileInfo ti = tile_info(p, g);
-      if (ti.unit != prev_unit) {
-        ++seg;
-        prev_unit = ti.unit;
-      }
       const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != ti.unit);
       if (!warp_wait(&bars->full[s], ph, abort_flag)) break;
-      const uint32_t base = sbase + s * STAGE + chunk_off;
-      uint32_t n = static_cast<uint32_t>(ti.n0) + rg;
+      const int row0 = 64 * tg + rg;
+      const uint32_t base = sbase + s * STAGE + chunk_off + static_cast<uint32_t>(row0 * 128);
+      uint32_t n = static_cast<uint32_t>(ti.n0) + row0;
       const uint32_t n_end = static_cast<uint32_t>(ti.n_end);
       uint32_t pt, ph_, pw;
       token_pos(p, n, pt, ph_, pw);
-#pragma unroll 2
-      for (int j = 0; j < TILE / 8; ++j) {
-        const uint32_t addr = base + static_cast<uint32_t>((rg + 8 * j) * 128);
-        uint4 raw = lds128(addr);
+#pragma unroll 4
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t addr = base + static_cast<uint32_t>(j * 8 * 128);
+        const uint4 raw = lds128(addr);
         const bool valid = n < n_end;
-        uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
         uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          float x0 = valid ? fmaxf(bf16lo(w[q]), 0.f) : 0.f;
-          float x1 = valid ? fmaxf(bf16hi(w[q]), 0.f) : 0.f;
+          const float x0 = valid ? fmaxf(bf16lo(w[q]), 0.f) : 0.f;
+          const float x1 = valid ? fmaxf(bf16hi(w[q]), 0.f) : 0.f;
           zacc[2 * q] += x0;
           zacc[2 * q + 1] += x1;
           const uint32_t pos = bd[q] == 0 ? pt : (bd[q] == 1 ? ph_ : pw);
@@ -210,9 +210,9 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->aready[s]);
       if (last) {
-        // z of this unit, one partial per row group rg; the combine kernel adds the 8 in order.
+        // z of this unit, one partial per row group; the combine kernel adds them in order.
         const int64_t slot = c * p.maxseg + (ti.unit - u_first);
-        float4* zd = reinterpret_cast<float4*>(partial + slot * SLOT + D * D + rg * D + 8 * ck);
+        float4* zd = reinterpret_cast<float4*>(partial + slot * SLOT + D * D + (tg * 8 + rg) * D + 8 * ck);
         zd[0] = make_float4(zacc[0], zacc[1], zacc[2], zacc[3]);
         zd[1] = make_float4(zacc[4], zacc[5], zacc[6], zacc[7]);
 #pragma unroll
