@@ -231,7 +231,7 @@ def main():
 
     # Marker events around each kernel of each timed step; recorded once here so their CUDA
     # handles exist before the timed region.
-    nmark = 4
+    nmark = 5
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nmark)] for _ in range(args.steps)]
     for row in evs:
         for e in row:
@@ -258,9 +258,10 @@ def main():
     assert la.device_error() == 0, "device-side error in the timed region"
 
     # Per-kernel durations inside the timed steps.
-    names = ["state_tc_kernel", "combine_kernel", "apply_tc_kernel"] if not args.simt and w.d == 128 \
-        and w.dtype == "bf16" else ["state_simt_kernel", "combine_kernel", "apply_simt_kernel"]
-    names = names[:launches_per_step]
+    tc = not args.simt and w.d == 128 and w.dtype == "bf16"
+    names = ["rope_table_kernel", "state_tc_kernel", "combine_kernel", "apply_tc_kernel"] if tc \
+        else ["state_simt_kernel", "combine_kernel", "apply_simt_kernel"]
+    assert len(names) == launches_per_step, (names, launches_per_step)
     per = {n: [] for n in names}
     for k in range(args.steps):
         for i, n in enumerate(names):
@@ -269,7 +270,7 @@ def main():
     tot = sum(kern_ms.values())
     elem = w.elem_bytes
     th = w.B * w.H * w.N
-    alg_bytes = {names[0]: 2 * th * w.d * elem, names[-1]: 3 * th * w.d * elem}
+    alg_bytes = {names[-3]: 2 * th * w.d * elem, names[-1]: 3 * th * w.d * elem}
     dominant = max((n for n in names if n in alg_bytes), key=lambda n: kern_ms[n])
     peak, peak_kind = measured_hbm()
     achieved = alg_bytes[dominant] / (kern_ms[dominant] * 1e-3) / 1e9

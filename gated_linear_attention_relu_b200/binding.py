@@ -25,7 +25,7 @@ STATUS = {
 EXPORTS = [
     "la_workspace_bytes", "la_workspace_bytes_for", "la_state_reduce", "la_state_scan", "la_apply",
     "la_forward_bidir", "la_forward_blockcausal", "la_status_string", "la_device_error",
-    "la_last_launch_count", "la_forward_marked",
+    "la_last_launch_count", "la_forward_marked", "la_selftest_host",
 ]
 
 
@@ -53,8 +53,8 @@ def load(path: Optional[str] = None):
     global _lib
     if _lib is not None:
         return _lib
-    path = path or LIB_PATH
-    if not os.path.exists(path):
+    path = path or os.environ.get("LA_LIBRARY") or LIB_PATH
+    if not os.path.exists(path) and path == LIB_PATH:
         from . import build as _build
 
         _build.build()
@@ -75,6 +75,7 @@ def load(path: Optional[str] = None):
         "la_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "la_device_error": (ctypes.c_int, [vp]),
         "la_last_launch_count": (ctypes.c_int, []),
+        "la_selftest_host": (ctypes.c_int, []),
         "la_forward_marked": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                              ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
     }

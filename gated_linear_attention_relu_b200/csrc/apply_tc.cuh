@@ -8,56 +8,117 @@
 // Q tile (K-major, 128B swizzle) and S the unit's state as a bf16 operand (N-major).  The
 // denominator, the divide and the gate run on the CUDA cores around it: the thread that
 // transforms row n of Q also owns TMEM lane n, so the denominator never leaves its register.
-// The rotation reads cos/sin from a per-band table (fp64-accurate, built by the combine
-// kernel), indexed [pair][position] so the 32 rows of a warp read consecutive entries.
+// The rotation reads cos/sin from a per-band table (fp64-accurate, built by the prep kernel),
+// indexed [pair][position] so the 32 rows of a warp read consecutive entries.
 //
 // Warps (one CTA per SM, persistent over a contiguous range of tiles):
-//   warp 0      TMA producer: Q and G tiles, plus the state operand once per unit (bulk copy)
-//   warp 1      MMA issuer
-//   warps 2-5   math group 0 (even local tiles), warps 6-9 math group 1 (odd local tiles):
-//               transform Q, then epilogue: TMEM -> registers, divide, gate, bf16, written in
-//               place over the staged G tile
-//   warp 10     TMA store of the finished O tile, then releases the G stage
+//   warpgroup 0   warp 0: TMA producer (Q and G tiles; the state operand once per unit)
+//                 warp 1: MMA issuer (and TMEM owner); warp 2: TMA store of finished O tiles
+//   warpgroups 1..NWG  math: group w takes local tiles i = w-1 (mod NWG): transform Q, then the
+//                 epilogue (TMEM -> registers, divide, gate, bf16) in place over the staged G tile
+// With three math groups the control warpgroup hands registers to the math groups
+// (setmaxnreg); the host checks the launch's register budget before launching.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
+
+#ifndef LA_AP_QST
+#define LA_AP_QST 2
+#endif
+#ifndef LA_AP_GST
+#define LA_AP_GST 2
+#endif
+#ifndef LA_AP_NSB
+#define LA_AP_NSB 2
+#endif
+#ifndef LA_AP_NWG
+#define LA_AP_NWG 2
+#endif
 
 namespace la {
 namespace ap {
 
 constexpr int TILE = 128;
 constexpr int D = 128;
-constexpr int QST = 2;   // Q stages (freed when the MMA has read them)
-constexpr int GST = 3;   // G / O stages (freed when the O tile has been stored)
-constexpr int NSB = 2;   // state operand buffers
-constexpr int THREADS = 352;
+constexpr int QST = LA_AP_QST;  // Q stages (freed when the MMA has read them)
+constexpr int GST = LA_AP_GST;  // G / O stages (freed when the O tile has been stored)
+constexpr int NSB = LA_AP_NSB;  // state operand buffers
+constexpr int NWG = LA_AP_NWG;  // math warpgroups
+constexpr int THREADS = 128 * (1 + NWG);
 constexpr uint32_t HALF = 128 * 128;
 constexpr uint32_t BUF = 2 * HALF;  // 32 KB: a 128 x 128 bf16 tile
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_G = OFF_Q + QST * BUF;
 constexpr uint32_t OFF_S = OFF_G + GST * BUF;
-constexpr uint32_t OFF_Z = OFF_S + NSB * BUF;
-constexpr uint32_t OFF_BAR = OFF_Z + NSB * 512;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
-constexpr uint32_t TMEM_COLS = 256;                    // one 128-column accumulator per math group
+constexpr uint32_t OFF_BAR = OFF_S + NSB * BUF;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // + alignment slack
+constexpr uint32_t TMEM_COLS = NWG <= 2 ? 256 : 512;   // one 128-column accumulator per math group
 constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/true);
+// Register split (used only with three or more math groups).  The launch grants REGS_LAUNCH per
+// thread (the largest multiple of 8 that fits 65536 / THREADS); the control warpgroup shrinks to
+// REGS_CTRL and the math groups grow to REGS_MATH, never asking for more than the launch granted.
+constexpr bool SPLIT_REGS = NWG >= 3;
+constexpr uint32_t REGS_LAUNCH = (65536 / THREADS) / 8 * 8;
+constexpr uint32_t REGS_CTRL = 56;
+constexpr uint32_t REGS_MATH = ((THREADS * REGS_LAUNCH - 128 * REGS_CTRL) / (128 * NWG)) / 8 * 8;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// Each Q / G stage must always serve the same math group: a group then never polls a stage's
+// barrier more than one phase ahead of it, so the parity test cannot alias.
+static_assert(QST % NWG == 0 && GST % NWG == 0, "stages must be a multiple of the math groups");
+static_assert(!SPLIT_REGS || 128 * REGS_CTRL + 128 * NWG * REGS_MATH <= THREADS * REGS_LAUNCH, "register split");
+static_assert(!SPLIT_REGS || (REGS_CTRL <= REGS_LAUNCH && REGS_LAUNCH <= REGS_MATH), "register split");
 
 struct Bars {
   uint64_t qfull[QST], aready[QST], qempty[QST];
   uint64_t gfull[GST], gempty[GST], ostaged[GST];
   uint64_t sfull[NSB], sfree[NSB];
-  uint64_t accfull[2], accempty[2];
+  uint64_t accfull[NWG], accempty[NWG];
   uint64_t final_;
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block too large");
+static_assert(sizeof(Bars) <= 512, "barrier block too large");
 
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+template <uint32_t R>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+
+// Transform of chunks [CK0, CK1) of one row, all in one RoPE band: q <- RoPE(ReLU(q)) in place,
+// den += ReLU(q) . z.  `tp` walks the band's [pair][position] table column of this row.
+template <int CK0, int CK1>
+__device__ __forceinline__ void transform_band(uint32_t qrow, uint32_t swz, const float* __restrict__ zg,
+                                               const float2* __restrict__ tp, int ext, float (&den4)[4]) {
+#pragma unroll 2
+  for (int ck = CK0; ck < CK1; ++ck) {
+    const uint32_t addr = qrow + (ck >> 3) * HALF + (((static_cast<uint32_t>(ck) & 7u) ^ swz) << 4);
+    const uint4 raw = lds128(addr);
+    const float4 za = __ldg(reinterpret_cast<const float4*>(zg + ck * 8));
+    const float4 zc = __ldg(reinterpret_cast<const float4*>(zg + ck * 8 + 4));
+    const float zz[8] = {za.x, za.y, za.z, za.w, zc.x, zc.y, zc.z, zc.w};
+    const uint32_t w[4] = {relu_bf16x2(raw.x), relu_bf16x2(raw.y), relu_bf16x2(raw.z), relu_bf16x2(raw.w)};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 cs = __ldg(tp + (4 * (ck - CK0) + q) * ext);
+      const float x0 = bf16lo(w[q]);
+      const float x1 = bf16hi(w[q]);
+      den4[q] = fmaf(x0, zz[2 * q], den4[q]);
+      den4[q] = fmaf(x1, zz[2 * q + 1], den4[q]);
+      o[q] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+    }
+    sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
+  }
 }
 
 template <int DT, int DH>
@@ -94,7 +155,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(&bars->sfull[s], 1);
       mbar_init(&bars->sfree[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < NWG; ++a) {
       mbar_init(&bars->accfull[a], 1);
       mbar_init(&bars->accempty[a], 4);
     }
@@ -116,9 +177,10 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (warp < 4) {
+    if constexpr (SPLIT_REGS) regs_dec<REGS_CTRL>();
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
       int64_t issued_q = 0, issued_g = 0, issued_s = 0;
       int64_t prev_unit = -1;
       for (int64_t g = g0; g < g1; ++g) {
@@ -128,9 +190,8 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const int64_t ku = ti.unit - u_first;
           const int b = static_cast<int>(ku % NSB);
           if (!mbar_wait(&bars->sfree[b], static_cast<uint32_t>(((ku / NSB) & 1) ^ 1), abort_flag)) break;
-          mbar_arrive_expect_tx(&bars->sfull[b], BUF + 512);
+          mbar_arrive_expect_tx(&bars->sfull[b], BUF);
           bulk_load(smem + OFF_S + b * BUF, simg + ti.unit * static_cast<int64_t>(BUF), BUF, &bars->sfull[b]);
-          bulk_load(smem + OFF_Z + b * 512, zimg + ti.unit * D, 512, &bars->sfull[b]);
           prev_unit = ti.unit;
           ++issued_s;
         }
@@ -157,19 +218,17 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int64_t j = (issued_s > NSB ? issued_s - NSB : 0); j < issued_s; ++j)
           mbar_wait_drain(&bars->sfull[j % NSB], static_cast<uint32_t>((j / NSB) & 1));
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       for (int64_t g = g0; g < g1; ++g) {
         const int64_t i = g - g0;
         const int64_t u = unit_of_tile(p, g);
         const int64_t ku = u - u_first;
         const int b = static_cast<int>(ku % NSB);
-        const int wg = static_cast<int>(i & 1);
+        const int wg = static_cast<int>(i % NWG);
         const int qs = static_cast<int>(i % QST);
         const uint32_t qph = static_cast<uint32_t>((i / QST) & 1);
-        if (!mbar_wait(&bars->accempty[wg], static_cast<uint32_t>(((i >> 1) & 1) ^ 1), abort_flag)) break;
+        if (!mbar_wait(&bars->accempty[wg], static_cast<uint32_t>(((i / NWG) & 1) ^ 1), abort_flag)) break;
         if (!mbar_wait(&bars->sfull[b], static_cast<uint32_t>((ku / NSB) & 1), abort_flag)) break;
         if (!mbar_wait(&bars->qfull[qs], qph, abort_flag)) break;
         if (!mbar_wait(&bars->aready[qs], qph, abort_flag)) break;
@@ -190,23 +249,40 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       mma_commit(&bars->final_);
       mbar_wait_drain(&bars->final_, 0);
+    } else if (warp == 2 && lane == 0) {
+      // ---------------------------------------------------------- TMA store of O
+      for (int64_t g = g0; g < g1; ++g) {
+        const int64_t i = g - g0;
+        const int gs = static_cast<int>(i % GST);
+        if (!mbar_wait(&bars->ostaged[gs], static_cast<uint32_t>((i / GST) & 1), abort_flag)) break;
+        const TileInfo ti = tile_info(p, g);
+        if ((ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N)) {
+          const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
+          tma_store_3d(&tmO, smem + OFF_G + gs * BUF, 0, n0, bh);
+          tma_store_3d(&tmO, smem + OFF_G + gs * BUF + HALF, 64, n0, bh);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        mbar_arrive(&bars->gempty[gs]);
+      }
+      bulk_wait_group0();
     }
-  } else if (warp < 10) {
+  } else {
     // ------------------------------------------------------------ math groups
-    const int wg = (warp - 2) >> 2;
+    if constexpr (SPLIT_REGS) regs_inc<REGS_MATH>();
+    const int wg = (warp >> 2) - 1;
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     const uint32_t swz = static_cast<uint32_t>(row & 7);
     const uint32_t row_off = static_cast<uint32_t>(row) * 128u;
     const int ext_t = static_cast<int>(p.T), ext_h = static_cast<int>(p.Hh), ext_w = static_cast<int>(p.W);
-    for (int64_t g = g0 + wg; g < g1; g += 2) {
+    for (int64_t g = g0 + wg; g < g1; g += NWG) {
       const int64_t i = g - g0;
       const TileInfo ti = tile_info(p, g);
-      const int64_t ku = ti.unit - u_first;
-      const int b = static_cast<int>(ku % NSB);
       const int qs = static_cast<int>(i % QST);
       const int gs = static_cast<int>(i % GST);
-      if (!warp_wait(&bars->sfull[b], static_cast<uint32_t>((ku / NSB) & 1), abort_flag)) break;
+      // z is read straight from the combine kernel's output (read-only here), so the math groups
+      // never wait on the state buffer's barrier; only the MMA issuer does.
       if (!warp_wait(&bars->qfull[qs], static_cast<uint32_t>((i / QST) & 1), abort_flag)) break;
 
       // -- transform: A = RoPE(ReLU(q)) in place, den = ReLU(q) . z
@@ -214,35 +290,41 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       uint32_t pt = 0, ph = 0, pw = 0;
       // Rows past the end of the head keep position 0 (their output is dropped).
       if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph, pw);
-      const int it = static_cast<int>(pt);
-      const int ih = static_cast<int>(rope.tab_off_h + ph);
-      const int iw = static_cast<int>(rope.tab_off_w + pw);
       const uint32_t qrow = sbase + OFF_Q + qs * BUF + row_off;
-      const uint32_t zb = sbase + OFF_Z + b * 512;
+      const float* zg = zimg + ti.unit * D;
       float den4[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (DT >= 0 && DH >= 0 && DT % 8 == 0 && DH % 8 == 0) {
+        transform_band<0, DT / 8>(qrow, swz, zg, tab + pt, ext_t, den4);
+        transform_band<DT / 8, (DT + DH) / 8>(qrow, swz, zg, tab + rope.tab_off_h + ph, ext_h, den4);
+        transform_band<(DT + DH) / 8, 16>(qrow, swz, zg, tab + rope.tab_off_w + pw, ext_w, den4);
+      } else {
+        const int it = static_cast<int>(pt);
+        const int ih = static_cast<int>(rope.tab_off_h + ph);
+        const int iw = static_cast<int>(rope.tab_off_w + pw);
+#pragma unroll 2
+        for (int ck = 0; ck < 16; ++ck) {
+          const uint32_t addr = qrow + (ck >> 3) * HALF + (((static_cast<uint32_t>(ck) & 7u) ^ swz) << 4);
+          const uint4 raw = lds128(addr);
+          const float4 za = __ldg(reinterpret_cast<const float4*>(zg + ck * 8));
+          const float4 zc = __ldg(reinterpret_cast<const float4*>(zg + ck * 8 + 4));
+          const float zz[8] = {za.x, za.y, za.z, za.w, zc.x, zc.y, zc.z, zc.w};
+          const uint32_t w[4] = {relu_bf16x2(raw.x), relu_bf16x2(raw.y), relu_bf16x2(raw.z), relu_bf16x2(raw.w)};
+          uint32_t o[4];
 #pragma unroll
-      for (int ck = 0; ck < 16; ++ck) {
-        const uint32_t addr = qrow + (ck >> 3) * HALF + (((static_cast<uint32_t>(ck) & 7u) ^ swz) << 4);
-        const uint4 raw = lds128(addr);
-        const float4 za = lds128f(zb + ck * 32);
-        const float4 zc = lds128f(zb + ck * 32 + 16);
-        const float zz[8] = {za.x, za.y, za.z, za.w, zc.x, zc.y, zc.z, zc.w};
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int pi = 4 * ck + q;
-          const int bnd = band_of<DT, DH>(pi, rope);
-          const int loc = pair_in_band<DT, DH>(pi, rope);
-          const int idx = bnd == 0 ? it + loc * ext_t : (bnd == 1 ? ih + loc * ext_h : iw + loc * ext_w);
-          const float2 cs = __ldg(tab + idx);
-          const float x0 = fmaxf(bf16lo(w[q]), 0.f);
-          const float x1 = fmaxf(bf16hi(w[q]), 0.f);
-          den4[q] = fmaf(x0, zz[2 * q], den4[q]);
-          den4[q] = fmaf(x1, zz[2 * q + 1], den4[q]);
-          o[q] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+          for (int q = 0; q < 4; ++q) {
+            const int pi = 4 * ck + q;
+            const int bnd = band_of<DT, DH>(pi, rope);
+            const int loc = pair_in_band<DT, DH>(pi, rope);
+            const int idx = bnd == 0 ? it + loc * ext_t : (bnd == 1 ? ih + loc * ext_h : iw + loc * ext_w);
+            const float2 cs = __ldg(tab + idx);
+            const float x0 = bf16lo(w[q]);
+            const float x1 = bf16hi(w[q]);
+            den4[q] = fmaf(x0, zz[2 * q], den4[q]);
+            den4[q] = fmaf(x1, zz[2 * q + 1], den4[q]);
+            o[q] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+          }
+          sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
         }
-        sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -251,7 +333,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const float hinv = 0.5f / ((den4[0] + den4[1]) + (den4[2] + den4[3]) + p.eps);
 
       // -- epilogue, in place over the G tile
-      if (!warp_wait(&bars->accfull[wg], static_cast<uint32_t>((i >> 1) & 1), abort_flag)) break;
+      if (!warp_wait(&bars->accfull[wg], static_cast<uint32_t>((i / NWG) & 1), abort_flag)) break;
       if (!warp_wait(&bars->gfull[gs], static_cast<uint32_t>((i / GST) & 1), abort_flag)) break;
       tc_fence_after();
       const bool tma_out = (ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N);
@@ -259,27 +341,25 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint32_t grow = sbase + OFF_G + gs * BUF + row_off;
       __nv_bfloat16* orow = O + (ti.bh * p.N + static_cast<int64_t>(n)) * D;
       const uint32_t taddr = tmem + static_cast<uint32_t>(wg) * 128u + (static_cast<uint32_t>(quarter * 32) << 16);
-#pragma unroll
-      for (int hv = 0; hv < 2; ++hv) {
-        uint32_t r0[32], r1[32];
-        tmem_ld_x32(taddr + hv * 64, r0);
-        tmem_ld_x32(taddr + hv * 64 + 32, r1);
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t r[32];
+        tmem_ld_x32(taddr + ch * 32, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const int ck = hv * 8 + cc;
+        for (int cc = 0; cc < 4; ++cc) {
+          const int ck = ch * 4 + cc;
           const uint32_t addr = grow + (ck >> 3) * HALF + (((static_cast<uint32_t>(ck) & 7u) ^ swz) << 4);
           const uint4 graw = lds128(addr);
-          const uint32_t gw[4] = {graw.x, graw.y, graw.z, graw.w};
+          // g/2 is exact in bf16, so halve the packed words before unpacking.
+          const uint32_t gw[4] = {half_bf16x2(graw.x), half_bf16x2(graw.y), half_bf16x2(graw.z), half_bf16x2(graw.w)};
           uint32_t o[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int col = (cc & 3) * 8 + 2 * q;
-            const float acc0 = __uint_as_float(cc < 4 ? r0[col] : r1[col]);
-            const float acc1 = __uint_as_float(cc < 4 ? r0[col + 1] : r1[col + 1]);
-            const float a0 = acc0 * hinv, a1 = acc1 * hinv;
-            const float t0 = tanh_approx(0.5f * bf16lo(gw[q]));
-            const float t1 = tanh_approx(0.5f * bf16hi(gw[q]));
+            const float a0 = __uint_as_float(r[cc * 8 + 2 * q]) * hinv;
+            const float a1 = __uint_as_float(r[cc * 8 + 2 * q + 1]) * hinv;
+            const float t0 = tanh_approx(bf16lo(gw[q]));
+            const float t1 = tanh_approx(bf16hi(gw[q]));
             o[q] = pack_bf16(fmaf(a0, t0, a0), fmaf(a1, t1, a1));
           }
           const uint4 ov = make_uint4(o[0], o[1], o[2], o[3]);
@@ -297,25 +377,6 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_arrive(&bars->accempty[wg]);
         mbar_arrive(&bars->ostaged[gs]);
       }
-    }
-  } else {
-    // ------------------------------------------------------------ TMA store of O
-    if (lane == 0) {
-      for (int64_t g = g0; g < g1; ++g) {
-        const int64_t i = g - g0;
-        const int gs = static_cast<int>(i % GST);
-        if (!mbar_wait(&bars->ostaged[gs], static_cast<uint32_t>((i / GST) & 1), abort_flag)) break;
-        const TileInfo ti = tile_info(p, g);
-        if ((ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N)) {
-          const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
-          tma_store_3d(&tmO, smem + OFF_G + gs * BUF, 0, n0, bh);
-          tma_store_3d(&tmO, smem + OFF_G + gs * BUF + HALF, 64, n0, bh);
-          bulk_commit_group();
-          bulk_wait_group_read0();
-        }
-        mbar_arrive(&bars->gempty[gs]);
-      }
-      bulk_wait_group0();
     }
   }
 

@@ -14,6 +14,36 @@
 
 namespace la {
 
+// Division by a run-time constant 1 <= d < 2^31, exact for every dividend n < 2^31:
+// with s = ceil(log2 d), mul = ceil(2^(31+s) / d) < 2^32 and q = floor(n * mul / 2^(31+s)).
+// (n * mul / 2^(31+s) = n/d + n*e/2^(31+s) with 0 <= e < 1, and the excess is below 2^-s <= 1/d,
+// so it never carries the quotient past the next integer.)
+struct FastDiv {
+  uint32_t d, mul, shift;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.mul = 0;
+  f.shift = 0;
+  if (d <= 1) return f;
+  uint32_t s = 0;
+  while ((uint64_t(1) << s) < d) ++s;
+  f.mul = static_cast<uint32_t>(((uint64_t(1) << (31 + s)) + d - 1) / d);
+  f.shift = s - 1;
+  return f;
+}
+
+__host__ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  if (f.d == 1) return n;
+#ifdef __CUDA_ARCH__
+  return __umulhi(n, f.mul) >> f.shift;
+#else
+  return static_cast<uint32_t>((uint64_t(n) * f.mul) >> 32) >> f.shift;
+#endif
+}
+
 struct Plan {
   int64_t BH;              // B * H
   int64_t N;               // tokens per head
@@ -30,6 +60,7 @@ struct Plan {
   int32_t d;
   int32_t zparts;          // partial z rows per slot (summed in order by the combine kernel)
   float eps;
+  FastDiv fd_tph, fd_tfull, fd_HW, fd_W;  // tiles_per_head, tiles_full, Hh*W, W
 };
 
 // Rotation parameters of the d/2 channel pairs (at most 64 for d = 128).
@@ -66,27 +97,32 @@ struct TileInfo {
   int64_t n_end;   // one past the last token of the tile's unit
 };
 
+// Tile indices, token indices and tile counts all stay below 2^31 (checked on the host), so the
+// per-tile bookkeeping uses 32-bit multiply-high division.
 __host__ __device__ inline TileInfo tile_info(const Plan& p, int64_t g) {
   TileInfo t;
-  t.bh = g / p.tiles_per_head;
-  int64_t r = g - t.bh * p.tiles_per_head;
-  int64_t blk = r / p.tiles_full;
-  if (blk > p.nblk - 1) blk = p.nblk - 1;
-  int64_t tib = r - blk * p.tiles_full;
-  int64_t start = blk * p.blk_tokens;
+  const uint32_t gg = static_cast<uint32_t>(g);
+  const uint32_t bh = fdiv(gg, p.fd_tph);
+  const uint32_t r = gg - bh * static_cast<uint32_t>(p.tiles_per_head);
+  uint32_t blk = fdiv(r, p.fd_tfull);
+  if (blk > static_cast<uint32_t>(p.nblk - 1)) blk = static_cast<uint32_t>(p.nblk - 1);
+  const uint32_t tib = r - blk * static_cast<uint32_t>(p.tiles_full);
+  const int64_t start = int64_t(blk) * p.blk_tokens;
   int64_t end = start + p.blk_tokens;
   if (end > p.N) end = p.N;
-  t.unit = t.bh * p.nblk + blk;
-  t.n0 = start + tib * p.tile;
+  t.bh = bh;
+  t.unit = int64_t(bh) * p.nblk + blk;
+  t.n0 = start + int64_t(tib) * p.tile;
   t.n_end = end;
   return t;
 }
 
 __host__ __device__ inline int64_t unit_of_tile(const Plan& p, int64_t g) {
-  int64_t bh = g / p.tiles_per_head;
-  int64_t blk = (g - bh * p.tiles_per_head) / p.tiles_full;
-  if (blk > p.nblk - 1) blk = p.nblk - 1;
-  return bh * p.nblk + blk;
+  const uint32_t gg = static_cast<uint32_t>(g);
+  const uint32_t bh = fdiv(gg, p.fd_tph);
+  uint32_t blk = fdiv(gg - bh * static_cast<uint32_t>(p.tiles_per_head), p.fd_tfull);
+  if (blk > static_cast<uint32_t>(p.nblk - 1)) blk = static_cast<uint32_t>(p.nblk - 1);
+  return int64_t(bh) * p.nblk + blk;
 }
 
 __host__ __device__ inline int64_t cta_start(const Plan& p, int64_t c) { return c * p.total / p.grid; }
@@ -106,12 +142,10 @@ __host__ __device__ inline void unit_tiles(const Plan& p, int64_t u, int64_t* fi
 
 // Grid position of token n, row-major over (T, Hh, W) with t slowest.
 __device__ __forceinline__ void token_pos(const Plan& p, uint32_t n, uint32_t& t, uint32_t& h, uint32_t& w) {
-  uint32_t hw = static_cast<uint32_t>(p.HW);
-  uint32_t W = static_cast<uint32_t>(p.W);
-  t = n / hw;
-  uint32_t rem = n - t * hw;
-  h = rem / W;
-  w = rem - h * W;
+  t = fdiv(n, p.fd_HW);
+  const uint32_t rem = n - t * static_cast<uint32_t>(p.HW);
+  h = fdiv(rem, p.fd_W);
+  w = rem - h * static_cast<uint32_t>(p.W);
 }
 
 // Advance a grid position by `step` tokens.

@@ -1,5 +1,6 @@
 // la_api.cu -- the C ABI declared in include/la.h: argument checks, work planning, TMA
 // descriptors and kernel launches.  Single translation unit: the kernels are included here.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -45,6 +46,8 @@ int validate(const la_problem* p) {
   if (n > double(kMaxTokens)) return LA_ERR_SHAPE;
   if (double(p->B) * double(p->H) > double(lim - 1)) return LA_ERR_SHAPE;
   if (double(p->B) * double(p->H) * n * double(p->d) > 4.0e18) return LA_ERR_SHAPE;
+  // Tile and token indices are 32-bit on the device: at most 2^31 - 1 tiles of >= 32 tokens.
+  if (double(p->B) * double(p->H) * (n / 32.0 + double(p->T) + 1.0) >= double(lim - 1)) return LA_ERR_SHAPE;
   return LA_OK;
 }
 
@@ -59,6 +62,13 @@ int check_ptr(const void* ptr, bool needed) {
 }
 
 // ------------------------------------------------------------------------------- planning
+void set_fastdiv(Plan& p) {
+  p.fd_tph = la::make_fastdiv(static_cast<uint32_t>(p.tiles_per_head > 0 ? p.tiles_per_head : 1));
+  p.fd_tfull = la::make_fastdiv(static_cast<uint32_t>(p.tiles_full > 0 ? p.tiles_full : 1));
+  p.fd_HW = la::make_fastdiv(static_cast<uint32_t>(p.HW > 0 ? p.HW : 1));
+  p.fd_W = la::make_fastdiv(static_cast<uint32_t>(p.W > 0 ? p.W : 1));
+}
+
 Plan build_plan(const la_problem& q, int64_t tile, int64_t grid_cap, int zparts) {
   Plan p;
   std::memset(&p, 0, sizeof p);
@@ -84,6 +94,7 @@ Plan build_plan(const la_problem& q, int64_t tile, int64_t grid_cap, int zparts)
     p.grid = 0;
     p.maxseg = 0;
     p.tiles_full = p.tiles_last = p.tiles_per_head = 0;
+    set_fastdiv(p);
     return p;
   }
   const int64_t full_len = p.blk_tokens < p.N ? p.blk_tokens : p.N;
@@ -93,6 +104,7 @@ Plan build_plan(const la_problem& q, int64_t tile, int64_t grid_cap, int zparts)
   p.tiles_per_head = (p.nblk - 1) * p.tiles_full + p.tiles_last;
   p.total = p.BH * p.tiles_per_head;
   p.grid = static_cast<int32_t>(p.total < grid_cap ? p.total : grid_cap);
+  set_fastdiv(p);
   int64_t maxseg = 0;
   for (int64_t c = 0; c < p.grid; ++c) {
     const int64_t a = la::cta_start(p, c), b = la::cta_start(p, c + 1);
@@ -196,12 +208,12 @@ EncodeTiledFn encode_fn() {
 
 // [BH, N, 128] bf16 viewed as a 3D tensor {128, N, BH}; boxes of 64 channels x 128 tokens,
 // 128-byte swizzle (the canonical UMMA operand layout).
-bool make_tmap(CUtensorMap* m, const void* base, int64_t BH, int64_t N) {
+bool make_tmap(CUtensorMap* m, const void* base, int64_t BH, int64_t N, uint32_t box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {128, cuuint64_t(N), cuuint64_t(BH)};
   cuuint64_t strides[2] = {128 * 2, cuuint64_t(N) * 128 * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -212,6 +224,17 @@ bool make_tmap(CUtensorMap* m, const void* base, int64_t BH, int64_t N) {
 int launched_ok() { return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
 
 // ------------------------------------------------------------------------------- launchers
+// cos/sin table shared by the tensor-core state and apply kernels, one entry per thread.
+int launch_table(const PlanSet& s, const la_problem& q, void* ws, cudaStream_t st, int* nl) {
+  if (!s.tc || s.tab_entries == 0) return LA_OK;
+  float2* tab = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + s.off_tab);
+  const Rope rope = make_rope(q);
+  const int64_t tblocks = (s.tab_entries + la::cmb::THREADS - 1) / la::cmb::THREADS;
+  la::cmb::rope_table_kernel<<<unsigned(tblocks), la::cmb::THREADS, 0, st>>>(s.ps, rope, tab);
+  ++*nl;
+  return launched_ok();
+}
+
 int launch_state(const PlanSet& s, const la_problem& q, const void* K, const void* V, void* ws,
                  cudaStream_t st, int* nl) {
   if (s.ps.total == 0) return LA_OK;
@@ -219,11 +242,13 @@ int launch_state(const PlanSet& s, const la_problem& q, const void* K, const voi
   const Rope rope = make_rope(q);
   if (s.tc) {
     CUtensorMap tk, tv;
-    if (!make_tmap(&tk, K, s.ps.BH, s.ps.N) || !make_tmap(&tv, V, s.ps.BH, s.ps.N)) return LA_ERR_CUDA;
+    if (!make_tmap(&tk, K, s.ps.BH, s.ps.N, la::st::TILE) || !make_tmap(&tv, V, s.ps.BH, s.ps.N, la::st::TILE))
+      return LA_ERR_CUDA;
+    const float2* tab = reinterpret_cast<const float2*>(static_cast<uint8_t*>(ws) + s.off_tab);
     auto kern = standard_bands(q) ? la::st::state_tc_kernel<32, 48> : la::st::state_tc_kernel<-1, -1>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::st::SMEM_BYTES) != cudaSuccess)
       return LA_ERR_CUDA;
-    kern<<<s.ps.grid, la::st::THREADS, la::st::SMEM_BYTES, st>>>(tk, tv, s.ps, rope, partial);
+    kern<<<s.ps.grid, la::st::THREADS, la::st::SMEM_BYTES, st>>>(tk, tv, s.ps, rope, tab, partial);
   } else {
 #define LA_STATE_SIMT(DD, TT)                                                                         \
   la::simt::state_simt_kernel<DD, TT><<<s.ps.grid, la::simt::THREADS, 0, st>>>(                      \
@@ -252,14 +277,10 @@ int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk
   const float* partial = reinterpret_cast<const float*>(w + s.off_partial);
   uint8_t* im = img ? w + s.off_img : nullptr;
   float* zim = img ? reinterpret_cast<float*>(w + s.off_zimg) : nullptr;
-  // The apply's cos/sin table is filled by extra blocks of the same launch.
-  const int64_t tab_n = img ? s.tab_entries : 0;
-  float2* tab = tab_n ? reinterpret_cast<float2*>(w + s.off_tab) : nullptr;
+  (void)q;
   const int64_t cblocks = (threads + la::cmb::THREADS - 1) / la::cmb::THREADS;
-  const int64_t tblocks = (tab_n + la::cmb::THREADS - 1) / la::cmb::THREADS;
-  const Rope rope = make_rope(q);
-  la::cmb::combine_kernel<<<unsigned(cblocks + tblocks), la::cmb::THREADS, 0, st>>>(
-      s.ps, partial, S_blk, z_blk, S_inc, z_inc, im, zim, rope, tab, cblocks);
+  la::cmb::combine_kernel<<<unsigned(cblocks), la::cmb::THREADS, 0, st>>>(s.ps, partial, S_blk, z_blk, S_inc,
+                                                                         z_inc, im, zim);
   ++*nl;
   return launched_ok();
 }
@@ -282,6 +303,15 @@ int launch_apply(const PlanSet& s, const la_problem& q, const void* Q, const voi
     auto kern = standard_bands(q) ? la::ap::apply_tc_kernel<32, 48> : la::ap::apply_tc_kernel<-1, -1>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::ap::SMEM_BYTES) != cudaSuccess)
       return LA_ERR_CUDA;
+    if (la::ap::SPLIT_REGS) {
+      // The math warpgroups grow their register files out of what the launch granted; refuse to
+      // launch unless the kernel really starts with the per-thread count the split assumes.
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != int(la::ap::REGS_LAUNCH) ||
+          int64_t(fa.numRegs) * la::ap::THREADS <
+              128 * (int64_t(la::ap::REGS_CTRL) + int64_t(la::ap::NWG) * la::ap::REGS_MATH))
+        return LA_ERR_CUDA;
+    }
     kern<<<s.pa.grid, la::ap::THREADS, la::ap::SMEM_BYTES, st>>>(
         tq, tg, to, s.pa, rope, w + s.off_img, reinterpret_cast<const float*>(w + s.off_zimg),
         reinterpret_cast<const float2*>(w + s.off_tab), static_cast<__nv_bfloat16*>(O));
@@ -354,6 +384,7 @@ int la_state_reduce(const la_problem* p, const void* K, const void* V, float* S,
   const PlanSet s = make_plans(*p, sm);
   if ((rc = check_ws(s, ws, ws_bytes))) return rc;
   int nl = 0;
+  if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
   if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
   if ((rc = launch_combine(s, *p, ws, S, z, nullptr, nullptr, false, stream, &nl))) return rc;
   g_last_launches = nl;
@@ -447,8 +478,11 @@ static int forward_common(const la_problem* p, const void* Q, const void* K, con
     if (i < nmarks && marks && marks[i]) cudaEventRecord(marks[i], stream);
   };
   mark(0);
+  if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
+  if (nl) mark(nl);
+  const int b0 = nl;
   if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
-  mark(nl);
+  if (nl != b0) mark(nl);
   const int before = nl;
   if ((rc = launch_combine(s, *p, ws, nullptr, nullptr, need_fp32 ? st_S : nullptr, need_fp32 ? st_z : nullptr,
                            s.tc, stream, &nl)))
@@ -515,5 +549,70 @@ int la_device_error(cudaStream_t stream) {
 }
 
 int la_last_launch_count(void) { return g_last_launches; }
+
+// Host-side self-check of the work decomposition: exact fast division, and every tile of a set
+// of problems owned by exactly one CTA with its partial slot in range.  Returns 0 on success.
+int la_selftest_host(void) {
+  // Fast division against exact division.
+  const uint32_t divs[] = {1, 2, 3, 5, 7, 12, 80, 127, 128, 129, 3600, 3601, 65535, 65536, 75600, 1000003,
+                           (1u << 30) + 1, (1u << 31) - 1};
+  uint64_t x = 88172645463325252ull;
+  for (uint32_t d : divs) {
+    const la::FastDiv f = la::make_fastdiv(d);
+    const uint32_t edge[] = {0, 1, d - 1, d, d + 1, 2 * d - 1, (1u << 31) - 1, (1u << 31) - 2};
+    for (uint32_t n : edge)
+      if (n < (1u << 31) && la::fdiv(n, f) != n / d) return 1;
+    for (int k = 0; k < 20000; ++k) {
+      x ^= x << 13; x ^= x >> 7; x ^= x << 17;
+      const uint32_t n = static_cast<uint32_t>(x) & 0x7fffffffu;
+      if (la::fdiv(n, f) != n / d) return 2;
+    }
+  }
+  // Decomposition invariants on assorted problems and SM counts.
+  struct Shape { int64_t B, H, T, Hh, W; int32_t bf; };
+  const Shape shapes[] = {{1, 32, 21, 45, 80, 0}, {1, 32, 81, 45, 80, 3}, {3, 70, 1, 2, 64, 0},
+                          {1, 2, 7, 6, 10, 2}, {2, 1, 3, 5, 30, 10}, {1, 1, 1, 1, 1, 0}, {1, 3, 6, 4, 33, 1}};
+  const int sms[] = {1, 7, 148, 1000};
+  for (const Shape& sh : shapes)
+    for (int sm : sms)
+      for (int64_t tile : {int64_t(32), int64_t(128)}) {
+        la_problem q;
+        std::memset(&q, 0, sizeof q);
+        q.B = sh.B; q.H = sh.H; q.T = sh.T; q.Hh = sh.Hh; q.W = sh.W; q.d = 128; q.dt = 32; q.dh = 48;
+        q.dw = 48; q.rope_base = 10000.0; q.eps = 1e-6f; q.block_frames = sh.bf; q.dtype = LA_BF16;
+        const Plan p = build_plan(q, tile, sm, 1);
+        int64_t covered = 0;
+        for (int64_t c = 0; c < p.grid; ++c) {
+          const int64_t a = la::cta_start(p, c), b = la::cta_start(p, c + 1);
+          if (b <= a) return 3;                       // every CTA owns at least one tile
+          for (int64_t g = a; g < b; ++g) {
+            if (la::cta_of(p, g) != c) return 4;      // ownership is consistent
+            const la::TileInfo ti = la::tile_info(p, g);
+            if (ti.unit - la::unit_of_tile(p, a) >= p.maxseg) return 5;
+            if (ti.n0 < 0 || ti.n0 >= ti.n_end || ti.n_end > p.N) return 6;
+            // the tile starts on its unit's 'tile' grid
+            const int64_t blk = ti.unit % p.nblk;
+            if ((ti.n0 - blk * p.blk_tokens) % p.tile != 0) return 7;
+            ++covered;
+          }
+        }
+        if (covered != p.total) return 8;
+        // Tiles of a unit are contiguous and cover its tokens.
+        for (int64_t u = 0; u < p.BH * p.nblk; ++u) {
+          int64_t first, count;
+          la::unit_tiles(p, u, &first, &count);
+          int64_t tok = 0;
+          for (int64_t g = first; g < first + count; ++g) {
+            const la::TileInfo ti = la::tile_info(p, g);
+            if (ti.unit != u) return 9;
+            tok += std::min<int64_t>(p.tile, ti.n_end - ti.n0);
+          }
+          const int64_t blk = u % p.nblk;
+          const int64_t len = std::min<int64_t>(p.blk_tokens, p.N - blk * p.blk_tokens);
+          if (tok != len) return 10;
+        }
+      }
+  return 0;
+}
 
 }  // extern "C"

@@ -243,6 +243,8 @@ __device__ __forceinline__ void store8(float* S, float* z, int64_t unit, int D, 
 // cos/sin of every (band, pair, position) the tensor-core apply reads, computed in fp64:
 // entry e of band b holds (cos, sin)(x * theta) for pair i = (e - off_b) / extent_b and
 // position x = (e - off_b) % extent_b.
+// Layout [band][pair][position]: the lanes of a warp, which hold consecutive tokens, read
+// consecutive positions of one pair.
 __device__ __forceinline__ void rope_table_entry(const Plan& p, const Rope& r, int64_t e, float2* tab) {
   int64_t i, x;
   int pair;
@@ -258,16 +260,16 @@ __device__ __forceinline__ void rope_table_entry(const Plan& p, const Rope& r, i
   tab[e] = make_float2(static_cast<float>(c), static_cast<float>(s));
 }
 
-// Blocks [0, comb_blocks) combine states; blocks past them (if any) fill the cos/sin table.
+// Builds the cos/sin table of the tensor-core kernels (one thread per entry).
+__global__ void __launch_bounds__(THREADS)
+rope_table_kernel(const Plan p, const __grid_constant__ Rope rope, float2* tab) {
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
+  if (e < rope.tab_entries) rope_table_entry(p, rope, e, tab);
+}
+
 __global__ void __launch_bounds__(THREADS)
 combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, float* z_blk, float* S_inc,
-               float* z_inc, uint8_t* img, float* zimg, const __grid_constant__ Rope rope, float2* tab,
-               int64_t comb_blocks) {
-  if (static_cast<int64_t>(blockIdx.x) >= comb_blocks) {
-    const int64_t e = (static_cast<int64_t>(blockIdx.x) - comb_blocks) * THREADS + threadIdx.x;
-    if (tab && e < rope.tab_entries) rope_table_entry(p, rope, e, tab);
-    return;
-  }
+               float* z_inc, uint8_t* img, float* zimg) {
   const int D = p.d;
   const int groups = (D * D + D) / 8;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;

@@ -221,6 +221,18 @@ __device__ __forceinline__ float4 lds128f(uint32_t saddr) {
 }
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// max(x, 0) on both bf16 halves of a word.
+__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t w) {
+  __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&w);
+  v = __hmax2(v, __float2bfloat162_rn(0.f));
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+// x / 2 on both bf16 halves of a word (exact unless a half underflows to a subnormal).
+__device__ __forceinline__ uint32_t half_bf16x2(uint32_t w) {
+  __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&w);
+  v = __hmul2(v, __float2bfloat162_rn(0.5f));
+  return *reinterpret_cast<uint32_t*>(&v);
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);

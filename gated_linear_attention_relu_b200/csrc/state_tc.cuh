@@ -11,7 +11,8 @@
 //   warp 0       TMA producer: K and V tiles (two 64-channel, 128-row, 128B-swizzled boxes each)
 //   warp 1       MMA issuer: 8 x tcgen05.mma per tile into one of two TMEM accumulators
 //   warps 2-9    transform, two groups of four warps splitting each tile's rows: ReLU + RoPE of
-//                K in place (bf16), z accumulated in registers
+//                K in place (bf16; cos/sin from the fp64-accurate table the prep kernel builds),
+//                z accumulated in registers
 //   warps 10-13  drain: TMEM accumulator -> fp32 partial S in global memory, once per unit
 // The staged K tile is already in the canonical 128B-swizzled MN-major operand layout, so the
 // transform rewrites it in place.
@@ -19,16 +20,27 @@
 #include "common.cuh"
 #include "sm100.cuh"
 
+#ifndef LA_ST_TILE
+#define LA_ST_TILE 128
+#endif
+#ifndef LA_ST_STAGES
+#define LA_ST_STAGES 3
+#endif
+#ifndef LA_ST_TGROUPS
+#define LA_ST_TGROUPS 2
+#endif
+
 namespace la {
 namespace st {
 
-constexpr int TILE = 128;
+constexpr int TILE = LA_ST_TILE;              // tokens per stage (the MMA K extent of one stage)
 constexpr int D = 128;
-constexpr int STAGES = 3;
-constexpr int TGROUPS = 2;                    // transform warpgroups
+constexpr int STAGES = LA_ST_STAGES;
+constexpr int TGROUPS = LA_ST_TGROUPS;        // transform warpgroups, each owning TILE/TGROUPS rows
+constexpr int GROUP_ROWS = TILE / TGROUPS;
 constexpr int THREADS = 32 * (2 + 4 * TGROUPS + 4);
-constexpr uint32_t HALF = 128 * 128;          // one 64-channel box of 128 rows x 128 B
-constexpr uint32_t BUF = 2 * HALF;            // 128 tokens x 128 channels bf16
+constexpr uint32_t HALF = TILE * 128;         // one 64-channel box of TILE rows x 128 B
+constexpr uint32_t BUF = 2 * HALF;            // TILE tokens x 128 channels bf16
 constexpr uint32_t STAGE = 2 * BUF;           // K + V
 constexpr uint32_t OFF_BAR = STAGES * STAGE;  // barriers after the stages
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
@@ -49,11 +61,14 @@ struct Bars {
   int abort_flag;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block too large");
+static_assert(TILE % 16 == 0 && TILE <= 256 && GROUP_ROWS % 8 == 0 && GROUP_ROWS * TGROUPS == TILE, "tile shape");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 template <int DT, int DH>
 __global__ void __launch_bounds__(THREADS, 1)
 state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                const Plan p, const __grid_constant__ Rope rope, float* __restrict__ partial) {
+                const Plan p, const __grid_constant__ Rope rope, const float2* __restrict__ tab,
+                float* __restrict__ partial) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
@@ -156,21 +171,35 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     }
   } else if (warp < DRAIN_WARP0) {
     // ------------------------------------------------------------ transform: ReLU + RoPE of K
-    const int tg = (warp - 2) >> 2;               // transform group: rows 64*tg .. 64*tg+63
-    const int tt = threadIdx.x - 64 - 128 * tg;   // 0..127 within the group
-    const int ck = tt & 15;                       // 8-channel chunk: channels 8ck .. 8ck+7
-    const int rg = tt >> 4;                       // rows 64tg + rg + 8j, j < 8 (row % 8 == rg)
+    // Group tg owns rows GROUP_ROWS*tg .. GROUP_ROWS*(tg+1)-1 of each tile.  Warp k of the group
+    // owns the 8-channel chunks 4k .. 4k+3; each lane walks rows GROUP_ROWS*tg + rg + 8j, so the
+    // 32 lanes of a load touch 8 consecutive tokens and the cos/sin table reads coalesce.
+    const int tg = (warp - 2) >> 2;
+    const int wk = (warp - 2) & 3;
+    const int ck = 4 * wk + (lane & 3);           // channels 8ck .. 8ck+7
+    // Each 8-lane phase of a 16-byte shared access covers rows r and r+4 (r = rg mod 4) and the
+    // 4 chunks: the swizzled positions (chunk ^ row) % 8 are then all distinct (no bank conflict).
+    const int rg = ((lane >> 2) & 1) * 4 + (lane >> 3);  // row % 8
     const uint32_t chunk_off = static_cast<uint32_t>((ck >> 3) * HALF + (((ck & 7) ^ rg) << 4));
-    float th[4];
-    int bd[4];
+    // With the band split a multiple of 8 channels, the 4 pairs of a chunk share one band, so the
+    // position is selected once per row.
+    constexpr bool UNIFORM = DT >= 0 && DH >= 0 && DT % 8 == 0 && DH % 8 == 0;
+    const int bnd0 = band_of<DT, DH>(4 * ck, rope);
+    const int ext0 = bnd0 == 0 ? static_cast<int>(p.T) : (bnd0 == 1 ? static_cast<int>(p.Hh) : static_cast<int>(p.W));
+    int bd[4], tix[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      th[q] = rope.theta[4 * ck + q];
-      bd[q] = band_of<DT, DH>(4 * ck + q, rope);
+      const int pi = 4 * ck + q;
+      bd[q] = band_of<DT, DH>(pi, rope);
+      const int loc = pair_in_band<DT, DH>(pi, rope);
+      tix[q] = bd[q] == 0 ? loc * static_cast<int>(p.T)
+                          : (bd[q] == 1 ? static_cast<int>(rope.tab_off_h) + loc * static_cast<int>(p.Hh)
+                                        : static_cast<int>(rope.tab_off_w) + loc * static_cast<int>(p.W));
     }
     float zacc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
+    const uint32_t N = static_cast<uint32_t>(p.N);
     for (int64_t g = g0; g < g1; ++g) {
       const int64_t i = g - g0;
       const int s = static_cast<int>(i % STAGES);
@@ -178,33 +207,44 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const TileInfo ti = tile_info(p, g);
       const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != ti.unit);
       if (!warp_wait(&bars->full[s], ph, abort_flag)) break;
-      const int row0 = 64 * tg + rg;
+      const int row0 = GROUP_ROWS * tg + rg;
       const uint32_t base = sbase + s * STAGE + chunk_off + static_cast<uint32_t>(row0 * 128);
-      uint32_t n = static_cast<uint32_t>(ti.n0) + row0;
+      const uint32_t n0 = static_cast<uint32_t>(ti.n0) + row0;
       const uint32_t n_end = static_cast<uint32_t>(ti.n_end);
-      uint32_t pt, ph_, pw;
-      token_pos(p, n, pt, ph_, pw);
+      // Branch-free over rows so the unrolled iterations' load chains overlap: rows past the end
+      // of the unit are zeroed with a select, and their (unused) position is clamped in range.
 #pragma unroll 4
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < GROUP_ROWS / 8; ++j) {
         const uint32_t addr = base + static_cast<uint32_t>(j * 8 * 128);
+        const uint32_t n = n0 + 8 * j;
+        const uint32_t keep = n < n_end ? 0xffffffffu : 0u;
         const uint4 raw = lds128(addr);
-        const bool valid = n < n_end;
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t pt, ph_, pw;
+        token_pos(p, n < N ? n : N - 1, pt, ph_, pw);
+        float2 cs[4];
+        if constexpr (UNIFORM) {
+          const float2* tp = tab + tix[0] + (bnd0 == 0 ? pt : (bnd0 == 1 ? ph_ : pw));
+#pragma unroll
+          for (int q = 0; q < 4; ++q) cs[q] = __ldg(tp + q * ext0);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t pos = bd[q] == 0 ? pt : (bd[q] == 1 ? ph_ : pw);
+            cs[q] = __ldg(tab + tix[q] + pos);
+          }
+        }
+        const uint32_t w[4] = {relu_bf16x2(raw.x) & keep, relu_bf16x2(raw.y) & keep,
+                               relu_bf16x2(raw.z) & keep, relu_bf16x2(raw.w) & keep};
         uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float x0 = valid ? fmaxf(bf16lo(w[q]), 0.f) : 0.f;
-          const float x1 = valid ? fmaxf(bf16hi(w[q]), 0.f) : 0.f;
+          const float x0 = bf16lo(w[q]);
+          const float x1 = bf16hi(w[q]);
           zacc[2 * q] += x0;
           zacc[2 * q + 1] += x1;
-          const uint32_t pos = bd[q] == 0 ? pt : (bd[q] == 1 ? ph_ : pw);
-          float sn, cs;
-          __sincosf(static_cast<float>(pos) * th[q], &sn, &cs);
-          o[q] = pack_bf16(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+          o[q] = pack_bf16(x0 * cs[q].x - x1 * cs[q].y, x0 * cs[q].y + x1 * cs[q].x);
         }
         sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
-        n += 8;
-        token_pos_advance(p, 8, pt, ph_, pw);
       }
       fence_proxy_async_smem();
       __syncwarp();

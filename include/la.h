@@ -138,6 +138,12 @@ int la_device_error(cudaStream_t stream);
 /* Number of kernels the last successful entry point on this host thread queued. */
 int la_last_launch_count(void);
 
+/* Host-only self-check of the library's work decomposition (no CUDA call): exact 32-bit
+ * fast division, and for a set of problem shapes every tile owned by exactly one CTA, every
+ * partial-state slot in range, and every unit's tiles covering its tokens.  Returns 0 on
+ * success, a positive code naming the failed check otherwise. */
+int la_selftest_host(void);
+
 #ifdef __cplusplus
 }
 #endif

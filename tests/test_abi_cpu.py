@@ -87,3 +87,8 @@ def test_workspace_sizes_are_consistent():
     assert la.workspace_bytes(bc, sm_count=148) >= 32 * 27 * (32768 + 512)
     assert la.workspace_bytes(la.Problem(B=1, H=1, T=1, Hh=1, W=1, d=40, bands=(8, 16, 16)), 148) == 0
     assert la.workspace_bytes(la.Problem(B=0, H=4, T=2, Hh=2, W=2), sm_count=148) >= 0
+
+
+def test_host_selftest_of_work_decomposition():
+    # Exact fast division and tile/segment bookkeeping, checked on the host by the library itself.
+    assert la.load().la_selftest_host() == 0

@@ -185,9 +185,11 @@ def test_launch_counts_and_device_error_word():
     Q, K, V, G = wl.generate(w, "cuda")
     p = _problem(w)
     la.forward_bidir(p, Q, K, V, G)
-    assert la.last_launch_count() == 3  # state, combine, apply
+    assert la.last_launch_count() == 4  # cos/sin table, state, combine, apply
     la.state_reduce(p, K, V)
-    assert la.last_launch_count() == 2  # state, combine
+    assert la.last_launch_count() == 3  # cos/sin table, state, combine
+    la.forward_bidir(la.Problem.from_workload(w, force_simt=True), Q, K, V, G)
+    assert la.last_launch_count() == 3  # state, combine, apply (CUDA cores)
     assert la.device_error() == 0
 
 
