@@ -25,7 +25,7 @@ STATUS = {
 EXPORTS = [
     "la_workspace_bytes", "la_workspace_bytes_for", "la_state_reduce", "la_state_scan", "la_apply",
     "la_forward_bidir", "la_forward_blockcausal", "la_status_string", "la_device_error",
-    "la_last_launch_count", "la_forward_marked", "la_selftest_host",
+    "la_last_launch_count", "la_forward_marked", "la_selftest_host", "la_forward_bidir_static",
 ]
 
 
@@ -76,6 +76,7 @@ def load(path: Optional[str] = None):
         "la_device_error": (ctypes.c_int, [vp]),
         "la_last_launch_count": (ctypes.c_int, []),
         "la_selftest_host": (ctypes.c_int, []),
+        "la_forward_bidir_static": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp]),
         "la_forward_marked": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                              ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
     }
@@ -224,6 +225,16 @@ def forward_bidir(p: Problem, Q, K, V, G, O=None, ws=None, stream=None):
     cp = p.c()
     _check(lib.la_forward_bidir(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(O), _ptr(ws),
                                 nbytes, _stream(stream)), "la_forward_bidir")
+    return O
+
+
+def forward_bidir_static(p: Problem, Q, K, V, G, O, stream=None):
+    """la_forward_bidir without a workspace: the library's fixed device scratch is used instead
+    (for callers that cannot allocate device memory).  ``O`` must be given; nothing is allocated."""
+    lib = load()
+    cp = p.c()
+    _check(lib.la_forward_bidir_static(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(O),
+                                       _stream(stream)), "la_forward_bidir_static")
     return O
 
 

@@ -550,6 +550,47 @@ int la_device_error(cudaStream_t stream) {
 
 int la_last_launch_count(void) { return g_last_launches; }
 
+}  // extern "C"
+
+// Fixed scratch for callers that cannot allocate (la_forward_bidir_static).  In host code the
+// symbol is only a handle: its device address is looked up per device with
+// cudaGetSymbolAddress, with that device current, and cached.
+static __device__ __align__(256) uint8_t g_la_static_ws[LA_STATIC_WORKSPACE_BYTES];
+
+namespace {
+std::mutex g_static_mu;
+constexpr int kMaxDevices = 256;
+void* g_static_ptr[kMaxDevices] = {};
+
+int static_workspace(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return LA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_la_static_ws) != cudaSuccess || !ptr) return LA_ERR_CUDA;
+    g_static_ptr[dev] = ptr;
+  }
+  *out = g_static_ptr[dev];
+  return LA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int la_forward_bidir_static(const la_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                            void* O, cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  if (p->block_frames != 0) return LA_ERR_SHAPE;
+  int dev = 0, sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LA_ERR_CUDA;
+  if ((rc = current_sm_count(&sm))) return rc;
+  if (make_plans(*p, sm).total > LA_STATIC_WORKSPACE_BYTES) return LA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if ((rc = static_workspace(dev, &ws))) return rc;
+  return forward_common(p, Q, K, V, G, O, nullptr, nullptr, ws, LA_STATIC_WORKSPACE_BYTES, stream);
+}
+
 // Host-side self-check of the work decomposition: exact fast division, and every tile of a set
 // of problems owned by exactly one CTA with its partial slot in range.  Returns 0 on success.
 int la_selftest_host(void) {

@@ -127,6 +127,28 @@ int la_forward_marked(const la_problem* p, const void* Q, const void* K, const v
                       const void* G, void* O, float* S_incl, float* z_incl, void* workspace,
                       size_t workspace_bytes, cudaStream_t stream, cudaEvent_t* marks, int nmarks);
 
+/* Bytes of the library's fixed device scratch used by la_forward_bidir_static(). */
+#define LA_STATIC_WORKSPACE_BYTES (32u << 20)
+
+/* la_forward_bidir() for callers that must not allocate device memory themselves: for example
+ * a plugin whose host framework owns every device allocation and forbids new ones while it
+ * executes, or a latency-critical service that fixes all of its memory at start-up.  This
+ * entry point takes no workspace and allocates nothing; it uses a scratch array of
+ * LA_STATIC_WORKSPACE_BYTES that is part of the library's device code.  (The pages describe no
+ * such call; it exists only for those callers.)
+ *  - The caller still passes Q, K, V, G and O (same rules as la_forward_bidir).
+ *  - The scratch lives in every GPU that loads the library, until the process exits.
+ *  - The first call on a device looks up the scratch's device address (a host-side query that
+ *    allocates nothing); make that first call before any stream capture.
+ *  - Problems whose workspace (la_workspace_bytes) exceeds LA_STATIC_WORKSPACE_BYTES are
+ *    rejected with LA_ERR_WORKSPACE before anything is launched.  B = 1, H = 32 at the
+ *    720p/5s and 720p/60s latent grids fits.
+ *  - All calls, on any stream, share the one scratch array, which keeps whatever the last call
+ *    left in it.  Nothing in it needs clearing (each call writes every byte it later reads),
+ *    but calls whose GPU work overlaps in time race on it: serialise them. */
+int la_forward_bidir_static(const la_problem* p, const void* Q, const void* K, const void* V,
+                            const void* G, void* O, cudaStream_t stream);
+
 /* Static description of a status code. */
 const char* la_status_string(int status);
 
