@@ -108,8 +108,6 @@ def test_rope_norm_identity_relative_composition():
 # --------------------------------------------------------------------------
 
 def test_linear_form_equals_brute_form_on_tiny_workload():
-    import torch
-
     w = wl.WORKLOADS["tiny_f32"]
     Q, K, V, G = (t.double().numpy() for t in wl.generate(w, "cpu"))
     O = orc.forward_bidir(Q, K, V, G, (w.T, w.Hh, w.W), w.bands, w.rope_base, w.eps)
@@ -117,7 +115,6 @@ def test_linear_form_equals_brute_form_on_tiny_workload():
     for h in range(w.H):
         ob = orc.forward_brute(Q[0, h], K[0, h], V[0, h], G[0, h], pos, w.bands, w.rope_base, w.eps)
         assert np.max(np.abs(ob - O[0, h])) <= 1e-12 * np.max(np.abs(ob))
-    del torch
 
 
 @pytest.mark.parametrize("grid,d,bands", [((3, 5, 7), 16, (4, 6, 6)), ((4, 4, 32), 32, (8, 12, 12)),
