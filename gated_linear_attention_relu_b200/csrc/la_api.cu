@@ -309,7 +309,7 @@ int launch_apply(const PlanSet& s, const la_problem& q, const void* Q, const voi
       cudaFuncAttributes fa;
       if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != int(la::ap::REGS_LAUNCH) ||
           int64_t(fa.numRegs) * la::ap::THREADS <
-              128 * (int64_t(la::ap::REGS_CTRL) + int64_t(la::ap::NWG) * la::ap::REGS_MATH))
+              128 * (int64_t(la::ap::REGS_CTRL) + int64_t(la::ap::MATH_WGS) * la::ap::REGS_MATH))
         return LA_ERR_CUDA;
     }
     kern<<<s.pa.grid, la::ap::THREADS, la::ap::SMEM_BYTES, st>>>(
