@@ -8,8 +8,7 @@
 // to tensor memory (thread n owns token n and TMEM lane n), so a staged Q tile is released as
 // soon as its rows are in registers; S is the unit's state as a bf16 operand (N-major) in shared
 // memory.  The denominator, the divide and the gate run on the CUDA cores.  The rotation reads
-// cos/sin from a per-band table (fp64-accurate, built by the prep kernel), indexed
-// [pair][position] so the 32 rows of a warp read consecutive entries.
+// cos/sin from per-band tables (fp64-accurate, built by the prep kernel).
 //
 // Warps (one CTA per SM, persistent over a contiguous range of tiles):
 //   warpgroup 0   warp 0: TMA producer of Q tiles (and the state operand once per unit)
@@ -68,7 +67,7 @@ constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/tru
 // 65536 / THREADS); the control warpgroup shrinks to REGS_CTRL and the math groups grow to
 // REGS_MATH, never asking for more than the launch granted.
 constexpr uint32_t REGS_LAUNCH = (65536 / THREADS) / 8 * 8;
-constexpr uint32_t REGS_CTRL = 56;
+constexpr uint32_t REGS_CTRL = 24;  // the single-lane control loops need few registers
 constexpr uint32_t REGS_MATH_FIT = ((THREADS * REGS_LAUNCH - 128 * REGS_CTRL) / (128 * MATH_WGS)) / 8 * 8;
 constexpr uint32_t REGS_MATH = REGS_MATH_FIT > 232 ? 232 : REGS_MATH_FIT;
 constexpr bool SPLIT_REGS = true;
@@ -109,35 +108,63 @@ __device__ __forceinline__ void regs_inc() {
 }
 
 // In place over half a row held in registers (channels [64 HF, 64 HF + 64) as 32 bf16 pairs,
-// already ReLU'd): a <- RoPE(a).  Returns the half's share of ReLU(q) . z (un-rotated).  Pair i of
-// band b at grid coordinate x reads the table entry at (band offset) + i_in_band * extent_b + x;
-// it, ih, iw carry the band offsets already.
+// already ReLU'd): a <- RoPE(a).  Returns the half's share of ReLU(q) . z (un-rotated).
+// (pt, ph, pw) is the token's grid position.
+//   Band split fixed at compile time: `tab2` holds two consecutive pairs of a band per 16-byte
+//   entry, t and h bands position-major and the w band [pair / 2][x], so a half row takes 16
+//   vector loads, most of them at constant offsets from one per-band base.
+//   Run-time split: pair i of band b at coordinate x reads `tab` at (band offset) +
+//   i_in_band * extent_b + x.
 template <int DT, int DH, int HF>
 __device__ __forceinline__ float transform_half(uint32_t (&a)[32], const float* __restrict__ zg,
-                                                const float2* __restrict__ tab, const Rope& rope, int it, int ih,
-                                                int iw, int ext_t, int ext_h, int ext_w) {
-  float den4[4] = {0.f, 0.f, 0.f, 0.f};
+                                                const float2* __restrict__ tab, const float4* __restrict__ tab2,
+                                                const Rope& rope, int pt, int ph, int pw, int ext_t, int ext_h,
+                                                int ext_w) {
+  uint64_t den2[4] = {0, 0, 0, 0};  // packed fp32 pairs: (even, odd) channel partial sums
+  if constexpr (DT >= 0 && DH >= 0) {
+    constexpr int DW = 128 - DT - DH;
+    static_assert(DT % 4 == 0 && DH % 4 == 0 && DW % 4 == 0, "bands of whole 16-byte entries");
+    const float4* bt = tab2 + pt * (DT / 4);
+    const float4* bh = tab2 + rope.tab_off_h / 2 + ph * (DH / 4);
+    const float4* bw = tab2 + rope.tab_off_w / 2 + pw;
 #pragma unroll
-  for (int c8 = 0; c8 < 8; ++c8) {
-    const float4 za = __ldg(reinterpret_cast<const float4*>(zg + c8 * 8));
-    const float4 zc = __ldg(reinterpret_cast<const float4*>(zg + c8 * 8 + 4));
-    const float zz[8] = {za.x, za.y, za.z, za.w, zc.x, zc.y, zc.z, zc.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j = 4 * c8 + q;
-      const int pi = 32 * HF + j;
+    for (int j = 0; j < 16; ++j) {
+      const int pi = 32 * HF + 2 * j;  // pairs pi, pi + 1 (same band: band edges are even)
       const int bnd = band_of<DT, DH>(pi, rope);
-      const int loc = pair_in_band<DT, DH>(pi, rope);
-      const int idx = bnd == 0 ? it + loc * ext_t : (bnd == 1 ? ih + loc * ext_h : iw + loc * ext_w);
-      const float2 cs = __ldg(tab + idx);
-      const float x0 = bf16lo(a[j]);
-      const float x1 = bf16hi(a[j]);
-      den4[q] = fmaf(x0, zz[2 * q], den4[q]);
-      den4[q] = fmaf(x1, zz[2 * q + 1], den4[q]);
-      a[j] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+      const int e = pair_in_band<DT, DH>(pi, rope) / 2;
+      const float4 cs = __ldg(bnd == 0 ? bt + e : (bnd == 1 ? bh + e : bw + e * ext_w));
+      const ulonglong2 z4 = __ldg(reinterpret_cast<const ulonglong2*>(zg + 4 * j));
+      const float x0 = bf16lo(a[2 * j]), x1 = bf16hi(a[2 * j]);
+      const float y0 = bf16lo(a[2 * j + 1]), y1 = bf16hi(a[2 * j + 1]);
+      den2[(2 * j) & 3] = fma2(pk(x0, x1), z4.x, den2[(2 * j) & 3]);
+      den2[(2 * j + 1) & 3] = fma2(pk(y0, y1), z4.y, den2[(2 * j + 1) & 3]);
+      a[2 * j] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+      a[2 * j + 1] = pack_bf16(y0 * cs.z - y1 * cs.w, y0 * cs.w + y1 * cs.z);
+    }
+  } else {
+    const int it = pt, ih = static_cast<int>(rope.tab_off_h) + ph, iw = static_cast<int>(rope.tab_off_w) + pw;
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+      const ulonglong2 za = __ldg(reinterpret_cast<const ulonglong2*>(zg + c8 * 8));
+      const ulonglong2 zc = __ldg(reinterpret_cast<const ulonglong2*>(zg + c8 * 8 + 4));
+      const uint64_t zz[4] = {za.x, za.y, zc.x, zc.y};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = 4 * c8 + q;
+        const int pi = 32 * HF + j;
+        const int bnd = band_of<DT, DH>(pi, rope);
+        const int loc = pair_in_band<DT, DH>(pi, rope);
+        const int idx = bnd == 0 ? it + loc * ext_t : (bnd == 1 ? ih + loc * ext_h : iw + loc * ext_w);
+        const float2 cs = __ldg(tab + idx);
+        const float x0 = bf16lo(a[j]);
+        const float x1 = bf16hi(a[j]);
+        den2[q] = fma2(pk(x0, x1), zz[q], den2[q]);
+        a[j] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+      }
     }
   }
-  return (den4[0] + den4[1]) + (den4[2] + den4[3]);
+  const float2 d0 = upk(den2[0]), d1 = upk(den2[1]), d2 = upk(den2[2]), d3 = upk(den2[3]);
+  return ((d0.x + d0.y) + (d1.x + d1.y)) + ((d2.x + d2.y) + (d3.x + d3.y));
 }
 
 template <int DT, int DH>
@@ -145,7 +172,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
                 const __grid_constant__ CUtensorMap tmO, const Plan p, const __grid_constant__ Rope rope,
                 const uint8_t* __restrict__ simg, const float* __restrict__ zimg,
-                const float2* __restrict__ tab, __nv_bfloat16* __restrict__ O) {
+                const float2* __restrict__ tab, const float4* __restrict__ tab2, __nv_bfloat16* __restrict__ O) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
@@ -345,10 +372,10 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // Rows past the end of the head keep position 0 (their output is dropped).
         if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph, pw);
         const float* zg = zimg + ti.unit * D + 64 * hf;
-        const int it = static_cast<int>(pt), ih = static_cast<int>(rope.tab_off_h + ph);
-        const int iw = static_cast<int>(rope.tab_off_w + pw);
-        const float dpart = hf == 0 ? transform_half<DT, DH, 0>(a, zg, tab, rope, it, ih, iw, ext_t, ext_h, ext_w)
-                                    : transform_half<DT, DH, 1>(a, zg, tab, rope, it, ih, iw, ext_t, ext_h, ext_w);
+        const int ipt = static_cast<int>(pt), iph = static_cast<int>(ph), ipw = static_cast<int>(pw);
+        const float dpart =
+            hf == 0 ? transform_half<DT, DH, 0>(a, zg, tab, tab2, rope, ipt, iph, ipw, ext_t, ext_h, ext_w)
+                    : transform_half<DT, DH, 1>(a, zg, tab, tab2, rope, ipt, iph, ipw, ext_t, ext_h, ext_w);
         // Swap partial denominators with the warp holding the other half of these rows (two
         // slots: a slot is rewritten only after the partner's next arrival, which follows its read).
         const uint32_t t_den = t_grp + DEN_COL + 2u * static_cast<uint32_t>(k & 1);
@@ -396,6 +423,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const bool valid = static_cast<int64_t>(n) < ti.n_end;
         const uint32_t grow = sbase + OFF_G + gs * BUF + row_off;
         __nv_bfloat16* orow = O + (ti.bh * p.N + static_cast<int64_t>(n)) * D + 64 * hf;
+        const uint64_t hh = pk(hinv_prev, hinv_prev);
         // The G row is read and overwritten in place, four chunks at a time: the loads of a batch
         // are all issued before its first store, so their latency is paid once per batch.
 #pragma unroll
@@ -413,11 +441,10 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             uint32_t ov[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const float h0 = __uint_as_float(r[c8 * 8 + 2 * q]) * hinv_prev;
-              const float h1 = __uint_as_float(r[c8 * 8 + 2 * q + 1]) * hinv_prev;
-              const float t0 = tanh_approx(bf16lo(gw[q]));
-              const float t1 = tanh_approx(bf16hi(gw[q]));
-              ov[q] = pack_bf16(fmaf(h0, t0, h0), fmaf(h1, t1, h1));
+              const uint64_t h = mul2(pk(__uint_as_float(r[c8 * 8 + 2 * q]), __uint_as_float(r[c8 * 8 + 2 * q + 1])), hh);
+              const uint64_t t = pk(tanh_approx(bf16lo(gw[q])), tanh_approx(bf16hi(gw[q])));
+              const float2 o2 = upk(fma2(h, t, h));
+              ov[q] = pack_bf16(o2.x, o2.y);
             }
             const uint4 o4 = make_uint4(ov[0], ov[1], ov[2], ov[3]);
             if (tma_out) {

@@ -115,12 +115,16 @@ Plan build_plan(const la_problem& q, int64_t tile, int64_t grid_cap, int zparts)
   return p;
 }
 
+// The band split of the production head (d = 128: t/h/w = 32/48/48) gets kernels with the split
+// fixed at compile time; any other split uses the run-time variant.
+bool standard_bands(const la_problem& q) { return q.d == 128 && q.dt == 32 && q.dh == 48 && q.dw == 48; }
+
 struct PlanSet {
   bool tc;            // tensor-core kernels (bf16, d = 128)
   Plan ps;            // state reduction
   Plan pa;            // apply
   int64_t units;      // B*H*nblk
-  size_t off_partial, off_states, off_img, off_zimg, off_tab, total;
+  size_t off_partial, off_states, off_img, off_zimg, off_tab, off_tab2, total;
   int64_t tab_entries;
 };
 
@@ -151,6 +155,8 @@ PlanSet make_plans(const la_problem& q, int sm_count) {
   s.tab_entries = (s.tc && s.pa.total > 0) ? (q.dt / 2) * q.T + (q.dh / 2) * q.Hh + (q.dw / 2) * q.W : 0;
   s.off_tab = off;
   off = align256(off + size_t(s.tab_entries) * 8);
+  s.off_tab2 = off;  // the same entries in the apply kernel's layout (standard band split only)
+  off = align256(off + (standard_bands(q) ? size_t(s.tab_entries) * 8 : 0));
   s.total = off;
   return s;
 }
@@ -177,9 +183,6 @@ Rope make_rope(const la_problem& q) {
   return r;
 }
 
-// The band split of the production head (d = 128: t/h/w = 32/48/48) gets kernels with the split
-// fixed at compile time; any other split uses the run-time variant.
-bool standard_bands(const la_problem& q) { return q.d == 128 && q.dt == 32 && q.dh == 48 && q.dw == 48; }
 
 // ------------------------------------------------------------------------------- CUDA helpers
 int current_sm_count(int* sm) {
@@ -230,7 +233,8 @@ int launch_table(const PlanSet& s, const la_problem& q, void* ws, cudaStream_t s
   float2* tab = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + s.off_tab);
   const Rope rope = make_rope(q);
   const int64_t tblocks = (s.tab_entries + la::cmb::THREADS - 1) / la::cmb::THREADS;
-  la::cmb::rope_table_kernel<<<unsigned(tblocks), la::cmb::THREADS, 0, st>>>(s.ps, rope, tab);
+  float2* tab2 = standard_bands(q) ? reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + s.off_tab2) : nullptr;
+  la::cmb::rope_table_kernel<<<unsigned(tblocks), la::cmb::THREADS, 0, st>>>(s.ps, rope, tab, tab2);
   ++*nl;
   return launched_ok();
 }
@@ -314,7 +318,8 @@ int launch_apply(const PlanSet& s, const la_problem& q, const void* Q, const voi
     }
     kern<<<s.pa.grid, la::ap::THREADS, la::ap::SMEM_BYTES, st>>>(
         tq, tg, to, s.pa, rope, w + s.off_img, reinterpret_cast<const float*>(w + s.off_zimg),
-        reinterpret_cast<const float2*>(w + s.off_tab), static_cast<__nv_bfloat16*>(O));
+        reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2),
+        static_cast<__nv_bfloat16*>(O));
   } else {
     const size_t smem = apply_simt_smem(q.d);
 #define LA_APPLY_SIMT(DD, TT)                                                                              \
@@ -439,7 +444,8 @@ int la_apply(const la_problem* p, const void* Q, const void* G, const float* S, 
     const Rope rope = make_rope(*p);
     la::cmb::pack_kernel<<<unsigned(pblocks + tblocks), la::cmb::THREADS, 0, stream>>>(
         s.units, 128, S, z, w + s.off_img, reinterpret_cast<float*>(w + s.off_zimg), s.pa, rope,
-        reinterpret_cast<float2*>(w + s.off_tab), pblocks);
+        reinterpret_cast<float2*>(w + s.off_tab),
+        standard_bands(*p) ? reinterpret_cast<float2*>(w + s.off_tab2) : nullptr, pblocks);
     ++nl;
     if ((rc = launched_ok())) return rc;
   }

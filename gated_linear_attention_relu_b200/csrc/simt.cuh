@@ -245,26 +245,38 @@ __device__ __forceinline__ void store8(float* S, float* z, int64_t unit, int D, 
 // position x = (e - off_b) % extent_b.
 // Layout [band][pair][position]: the lanes of a warp, which hold consecutive tokens, read
 // consecutive positions of one pair.
-__device__ __forceinline__ void rope_table_entry(const Plan& p, const Rope& r, int64_t e, float2* tab) {
+__device__ __forceinline__ void rope_table_entry(const Plan& p, const Rope& r, int64_t e, float2* tab,
+                                                 float2* tab2) {
   int64_t i, x;
-  int pair;
+  int pair, band;
   if (e < r.tab_off_h) {
-    i = e / p.T; x = e - i * p.T; pair = static_cast<int>(i);
+    i = e / p.T; x = e - i * p.T; pair = static_cast<int>(i); band = 0;
   } else if (e < r.tab_off_w) {
-    i = (e - r.tab_off_h) / p.Hh; x = (e - r.tab_off_h) - i * p.Hh; pair = r.dt / 2 + static_cast<int>(i);
+    i = (e - r.tab_off_h) / p.Hh; x = (e - r.tab_off_h) - i * p.Hh; pair = r.dt / 2 + static_cast<int>(i); band = 1;
   } else {
     i = (e - r.tab_off_w) / p.W; x = (e - r.tab_off_w) - i * p.W; pair = (r.dt + r.dh) / 2 + static_cast<int>(i);
+    band = 2;
   }
   double s, c;
   sincos(static_cast<double>(x) * r.theta_d[pair], &s, &c);
-  tab[e] = make_float2(static_cast<float>(c), static_cast<float>(s));
+  const float2 v = make_float2(static_cast<float>(c), static_cast<float>(s));
+  tab[e] = v;
+  if (tab2) {
+    // Second layout (even pair counts per band only): two consecutive pairs of a band per
+    // 16-byte entry; t and h bands position-major ([x][pair]), w band [pair / 2][x].
+    int64_t e2;
+    if (band == 0) e2 = x * (r.dt / 2) + i;
+    else if (band == 1) e2 = r.tab_off_h + x * (r.dh / 2) + i;
+    else e2 = r.tab_off_w + ((i >> 1) * p.W + x) * 2 + (i & 1);
+    tab2[e2] = v;
+  }
 }
 
 // Builds the cos/sin table of the tensor-core kernels (one thread per entry).
 __global__ void __launch_bounds__(THREADS)
-rope_table_kernel(const Plan p, const __grid_constant__ Rope rope, float2* tab) {
+rope_table_kernel(const Plan p, const __grid_constant__ Rope rope, float2* tab, float2* tab2) {
   const int64_t e = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
-  if (e < rope.tab_entries) rope_table_entry(p, rope, e, tab);
+  if (e < rope.tab_entries) rope_table_entry(p, rope, e, tab, tab2);
 }
 
 __global__ void __launch_bounds__(THREADS)
@@ -341,10 +353,11 @@ scan_kernel(int64_t BH, int64_t nblk, int D, float* S, float* z) {
 // bf16 operand image of given fp32 states (for the tensor-core apply called on its own).
 __global__ void __launch_bounds__(THREADS)
 pack_kernel(int64_t units, int D, const float* __restrict__ S, const float* __restrict__ z, uint8_t* img,
-            float* zimg, const Plan p, const __grid_constant__ Rope rope, float2* tab, int64_t pack_blocks) {
+            float* zimg, const Plan p, const __grid_constant__ Rope rope, float2* tab, float2* tab2,
+            int64_t pack_blocks) {
   if (static_cast<int64_t>(blockIdx.x) >= pack_blocks) {
     const int64_t e = (static_cast<int64_t>(blockIdx.x) - pack_blocks) * THREADS + threadIdx.x;
-    if (tab && e < rope.tab_entries) rope_table_entry(p, rope, e, tab);
+    if (tab && e < rope.tab_entries) rope_table_entry(p, rope, e, tab, tab2);
     return;
   }
   const int groups = (D * D + D) / 8;
