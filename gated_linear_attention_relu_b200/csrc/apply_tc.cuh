@@ -224,11 +224,15 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // The state image, z and the cos/sin tables come from the kernels before this one: the threads
+  // that read them wait for those kernels; the G loads start at once.
+  pdl_trigger();
 
   if (warp < 4) {
     regs_dec<REGS_CTRL>();
     if (warp == 0 && lane == 0) {
       // ---------------------------------------------------------- TMA producer: state, Q
+      pdl_wait();
       int64_t issued_q = 0, issued_s = 0;
       int64_t prev_unit = -1;
       for (int64_t g = g0; g < g1; ++g) {
@@ -341,6 +345,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t t_a = t_grp + A_COL + 32u * hf;
     const int ext_t = static_cast<int>(p.T), ext_h = static_cast<int>(p.Hh), ext_w = static_cast<int>(p.W);
     uint64_t* denx = &bars->denx[m][quarter];
+    pdl_wait();
     int64_t g_prev = -1;
     uint32_t k_prev = 0;
     float hinv_prev = 0.f;

@@ -226,6 +226,27 @@ bool make_tmap(CUtensorMap* m, const void* base, int64_t BH, int64_t N, uint32_t
 
 int launched_ok() { return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
 
+// Launches `kern`; with `pdl` it may start while the previous kernel in the stream is still
+// running (programmatic stream serialization).  Only kernels whose predecessor in the stream is
+// one of this library's own kernels get `pdl`, and each of them calls pdl_wait() before reading
+// anything produced before it; what they read earlier (K, V, G) was produced before the first
+// kernel of the call, which is launched normally.
+template <typename... KArgs, typename... Args>
+int launch_k(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st, bool pdl,
+             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------------------- launchers
 // cos/sin table shared by the tensor-core state and apply kernels, one entry per thread.
 int launch_table(const PlanSet& s, const la_problem& q, void* ws, cudaStream_t st, int* nl) {
@@ -252,7 +273,12 @@ int launch_state(const PlanSet& s, const la_problem& q, const void* K, const voi
     auto kern = standard_bands(q) ? la::st::state_tc_kernel<32, 48> : la::st::state_tc_kernel<-1, -1>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::st::SMEM_BYTES) != cudaSuccess)
       return LA_ERR_CUDA;
-    kern<<<s.ps.grid, la::st::THREADS, la::st::SMEM_BYTES, st>>>(tk, tv, s.ps, rope, tab, partial);
+    const float4* tab2 =
+        standard_bands(q) ? reinterpret_cast<const float4*>(static_cast<uint8_t*>(ws) + s.off_tab2) : nullptr;
+    // The cos/sin table kernel runs just before (same condition: tensor-core path, tokens > 0).
+    if (launch_k(kern, unsigned(s.ps.grid), la::st::THREADS, la::st::SMEM_BYTES, st, true, tk, tv, s.ps, rope,
+                 tab, tab2, partial))
+      return LA_ERR_CUDA;
   } else {
 #define LA_STATE_SIMT(DD, TT)                                                                         \
   la::simt::state_simt_kernel<DD, TT><<<s.ps.grid, la::simt::THREADS, 0, st>>>(                      \
@@ -283,8 +309,11 @@ int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk
   float* zim = img ? reinterpret_cast<float*>(w + s.off_zimg) : nullptr;
   (void)q;
   const int64_t cblocks = (threads + la::cmb::THREADS - 1) / la::cmb::THREADS;
-  la::cmb::combine_kernel<<<unsigned(cblocks), la::cmb::THREADS, 0, st>>>(s.ps, partial, S_blk, z_blk, S_inc,
-                                                                         z_inc, im, zim);
+  // After the tensor-core state kernel (if it ran) the combine kernel may launch early; it waits
+  // for that kernel before its first read.
+  if (launch_k(la::cmb::combine_kernel, unsigned(cblocks), la::cmb::THREADS, 0, st, s.tc && s.ps.total > 0,
+               s.ps, partial, S_blk, z_blk, S_inc, z_inc, im, zim))
+    return LA_ERR_CUDA;
   ++*nl;
   return launched_ok();
 }
@@ -316,10 +345,12 @@ int launch_apply(const PlanSet& s, const la_problem& q, const void* Q, const voi
               128 * (int64_t(la::ap::REGS_CTRL) + int64_t(la::ap::MATH_WGS) * la::ap::REGS_MATH))
         return LA_ERR_CUDA;
     }
-    kern<<<s.pa.grid, la::ap::THREADS, la::ap::SMEM_BYTES, st>>>(
-        tq, tg, to, s.pa, rope, w + s.off_img, reinterpret_cast<const float*>(w + s.off_zimg),
-        reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2),
-        static_cast<__nv_bfloat16*>(O));
+    // Called right after the combine kernel (forward) or the pack kernel (apply on its own).
+    if (launch_k(kern, unsigned(s.pa.grid), la::ap::THREADS, la::ap::SMEM_BYTES, st, true, tq, tg, to, s.pa, rope,
+                 static_cast<const uint8_t*>(w + s.off_img), reinterpret_cast<const float*>(w + s.off_zimg),
+                 reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2),
+                 static_cast<__nv_bfloat16*>(O)))
+      return LA_ERR_CUDA;
   } else {
     const size_t smem = apply_simt_smem(q.d);
 #define LA_APPLY_SIMT(DD, TT)                                                                              \

@@ -275,6 +275,7 @@ __device__ __forceinline__ void rope_table_entry(const Plan& p, const Rope& r, i
 // Builds the cos/sin table of the tensor-core kernels (one thread per entry).
 __global__ void __launch_bounds__(THREADS)
 rope_table_kernel(const Plan p, const __grid_constant__ Rope rope, float2* tab, float2* tab2) {
+  pdl_trigger();
   const int64_t e = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
   if (e < rope.tab_entries) rope_table_entry(p, rope, e, tab, tab2);
 }
@@ -282,6 +283,9 @@ rope_table_kernel(const Plan p, const __grid_constant__ Rope rope, float2* tab, 
 __global__ void __launch_bounds__(THREADS)
 combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, float* z_blk, float* S_inc,
                float* z_inc, uint8_t* img, float* zimg) {
+  // Every thread reads the state kernel's partial sums: wait for that kernel first.
+  pdl_trigger();
+  pdl_wait();
   const int D = p.d;
   const int groups = (D * D + D) / 8;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
@@ -301,6 +305,8 @@ combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, fl
     if (p.total > 0) unit_tiles(p, u, &first, &count);
     if (count > 0) {
       const int64_t c0 = cta_of(p, first), c1 = cta_of(p, first + count - 1);
+      // (unrolled so that the loads of several slots are in flight together)
+#pragma unroll 4
       for (int64_t cc = c0; cc <= c1; ++cc) {
         const int64_t k = u - unit_of_tile(p, cta_start(p, cc));
         const float* src = partial + (cc * p.maxseg + k) * slot_floats;

@@ -92,6 +92,14 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   }
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the kernel before it
+// in the stream is still running.  pdl_wait() returns once that kernel has completed and its
+// memory is visible; a thread must call it before reading anything that kernel wrote.
+// pdl_trigger() lets the next kernel start launching.  Both are no-ops without such a launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- proxy fences, named barriers
 // Makes this thread's generic-proxy shared-memory writes visible to the async proxy (TMA, tcgen05).
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -279,6 +287,11 @@ __device__ __forceinline__ float2 upk(uint64_t r) {
 __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
