@@ -230,6 +230,8 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     uint64_t zacc[4] = {0, 0, 0, 0};  // packed fp32 pairs: z of channels (8ck + 2q, 8ck + 2q + 1)
     pdl_wait();
     const uint32_t N = static_cast<uint32_t>(p.N);
+    const uint32_t Wd = static_cast<uint32_t>(p.W), Hd = static_cast<uint32_t>(p.Hh);
+    const bool step_ok = Wd >= 8;  // incremental positions need at most one wrap per 8 rows
     for (int64_t g = g0; g < g1; ++g) {
       const int64_t i = g - g0;
       const int s = static_cast<int>(i % KST);
@@ -241,16 +243,10 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const uint32_t base = sbase + OFF_K + s * BUF + chunk_off + static_cast<uint32_t>(row0 * 128);
       const uint32_t n0 = static_cast<uint32_t>(ti.n0) + row0;
       const uint32_t n_end = static_cast<uint32_t>(ti.n_end);
-      // Branch-free over rows so the unrolled iterations' load chains overlap: rows past the end
-      // of the unit are zeroed with a select, and their (unused) position is clamped in range.
-#pragma unroll 4
-      for (int j = 0; j < GROUP_ROWS / 8; ++j) {
-        const uint32_t addr = base + static_cast<uint32_t>(j * 8 * 128);
-        const uint32_t n = n0 + 8 * j;
-        const uint32_t keep = n < n_end ? 0xffffffffu : 0u;
+      // One 8-channel chunk of one row: ReLU (rows past the unit's end zeroed by `keep`), RoPE with
+      // the chunk's cos/sin, z, written back in place.
+      auto item = [&](uint32_t addr, uint32_t keep, uint32_t pt, uint32_t ph_, uint32_t pw) {
         const uint4 raw = lds128(addr);
-        uint32_t pt, ph_, pw;
-        token_pos(p, n < N ? n : N - 1, pt, ph_, pw);
         float2 cs[4];
         if constexpr (UNIFORM) {
           const int x = static_cast<int>(bnd0 == 0 ? pt : (bnd0 == 1 ? ph_ : pw));
@@ -278,6 +274,33 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
           o[q] = pack_bf16(x0 * cs[q].x - x1 * cs[q].y, x0 * cs[q].y + x1 * cs[q].x);
         }
         sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
+      };
+      if (ti.n0 + TILE <= ti.n_end && step_ok) {
+        // Whole tile inside the unit (warp-uniform): no masking, and the position of row n + 8
+        // follows from that of row n with at most one wrap of w (W >= 8).
+        uint32_t pt, ph_, pw;
+        token_pos(p, n0, pt, ph_, pw);
+#pragma unroll 4
+        for (int j = 0; j < GROUP_ROWS / 8; ++j) {
+          item(base + static_cast<uint32_t>(j * 8 * 128), 0xffffffffu, pt, ph_, pw);
+          pw += 8;
+          const bool wrap = pw >= Wd;
+          pw = wrap ? pw - Wd : pw;
+          ph_ += wrap ? 1u : 0u;
+          const bool wrap2 = ph_ >= Hd;
+          ph_ = wrap2 ? 0u : ph_;
+          pt += wrap2 ? 1u : 0u;
+        }
+      } else {
+        // Branch-free over rows so the unrolled iterations' load chains overlap: rows past the
+        // end of the unit are zeroed with a select, and their (unused) position is clamped.
+#pragma unroll 4
+        for (int j = 0; j < GROUP_ROWS / 8; ++j) {
+          const uint32_t n = n0 + 8 * j;
+          uint32_t pt, ph_, pw;
+          token_pos(p, n < N ? n : N - 1, pt, ph_, pw);
+          item(base + static_cast<uint32_t>(j * 8 * 128), n < n_end ? 0xffffffffu : 0u, pt, ph_, pw);
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
