@@ -26,6 +26,7 @@ EXPORTS = [
     "la_workspace_bytes", "la_workspace_bytes_for", "la_state_reduce", "la_state_scan", "la_apply",
     "la_forward_bidir", "la_forward_blockcausal", "la_status_string", "la_device_error",
     "la_last_launch_count", "la_forward_marked", "la_selftest_host", "la_forward_bidir_static",
+    "la_state_update",
 ]
 
 
@@ -36,6 +37,7 @@ class LaProblem(ctypes.Structure):
         ("d", ctypes.c_int32), ("dt", ctypes.c_int32), ("dh", ctypes.c_int32), ("dw", ctypes.c_int32),
         ("rope_base", ctypes.c_double), ("eps", ctypes.c_float),
         ("block_frames", ctypes.c_int32), ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32),
+        ("t0", ctypes.c_int64),
     ]
 
 
@@ -69,6 +71,7 @@ def load(path: Optional[str] = None):
         "la_workspace_bytes_for": (sz, [P, ctypes.c_int]),
         "la_state_reduce": (ctypes.c_int, [P, vp, vp, vp, vp, vp, sz, vp]),
         "la_state_scan": (ctypes.c_int, [P, vp, vp, vp]),
+        "la_state_update": (ctypes.c_int, [P, vp, vp, vp, vp, vp, sz, vp]),
         "la_apply": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_bidir": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_blockcausal": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -109,6 +112,7 @@ class Problem:
     block_frames: int = 0
     dtype: str = "bf16"
     force_simt: bool = False
+    t0: int = 0  # global index of frame 0 (the t band rotates at t0 + t)
 
     @property
     def N(self) -> int:
@@ -129,7 +133,7 @@ class Problem:
         return LaProblem(self.B, self.H, self.T, self.Hh, self.W, self.d, self.bands[0], self.bands[1],
                          self.bands[2], float(self.rope_base), float(self.eps), int(self.block_frames),
                          LA_BF16 if self.dtype == "bf16" else LA_F32,
-                         LA_FLAG_FORCE_SIMT if self.force_simt else 0)
+                         LA_FLAG_FORCE_SIMT if self.force_simt else 0, int(self.t0))
 
 
 def _ptr(t) -> Optional[int]:
@@ -186,6 +190,21 @@ def state_reduce(p: Problem, K, V, S=None, z=None, ws=None, stream=None):
     cp = p.c()
     _check(lib.la_state_reduce(ctypes.byref(cp), _ptr(K), _ptr(V), _ptr(S), _ptr(z), _ptr(ws), nbytes,
                                _stream(stream)), "la_state_reduce")
+    return S, z
+
+
+def state_update(p: Problem, K, V, S, z, ws=None, stream=None):
+    """Cache update of block-autoregressive generation: S += sum phi(K)^T V, z += sum ReLU(K)
+    over the call's tokens, in place (S [B,H,d,d], z [B,H,d] fp32; ``p.block_frames`` = 0 and
+    ``p.t0`` = the block's first global frame)."""
+    lib = load()
+    if ws is None:
+        ws, nbytes = workspace(p, K.device)
+    else:
+        nbytes = ws.numel()
+    cp = p.c()
+    _check(lib.la_state_update(ctypes.byref(cp), _ptr(K), _ptr(V), _ptr(S), _ptr(z), _ptr(ws), nbytes,
+                               _stream(stream)), "la_state_update")
     return S, z
 
 

@@ -72,6 +72,7 @@ struct Rope {
   // cos/sin table (float2 entries), band-major then pair then position:
   //   t band: [dt/2][T] at 0, h band: [dh/2][Hh] at off_h, w band: [dw/2][W] at off_w.
   int64_t tab_off_h, tab_off_w, tab_entries;
+  int64_t t_offset;     // global index of frame 0: the t band rotates at t_offset + t
 };
 
 // Band (0: t, 1: h, 2: w) of channel pair `pair`.  DT/DH >= 0 fix the split at compile time.

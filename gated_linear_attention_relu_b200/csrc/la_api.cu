@@ -42,6 +42,7 @@ int validate(const la_problem* p) {
   // Overflow-safe size checks.
   const int64_t lim = int64_t(1) << 31;
   if (p->T >= lim || p->Hh >= lim || p->W >= lim || p->B >= lim || p->H >= lim) return LA_ERR_SHAPE;
+  if (p->t0 < 0 || p->t0 + p->T >= lim) return LA_ERR_SHAPE;
   const double n = double(p->T) * double(p->Hh) * double(p->W);
   if (n > double(kMaxTokens)) return LA_ERR_SHAPE;
   if (double(p->B) * double(p->H) > double(lim - 1)) return LA_ERR_SHAPE;
@@ -180,6 +181,7 @@ Rope make_rope(const la_problem& q) {
   r.tab_off_h = int64_t(q.dt / 2) * q.T;
   r.tab_off_w = r.tab_off_h + int64_t(q.dh / 2) * q.Hh;
   r.tab_entries = r.tab_off_w + int64_t(q.dw / 2) * q.W;
+  r.t_offset = q.t0;
   return r;
 }
 
@@ -299,7 +301,7 @@ int launch_state(const PlanSet& s, const la_problem& q, const void* K, const voi
 }
 
 int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk, float* z_blk, float* S_inc,
-                   float* z_inc, bool img, cudaStream_t st, int* nl) {
+                   float* z_inc, bool img, cudaStream_t st, int* nl, bool accumulate = false) {
   const int64_t groups = (int64_t(s.ps.d) * s.ps.d + s.ps.d) / 8;
   const int64_t threads = s.ps.BH * groups;
   if (threads == 0 || s.ps.nblk == 0) return LA_OK;
@@ -312,7 +314,7 @@ int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk
   // After the tensor-core state kernel (if it ran) the combine kernel may launch early; it waits
   // for that kernel before its first read.
   if (launch_k(la::cmb::combine_kernel, unsigned(cblocks), la::cmb::THREADS, 0, st, s.tc && s.ps.total > 0,
-               s.ps, partial, S_blk, z_blk, S_inc, z_inc, im, zim))
+               s.ps, partial, S_blk, z_blk, S_inc, z_inc, im, zim, accumulate ? 1 : 0))
     return LA_ERR_CUDA;
   ++*nl;
   return launched_ok();
@@ -423,6 +425,29 @@ int la_state_reduce(const la_problem* p, const void* K, const void* V, float* S,
   if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
   if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
   if ((rc = launch_combine(s, *p, ws, S, z, nullptr, nullptr, false, stream, &nl))) return rc;
+  g_last_launches = nl;
+  return LA_OK;
+}
+
+int la_state_update(const la_problem* p, const void* K, const void* V, float* S, float* z, void* ws,
+                    size_t ws_bytes, cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  if (p->block_frames != 0) return LA_ERR_SHAPE;
+  const bool has_tok = elems(*p) > 0;
+  const bool has_state = state_units(*p) > 0;
+  if ((rc = check_ptr(K, has_tok)) || (rc = check_ptr(V, has_tok)) || (rc = check_ptr(S, has_state)) ||
+      (rc = check_ptr(z, has_state)))
+    return rc;
+  int sm = 0;
+  if ((rc = current_sm_count(&sm))) return rc;
+  const PlanSet s = make_plans(*p, sm);
+  if ((rc = check_ws(s, ws, ws_bytes))) return rc;
+  int nl = 0;
+  if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
+  if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
+  // No tokens: the state reduction queues nothing and the carried state stays as it is.
+  if (has_tok && (rc = launch_combine(s, *p, ws, nullptr, nullptr, S, z, false, stream, &nl, true))) return rc;
   g_last_launches = nl;
   return LA_OK;
 }

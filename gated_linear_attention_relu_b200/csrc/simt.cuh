@@ -80,7 +80,9 @@ state_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const Plan p
         token_pos(p, static_cast<uint32_t>(n), pt, ph, pw);
       }
       float cs, sn;
-      rope_cs(static_cast<double>(axis_pos(rope.band[pi], pt, ph, pw)), rope.theta_d[pi], cs, sn);
+      rope_cs(static_cast<double>(axis_pos(rope.band[pi], pt, ph, pw)) +
+                  (rope.band[pi] == 0 ? static_cast<double>(rope.t_offset) : 0.0),
+              rope.theta_d[pi], cs, sn);
       kp[r][2 * pi] = x0;
       kp[r][2 * pi + 1] = x1;
       kr[r][2 * pi] = x0 * cs - x1 * sn;
@@ -163,7 +165,9 @@ apply_simt_kernel(const T* __restrict__ Q, const T* __restrict__ G, const float*
         token_pos(p, static_cast<uint32_t>(n), pt, ph, pw);
       }
       float cs, sn;
-      rope_cs(static_cast<double>(axis_pos(rope.band[pi], pt, ph, pw)), rope.theta_d[pi], cs, sn);
+      rope_cs(static_cast<double>(axis_pos(rope.band[pi], pt, ph, pw)) +
+                  (rope.band[pi] == 0 ? static_cast<double>(rope.t_offset) : 0.0),
+              rope.theta_d[pi], cs, sn);
       qp[r * (D + 1) + 2 * pi] = x0;
       qp[r * (D + 1) + 2 * pi + 1] = x1;
       qr[r * (D + 1) + 2 * pi] = x0 * cs - x1 * sn;
@@ -258,7 +262,8 @@ __device__ __forceinline__ void rope_table_entry(const Plan& p, const Rope& r, i
     band = 2;
   }
   double s, c;
-  sincos(static_cast<double>(x) * r.theta_d[pair], &s, &c);
+  const int64_t xg = band == 0 ? x + r.t_offset : x;  // t rotates at its global frame index
+  sincos(static_cast<double>(xg) * r.theta_d[pair], &s, &c);
   const float2 v = make_float2(static_cast<float>(c), static_cast<float>(s));
   tab[e] = v;
   if (tab2) {
@@ -282,7 +287,7 @@ rope_table_kernel(const Plan p, const __grid_constant__ Rope rope, float2* tab, 
 
 __global__ void __launch_bounds__(THREADS)
 combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, float* z_blk, float* S_inc,
-               float* z_inc, uint8_t* img, float* zimg) {
+               float* z_inc, uint8_t* img, float* zimg, int accumulate) {
   // Every thread reads the state kernel's partial sums: wait for that kernel first.
   pdl_trigger();
   pdl_wait();
@@ -296,6 +301,14 @@ combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, fl
   float run[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) run[e] = 0.f;
+  if (accumulate) {
+    // Cache update: the running sum starts from the carried state in S_inc / z_inc (one unit per
+    // head), which is then overwritten with carried + this call's sum.
+    const float* src = (e0 < D * D) ? S_inc + bh * D * D + e0 : z_inc + bh * D + (e0 - D * D);
+    const float4 a = reinterpret_cast<const float4*>(src)[0], b = reinterpret_cast<const float4*>(src)[1];
+    run[0] = a.x; run[1] = a.y; run[2] = a.z; run[3] = a.w;
+    run[4] = b.x; run[5] = b.y; run[6] = b.z; run[7] = b.w;
+  }
   for (int64_t blk = 0; blk < p.nblk; ++blk) {
     const int64_t u = bh * p.nblk + blk;
     float acc[8];

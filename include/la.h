@@ -78,6 +78,9 @@ typedef struct {
   int32_t block_frames;  /* 0: bidirectional; > 0: latent frames per causal block */
   int32_t dtype;         /* la_dtype of Q, K, V, G and O */
   uint32_t flags;        /* LA_FLAG_* */
+  int64_t t0;            /* global index of latent frame 0 (>= 0): the t band rotates at t0 + t.
+                            0 for a whole video; the first frame of the block when a
+                            block-autoregressive generator processes one block per call. */
 } la_problem;
 
 /* Bytes of device workspace the calls below need for this problem on the CURRENT
@@ -92,6 +95,17 @@ size_t la_workspace_bytes_for(const la_problem* p, int sm_count);
  * per-block states): writes S [B,H,nblk,d,d] and z [B,H,nblk,d], fp32.  In block-causal
  * mode these are the states of each block alone (not prefixed).  K, V: [B,H,N,d]. */
 int la_state_reduce(const la_problem* p, const void* K, const void* V, float* S, float* z,
+                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Constant-memory cache update for block-autoregressive generation (SANA-Video Sec. 3.4,
+ * Algorithm 1: after a block is generated, its keys and values are folded into the cache):
+ *   S += sum_n phi(K_n)^T V_n,   z += sum_n ReLU(K_n)   over all N tokens of the call, in place.
+ * S: [B,H,d,d], z: [B,H,d], fp32, the carried cache (zeros before the first block).  The call's
+ * frames form one block: p->block_frames must be 0; set p->t0 to the block's first global frame
+ * so its keys rotate at their global t.  Then la_apply with the same problem and the updated
+ * cache gives the block's outputs (a block sees itself and every earlier block), matching
+ * la_forward_blockcausal on the whole video up to rounding.  K, V: [B,H,N,d]. */
+int la_state_update(const la_problem* p, const void* K, const void* V, float* S, float* z,
                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* In-place inclusive prefix over blocks (SANA-Video Sec. 3.4: the cache after block j

@@ -48,6 +48,8 @@ def _call_bidir(p, ptrs=(16, 16, 16, 16, 16)):
     (dict(rope_base=0.0), 2),
     (dict(block_frames=2), 2),          # la_forward_bidir wants block_frames == 0
     (dict(T=100000, Hh=1000, W=1000), 2),  # N beyond 2^31 tokens
+    (dict(t0=-1), 2),                   # frame offset must be >= 0
+    (dict(t0=2**31 - 3), 2),            # t0 + T beyond 2^31
 ])
 def test_invalid_problems_rejected_before_cuda(kw, status):
     args = dict(B=1, H=2, T=3, Hh=4, W=5)
@@ -92,3 +94,13 @@ def test_workspace_sizes_are_consistent():
 def test_host_selftest_of_work_decomposition():
     # Exact fast division and tile/segment bookkeeping, checked on the host by the library itself.
     assert la.load().la_selftest_host() == 0
+
+
+def test_state_update_rejects_block_causal_problems_before_cuda():
+    lib = la.load()
+    cp = la.Problem(B=1, H=2, T=3, Hh=4, W=5, block_frames=1).c()
+    assert lib.la_state_update(ctypes.byref(cp), 16, 16, 16, 16, 16, 1 << 30, None) == 2
+    cp = la.Problem(B=1, H=2, T=3, Hh=4, W=5, t0=-2).c()
+    assert lib.la_state_update(ctypes.byref(cp), 16, 16, 16, 16, 16, 1 << 30, None) == 2
+    cp = la.Problem(B=1, H=2, T=3, Hh=4, W=5, t0=4).c()
+    assert lib.la_state_update(ctypes.byref(cp), None, 16, 16, 16, 16, 1 << 30, None) == 1

@@ -335,3 +335,30 @@ def test_planted_transposed_state_is_caught_by_brute_form():
     bad = orc.head_apply(q, g, S.T, z, pos, bands, 10000.0, 1e-6)
     ob = orc.forward_brute(q, k, v, g, pos, bands, 10000.0, 1e-6)
     assert np.max(np.abs(bad - ob)) > 1e-3 * np.max(np.abs(ob))
+
+
+def test_streaming_cache_restatement_equals_block_causal_form():
+    """Algorithm 1 of the block-causal paper, restated: carry (S, z), fold each block's keys and
+    values in (RoPE at global frame indices), then apply the block against the carried state.
+    This must reproduce the block-causal operator exactly (up to fp64 rounding)."""
+    rng = np.random.default_rng(11)
+    T, Hh, W, d, bands, bf = 7, 3, 4, 16, (4, 6, 6), 2
+    N = T * Hh * W
+    q, k, v, g = (rng.standard_normal((1, 1, N, d)) for _ in range(4))
+    ref = orc.forward_blockcausal(q, k, v, g, (T, Hh, W), bands, 10000.0, 1e-6, block_frames=bf)[0, 0]
+    S, z = np.zeros((d, d)), np.zeros(d)
+    out = []
+    for t0 in range(0, T, bf):
+        t1 = min(T, t0 + bf)
+        sl = slice(t0 * Hh * W, t1 * Hh * W)
+        pos = orc.grid_positions(t1 - t0, Hh, W)
+        pos[:, 0] += t0
+        Sb, zb = orc.head_state(k[0, 0, sl], v[0, 0, sl], pos, bands, 10000.0)
+        S, z = S + Sb, z + zb
+        out.append(orc.head_apply(q[0, 0, sl], g[0, 0, sl], S, z, pos, bands, 10000.0, 1e-6))
+    assert np.allclose(np.concatenate(out), ref, rtol=1e-12, atol=1e-14)
+    # Positions local to the block (t0 ignored) give a different result: the offset matters.
+    pos_local = orc.grid_positions(T - 6, Hh, W)
+    sl = slice(6 * Hh * W, N)
+    bad = orc.head_apply(q[0, 0, sl], g[0, 0, sl], S, z, pos_local, bands, 10000.0, 1e-6)
+    assert not np.allclose(bad, ref[sl], rtol=1e-3)
