@@ -43,6 +43,11 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work of the oracle baseline")
+    ap.add_argument("--gated", action="store_true",
+                    help="full gated form: write gate beta [B,H,N] and RMSNorm before the output gate")
+    ap.add_argument("--stream", action="store_true",
+                    help="block-causal workloads: one call pair per block (la_state_update + la_apply "
+                         "on a carried cache), as a block-autoregressive generator runs")
     return ap.parse_args()
 
 
@@ -228,6 +233,46 @@ def main():
     if w.block_frames > 0:
         S_incl = torch.empty((w.B, w.H, w.nblk, w.d, w.d), dtype=torch.float32, device=dev)
         z_incl = torch.empty((w.B, w.H, w.nblk, w.d), dtype=torch.float32, device=dev)
+    gates = {}
+    if args.gated:
+        beta, gamma = wl.generate_gates(w, dev, seed=w.seed + 7 + 1000 * rank)
+        gates = dict(beta=beta, gamma=gamma, rms_norm=True, norm_eps=1e-6)
+    if args.stream and w.block_frames <= 0:
+        raise SystemExit("--stream needs a block-causal workload")
+
+    if args.stream:
+        # One block per call pair, on contiguous per-block tensors cut out before timing (a
+        # generator produces each block's tensors as it goes).
+        HW = w.Hh * w.W
+        blocks = []
+        for t0 in range(0, w.T, w.block_frames):
+            t1 = min(w.T, t0 + w.block_frames)
+            sl = slice(t0 * HW, t1 * HW)
+            pb = la.Problem.from_workload(w, T=t1 - t0, block_frames=0, t0=t0)
+            blocks.append((pb, [x[:, :, sl].contiguous() for x in (Q, K, V, G)], torch.empty_like(Q[:, :, sl])))
+        ws_s, _ = la.workspace(blocks[0][0], dev)
+        S_c = torch.empty((w.B, w.H, w.d, w.d), dtype=torch.float32, device=dev)
+        z_c = torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=dev)
+        counter = {"launches": 0}
+
+        def forward_plain():
+            S_c.zero_()
+            z_c.zero_()
+            n = 0
+            for pb, (qb, kb, vb, gb), ob in blocks:
+                la.state_update(pb, kb, vb, S_c, z_c, ws=ws_s)
+                n += la.last_launch_count()
+                la.apply(pb, qb, gb, S_c, z_c, O=ob, ws=ws_s)
+                n += la.last_launch_count()
+            counter["launches"] = n
+    else:
+        def forward_plain():
+            if args.gated:
+                la.forward_gated(p, Q, K, V, G, O=O, ws=ws, S_incl=S_incl, z_incl=z_incl, **gates)
+            elif w.block_frames > 0:
+                la.forward_blockcausal(p, Q, K, V, G, O=O, ws=ws, S_incl=S_incl, z_incl=z_incl)
+            else:
+                la.forward_bidir(p, Q, K, V, G, O=O, ws=ws)
 
     # Marker events around each kernel of each timed step; recorded once here so their CUDA
     # handles exist before the timed region.
@@ -236,21 +281,18 @@ def main():
     for row in evs:
         for e in row:
             e.record(stream)
-    for _ in range(max(3, args.warmup)):
-        la.forward_marked(p, Q, K, V, G, O, ws, evs[0], S_incl, z_incl)
-    launches_per_step = la.last_launch_count()
+    if not args.stream:
+        for _ in range(max(3, args.warmup)):
+            la.forward_marked(p, Q, K, V, G, O, ws, evs[0], S_incl, z_incl, **gates)
+        launches_per_step = la.last_launch_count()
     torch.cuda.synchronize()
     assert la.device_error() == 0, "device-side error during warm-up"
-
-    def forward_plain():
-        if w.block_frames > 0:
-            la.forward_blockcausal(p, Q, K, V, G, O=O, ws=ws, S_incl=S_incl, z_incl=z_incl)
-        else:
-            la.forward_bidir(p, Q, K, V, G, O=O, ws=ws)
 
     for _ in range(max(3, args.warmup)):
         forward_plain()
     torch.cuda.synchronize()
+    if args.stream:
+        launches_per_step = counter["launches"]
 
     # Timed region (the headline): K steps of the public forward call, bracketed by a barrier and
     # a synchronize on both sides.  No events sit between the kernels of a step, so each kernel
@@ -272,63 +314,78 @@ def main():
     # Second timed region, same K steps with an event before and after every kernel: the
     # per-kernel durations and the dominant kernel's roofline come from here.  (An event between
     # two kernels keeps the second from starting early, so these steps run a little longer.)
-    ldist.barrier(dev)
-    torch.cuda.synchronize()
-    m_start, m_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    m_start.record(stream)
-    for k in range(args.steps):
-        la.forward_marked(p, Q, K, V, G, O, ws, evs[k], S_incl, z_incl)
-    m_end.record(stream)
-    torch.cuda.synchronize()
-    ldist.barrier(dev)
-    marked_ms = m_start.elapsed_time(m_end) / args.steps
-    assert la.device_error() == 0, "device-side error in the marked region"
+    marked_ms = None
+    if not args.stream:
+        ldist.barrier(dev)
+        torch.cuda.synchronize()
+        m_start, m_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m_start.record(stream)
+        for k in range(args.steps):
+            la.forward_marked(p, Q, K, V, G, O, ws, evs[k], S_incl, z_incl, **gates)
+        m_end.record(stream)
+        torch.cuda.synchronize()
+        ldist.barrier(dev)
+        marked_ms = m_start.elapsed_time(m_end) / args.steps
+        assert la.device_error() == 0, "device-side error in the marked region"
 
-    # Per-kernel durations inside the timed steps.
-    tc = not args.simt and w.d == 128 and w.dtype == "bf16"
-    names = ["rope_table_kernel", "state_tc_kernel", "combine_kernel", "apply_tc_kernel"] if tc \
-        else ["state_simt_kernel", "combine_kernel", "apply_simt_kernel"]
-    assert len(names) == launches_per_step, (names, launches_per_step)
-    per = {n: [] for n in names}
-    for k in range(args.steps):
-        for i, n in enumerate(names):
-            per[n].append(evs[k][i].elapsed_time(evs[k][i + 1]))
-    kern_ms = {n: sum(v) / len(v) for n, v in per.items()}
-    tot = sum(kern_ms.values())
     elem = w.elem_bytes
     th = w.B * w.H * w.N
-    alg_bytes = {names[-3]: 2 * th * w.d * elem, names[-1]: 3 * th * w.d * elem}
-    dominant = max((n for n in names if n in alg_bytes), key=lambda n: kern_ms[n])
     peak, peak_kind = measured_hbm()
-    achieved = alg_bytes[dominant] / (kern_ms[dominant] * 1e-3) / 1e9
-    traffic_rec, _ = kernel_traffic(dominant)
-    traffic = None
-    if traffic_rec is not None and traffic_rec.get("workload") == w.name:
-        traffic = traffic_rec.get("bytes_per_launch")
-
     value = world * th * args.steps / (t_max * 1e-3)
     ms_per_step = t_max / args.steps
-    roof_all = w.min_bytes / (ms_per_step * 1e-3) / 1e9
+    # bytes_min: Q, K, V, G read once and O written once (+ the write gate when gated).
+    min_bytes = w.min_bytes + (th * elem if args.gated else 0)
+    roof_all = min_bytes / (ms_per_step * 1e-3) / 1e9
 
+    if args.stream:
+        # No events can sit inside la_state_update / la_apply, so the roofline is the whole step's.
+        kernels, dominant, alg, achieved, traffic = {}, "whole step (per-block calls)", min_bytes, roof_all, None
+    else:
+        # Per-kernel durations inside the timed steps of the second region.
+        tc = not args.simt and w.d == 128 and w.dtype == "bf16"
+        names = ["rope_table_kernel", "state_tc_kernel", "combine_kernel", "apply_tc_kernel"] if tc \
+            else ["state_simt_kernel", "combine_kernel", "apply_simt_kernel"]
+        assert len(names) == launches_per_step, (names, launches_per_step)
+        per = {n: [] for n in names}
+        for k in range(args.steps):
+            for i, n in enumerate(names):
+                per[n].append(evs[k][i].elapsed_time(evs[k][i + 1]))
+        kern_ms = {n: sum(v) / len(v) for n, v in per.items()}
+        tot = sum(kern_ms.values())
+        alg_bytes = {names[-3]: (2 * w.d + (1 if args.gated else 0)) * th * elem, names[-1]: 3 * th * w.d * elem}
+        dominant = max((n for n in names if n in alg_bytes), key=lambda n: kern_ms[n])
+        alg = alg_bytes[dominant]
+        achieved = alg / (kern_ms[dominant] * 1e-3) / 1e9
+        traffic_rec, _ = kernel_traffic(dominant)
+        traffic = None
+        if traffic_rec is not None and traffic_rec.get("workload") == w.name and not args.gated:
+            traffic = traffic_rec.get("bytes_per_launch")
+        kernels = {n: {"ms": kern_ms[n], "share": kern_ms[n] / tot if tot else None} for n in names}
+
+    config = config_of(w, world)
+    if args.gated:
+        config["gated"] = "write gate beta [B,H,N] + RMSNorm (gamma [d]) before the output gate"
+    if args.stream:
+        config["stream"] = f"{len(blocks)} blocks, la_state_update + la_apply per block on a carried cache"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
-        "config": config_of(w, world),
+        "config": config,
         "hbm_roofline_frac_8tbs": roof_all / NOMINAL_HBM_GBS,
         "hbm_roofline_frac_measured": roof_all / peak,
         "achieved_gbs_whole_step": roof_all,
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": alg_bytes[dominant]},
-        "kernels": {n: {"ms": kern_ms[n], "share": kern_ms[n] / tot if tot else None} for n in names},
+                     "algorithmic_bytes_per_launch": alg},
+        "kernels": kernels,
         "kernels_region": {"ms_per_step": marked_ms, "note": "second timed region, events around every kernel"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
 
-    if not args.no_e2e:
-        line["e2e"] = e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world)
+    if not args.no_e2e and not args.stream:
+        line["e2e"] = e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, times = oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -340,20 +397,26 @@ def main():
     return 0
 
 
-def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world):
+def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None):
     """Same metric through the public API with the inputs in pinned host memory: every step
-    copies Q, K, V, G host->device, runs the operator and copies O device->host."""
+    copies Q, K, V, G (and the write gate when gated) host->device, runs the operator and copies
+    O device->host."""
     import torch
 
-    hosts = [t.cpu().pin_memory() for t in (Q, K, V, G)]
+    gates = gates or {}
+    srcs = [Q, K, V, G] + ([gates["beta"]] if "beta" in gates else [])
+    hosts = [t.cpu().pin_memory() for t in srcs]
     Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
     steps = max(3, min(args.steps, 10))
     stream = torch.cuda.current_stream()
 
     def step():
-        for hsrc, dst in zip(hosts, (Q, K, V, G)):
+        for hsrc, dst in zip(hosts, srcs):
             dst.copy_(hsrc, non_blocking=True)
-        la.forward(p, Q, K, V, G, O=O, ws=ws)
+        if gates:
+            la.forward_gated(p, Q, K, V, G, O=O, ws=ws, **gates)
+        else:
+            la.forward(p, Q, K, V, G, O=O, ws=ws)
         Oh.copy_(O, non_blocking=True)
 
     for _ in range(2):
@@ -368,9 +431,9 @@ def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world):
     torch.cuda.synchronize()
     t = ldist.max_over_ranks(s.elapsed_time(e), dev)
     th = w.B * w.H * w.N
-    nbytes = Q.numel() * Q.element_size()
-    return {"value": world * th * steps / (t * 1e-3), "unit": UNIT, "h2d_bytes_per_step": 4 * nbytes,
-            "d2h_bytes_per_step": nbytes, "steps": steps}
+    h2d = sum(x.numel() * x.element_size() for x in srcs)
+    return {"value": world * th * steps / (t * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": O.numel() * O.element_size(), "steps": steps}
 
 
 if __name__ == "__main__":

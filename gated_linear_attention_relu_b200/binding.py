@@ -26,7 +26,7 @@ EXPORTS = [
     "la_workspace_bytes", "la_workspace_bytes_for", "la_state_reduce", "la_state_scan", "la_apply",
     "la_forward_bidir", "la_forward_blockcausal", "la_status_string", "la_device_error",
     "la_last_launch_count", "la_forward_marked", "la_selftest_host", "la_forward_bidir_static",
-    "la_state_update",
+    "la_state_update", "la_forward_gated",
 ]
 
 
@@ -38,6 +38,13 @@ class LaProblem(ctypes.Structure):
         ("rope_base", ctypes.c_double), ("eps", ctypes.c_float),
         ("block_frames", ctypes.c_int32), ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32),
         ("t0", ctypes.c_int64),
+    ]
+
+
+class LaGates(ctypes.Structure):
+    _fields_ = [
+        ("beta", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("norm_eps", ctypes.c_float),
+        ("rms_norm", ctypes.c_int32),
     ]
 
 
@@ -72,6 +79,7 @@ def load(path: Optional[str] = None):
         "la_state_reduce": (ctypes.c_int, [P, vp, vp, vp, vp, vp, sz, vp]),
         "la_state_scan": (ctypes.c_int, [P, vp, vp, vp]),
         "la_state_update": (ctypes.c_int, [P, vp, vp, vp, vp, vp, sz, vp]),
+        "la_forward_gated": (ctypes.c_int, [P, ctypes.POINTER(LaGates), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_apply": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_bidir": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_blockcausal": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -80,7 +88,7 @@ def load(path: Optional[str] = None):
         "la_last_launch_count": (ctypes.c_int, []),
         "la_selftest_host": (ctypes.c_int, []),
         "la_forward_bidir_static": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp]),
-        "la_forward_marked": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+        "la_forward_marked": (ctypes.c_int, [P, ctypes.POINTER(LaGates), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                              ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
@@ -280,6 +288,33 @@ def forward_blockcausal(p: Problem, Q, K, V, G, O=None, S_incl=None, z_incl=None
     return O
 
 
+def forward_gated(p: Problem, Q, K, V, G, beta=None, gamma=None, rms_norm=False, norm_eps=1e-6, O=None,
+                  S_incl=None, z_incl=None, ws=None, return_states=False, stream=None):
+    """The full gated form: write gate ``beta`` [B,H,N] (problem dtype) on the state, and RMSNorm
+    (weight ``gamma`` [d] fp32, or None) of num/den before the output gate when ``rms_norm``.
+    Bidirectional or block-causal as ``p.block_frames`` says."""
+    import torch
+
+    lib = load()
+    if O is None:
+        O = torch.empty_like(Q)
+    if return_states and S_incl is None:
+        S_incl = torch.empty((p.B, p.H, p.nblk, p.d, p.d), dtype=torch.float32, device=Q.device)
+        z_incl = torch.empty((p.B, p.H, p.nblk, p.d), dtype=torch.float32, device=Q.device)
+    if ws is None:
+        ws, nbytes = workspace(p, Q.device)
+    else:
+        nbytes = ws.numel()
+    cp = p.c()
+    gates = LaGates(_ptr(beta), _ptr(gamma), float(norm_eps), 1 if rms_norm else 0)
+    _check(lib.la_forward_gated(ctypes.byref(cp), ctypes.byref(gates), _ptr(Q), _ptr(K), _ptr(V), _ptr(G),
+                                _ptr(O), _ptr(S_incl), _ptr(z_incl), _ptr(ws), nbytes, _stream(stream)),
+           "la_forward_gated")
+    if return_states:
+        return O, S_incl, z_incl
+    return O
+
+
 def forward(p: Problem, Q, K, V, G, **kw):
     """Bidirectional or block-causal, as ``p.block_frames`` says."""
     if p.block_frames > 0:
@@ -287,7 +322,8 @@ def forward(p: Problem, Q, K, V, G, **kw):
     return forward_bidir(p, Q, K, V, G, **kw)
 
 
-def forward_marked(p: Problem, Q, K, V, G, O, ws, events, S_incl=None, z_incl=None, stream=None):
+def forward_marked(p: Problem, Q, K, V, G, O, ws, events, S_incl=None, z_incl=None, stream=None, beta=None,
+                   gamma=None, rms_norm=False, norm_eps=1e-6):
     """Forward pass recording ``events[0]`` before the first kernel and ``events[i]`` after kernel i.
 
     ``events`` are ``torch.cuda.Event(enable_timing=True)`` objects; each is recorded once on
@@ -302,7 +338,8 @@ def forward_marked(p: Problem, Q, K, V, G, O, ws, events, S_incl=None, z_incl=No
             e.record(st)
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     cp = p.c()
-    _check(lib.la_forward_marked(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(O),
+    gates = LaGates(_ptr(beta), _ptr(gamma), float(norm_eps), 1 if rms_norm else 0)
+    _check(lib.la_forward_marked(ctypes.byref(cp), ctypes.byref(gates), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(O),
                                  _ptr(S_incl), _ptr(z_incl), _ptr(ws), ws.numel(), st.cuda_stream,
                                  arr, len(events)), "la_forward_marked")
     return O

@@ -62,6 +62,7 @@ constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t GROUP_COLS = 256, ACC_COL = 0, A_COL = 128;
 constexpr uint32_t DEN_COL = 192;  // + 2 * slot + half: partial denominators (fp32, lane = row)
+constexpr uint32_t RMS_COL = 196;  // + 2 * slot + half: partial sums of squares (RMSNorm)
 constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/true);
 // Register split: the launch grants REGS_LAUNCH per thread (the largest multiple of 8 that fits
 // 65536 / THREADS); the control warpgroup shrinks to REGS_CTRL and the math groups grow to
@@ -76,7 +77,9 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 // serves the same group and no group polls a stage's barrier more than one phase ahead (which
 // would alias the parity test).
 static_assert(QST % NWG == 0 && GST % NWG == 0, "stages must be a multiple of the math groups");
-static_assert(NWG * GROUP_COLS <= TMEM_COLS && A_COL + 64 <= DEN_COL && DEN_COL + 4 <= GROUP_COLS, "TMEM columns");
+static_assert(NWG * GROUP_COLS <= TMEM_COLS && A_COL + 64 <= DEN_COL && DEN_COL + 4 <= RMS_COL &&
+                  RMS_COL + 4 <= GROUP_COLS,
+              "TMEM columns");
 static_assert(128 * REGS_CTRL + 128 * MATH_WGS * REGS_MATH <= THREADS * REGS_LAUNCH, "register split");
 static_assert(REGS_CTRL <= REGS_LAUNCH && REGS_LAUNCH <= REGS_MATH, "register split");
 
@@ -86,6 +89,7 @@ struct Bars {
   uint64_t sfull[NSB], sfree[NSB];
   uint64_t aready[NWG], afree[NWG], accfull[NWG], accempty[NWG];
   uint64_t denx[NWG][4];  // the two warps holding the halves of rows 32q .. 32q+31 of group m
+  uint64_t rmsx[NWG][4];  // the same pairs, for the RMSNorm sums of squares
   uint64_t final_;
   uint32_t tmem_base;
   int abort_flag;
@@ -167,12 +171,15 @@ __device__ __forceinline__ float transform_half(uint32_t (&a)[32], const float* 
   return ((d0.x + d0.y) + (d1.x + d1.y)) + ((d2.x + d2.y) + (d3.x + d3.y));
 }
 
-template <int DT, int DH>
+// RMS: RMSNorm of y = num / den over the row's 128 channels before the gate (SANA-Video 2.0,
+// Eq. (1)), y / sqrt(mean(y^2) + norm_eps) * gamma (gamma may be null: 1).
+template <int DT, int DH, bool RMS>
 __global__ void __launch_bounds__(THREADS, 1)
 apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
                 const __grid_constant__ CUtensorMap tmO, const Plan p, const __grid_constant__ Rope rope,
                 const uint8_t* __restrict__ simg, const float* __restrict__ zimg,
-                const float2* __restrict__ tab, const float4* __restrict__ tab2, __nv_bfloat16* __restrict__ O) {
+                const float2* __restrict__ tab, const float4* __restrict__ tab2, const float* __restrict__ gamma,
+                float norm_eps, __nv_bfloat16* __restrict__ O) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
@@ -205,7 +212,10 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(&bars->afree[m], 1);
       mbar_init(&bars->accfull[m], 1);
       mbar_init(&bars->accempty[m], 8);
-      for (int q = 0; q < 4; ++q) mbar_init(&bars->denx[m][q], 2);
+      for (int q = 0; q < 4; ++q) {
+        mbar_init(&bars->denx[m][q], 2);
+        mbar_init(&bars->rmsx[m][q], 2);
+      }
     }
     mbar_init(&bars->final_, 1);
     bars->abort_flag = 0;
@@ -345,6 +355,9 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t t_a = t_grp + A_COL + 32u * hf;
     const int ext_t = static_cast<int>(p.T), ext_h = static_cast<int>(p.Hh), ext_w = static_cast<int>(p.W);
     uint64_t* denx = &bars->denx[m][quarter];
+    uint64_t* rmsx = &bars->rmsx[m][quarter];
+    const bool use_gamma = RMS && gamma != nullptr;
+    const float* gm = use_gamma ? gamma + 64 * hf : nullptr;
     pdl_wait();
     int64_t g_prev = -1;
     uint32_t k_prev = 0;
@@ -422,13 +435,39 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->accempty[m]);
+        float scale = hinv_prev;  // h = acc * scale (* gamma)
+        if constexpr (RMS) {
+          // Sum of squares of this half of the row, swapped with the other half through TMEM
+          // (two slots, as for the denominators).  y = acc / den = 2 h, so mean(y^2) =
+          // 4 hinv^2 ss / 128 and the normalised h = acc * hinv / sqrt(mean(y^2) + norm_eps).
+          uint64_t s2[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const uint64_t a2 = pk(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
+            s2[c & 3] = fma2(a2, a2, s2[c & 3]);
+          }
+          const float2 e0 = upk(s2[0]), e1 = upk(s2[1]), e2 = upk(s2[2]), e3 = upk(s2[3]);
+          const float ss_half = ((e0.x + e0.y) + (e1.x + e1.y)) + ((e2.x + e2.y) + (e3.x + e3.y));
+          const uint32_t t_rms = t_grp + RMS_COL + 2u * (k_prev & 1u);
+          tmem_st_x1(t_rms + hf, __float_as_uint(ss_half));
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(rmsx);
+          if (!warp_wait(rmsx, k_prev & 1u, abort_flag)) break;
+          tc_fence_after();
+          const float other = __uint_as_float(tmem_ld_x1(t_rms + (hf ^ 1)));
+          tmem_ld_wait();
+          const float ss = hf == 0 ? ss_half + other : other + ss_half;
+          scale = hinv_prev * rsqrtf(4.f * hinv_prev * hinv_prev * ss * (1.f / D) + norm_eps);
+        }
         if (!warp_wait(&bars->gfull[gs], static_cast<uint32_t>((i / GST) & 1), abort_flag)) break;
         const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
         const bool tma_out = (ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N);
         const bool valid = static_cast<int64_t>(n) < ti.n_end;
         const uint32_t grow = sbase + OFF_G + gs * BUF + row_off;
         __nv_bfloat16* orow = O + (ti.bh * p.N + static_cast<int64_t>(n)) * D + 64 * hf;
-        const uint64_t hh = pk(hinv_prev, hinv_prev);
+        const uint64_t hh = pk(scale, scale);
         // The G row is read and overwritten in place, four chunks at a time: the loads of a batch
         // are all issued before its first store, so their latency is paid once per batch.
 #pragma unroll
@@ -444,9 +483,16 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const uint32_t gw[4] = {half_bf16x2(graw[c4].x), half_bf16x2(graw[c4].y), half_bf16x2(graw[c4].z),
                                     half_bf16x2(graw[c4].w)};
             uint32_t ov[4];
+            ulonglong2 gw01 = make_ulonglong2(0, 0), gw23 = make_ulonglong2(0, 0);
+            if (use_gamma) {
+              gw01 = __ldg(reinterpret_cast<const ulonglong2*>(gm + 8 * c8));
+              gw23 = __ldg(reinterpret_cast<const ulonglong2*>(gm + 8 * c8 + 4));
+            }
+            const uint64_t gpair[4] = {gw01.x, gw01.y, gw23.x, gw23.y};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const uint64_t h = mul2(pk(__uint_as_float(r[c8 * 8 + 2 * q]), __uint_as_float(r[c8 * 8 + 2 * q + 1])), hh);
+              uint64_t h = mul2(pk(__uint_as_float(r[c8 * 8 + 2 * q]), __uint_as_float(r[c8 * 8 + 2 * q + 1])), hh);
+              if (use_gamma) h = mul2(h, gpair[q]);
               const uint64_t t = pk(tanh_approx(bf16lo(gw[q])), tanh_approx(bf16hi(gw[q])));
               const float2 o2 = upk(fma2(h, t, h));
               ov[q] = pack_bf16(o2.x, o2.y);

@@ -249,6 +249,14 @@ int launch_k(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
+// Optional terms of the full gated form (la_gates), as the launchers see them.
+struct Gates {
+  const void* beta = nullptr;   // [B,H,N] write gate, problem dtype; null: 1
+  const float* gamma = nullptr; // [d] RMSNorm weight; null: 1
+  float norm_eps = 0.f;
+  bool rms = false;
+};
+
 // ------------------------------------------------------------------------------- launchers
 // cos/sin table shared by the tensor-core state and apply kernels, one entry per thread.
 int launch_table(const PlanSet& s, const la_problem& q, void* ws, cudaStream_t st, int* nl) {
@@ -263,7 +271,7 @@ int launch_table(const PlanSet& s, const la_problem& q, void* ws, cudaStream_t s
 }
 
 int launch_state(const PlanSet& s, const la_problem& q, const void* K, const void* V, void* ws,
-                 cudaStream_t st, int* nl) {
+                 cudaStream_t st, int* nl, const void* beta = nullptr) {
   if (s.ps.total == 0) return LA_OK;
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + s.off_partial);
   const Rope rope = make_rope(q);
@@ -272,19 +280,20 @@ int launch_state(const PlanSet& s, const la_problem& q, const void* K, const voi
     if (!make_tmap(&tk, K, s.ps.BH, s.ps.N, la::st::TILE) || !make_tmap(&tv, V, s.ps.BH, s.ps.N, la::st::TILE))
       return LA_ERR_CUDA;
     const float2* tab = reinterpret_cast<const float2*>(static_cast<uint8_t*>(ws) + s.off_tab);
-    auto kern = standard_bands(q) ? la::st::state_tc_kernel<32, 48> : la::st::state_tc_kernel<-1, -1>;
+    auto kern = standard_bands(q) ? (beta ? la::st::state_tc_kernel<32, 48, true> : la::st::state_tc_kernel<32, 48, false>)
+                                  : (beta ? la::st::state_tc_kernel<-1, -1, true> : la::st::state_tc_kernel<-1, -1, false>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::st::SMEM_BYTES) != cudaSuccess)
       return LA_ERR_CUDA;
     const float4* tab2 =
         standard_bands(q) ? reinterpret_cast<const float4*>(static_cast<uint8_t*>(ws) + s.off_tab2) : nullptr;
     // The cos/sin table kernel runs just before (same condition: tensor-core path, tokens > 0).
     if (launch_k(kern, unsigned(s.ps.grid), la::st::THREADS, la::st::SMEM_BYTES, st, true, tk, tv, s.ps, rope,
-                 tab, tab2, partial))
+                 tab, tab2, static_cast<const __nv_bfloat16*>(beta), partial))
       return LA_ERR_CUDA;
   } else {
 #define LA_STATE_SIMT(DD, TT)                                                                         \
   la::simt::state_simt_kernel<DD, TT><<<s.ps.grid, la::simt::THREADS, 0, st>>>(                      \
-      static_cast<const TT*>(K), static_cast<const TT*>(V), s.ps, rope, partial)
+      static_cast<const TT*>(K), static_cast<const TT*>(V), static_cast<const TT*>(beta), s.ps, rope, partial)
     if (q.dtype == LA_BF16) {
       if (q.d == 32) LA_STATE_SIMT(32, __nv_bfloat16);
       else if (q.d == 64) LA_STATE_SIMT(64, __nv_bfloat16);
@@ -326,7 +335,7 @@ size_t apply_simt_smem(int d) {
 }
 
 int launch_apply(const PlanSet& s, const la_problem& q, const void* Q, const void* G, const float* S,
-                 const float* z, void* O, void* ws, cudaStream_t st, int* nl) {
+                 const float* z, void* O, void* ws, cudaStream_t st, int* nl, const Gates& gt = Gates()) {
   if (s.pa.total == 0) return LA_OK;
   const Rope rope = make_rope(q);
   if (s.tc) {
@@ -335,7 +344,8 @@ int launch_apply(const PlanSet& s, const la_problem& q, const void* Q, const voi
     if (!make_tmap(&tq, Q, s.pa.BH, s.pa.N) || !make_tmap(&tg, G, s.pa.BH, s.pa.N) ||
         !make_tmap(&to, O, s.pa.BH, s.pa.N))
       return LA_ERR_CUDA;
-    auto kern = standard_bands(q) ? la::ap::apply_tc_kernel<32, 48> : la::ap::apply_tc_kernel<-1, -1>;
+    auto kern = standard_bands(q) ? (gt.rms ? la::ap::apply_tc_kernel<32, 48, true> : la::ap::apply_tc_kernel<32, 48, false>)
+                                  : (gt.rms ? la::ap::apply_tc_kernel<-1, -1, true> : la::ap::apply_tc_kernel<-1, -1, false>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::ap::SMEM_BYTES) != cudaSuccess)
       return LA_ERR_CUDA;
     if (la::ap::SPLIT_REGS) {
@@ -351,7 +361,7 @@ int launch_apply(const PlanSet& s, const la_problem& q, const void* Q, const voi
     if (launch_k(kern, unsigned(s.pa.grid), la::ap::THREADS, la::ap::SMEM_BYTES, st, true, tq, tg, to, s.pa, rope,
                  static_cast<const uint8_t*>(w + s.off_img), reinterpret_cast<const float*>(w + s.off_zimg),
                  reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2),
-                 static_cast<__nv_bfloat16*>(O)))
+                 gt.gamma, gt.norm_eps, static_cast<__nv_bfloat16*>(O)))
       return LA_ERR_CUDA;
   } else {
     const size_t smem = apply_simt_smem(q.d);
@@ -361,7 +371,8 @@ int launch_apply(const PlanSet& s, const la_problem& q, const void* Q, const voi
                              int(smem)) != cudaSuccess)                                                    \
       return LA_ERR_CUDA;                                                                                  \
     la::simt::apply_simt_kernel<DD, TT><<<s.pa.grid, la::simt::THREADS, smem, st>>>(                       \
-        static_cast<const TT*>(Q), static_cast<const TT*>(G), S, z, static_cast<TT*>(O), s.pa, rope);      \
+        static_cast<const TT*>(Q), static_cast<const TT*>(G), S, z, static_cast<TT*>(O), s.pa, rope,       \
+        gt.rms ? 1 : 0, gt.gamma, gt.norm_eps);                                                            \
   } while (0)
     if (q.dtype == LA_BF16) {
       if (q.d == 32) LA_APPLY_SIMT(32, __nv_bfloat16);
@@ -512,12 +523,14 @@ int la_apply(const la_problem* p, const void* Q, const void* G, const float* S, 
 
 static int forward_common(const la_problem* p, const void* Q, const void* K, const void* V, const void* G,
                           void* O, float* S_incl, float* z_incl, void* ws, size_t ws_bytes, cudaStream_t stream,
-                          cudaEvent_t* marks = nullptr, int nmarks = 0) {
+                          cudaEvent_t* marks = nullptr, int nmarks = 0, const Gates& gt = Gates()) {
   int rc;
   const bool has_tok = elems(*p) > 0;
   if ((rc = check_ptr(Q, has_tok)) || (rc = check_ptr(K, has_tok)) || (rc = check_ptr(V, has_tok)) ||
       (rc = check_ptr(G, has_tok)) || (rc = check_ptr(O, has_tok)))
     return rc;
+  if (gt.beta && !aligned16(gt.beta)) return LA_ERR_ALIGN;
+  if (gt.gamma && !aligned16(gt.gamma)) return LA_ERR_ALIGN;
   if (S_incl && !aligned16(S_incl)) return LA_ERR_ALIGN;
   if (z_incl && !aligned16(z_incl)) return LA_ERR_ALIGN;
   if ((S_incl == nullptr) != (z_incl == nullptr)) return LA_ERR_NULL;
@@ -543,7 +556,7 @@ static int forward_common(const la_problem* p, const void* Q, const void* K, con
   if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
   if (nl) mark(nl);
   const int b0 = nl;
-  if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
+  if ((rc = launch_state(s, *p, K, V, ws, stream, &nl, gt.beta))) return rc;
   if (nl != b0) mark(nl);
   const int before = nl;
   if ((rc = launch_combine(s, *p, ws, nullptr, nullptr, need_fp32 ? st_S : nullptr, need_fp32 ? st_z : nullptr,
@@ -552,7 +565,7 @@ static int forward_common(const la_problem* p, const void* Q, const void* K, con
   if (nl != before) mark(nl);
   if (has_tok) {
     const int b2 = nl;
-    if ((rc = launch_apply(s, *p, Q, G, st_S, st_z, O, ws, stream, &nl))) return rc;
+    if ((rc = launch_apply(s, *p, Q, G, st_S, st_z, O, ws, stream, &nl, gt))) return rc;
     if (nl != b2) mark(nl);
   }
   g_last_launches = nl;
@@ -575,14 +588,40 @@ int la_forward_blockcausal(const la_problem* p, const void* Q, const void* K, co
   return forward_common(p, Q, K, V, G, O, S_incl, z_incl, ws, ws_bytes, stream);
 }
 
-int la_forward_marked(const la_problem* p, const void* Q, const void* K, const void* V, const void* G, void* O,
-                      float* S_incl, float* z_incl, void* ws, size_t ws_bytes, cudaStream_t stream, cudaEvent_t* marks,
-                      int nmarks) {
+// Checks and converts la_gates (NULL: no optional terms).
+static int read_gates(const la_gates* gates, Gates* gt) {
+  *gt = Gates();
+  if (!gates) return LA_OK;
+  if (gates->rms_norm != 0 && gates->rms_norm != 1) return LA_ERR_UNSUPPORTED;
+  if (gates->rms_norm && (!std::isfinite(gates->norm_eps) || gates->norm_eps < 0.f)) return LA_ERR_SHAPE;
+  gt->beta = gates->beta;
+  gt->rms = gates->rms_norm == 1;
+  gt->gamma = gt->rms ? gates->gamma : nullptr;
+  gt->norm_eps = gates->norm_eps;
+  return LA_OK;
+}
+
+int la_forward_gated(const la_problem* p, const la_gates* gates, const void* Q, const void* K, const void* V,
+                     const void* G, void* O, float* S_incl, float* z_incl, void* ws, size_t ws_bytes,
+                     cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  if (p->block_frames == 0 && (S_incl || z_incl)) return LA_ERR_SHAPE;
+  Gates gt;
+  if ((rc = read_gates(gates, &gt))) return rc;
+  return forward_common(p, Q, K, V, G, O, S_incl, z_incl, ws, ws_bytes, stream, nullptr, 0, gt);
+}
+
+int la_forward_marked(const la_problem* p, const la_gates* gates, const void* Q, const void* K, const void* V,
+                      const void* G, void* O, float* S_incl, float* z_incl, void* ws, size_t ws_bytes,
+                      cudaStream_t stream, cudaEvent_t* marks, int nmarks) {
   int rc = validate(p);
   if (rc) return rc;
   if (nmarks < 0 || (nmarks > 0 && !marks)) return LA_ERR_NULL;
   if (p->block_frames == 0 && (S_incl || z_incl)) return LA_ERR_SHAPE;
-  return forward_common(p, Q, K, V, G, O, S_incl, z_incl, ws, ws_bytes, stream, marks, nmarks);
+  Gates gt;
+  if ((rc = read_gates(gates, &gt))) return rc;
+  return forward_common(p, Q, K, V, G, O, S_incl, z_incl, ws, ws_bytes, stream, marks, nmarks, gt);
 }
 
 const char* la_status_string(int status) {

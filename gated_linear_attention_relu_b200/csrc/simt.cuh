@@ -43,7 +43,7 @@ __device__ __forceinline__ uint32_t axis_pos(int band, uint32_t t, uint32_t h, u
 // State: per CTA, partial S (D x D) and z (D) for every unit it touches, into partial slots.
 template <int D, typename T>
 __global__ void __launch_bounds__(THREADS)
-state_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const Plan p,
+state_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ beta, const Plan p,
                   const __grid_constant__ Rope rope, float* __restrict__ partial) {
   constexpr int R = D / 16;  // each thread owns an R x R block of S
   __shared__ float kr[TS][D];
@@ -83,10 +83,12 @@ state_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const Plan p
       rope_cs(static_cast<double>(axis_pos(rope.band[pi], pt, ph, pw)) +
                   (rope.band[pi] == 0 ? static_cast<double>(rope.t_offset) : 0.0),
               rope.theta_d[pi], cs, sn);
+      // Write gate (optional): scales the rotated key only; z keeps ReLU(k).
+      const float b = (beta && n < ti.n_end) ? to_f(beta[ti.bh * p.N + n]) : 1.f;
       kp[r][2 * pi] = x0;
       kp[r][2 * pi + 1] = x1;
-      kr[r][2 * pi] = x0 * cs - x1 * sn;
-      kr[r][2 * pi + 1] = x0 * sn + x1 * cs;
+      kr[r][2 * pi] = (x0 * cs - x1 * sn) * b;
+      kr[r][2 * pi + 1] = (x0 * sn + x1 * cs) * b;
       vs[r][2 * pi] = v0;
       vs[r][2 * pi + 1] = v1;
     }
@@ -130,7 +132,7 @@ template <int D, typename T>
 __global__ void __launch_bounds__(THREADS)
 apply_simt_kernel(const T* __restrict__ Q, const T* __restrict__ G, const float* __restrict__ S,
                   const float* __restrict__ z, T* __restrict__ O, const Plan p,
-                  const __grid_constant__ Rope rope) {
+                  const __grid_constant__ Rope rope, int rms, const float* __restrict__ gamma, float norm_eps) {
   extern __shared__ float sm[];
   float* Ss = sm;                   // [D][D]
   float* zs = Ss + D * D;           // [D]
@@ -192,6 +194,17 @@ apply_simt_kernel(const T* __restrict__ Q, const T* __restrict__ G, const float*
       for (int j = 0; j < CW; ++j) ot[r_own * (D + 1) + cg * CW + j] = acc[j];
     }
     __syncthreads();
+    if (rms) {
+      // RMSNorm of y = num / den over the row's D channels, before the gate: fold
+      // 1 / sqrt(mean(y^2) + norm_eps) into the row's scale.
+      if (tid < TS) {
+        float ss = 0.f;
+        for (int v = 0; v < D; ++v) ss = fmaf(ot[tid * (D + 1) + v], ot[tid * (D + 1) + v], ss);
+        const float iv = inv[tid];
+        inv[tid] = iv * rsqrtf(iv * iv * ss / static_cast<float>(D) + norm_eps);
+      }
+      __syncthreads();
+    }
     const T* gb = G + (ti.bh * p.N) * D;
     T* ob = O + (ti.bh * p.N) * D;
     for (int e = tid; e < TS * D; e += THREADS) {
@@ -200,7 +213,8 @@ apply_simt_kernel(const T* __restrict__ Q, const T* __restrict__ G, const float*
       if (n < ti.n_end) {
         const float gv = to_f(gb[n * D + v]);
         const float sig = 1.0f / (1.0f + expf(-gv));
-        ob[n * D + v] = from_f<T>(ot[r * (D + 1) + v] * inv[r] * sig);
+        const float gm = (rms && gamma) ? gamma[v] : 1.f;
+        ob[n * D + v] = from_f<T>(ot[r * (D + 1) + v] * inv[r] * gm * sig);
       }
     }
   }

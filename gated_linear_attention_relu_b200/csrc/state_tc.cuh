@@ -75,11 +75,14 @@ static_assert(sizeof(Bars) <= 512, "barrier block too large");
 static_assert(TILE % 16 == 0 && TILE <= 256 && GROUP_ROWS % 8 == 0 && GROUP_ROWS * TGROUPS == TILE, "tile shape");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-template <int DT, int DH>
+// BETA: each token's rotated key is scaled by its write gate beta_n before the contraction
+// (SANA-Video 2.0, Eq. (1): S = sum_n v_n (beta_n k_n^r)^T); z stays un-gated.
+template <int DT, int DH, bool BETA>
 __global__ void __launch_bounds__(THREADS, 1)
 state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const Plan p, const __grid_constant__ Rope rope, const float2* __restrict__ tab,
-                const float4* __restrict__ tab2, float* __restrict__ partial) {
+                const float4* __restrict__ tab2, const __nv_bfloat16* __restrict__ beta,
+                float* __restrict__ partial) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
@@ -245,7 +248,8 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const uint32_t n_end = static_cast<uint32_t>(ti.n_end);
       // One 8-channel chunk of one row: ReLU (rows past the unit's end zeroed by `keep`), RoPE with
       // the chunk's cos/sin, z, written back in place.
-      auto item = [&](uint32_t addr, uint32_t keep, uint32_t pt, uint32_t ph_, uint32_t pw) {
+      const __nv_bfloat16* beta_h = BETA ? beta + ti.bh * p.N : nullptr;
+      auto item = [&](uint32_t addr, uint32_t keep, uint32_t n, uint32_t pt, uint32_t ph_, uint32_t pw) {
         const uint4 raw = lds128(addr);
         float2 cs[4];
         if constexpr (UNIFORM) {
@@ -262,6 +266,12 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             const uint32_t pos = bd[q] == 0 ? pt : (bd[q] == 1 ? ph_ : pw);
             cs[q] = __ldg(tab + tix[q] + pos);
           }
+        }
+        if constexpr (BETA) {
+          // The gate scales the rotated key: fold it into this row's cos/sin.
+          const float b = __bfloat162float(beta_h[n]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) cs[q] = make_float2(cs[q].x * b, cs[q].y * b);
         }
         const uint32_t w[4] = {relu_bf16x2(raw.x) & keep, relu_bf16x2(raw.y) & keep,
                                relu_bf16x2(raw.z) & keep, relu_bf16x2(raw.w) & keep};
@@ -282,7 +292,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         token_pos(p, n0, pt, ph_, pw);
 #pragma unroll 4
         for (int j = 0; j < GROUP_ROWS / 8; ++j) {
-          item(base + static_cast<uint32_t>(j * 8 * 128), 0xffffffffu, pt, ph_, pw);
+          item(base + static_cast<uint32_t>(j * 8 * 128), 0xffffffffu, n0 + 8 * j, pt, ph_, pw);
           pw += 8;
           const bool wrap = pw >= Wd;
           pw = wrap ? pw - Wd : pw;
@@ -297,9 +307,10 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 #pragma unroll 4
         for (int j = 0; j < GROUP_ROWS / 8; ++j) {
           const uint32_t n = n0 + 8 * j;
+          const uint32_t nc = n < N ? n : N - 1;
           uint32_t pt, ph_, pw;
-          token_pos(p, n < N ? n : N - 1, pt, ph_, pw);
-          item(base + static_cast<uint32_t>(j * 8 * 128), n < n_end ? 0xffffffffu : 0u, pt, ph_, pw);
+          token_pos(p, nc, pt, ph_, pw);
+          item(base + static_cast<uint32_t>(j * 8 * 128), n < n_end ? 0xffffffffu : 0u, nc, pt, ph_, pw);
         }
       }
       fence_proxy_async_smem();

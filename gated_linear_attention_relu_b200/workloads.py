@@ -147,6 +147,20 @@ def generate(w: Workload, device="cpu", seed: Optional[int] = None,
     return tuple(out)
 
 
+
+def generate_gates(w: Workload, device="cpu", seed: Optional[int] = None):
+    """Draw the optional inputs of the full gated form for workload ``w``: the write gate beta
+    [B, H, N] uniform in [0, 1) (rounded to ``w.dtype``) and an RMSNorm weight gamma [d] fp32,
+    1 + 0.1 N(0, 1).  Seeded with ``w.seed + 7`` (or ``seed``), independent of ``generate``."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed((w.seed + 7) if seed is None else seed)
+    beta = torch.rand((w.B, w.H, w.N), generator=g, device=device, dtype=torch.float32)
+    gamma = 1.0 + 0.1 * torch.randn((w.d,), generator=g, device=device, dtype=torch.float32)
+    return beta.to(_torch_dtype(w.dtype)).contiguous(), gamma.contiguous()
+
+
 def custom(name: str, B: int, H: int, T: int, Hh: int, W: int, d: int = 128,
            bands: Optional[Tuple[int, int, int]] = None, dtype: str = "bf16", seed: int = 7,
            qkv_scale: Optional[float] = None, k_shift: float = 0.0, block_frames: int = 0,

@@ -132,14 +132,37 @@ int la_forward_blockcausal(const la_problem* p, const void* Q, const void* K, co
                            const void* G, void* O, float* S_incl, float* z_incl,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Optional terms of the full gated form (SANA-Video 2.0, Sec. 2, Eq. (1)):
+ *   S = sum_n beta_n phi(K_n)^T V_n            (write gate; z keeps the un-gated ReLU(K_n):
+ *                                               Eq. (1)'s denominator has no beta)
+ *   O_n = RMSNorm((phi(Q_n) S) / (ReLU(Q_n) . z + eps)) * sigmoid(G_n)
+ *   RMSNorm(y) = y / sqrt(mean_c(y_c^2) + norm_eps) * gamma   (over the d channels of a row)
+ * RMSNorm sits before the output gate as in Eq. (1); W_o stays outside the operator. */
+typedef struct {
+  const void* beta;   /* [B,H,N] write gate per token, in the problem's dtype; NULL: beta = 1 */
+  const float* gamma; /* [d] fp32 RMSNorm weight (shared by all heads); NULL: gamma = 1 */
+  float norm_eps;     /* RMSNorm epsilon (finite, >= 0), e.g. 1e-6; used when rms_norm = 1 */
+  int32_t rms_norm;   /* 1: apply RMSNorm before the gate; 0: no RMSNorm */
+} la_gates;
+
+/* The whole operator with the optional terms of la_gates: bidirectional if p->block_frames
+ * == 0 (then S_incl and z_incl must be NULL), else block-causal with the same arguments as
+ * la_forward_blockcausal (S_incl / z_incl receive the gated inclusive states when non-NULL).
+ * gates == NULL, or beta == NULL with rms_norm == 0, computes exactly what la_forward_bidir /
+ * la_forward_blockcausal compute.  beta and gamma must be 16-byte aligned when given. */
+int la_forward_gated(const la_problem* p, const la_gates* gates, const void* Q, const void* K,
+                     const void* V, const void* G, void* O, float* S_incl, float* z_incl,
+                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* The whole operator (bidirectional if p->block_frames == 0, else block-causal, with the
- * same arguments as la_forward_bidir / la_forward_blockcausal) with timing marks: records
- * marks[0] on `stream` before the first kernel and marks[i] right after the i-th kernel it
- * queues, for every i < nmarks.  The events are created and owned by the caller.  Used to time
- * the individual kernels of one forward pass with CUDA events. */
-int la_forward_marked(const la_problem* p, const void* Q, const void* K, const void* V,
-                      const void* G, void* O, float* S_incl, float* z_incl, void* workspace,
-                      size_t workspace_bytes, cudaStream_t stream, cudaEvent_t* marks, int nmarks);
+ * same arguments as la_forward_gated; gates may be NULL) with timing marks: records marks[0]
+ * on `stream` before the first kernel and marks[i] right after the i-th kernel it queues, for
+ * every i < nmarks.  The events are created and owned by the caller.  Used to time the
+ * individual kernels of one forward pass with CUDA events. */
+int la_forward_marked(const la_problem* p, const la_gates* gates, const void* Q, const void* K,
+                      const void* V, const void* G, void* O, float* S_incl, float* z_incl,
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                      cudaEvent_t* marks, int nmarks);
 
 /* Bytes of the library's fixed device scratch used by la_forward_bidir_static(). */
 #define LA_STATIC_WORKSPACE_BYTES (32u << 20)

@@ -12,9 +12,12 @@ What it computes, per (batch, head), written out as plainly as possible:
   numerator; the denominator uses the un-rotated ReLU features.
 * State, normaliser, gate -- "SANA-Video 2.0: Hybrid Linear Attention with
   Attention Residuals for Efficient Video Generation", Sec. 2, Eq. (1):
-  S = sum_n k_n^r v_n^T, o_j = (q_j^r S) / (sum_n phi(k_n).phi(q_j) + eps)
-  * sigmoid(g_j), with the write gate beta fixed to 1 and RMSNorm / W_o left
-  out (they sit outside this operator).
+  S = sum_n beta_n k_n^r v_n^T, o_j = RMSNorm((q_j^r S) / (sum_n phi(k_n).phi(q_j)
+  + eps)) * sigmoid(g_j).  By default beta = 1 and there is no RMSNorm (the
+  operator's main form); both are optional arguments (``beta`` per token,
+  ``rms = (gamma, norm_eps)``).  beta scales only the state: the denominator of
+  Eq. (1) has none.  RMSNorm sits before the gate, as in Eq. (1) of that page
+  (the page's other rendering puts it after the gate); W_o is outside.
 * Block-causal mode -- "SANA-Video" Sec. 3.4 (causal linear attention with a
   constant-memory cache, and Algorithm 1's per-block cache update): a token
   in block b reads the sum of the states of blocks 0..b, its own block
@@ -37,7 +40,7 @@ import numpy as np
 __all__ = [
     "band_frequencies", "grid_positions", "relu", "sigmoid", "rope3d",
     "head_state", "head_apply", "forward_positions", "forward_bidir",
-    "block_of_tokens", "block_states", "forward_blockcausal", "forward_brute",
+    "block_of_tokens", "block_states", "forward_blockcausal", "forward_brute", "rms_norm",
 ]
 
 
@@ -88,33 +91,49 @@ def rope3d(x: np.ndarray, pos: np.ndarray, bands, base: float) -> np.ndarray:
     return y
 
 
-def head_state(k: np.ndarray, v: np.ndarray, pos: np.ndarray, bands, base: float):
-    """S = sum_n RoPE(ReLU(k_n))^T v_n (d x d) and z = sum_n ReLU(k_n) (d) over the given tokens."""
+def head_state(k: np.ndarray, v: np.ndarray, pos: np.ndarray, bands, base: float, beta=None):
+    """S = sum_n beta_n RoPE(ReLU(k_n))^T v_n (d x d) and z = sum_n ReLU(k_n) (d) over the given
+    tokens (beta = 1 when None; z is never gated)."""
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     kp = relu(k)
     kr = rope3d(kp, pos, bands, base)
+    if beta is not None:
+        kr = kr * np.asarray(beta, dtype=np.float64)[:, None]
     S = kr.T @ v
     z = kp.sum(axis=0)
     return S, z
 
 
+def rms_norm(y: np.ndarray, gamma, norm_eps: float) -> np.ndarray:
+    """Row-wise RMSNorm over the channels: y / sqrt(mean(y^2) + norm_eps) * gamma (gamma = 1 if None)."""
+    y = np.asarray(y, dtype=np.float64)
+    out = y / np.sqrt(np.mean(y * y, axis=-1, keepdims=True) + float(norm_eps))
+    if gamma is not None:
+        out = out * np.asarray(gamma, dtype=np.float64)
+    return out
+
+
 def head_apply(q: np.ndarray, g: np.ndarray, S: np.ndarray, z: np.ndarray, pos: np.ndarray,
-               bands, base: float, eps: float) -> np.ndarray:
-    """o_n = (RoPE(ReLU(q_n)) S) / (ReLU(q_n) . z + eps) * sigmoid(g_n)."""
+               bands, base: float, eps: float, rms=None) -> np.ndarray:
+    """o_n = (RoPE(ReLU(q_n)) S) / (ReLU(q_n) . z + eps) * sigmoid(g_n); with ``rms = (gamma,
+    norm_eps)`` the quotient is RMS-normalised before the gate."""
     q = np.asarray(q, dtype=np.float64)
     g = np.asarray(g, dtype=np.float64)
     qp = relu(q)
     qr = rope3d(qp, pos, bands, base)
     num = qr @ S
     den = qp @ z + float(eps)
-    return num / den[:, None] * sigmoid(g)
+    y = num / den[:, None]
+    if rms is not None:
+        y = rms_norm(y, rms[0], rms[1])
+    return y * sigmoid(g)
 
 
-def forward_positions(q, k, v, g, pos, bands, base, eps):
+def forward_positions(q, k, v, g, pos, bands, base, eps, beta=None, rms=None):
     """Bidirectional output of one head whose tokens sit at explicit positions ``pos``."""
-    S, z = head_state(k, v, pos, bands, base)
-    return head_apply(q, g, S, z, pos, bands, base, eps)
+    S, z = head_state(k, v, pos, bands, base, beta)
+    return head_apply(q, g, S, z, pos, bands, base, eps, rms)
 
 
 def _heads(x):
@@ -123,8 +142,8 @@ def _heads(x):
     return x.reshape(B * H, N, d)
 
 
-def forward_bidir(Q, K, V, G, grid, bands, base=10000.0, eps=1e-6, return_state=False):
-    """Bidirectional mixer over [B, H, N, d] inputs on a (T, Hh, W) latent grid."""
+def forward_bidir(Q, K, V, G, grid, bands, base=10000.0, eps=1e-6, return_state=False, beta=None, rms=None):
+    """Bidirectional mixer over [B, H, N, d] inputs on a (T, Hh, W) latent grid (``beta``: [B, H, N])."""
     T, Hh, W = grid
     pos = grid_positions(T, Hh, W)
     B, H, N, d = np.shape(Q)
@@ -133,9 +152,10 @@ def forward_bidir(Q, K, V, G, grid, bands, base=10000.0, eps=1e-6, return_state=
     O = np.empty((B * H, N, d))
     Ss = np.empty((B * H, d, d))
     zs = np.empty((B * H, d))
+    bt = None if beta is None else np.asarray(beta, dtype=np.float64).reshape(B * H, N)
     for u in range(B * H):
-        Ss[u], zs[u] = head_state(k[u], v[u], pos, bands, base)
-        O[u] = head_apply(q[u], g[u], Ss[u], zs[u], pos, bands, base, eps)
+        Ss[u], zs[u] = head_state(k[u], v[u], pos, bands, base, None if bt is None else bt[u])
+        O[u] = head_apply(q[u], g[u], Ss[u], zs[u], pos, bands, base, eps, rms)
     O = O.reshape(B, H, N, d)
     if return_state:
         return O, Ss.reshape(B, H, d, d), zs.reshape(B, H, d)
@@ -147,7 +167,7 @@ def block_of_tokens(pos: np.ndarray, block_frames: int) -> np.ndarray:
     return pos[:, 0] // int(block_frames)
 
 
-def block_states(k, v, pos, bands, base, block_frames):
+def block_states(k, v, pos, bands, base, block_frames, beta=None):
     """Per-block states (not prefixed) of one head: S_b, z_b for b = 0..nblk-1."""
     blk = block_of_tokens(pos, block_frames)
     nblk = int(blk.max()) + 1 if len(blk) else 0
@@ -156,12 +176,12 @@ def block_states(k, v, pos, bands, base, block_frames):
     zb = np.zeros((nblk, d))
     for b in range(nblk):
         sel = blk == b
-        Sb[b], zb[b] = head_state(k[sel], v[sel], pos[sel], bands, base)
+        Sb[b], zb[b] = head_state(k[sel], v[sel], pos[sel], bands, base, None if beta is None else beta[sel])
     return Sb, zb
 
 
 def forward_blockcausal(Q, K, V, G, grid, bands, base=10000.0, eps=1e-6, block_frames=1,
-                        return_state=False):
+                        return_state=False, beta=None, rms=None):
     """Block-causal mixer: a token of block b reads sum_{b' <= b} (S_b', z_b').
 
     Returns O and, if asked, the inclusive per-block states [B, H, nblk, d, d] and
@@ -176,8 +196,9 @@ def forward_blockcausal(Q, K, V, G, grid, bands, base=10000.0, eps=1e-6, block_f
     O = np.empty((B * H, N, d))
     Sinc = np.empty((B * H, nblk, d, d))
     zinc = np.empty((B * H, nblk, d))
+    bt = None if beta is None else np.asarray(beta, dtype=np.float64).reshape(B * H, N)
     for u in range(B * H):
-        Sb, zb = block_states(k[u], v[u], pos, bands, base, block_frames)
+        Sb, zb = block_states(k[u], v[u], pos, bands, base, block_frames, None if bt is None else bt[u])
         S_run = np.zeros((d, d))
         z_run = np.zeros(d)
         for b in range(nblk):
@@ -185,15 +206,16 @@ def forward_blockcausal(Q, K, V, G, grid, bands, base=10000.0, eps=1e-6, block_f
             z_run = z_run + zb[b]
             Sinc[u, b], zinc[u, b] = S_run, z_run
             sel = blk == b
-            O[u][sel] = head_apply(q[u][sel], g[u][sel], S_run, z_run, pos[sel], bands, base, eps)
+            O[u][sel] = head_apply(q[u][sel], g[u][sel], S_run, z_run, pos[sel], bands, base, eps, rms)
     O = O.reshape(B, H, N, d)
     if return_state:
         return O, Sinc.reshape(B, H, nblk, d, d), zinc.reshape(B, H, nblk, d)
     return O
 
 
-def forward_brute(q, k, v, g, pos, bands, base, eps, visible=None):
-    """O(N^2) form of one head: o_n = sum_m (q_n^r . k_m^r) v_m / (sum_m q_n^+ . k_m^+ + eps) * sigmoid(g_n).
+def forward_brute(q, k, v, g, pos, bands, base, eps, visible=None, beta=None, rms=None):
+    """O(N^2) form of one head: o_n = sum_m beta_m (q_n^r . k_m^r) v_m / (sum_m q_n^+ . k_m^+ + eps)
+    * sigmoid(g_n) (the quotient RMS-normalised first when ``rms = (gamma, norm_eps)``).
 
     ``visible[n, m]`` (bool) restricts which keys token n reads; None means all.
     This is the pair-wise form the linear one is the associative rewrite of.
@@ -209,6 +231,11 @@ def forward_brute(q, k, v, g, pos, bands, base, eps, visible=None):
     for n in range(N):
         m = np.arange(N) if visible is None else np.nonzero(visible[n])[0]
         a = kr[m] @ qr[n]  # rotated similarities
+        if beta is not None:
+            a = a * np.asarray(beta, dtype=np.float64)[m]
         b = kp[m] @ qp[n]  # un-rotated similarities
-        out[n] = (a @ v[m]) / (b.sum() + float(eps)) * sigmoid(g[n])
+        y = (a @ v[m]) / (b.sum() + float(eps))
+        if rms is not None:
+            y = rms_norm(y, rms[0], rms[1])
+        out[n] = y * sigmoid(g[n])
     return out

@@ -23,16 +23,17 @@ def rel_err(got: np.ndarray, ref: np.ndarray) -> float:
     return float(np.max(np.abs(got - ref))) / (scale if scale > 0 else 1.0)
 
 
-def oracle_head(w, q, k, v, g, tokens=None):
+def oracle_head(w, q, k, v, g, tokens=None, beta=None, rms=None):
     """Oracle output rows (all, or the listed token indices) and the per-block inclusive states
-    of one head.  q, k, v, g: (N, d) float64 arrays of that head."""
+    of one head.  q, k, v, g: (N, d) float64 arrays of that head; ``beta`` (N,) and ``rms``
+    (gamma, norm_eps) are the optional terms of the full gated form."""
     pos = orc.grid_positions(w.T, w.Hh, w.W)
     if w.block_frames <= 0:
-        S, z = orc.head_state(k, v, pos, w.bands, w.rope_base)
+        S, z = orc.head_state(k, v, pos, w.bands, w.rope_base, beta)
         Sinc, zinc = S[None], z[None]
         blk = np.zeros(w.N, dtype=np.int64)
     else:
-        Sb, zb = orc.block_states(k, v, pos, w.bands, w.rope_base, w.block_frames)
+        Sb, zb = orc.block_states(k, v, pos, w.bands, w.rope_base, w.block_frames, beta)
         Sinc, zinc = np.cumsum(Sb, axis=0), np.cumsum(zb, axis=0)
         blk = orc.block_of_tokens(pos, w.block_frames)
     idx = np.arange(w.N) if tokens is None else np.asarray(tokens)
@@ -40,7 +41,8 @@ def oracle_head(w, q, k, v, g, tokens=None):
     for b in np.unique(blk[idx]):
         sel = blk[idx] == b
         rows = idx[sel]
-        out[sel] = orc.head_apply(q[rows], g[rows], Sinc[b], zinc[b], pos[rows], w.bands, w.rope_base, w.eps)
+        out[sel] = orc.head_apply(q[rows], g[rows], Sinc[b], zinc[b], pos[rows], w.bands, w.rope_base, w.eps,
+                                  rms)
     return out, Sinc, zinc
 
 

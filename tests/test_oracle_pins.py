@@ -362,3 +362,79 @@ def test_streaming_cache_restatement_equals_block_causal_form():
     sl = slice(6 * Hh * W, N)
     bad = orc.head_apply(q[0, 0, sl], g[0, 0, sl], S, z, pos_local, bands, 10000.0, 1e-6)
     assert not np.allclose(bad, ref[sl], rtol=1e-3)
+
+
+# ----------------------------------------------------------------- full Eq. (1): write gate, RMSNorm
+
+def _rand_head(rng, N, d):
+    return [rng.standard_normal((N, d)) for _ in range(4)]
+
+
+def test_gated_linear_form_equals_brute_form():
+    """beta and RMSNorm in the linear form agree with the pair-wise form (SANA-Video 2.0, Eq. (1))."""
+    rng = np.random.default_rng(21)
+    T, Hh, W, d, bands = 3, 2, 5, 16, (4, 6, 6)
+    pos = orc.grid_positions(T, Hh, W)
+    q, k, v, g = _rand_head(rng, T * Hh * W, d)
+    beta = rng.uniform(0.0, 1.0, T * Hh * W)
+    gamma = 1.0 + 0.1 * rng.standard_normal(d)
+    for b_, rms in ((beta, None), (None, (gamma, 1e-6)), (beta, (gamma, 1e-6)), (beta, (None, 0.0))):
+        lin = orc.forward_positions(q, k, v, g, pos, bands, 10000.0, 1e-6, beta=b_, rms=rms)
+        bru = orc.forward_brute(q, k, v, g, pos, bands, 10000.0, 1e-6, beta=b_, rms=rms)
+        assert np.allclose(lin, bru, rtol=1e-11, atol=1e-13)
+
+
+def test_write_gate_two_token_closed_form():
+    """Two tokens at one position, q = k_0 = k_1 = e_0, beta = (1, 0), g = 0: the gate removes
+    token 1 from the numerator only, so o = v_0 / (2 + eps) / 2.  (Gating the denominator too,
+    a plausible misreading, would give v_0 / (1 + eps) / 2.)"""
+    d, bands = 8, (2, 2, 4)
+    e0 = np.zeros(d); e0[0] = 1.0
+    q = np.array([e0, e0]); k = np.array([e0, e0])
+    v = np.array([[1.0, -2.0, 3.0, 0.5, 0.0, 1.0, 2.0, -1.0], [5.0, 5.0, 5.0, 5.0, 5.0, 5.0, 5.0, 5.0]])
+    g = np.zeros((2, d))
+    pos = np.array([[1, 2, 3], [1, 2, 3]])
+    out = orc.forward_positions(q, k, v, g, pos, bands, 10000.0, 1e-6, beta=np.array([1.0, 0.0]))
+    assert np.allclose(out[0], v[0] / (2.0 + 1e-6) / 2.0, rtol=1e-13)
+    assert not np.allclose(out[0], v[0] / (1.0 + 1e-6) / 2.0, rtol=1e-3)
+    # beta = 1 everywhere is the plain operator
+    plain = orc.forward_positions(q, k, v, g, pos, bands, 10000.0, 1e-6)
+    ones = orc.forward_positions(q, k, v, g, pos, bands, 10000.0, 1e-6, beta=np.ones(2))
+    assert np.array_equal(plain, ones)
+
+
+def test_rms_norm_single_token_closed_form():
+    """N = 1: y = a v with a = s / (s + eps); with norm_eps = 0 the factor a cancels and
+    RMSNorm(y) = v / sqrt(mean(v^2)) * gamma.  v = (3, 4, 0, ...) over d = 8 has mean(v^2) = 25/8."""
+    d, bands = 8, (2, 2, 4)
+    q = np.zeros((1, d)); q[0, 0] = 2.0
+    k = np.zeros((1, d)); k[0, 0] = 3.0
+    v = np.zeros((1, d)); v[0, 0], v[0, 1] = 3.0, 4.0
+    g = np.zeros((1, d))
+    gamma = np.array([1.0, 2.0, 1.0, 1.0, 1.0, 1.0, 1.0, 1.0])
+    out = orc.forward_positions(q, k, v, g, np.array([[4, 0, 7]]), bands, 10000.0, 1e-6, rms=(gamma, 0.0))
+    expect = np.zeros(d)
+    expect[0] = 3.0 / np.sqrt(25.0 / 8.0) * 0.5
+    expect[1] = 8.0 / np.sqrt(25.0 / 8.0) * 0.5
+    assert np.allclose(out[0], expect, rtol=1e-12, atol=1e-15)
+
+
+def test_rms_norm_invariances_and_placement():
+    rng = np.random.default_rng(23)
+    T, Hh, W, d, bands = 2, 3, 4, 16, (4, 6, 6)
+    pos = orc.grid_positions(T, Hh, W)
+    q, k, v, g = _rand_head(rng, T * Hh * W, d)
+    rms = (None, 0.0)
+    base = orc.forward_positions(q, k, v, g, pos, bands, 10000.0, 1e-6, rms=rms)
+    # scale of V (and of the write gate) drops out of a normalised row
+    assert np.allclose(orc.forward_positions(q, k, 7.5 * v, g, pos, bands, 10000.0, 1e-6, rms=rms), base,
+                       rtol=1e-12)
+    assert np.allclose(orc.forward_positions(q, k, v, g, pos, bands, 10000.0, 1e-6, beta=np.full(len(q), 0.3),
+                                             rms=rms), base, rtol=1e-12)
+    # every row of O / sigmoid(G) has unit RMS (gamma = 1, norm_eps = 0)
+    y = base / orc.sigmoid(g)
+    assert np.allclose(np.sqrt(np.mean(y * y, axis=1)), 1.0, rtol=1e-12)
+    # placement: normalising after the gate (the other rendering of Eq. (1)) is a different result
+    plain = orc.forward_positions(q, k, v, g, pos, bands, 10000.0, 1e-6)
+    after = orc.rms_norm(plain, None, 0.0)
+    assert not np.allclose(after, base, rtol=1e-3)
