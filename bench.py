@@ -46,8 +46,8 @@ def parse():
     ap.add_argument("--gated", action="store_true",
                     help="full gated form: write gate beta [B,H,N] and RMSNorm before the output gate")
     ap.add_argument("--stream", action="store_true",
-                    help="block-causal workloads: one call pair per block (la_state_update + la_apply "
-                         "on a carried cache), as a block-autoregressive generator runs")
+                    help="block-causal workloads: one la_block_step call per block on a carried cache, "
+                         "as a block-autoregressive generator runs")
     return ap.parse_args()
 
 
@@ -260,9 +260,7 @@ def main():
             z_c.zero_()
             n = 0
             for pb, (qb, kb, vb, gb), ob in blocks:
-                la.state_update(pb, kb, vb, S_c, z_c, ws=ws_s)
-                n += la.last_launch_count()
-                la.apply(pb, qb, gb, S_c, z_c, O=ob, ws=ws_s)
+                la.block_step(pb, qb, kb, vb, gb, S_c, z_c, O=ob, ws=ws_s)
                 n += la.last_launch_count()
             counter["launches"] = n
     else:
@@ -366,7 +364,7 @@ def main():
     if args.gated:
         config["gated"] = "write gate beta [B,H,N] + RMSNorm (gamma [d]) before the output gate"
     if args.stream:
-        config["stream"] = f"{len(blocks)} blocks, la_state_update + la_apply per block on a carried cache"
+        config["stream"] = f"{len(blocks)} blocks, one la_block_step per block on a carried cache"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",

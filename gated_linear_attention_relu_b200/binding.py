@@ -26,7 +26,7 @@ EXPORTS = [
     "la_workspace_bytes", "la_workspace_bytes_for", "la_state_reduce", "la_state_scan", "la_apply",
     "la_forward_bidir", "la_forward_blockcausal", "la_status_string", "la_device_error",
     "la_last_launch_count", "la_forward_marked", "la_selftest_host", "la_forward_bidir_static",
-    "la_state_update", "la_forward_gated",
+    "la_state_update", "la_forward_gated", "la_block_step",
 ]
 
 
@@ -79,6 +79,7 @@ def load(path: Optional[str] = None):
         "la_state_reduce": (ctypes.c_int, [P, vp, vp, vp, vp, vp, sz, vp]),
         "la_state_scan": (ctypes.c_int, [P, vp, vp, vp]),
         "la_state_update": (ctypes.c_int, [P, vp, vp, vp, vp, vp, sz, vp]),
+        "la_block_step": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_gated": (ctypes.c_int, [P, ctypes.POINTER(LaGates), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_apply": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_bidir": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -214,6 +215,24 @@ def state_update(p: Problem, K, V, S, z, ws=None, stream=None):
     _check(lib.la_state_update(ctypes.byref(cp), _ptr(K), _ptr(V), _ptr(S), _ptr(z), _ptr(ws), nbytes,
                                _stream(stream)), "la_state_update")
     return S, z
+
+
+def block_step(p: Problem, Q, K, V, G, S, z, O=None, ws=None, stream=None):
+    """One block of block-autoregressive generation: fold the block into the carried cache
+    (S [B,H,d,d], z [B,H,d], in place) and return its outputs against the updated cache."""
+    import torch
+
+    lib = load()
+    if O is None:
+        O = torch.empty_like(Q)
+    if ws is None:
+        ws, nbytes = workspace(p, Q.device)
+    else:
+        nbytes = ws.numel()
+    cp = p.c()
+    _check(lib.la_block_step(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(O), _ptr(S), _ptr(z),
+                             _ptr(ws), nbytes, _stream(stream)), "la_block_step")
+    return O
 
 
 def state_scan(p: Problem, S, z, stream=None):

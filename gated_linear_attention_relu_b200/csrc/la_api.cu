@@ -463,6 +463,35 @@ int la_state_update(const la_problem* p, const void* K, const void* V, float* S,
   return LA_OK;
 }
 
+int la_block_step(const la_problem* p, const void* Q, const void* K, const void* V, const void* G, void* O,
+                  float* S, float* z, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  if (p->block_frames != 0) return LA_ERR_SHAPE;
+  const bool has_tok = elems(*p) > 0;
+  const bool has_state = state_units(*p) > 0;
+  if ((rc = check_ptr(Q, has_tok)) || (rc = check_ptr(K, has_tok)) || (rc = check_ptr(V, has_tok)) ||
+      (rc = check_ptr(G, has_tok)) || (rc = check_ptr(O, has_tok)) || (rc = check_ptr(S, has_state)) ||
+      (rc = check_ptr(z, has_state)))
+    return rc;
+  if (!has_tok) {
+    g_last_launches = 0;
+    return LA_OK;
+  }
+  int sm = 0;
+  if ((rc = current_sm_count(&sm))) return rc;
+  const PlanSet s = make_plans(*p, sm);
+  if ((rc = check_ws(s, ws, ws_bytes))) return rc;
+  int nl = 0;
+  if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
+  if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
+  // carried + this block -> S, z (and the tensor-core apply's operand image)
+  if ((rc = launch_combine(s, *p, ws, nullptr, nullptr, S, z, s.tc, stream, &nl, true))) return rc;
+  if ((rc = launch_apply(s, *p, Q, G, S, z, O, ws, stream, &nl))) return rc;
+  g_last_launches = nl;
+  return LA_OK;
+}
+
 int la_state_scan(const la_problem* p, float* S, float* z, cudaStream_t stream) {
   int rc = validate(p);
   if (rc) return rc;

@@ -108,6 +108,16 @@ int la_state_reduce(const la_problem* p, const void* K, const void* V, float* S,
 int la_state_update(const la_problem* p, const void* K, const void* V, float* S, float* z,
                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* One step of block-autoregressive generation in one call (SANA-Video Sec. 3.4, Algorithm 1):
+ * folds the block into the carried cache exactly like la_state_update, then computes the
+ * block's outputs against the updated cache exactly like la_apply, with one cos/sin table and
+ * one state image for both (4 kernels).  Same arguments and rules as those two calls:
+ * p->block_frames == 0, p->t0 = the block's first global frame, S [B,H,d,d] and z [B,H,d]
+ * read-modified-written.  Q, K, V, G, O: [B,H,N,d] of the block. */
+int la_block_step(const la_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                  void* O, float* S, float* z, void* workspace, size_t workspace_bytes,
+                  cudaStream_t stream);
+
 /* In-place inclusive prefix over blocks (SANA-Video Sec. 3.4: the cache after block j
  * is the sum of the states of blocks 0..j).  S: [B,H,nblk,d,d], z: [B,H,nblk,d].
  * A no-op in bidirectional mode. */

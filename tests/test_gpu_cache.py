@@ -99,3 +99,27 @@ def test_frame_offset_shifts_positions():
                                     w.bands, w.rope_base, w.eps)
         assert rel_err(to64(O5[0, h]), ref) <= tol_for(w.dtype)
     assert not torch.equal(O5, O0)
+
+
+@pytest.mark.parametrize("w", CASES[:3], ids=lambda w: w.name)
+def test_block_step_matches_two_call_path(w):
+    """la_block_step (one call per block) computes what la_state_update + la_apply compute."""
+    Q, K, V, G = wl.generate(w, "cuda")
+    O_two, caches = _stream_blocks(w, Q, K, V, G)
+    HW = w.Hh * w.W
+    S = torch.zeros((w.B, w.H, w.d, w.d), dtype=torch.float32, device="cuda")
+    z = torch.zeros((w.B, w.H, w.d), dtype=torch.float32, device="cuda")
+    outs = []
+    for t0 in range(0, w.T, w.block_frames):
+        t1 = min(w.T, t0 + w.block_frames)
+        sl = slice(t0 * HW, t1 * HW)
+        pb = la.Problem.from_workload(w, T=t1 - t0, block_frames=0, t0=t0)
+        qb, kb, vb, gb = (x[:, :, sl].contiguous() for x in (Q, K, V, G))
+        outs.append(la.block_step(pb, qb, kb, vb, gb, S, z))
+        assert la.last_launch_count() == (4 if w.d == 128 and w.dtype == "bf16" else 3)
+    O = torch.cat(outs, dim=2)
+    torch.cuda.synchronize()
+    assert la.device_error() == 0
+    # Same kernels, same order of every sum: identical results.
+    assert torch.equal(O, O_two)
+    assert torch.equal(S, caches[-1][0][:, :, 0]) and torch.equal(z, caches[-1][1][:, :, 0])
