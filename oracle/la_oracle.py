@@ -22,6 +22,8 @@ What it computes, per (batch, head), written out as plainly as possible:
   constant-memory cache, and Algorithm 1's per-block cache update): a token
   in block b reads the sum of the states of blocks 0..b, its own block
   included.
+* Token-causal mode -- the same section's causal form, token by token: token n
+  reads the states of tokens 0..n (itself included) in the flattened order.
 
 Readings where the pages are silent (each one is listed in the design notes):
 3D RoPE splits d into consecutive t / h / w bands; pair i of a band of width D
@@ -41,6 +43,7 @@ __all__ = [
     "band_frequencies", "grid_positions", "relu", "sigmoid", "rope3d",
     "head_state", "head_apply", "forward_positions", "forward_bidir",
     "block_of_tokens", "block_states", "forward_blockcausal", "forward_brute", "rms_norm",
+    "tokencausal_rows", "forward_tokencausal",
 ]
 
 
@@ -239,3 +242,49 @@ def forward_brute(q, k, v, g, pos, bands, base, eps, visible=None, beta=None, rm
             y = rms_norm(y, rms[0], rms[1])
         out[n] = y * sigmoid(g[n])
     return out
+
+
+def tokencausal_rows(q, k, v, g, pos, bands, base, eps, rows=None, chunk=1024):
+    """Token-causal output of one head at the listed token indices (all when None):
+    o_n = (RoPE(q_n^+) S_{<=n}) / (q_n^+ . z_{<=n} + eps) * sigmoid(g_n), with
+    S_{<=n} = sum_{m<=n} RoPE(k_m^+)^T v_m and z_{<=n} = sum_{m<=n} k_m^+.
+
+    Walks the tokens in order, carrying (S, z) across chunks of ``chunk`` tokens; inside a chunk
+    the rows up to n are summed explicitly."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    N, d = q.shape
+    want = np.arange(N) if rows is None else np.sort(np.asarray(rows))
+    out = {}
+    S = np.zeros((d, d))
+    z = np.zeros(d)
+    for c0 in range(0, N, chunk):
+        c1 = min(N, c0 + chunk)
+        kp = relu(k[c0:c1])
+        kr = rope3d(kp, pos[c0:c1], bands, base)
+        sel = want[(want >= c0) & (want < c1)]
+        if len(sel):
+            qp = relu(q[sel])
+            qr = rope3d(qp, pos[sel], bands, base)
+            for i, n in enumerate(sel):
+                j = n - c0 + 1  # rows c0..n of this chunk
+                num = qr[i] @ S + (kr[:j] @ qr[i]) @ v[c0:c0 + j]
+                den = qp[i] @ z + (kp[:j] @ qp[i]).sum() + float(eps)
+                out[int(n)] = num / den * sigmoid(g[n])
+        S = S + kr.T @ v[c0:c1]
+        z = z + kp.sum(axis=0)
+    return np.array([out[int(n)] for n in (np.arange(N) if rows is None else np.asarray(rows))])
+
+
+def forward_tokencausal(Q, K, V, G, grid, bands, base=10000.0, eps=1e-6):
+    """Token-causal mixer over [B, H, N, d] inputs on a (T, Hh, W) latent grid."""
+    T, Hh, W = grid
+    pos = grid_positions(T, Hh, W)
+    B, H, N, d = np.shape(Q)
+    q, k, v, g = _heads(Q), _heads(K), _heads(V), _heads(G)
+    O = np.empty((B * H, N, d))
+    for u in range(B * H):
+        O[u] = tokencausal_rows(q[u], k[u], v[u], g[u], pos, bands, base, eps)
+    return O.reshape(B, H, N, d)

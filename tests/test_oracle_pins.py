@@ -438,3 +438,44 @@ def test_rms_norm_invariances_and_placement():
     plain = orc.forward_positions(q, k, v, g, pos, bands, 10000.0, 1e-6)
     after = orc.rms_norm(plain, None, 0.0)
     assert not np.allclose(after, base, rtol=1e-3)
+
+
+# ----------------------------------------------------------------- token-causal form
+
+def test_tokencausal_linear_form_equals_masked_brute_form():
+    rng = np.random.default_rng(31)
+    for T, Hh, W, d, bands, chunk in ((3, 2, 5, 16, (4, 6, 6), 7), (2, 3, 4, 8, (2, 2, 4), 1000)):
+        N = T * Hh * W
+        pos = orc.grid_positions(T, Hh, W)
+        q, k, v, g = (rng.standard_normal((N, d)) for _ in range(4))
+        lin = orc.tokencausal_rows(q, k, v, g, pos, bands, 10000.0, 1e-6, chunk=chunk)
+        mask = np.tril(np.ones((N, N), dtype=bool))
+        bru = orc.forward_brute(q, k, v, g, pos, bands, 10000.0, 1e-6, visible=mask)
+        assert np.allclose(lin, bru, rtol=1e-11, atol=1e-13)
+        # sampled rows agree with the full evaluation
+        rows = [0, 5, N - 1, 13]
+        assert np.allclose(orc.tokencausal_rows(q, k, v, g, pos, bands, 10000.0, 1e-6, rows=rows, chunk=4),
+                           lin[rows], rtol=1e-12)
+
+
+def test_tokencausal_first_last_and_causality():
+    rng = np.random.default_rng(37)
+    T, Hh, W, d, bands = 2, 3, 5, 16, (4, 6, 6)
+    N = T * Hh * W
+    Q, K, V, G = (rng.standard_normal((1, 1, N, d)) for _ in range(4))
+    O = orc.forward_tokencausal(Q, K, V, G, (T, Hh, W), bands)[0, 0]
+    bid = orc.forward_bidir(Q, K, V, G, (T, Hh, W), bands)[0, 0]
+    # the last token sees every token: bidirectional output
+    assert np.allclose(O[-1], bid[-1], rtol=1e-12)
+    # the first token sees only itself: single-token closed form (same position: rotation cancels)
+    qp, kp = np.maximum(Q[0, 0, 0], 0), np.maximum(K[0, 0, 0], 0)
+    s = qp @ kp
+    assert np.allclose(O[0], s / (s + 1e-6) * V[0, 0, 0] / (1 + np.exp(-G[0, 0, 0])), rtol=1e-10)
+    # changing token j changes no output before j
+    j = 11
+    K2, V2 = K.copy(), V.copy()
+    K2[0, 0, j] += 1.0
+    V2[0, 0, j] -= 2.0
+    O2 = orc.forward_tokencausal(Q, K2, V2, G, (T, Hh, W), bands)[0, 0]
+    assert np.array_equal(O2[:j], O[:j])
+    assert not np.allclose(O2[j:], O[j:])
