@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work of the oracle baseline")
     ap.add_argument("--gated", action="store_true",
                     help="full gated form: write gate beta [B,H,N] and RMSNorm before the output gate")
+    ap.add_argument("--causal", action="store_true",
+                    help="token-causal operator (token n reads tokens 0..n) on a bidirectional workload's shape")
     ap.add_argument("--stream", action="store_true",
                     help="block-causal workloads: one la_block_step call per block on a carried cache, "
                          "as a block-autoregressive generator runs")
@@ -222,7 +224,7 @@ def main():
     dev = torch.device("cuda", local)
     ldist.init("nccl")
     w = wl.WORKLOADS[args.workload]
-    p = la.Problem.from_workload(w, force_simt=args.simt)
+    p = la.Problem.from_workload(w, force_simt=args.simt, token_causal=args.causal)
     la.load()
 
     Q, K, V, G = wl.generate(w, dev, seed=w.seed + 1000 * rank)
@@ -263,6 +265,12 @@ def main():
                 la.block_step(pb, qb, kb, vb, gb, S_c, z_c, O=ob, ws=ws_s)
                 n += la.last_launch_count()
             counter["launches"] = n
+    elif args.causal:
+        if w.block_frames > 0 or args.gated:
+            raise SystemExit("--causal takes a bidirectional workload and no --gated")
+
+        def forward_plain():
+            la.forward_tokencausal(p, Q, K, V, G, O=O, ws=ws)
     else:
         def forward_plain():
             if args.gated:
@@ -341,8 +349,12 @@ def main():
     else:
         # Per-kernel durations inside the timed steps of the second region.
         tc = not args.simt and w.d == 128 and w.dtype == "bf16"
-        names = ["rope_table_kernel", "state_tc_kernel", "combine_kernel", "apply_tc_kernel"] if tc \
-            else ["state_simt_kernel", "combine_kernel", "apply_simt_kernel"]
+        if args.causal:
+            names = ["rope_table_kernel", "state_tc_kernel", "start_kernel", "causal_tc_kernel"]
+        elif tc:
+            names = ["rope_table_kernel", "state_tc_kernel", "combine_kernel", "apply_tc_kernel"]
+        else:
+            names = ["state_simt_kernel", "combine_kernel", "apply_simt_kernel"]
         assert len(names) == launches_per_step, (names, launches_per_step)
         per = {n: [] for n in names}
         for k in range(args.steps):
@@ -350,7 +362,10 @@ def main():
                 per[n].append(evs[k][i].elapsed_time(evs[k][i + 1]))
         kern_ms = {n: sum(v) / len(v) for n, v in per.items()}
         tot = sum(kern_ms.values())
-        alg_bytes = {names[-3]: (2 * w.d + (1 if args.gated else 0)) * th * elem, names[-1]: 3 * th * w.d * elem}
+        # the token-causal kernel reads Q, K, V, G and writes O; the apply kernel reads Q, G, writes O
+        state_name = next(n for n in names if n.startswith("state_"))
+        alg_bytes = {state_name: (2 * w.d + (1 if args.gated else 0)) * th * elem,
+                     names[-1]: (5 if args.causal else 3) * th * w.d * elem}
         dominant = max((n for n in names if n in alg_bytes), key=lambda n: kern_ms[n])
         alg = alg_bytes[dominant]
         achieved = alg / (kern_ms[dominant] * 1e-3) / 1e9
@@ -363,6 +378,8 @@ def main():
     config = config_of(w, world)
     if args.gated:
         config["gated"] = "write gate beta [B,H,N] + RMSNorm (gamma [d]) before the output gate"
+    if args.causal:
+        config["mode"] = "token-causal (token n reads tokens 0..n; K and V are read by both passes)"
     if args.stream:
         config["stream"] = f"{len(blocks)} blocks, one la_block_step per block on a carried cache"
     line = {
@@ -383,7 +400,7 @@ def main():
     }
 
     if not args.no_e2e and not args.stream:
-        line["e2e"] = e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates)
+        line["e2e"] = e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates, causal=args.causal)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, times = oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -395,7 +412,7 @@ def main():
     return 0
 
 
-def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None):
+def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None, causal=False):
     """Same metric through the public API with the inputs in pinned host memory: every step
     copies Q, K, V, G (and the write gate when gated) host->device, runs the operator and copies
     O device->host."""
@@ -413,6 +430,8 @@ def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None):
             dst.copy_(hsrc, non_blocking=True)
         if gates:
             la.forward_gated(p, Q, K, V, G, O=O, ws=ws, **gates)
+        elif causal:
+            la.forward_tokencausal(p, Q, K, V, G, O=O, ws=ws)
         else:
             la.forward(p, Q, K, V, G, O=O, ws=ws)
         Oh.copy_(O, non_blocking=True)

@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(HERE, "liblinattn.so")
 
 LA_BF16, LA_F32 = 0, 1
 LA_FLAG_FORCE_SIMT = 1
+LA_FLAG_TOKEN_CAUSAL = 2
 
 STATUS = {
     0: "LA_OK", 1: "LA_ERR_NULL", 2: "LA_ERR_SHAPE", 3: "LA_ERR_BANDS", 4: "LA_ERR_ALIGN",
@@ -26,7 +27,7 @@ EXPORTS = [
     "la_workspace_bytes", "la_workspace_bytes_for", "la_state_reduce", "la_state_scan", "la_apply",
     "la_forward_bidir", "la_forward_blockcausal", "la_status_string", "la_device_error",
     "la_last_launch_count", "la_forward_marked", "la_selftest_host", "la_forward_bidir_static",
-    "la_state_update", "la_forward_gated", "la_block_step",
+    "la_state_update", "la_forward_gated", "la_block_step", "la_forward_tokencausal",
 ]
 
 
@@ -80,6 +81,7 @@ def load(path: Optional[str] = None):
         "la_state_scan": (ctypes.c_int, [P, vp, vp, vp]),
         "la_state_update": (ctypes.c_int, [P, vp, vp, vp, vp, vp, sz, vp]),
         "la_block_step": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "la_forward_tokencausal": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_gated": (ctypes.c_int, [P, ctypes.POINTER(LaGates), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_apply": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_bidir": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -121,7 +123,8 @@ class Problem:
     block_frames: int = 0
     dtype: str = "bf16"
     force_simt: bool = False
-    t0: int = 0  # global index of frame 0 (the t band rotates at t0 + t)
+    t0: int = 0
+    token_causal: bool = False  # la_forward_marked runs the token-causal operator  # global index of frame 0 (the t band rotates at t0 + t)
 
     @property
     def N(self) -> int:
@@ -142,7 +145,8 @@ class Problem:
         return LaProblem(self.B, self.H, self.T, self.Hh, self.W, self.d, self.bands[0], self.bands[1],
                          self.bands[2], float(self.rope_base), float(self.eps), int(self.block_frames),
                          LA_BF16 if self.dtype == "bf16" else LA_F32,
-                         LA_FLAG_FORCE_SIMT if self.force_simt else 0, int(self.t0))
+                         (LA_FLAG_FORCE_SIMT if self.force_simt else 0) |
+                         (LA_FLAG_TOKEN_CAUSAL if self.token_causal else 0), int(self.t0))
 
 
 def _ptr(t) -> Optional[int]:
@@ -334,6 +338,23 @@ def forward_gated(p: Problem, Q, K, V, G, beta=None, gamma=None, rms_norm=False,
     return O
 
 
+def forward_tokencausal(p: Problem, Q, K, V, G, O=None, ws=None, stream=None):
+    """Token-causal operator: token n reads the states of tokens 0..n (bf16, d = 128)."""
+    import torch
+
+    lib = load()
+    if O is None:
+        O = torch.empty_like(Q)
+    if ws is None:
+        ws, nbytes = workspace(p, Q.device)
+    else:
+        nbytes = ws.numel()
+    cp = p.c()
+    _check(lib.la_forward_tokencausal(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(O), _ptr(ws),
+                                      nbytes, _stream(stream)), "la_forward_tokencausal")
+    return O
+
+
 def forward(p: Problem, Q, K, V, G, **kw):
     """Bidirectional or block-causal, as ``p.block_frames`` says."""
     if p.block_frames > 0:
@@ -357,8 +378,8 @@ def forward_marked(p: Problem, Q, K, V, G, O, ws, events, S_incl=None, z_incl=No
             e.record(st)
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     cp = p.c()
-    gates = LaGates(_ptr(beta), _ptr(gamma), float(norm_eps), 1 if rms_norm else 0)
-    _check(lib.la_forward_marked(ctypes.byref(cp), ctypes.byref(gates), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(O),
+    gates = LaGates(_ptr(beta), _ptr(gamma), float(norm_eps), 1 if rms_norm else 0) if (beta is not None or rms_norm) else None
+    _check(lib.la_forward_marked(ctypes.byref(cp), None if gates is None else ctypes.byref(gates), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(O),
                                  _ptr(S_incl), _ptr(z_incl), _ptr(ws), ws.numel(), st.cuda_stream,
                                  arr, len(events)), "la_forward_marked")
     return O

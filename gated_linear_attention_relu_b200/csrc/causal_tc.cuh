@@ -1,0 +1,469 @@
+// causal_tc.cuh -- token-causal operator on the 5th-generation tensor cores (bf16, d = 128).
+//
+// Token n reads the states of tokens 0..n of its head in the flattened order (the causal form
+// of "SANA-Video: Efficient Video Generation with Block Linear Diffusion Transformer", Sec. 3.4,
+// taken token by token):
+//   O_n = (phi(q_n) S_{<=n}) / (q_n^+ . z_{<=n} + eps) * sigmoid(g_n),
+//   S_{<=n} = sum_{m<=n} phi(k_m)^T v_m,  z_{<=n} = sum_{m<=n} k_m^+,  phi = RoPE3D(ReLU(.)).
+//
+// Chunkwise form.  The tiles of every head are split into contiguous segments, one per
+// persistent CTA (the same split as the state kernel's, whose per-segment sums the start
+// kernel prefix-sums into each CTA's starting state).  A CTA walks its 128-token chunks in order
+// carrying S (fp32, in TMEM) and z (fp32, channel k in thread k); for chunk c with rows n, m:
+//   D   = Q^+ K^+^T                     (tensor cores; masked row sums -> intra-chunk denominator)
+//   num = phi(Q) S_prev + (P o M) V,    P = phi(Q) phi(K)^T, M_nm = [m <= n]
+//   den = q_n^+ . z_prev + sum_{m<=n} D_nm + eps
+//   S  += phi(K)^T V,  z += column sums of K^+
+// P o M goes back to TMEM as bf16 and is the A operand of the P V product; S_prev is the bf16
+// image of the carried state in shared memory (rewritten after every chunk).
+//
+// Warps: 0-3 own the chunk's rows (thread = token = TMEM lane); warp 4 issues the TMA copies and
+// the MMAs.  One chunk at a time (each phase waits for the previous one): this first version
+// favours clarity over overlap.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace la {
+namespace ca {
+
+constexpr int TILE = 128;
+constexpr int D = 128;
+constexpr int THREADS = 160;
+constexpr uint32_t HALF = 128 * 128;
+constexpr uint32_t BUF = 2 * HALF;
+constexpr uint32_t OFF_Q = 0, OFF_K = BUF, OFF_V = 2 * BUF, OFF_G = 3 * BUF, OFF_S = 4 * BUF;
+constexpr uint32_t OFF_Z = 5 * BUF;  // z of the tokens before the chunk, [128] fp32
+constexpr uint32_t OFF_BAR = OFF_Z + 512;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_S = 0, COL_ND = 128, COL_P = 256;  // carried S; D then num; P (then bf16 P)
+constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/false);
+constexpr uint32_t IDESC_QS = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/true);
+constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, /*a_mn=*/true, /*b_mn=*/true);
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+struct Bars {
+  uint64_t full;      // Q, K, V, G of the chunk landed
+  uint64_t relu;      // math: Q^+ and K^+ written in place (4 warps)
+  uint64_t zsync1;    // math: every row's K^+ written (4 warps), before the column reads
+  uint64_t zsync;     // math: z published and K^+ columns read (4 warps)
+  uint64_t dready;    // MMA: D = Q^+ K^+^T done (and its operand reads)
+  uint64_t rot;       // math: phi(Q), phi(K) written in place (4 warps)
+  uint64_t pready;    // MMA: num (inter), P and the S update done
+  uint64_t pw;        // math: masked P written to TMEM as bf16 (4 warps)
+  uint64_t numready;  // MMA: num += P V done
+  uint64_t out;       // math: O staged over G, S image rewritten (4 warps)
+  uint64_t final_;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block too large");
+
+// K-major operand (rows of 128 channels, 128B swizzle, two 64-channel halves): K step kk.
+__device__ __forceinline__ uint64_t desc_k(uint32_t base, int kk) {
+  return smem_desc_sw128(base + static_cast<uint32_t>(kk >> 2) * HALF + static_cast<uint32_t>(kk & 3) * 32u, 16,
+                         1024);
+}
+// MN-major operand (the same row layout read along rows): K step kk = rows 16kk .. 16kk+15.
+__device__ __forceinline__ uint64_t desc_mn(uint32_t base, int kk) {
+  return smem_desc_sw128(base + static_cast<uint32_t>(kk) * 2048u, HALF, 1024);
+}
+// Shared-memory address of 16-byte chunk ck (0..15) of row r in that layout.
+__device__ __forceinline__ uint32_t row_chunk(uint32_t base, int r, int ck) {
+  return base + static_cast<uint32_t>(ck >> 3) * HALF + static_cast<uint32_t>(r) * 128u +
+         ((static_cast<uint32_t>(ck & 7) ^ static_cast<uint32_t>(r & 7)) << 4);
+}
+
+__device__ __forceinline__ float sigmoid_tanh(float g) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(0.5f * g));
+  return 0.5f + 0.5f * y;
+}
+
+// In place over one row (64 bf16 pairs, already ReLU'd): a <- RoPE(a) at grid position (pt, ph, pw).
+template <int DT, int DH>
+__device__ __forceinline__ void rotate_row(uint32_t (&a)[64], const float2* __restrict__ tab,
+                                           const float4* __restrict__ tab2, const Rope& rope, const Plan& p,
+                                           int pt, int ph, int pw) {
+  if constexpr (DT >= 0 && DH >= 0) {
+    constexpr int DW = 128 - DT - DH;
+    static_assert(DT % 4 == 0 && DH % 4 == 0 && DW % 4 == 0, "bands of whole 16-byte entries");
+    const float4* bt = tab2 + pt * (DT / 4);
+    const float4* bh = tab2 + rope.tab_off_h / 2 + ph * (DH / 4);
+    const float4* bw = tab2 + rope.tab_off_w / 2 + pw;
+    const int W = static_cast<int>(p.W);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int pi = 2 * j;
+      const int bnd = band_of<DT, DH>(pi, rope);
+      const int e = pair_in_band<DT, DH>(pi, rope) / 2;
+      const float4 cs = __ldg(bnd == 0 ? bt + e : (bnd == 1 ? bh + e : bw + e * W));
+      const float x0 = bf16lo(a[pi]), x1 = bf16hi(a[pi]);
+      const float y0 = bf16lo(a[pi + 1]), y1 = bf16hi(a[pi + 1]);
+      a[pi] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+      a[pi + 1] = pack_bf16(y0 * cs.z - y1 * cs.w, y0 * cs.w + y1 * cs.z);
+    }
+  } else {
+    const int ext[3] = {static_cast<int>(p.T), static_cast<int>(p.Hh), static_cast<int>(p.W)};
+    const int off[3] = {0, static_cast<int>(rope.tab_off_h), static_cast<int>(rope.tab_off_w)};
+    const int pos[3] = {pt, ph, pw};
+#pragma unroll 4
+    for (int pi = 0; pi < 64; ++pi) {
+      const int bnd = band_of<DT, DH>(pi, rope);
+      const int loc = pair_in_band<DT, DH>(pi, rope);
+      const float2 cs = __ldg(tab + off[bnd] + loc * ext[bnd] + pos[bnd]);
+      const float x0 = bf16lo(a[pi]), x1 = bf16hi(a[pi]);
+      a[pi] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+    }
+  }
+}
+
+template <int DT, int DH>
+__global__ void __launch_bounds__(THREADS, 1)
+causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
+                 const __grid_constant__ CUtensorMap tmO, const Plan p, const __grid_constant__ Rope rope,
+                 const float* __restrict__ start, const float2* __restrict__ tab,
+                 const float4* __restrict__ tab2) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
+  float* zs = reinterpret_cast<float*>(smem + OFF_Z);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t c = blockIdx.x;
+  const int64_t g0 = cta_start(p, c);
+  const int64_t g1 = cta_start(p, c + 1);
+  volatile int* abort_flag = &bars->abort_flag;
+
+  // Does this CTA's first unit start in an earlier CTA (then the start kernel summed its state)?
+  bool has_start = false;
+  if (g0 < g1) {
+    int64_t first = 0, count = 0;
+    unit_tiles(p, unit_of_tile(p, g0), &first, &count);
+    has_start = cta_of(p, first) != c;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->full, 1);
+    mbar_init(&bars->relu, 4);
+    mbar_init(&bars->zsync1, 4);
+    mbar_init(&bars->zsync, 4);
+    mbar_init(&bars->dready, 1);
+    mbar_init(&bars->rot, 4);
+    mbar_init(&bars->pready, 1);
+    mbar_init(&bars->pw, 4);
+    mbar_init(&bars->numready, 1);
+    mbar_init(&bars->out, 4);
+    mbar_init(&bars->final_, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(&bars->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  pdl_trigger();
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA + MMA issue
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmG);
+      tma_prefetch_desc(&tmO);
+      int64_t prev_unit = -1;
+      int64_t issued = 0;
+      TileInfo tprev{};
+      bool ok = true;
+      for (int64_t g = g0; g < g1 && ok; ++g) {
+        const int64_t i = g - g0;
+        const uint32_t ph = static_cast<uint32_t>(i & 1);
+        const TileInfo ti = tile_info(p, g);
+        const bool first = ti.unit != prev_unit;
+        const bool zero_start = first && !(g == g0 && has_start);
+        prev_unit = ti.unit;
+        if (i > 0) {
+          // The previous chunk is finished: store its O (staged over G), then reuse the buffers.
+          if (!mbar_wait(&bars->out, static_cast<uint32_t>((i - 1) & 1), abort_flag)) break;
+          const int32_t pn0 = static_cast<int32_t>(tprev.n0), pbh = static_cast<int32_t>(tprev.bh);
+          tma_store_3d(&tmO, smem + OFF_G, 0, pn0, pbh);
+          tma_store_3d(&tmO, smem + OFF_G + HALF, 64, pn0, pbh);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        tprev = ti;
+        mbar_arrive_expect_tx(&bars->full, 4 * BUF);
+        const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
+        tma_load_3d(smem + OFF_Q, &tmQ, 0, n0, bh, &bars->full);
+        tma_load_3d(smem + OFF_Q + HALF, &tmQ, 64, n0, bh, &bars->full);
+        tma_load_3d(smem + OFF_K, &tmK, 0, n0, bh, &bars->full);
+        tma_load_3d(smem + OFF_K + HALF, &tmK, 64, n0, bh, &bars->full);
+        tma_load_3d(smem + OFF_V, &tmV, 0, n0, bh, &bars->full);
+        tma_load_3d(smem + OFF_V + HALF, &tmV, 64, n0, bh, &bars->full);
+        tma_load_3d(smem + OFF_G, &tmG, 0, n0, bh, &bars->full);
+        tma_load_3d(smem + OFF_G + HALF, &tmG, 64, n0, bh, &bars->full);
+        ++issued;
+        // D = Q^+ K^+^T
+        if (!mbar_wait(&bars->relu, ph, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + COL_ND, desc_k(sbase + OFF_Q, kk), desc_k(sbase + OFF_K, kk), IDESC_QK, kk > 0 ? 1u : 0u);
+        mma_commit(&bars->dready);
+        // num = phi(Q) S_prev;  P = phi(Q) phi(K)^T;  S += phi(K)^T V
+        if (!mbar_wait(&bars->rot, ph, abort_flag)) break;
+        tc_fence_after();
+        if (!zero_start) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16(tmem + COL_ND, desc_k(sbase + OFF_Q, kk), desc_mn(sbase + OFF_S, kk), IDESC_QS,
+                     kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + COL_P, desc_k(sbase + OFF_Q, kk), desc_k(sbase + OFF_K, kk), IDESC_QK, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + COL_S, desc_mn(sbase + OFF_K, kk), desc_mn(sbase + OFF_V, kk), IDESC_KV,
+                   (kk > 0 || !zero_start) ? 1u : 0u);
+        mma_commit(&bars->pready);
+        // num += (P o M) V
+        if (!mbar_wait(&bars->pw, ph, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + COL_ND, tmem + COL_P + 8u * kk, desc_mn(sbase + OFF_V, kk), IDESC_QS,
+                      (kk > 0 || !zero_start) ? 1u : 0u);
+        mma_commit(&bars->numready);
+      }
+      // Store the last chunk's O.
+      if (issued > 0 && !*abort_flag &&
+          mbar_wait(&bars->out, static_cast<uint32_t>((issued - 1) & 1), abort_flag)) {
+        const int32_t pn0 = static_cast<int32_t>(tprev.n0), pbh = static_cast<int32_t>(tprev.bh);
+        tma_store_3d(&tmO, smem + OFF_G, 0, pn0, pbh);
+        tma_store_3d(&tmO, smem + OFF_G + HALF, 64, pn0, pbh);
+        bulk_commit_group();
+      }
+      bulk_wait_group0();
+      if (*abort_flag && issued > 0) mbar_wait_drain(&bars->full, static_cast<uint32_t>((issued - 1) & 1));
+      mma_commit(&bars->final_);
+      mbar_wait_drain(&bars->final_, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ rows (warps 0-3)
+    const int row = threadIdx.x;  // token row of the chunk = TMEM lane; also channel k for z and S
+    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t t_s = tmem + COL_S + lane_bits, t_nd = tmem + COL_ND + lane_bits, t_p = tmem + COL_P + lane_bits;
+    float zk = 0.f;  // z of channel `row` over the tokens before the chunk
+    pdl_wait();      // the start states and the cos/sin tables come from the kernels before
+    if (g0 < g1 && has_start) {
+      // Carried state at the segment start: fp32 row `row` of S into TMEM, its bf16 image, z.
+      const float* src = start + c * (D * D + D);
+      uint32_t r[32];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(src[row * D + 32 * j + e]);
+        tmem_st_x16(t_s + 32 * j, &r[0]);
+        tmem_st_x16(t_s + 32 * j + 16, &r[16]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int ck = 4 * j + e;
+          sts128(row_chunk(sbase + OFF_S, row, ck),
+                 make_uint4(pack_bf16(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
+                            pack_bf16(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
+                            pack_bf16(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
+                            pack_bf16(__uint_as_float(r[8 * e + 6]), __uint_as_float(r[8 * e + 7]))));
+        }
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      zk = src[D * D + row];
+    }
+    int64_t prev_unit = -1;
+    for (int64_t g = g0; g < g1; ++g) {
+      const int64_t i = g - g0;
+      const uint32_t ph = static_cast<uint32_t>(i & 1);
+      const TileInfo ti = tile_info(p, g);
+      if (ti.unit != prev_unit && !(g == g0 && has_start)) zk = 0.f;  // a head starting in this CTA
+      prev_unit = ti.unit;
+      if (!warp_wait(&bars->full, ph, abort_flag)) break;
+      // ReLU of Q and K in place; q^+ kept in registers.
+      uint32_t qa[64];
+#pragma unroll
+      for (int ck = 0; ck < 16; ++ck) {
+        const uint32_t aq = row_chunk(sbase + OFF_Q, row, ck);
+        const uint4 rq = lds128(aq);
+        qa[4 * ck] = relu_bf16x2(rq.x);
+        qa[4 * ck + 1] = relu_bf16x2(rq.y);
+        qa[4 * ck + 2] = relu_bf16x2(rq.z);
+        qa[4 * ck + 3] = relu_bf16x2(rq.w);
+        sts128(aq, make_uint4(qa[4 * ck], qa[4 * ck + 1], qa[4 * ck + 2], qa[4 * ck + 3]));
+        const uint32_t ak = row_chunk(sbase + OFF_K, row, ck);
+        const uint4 rk = lds128(ak);
+        sts128(ak, make_uint4(relu_bf16x2(rk.x), relu_bf16x2(rk.y), relu_bf16x2(rk.z), relu_bf16x2(rk.w)));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars->relu);
+        mbar_arrive(&bars->zsync1);
+      }
+      // z before the chunk, published for every row's denominator; then this chunk's K^+ column
+      // (thread `row` sums channel `row` over the chunk's rows, once every row is ReLU'd).
+      zs[row] = zk;
+      if (!warp_wait(&bars->zsync1, ph, abort_flag)) break;
+      {
+        const int kc = row;  // channel
+        const uint32_t kbase = sbase + OFF_K + static_cast<uint32_t>(kc >> 6) * HALF;
+        const uint32_t cchunk = static_cast<uint32_t>((kc & 63) >> 3), cbyte = static_cast<uint32_t>(kc & 7) * 2u;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int m = 0; m < TILE; ++m) {
+          uint16_t hv;
+          asm volatile("ld.shared.u16 %0, [%1];"
+                       : "=h"(hv)
+                       : "r"(kbase + static_cast<uint32_t>(m) * 128u + ((cchunk ^ static_cast<uint32_t>(m & 7)) << 4) +
+                             cbyte));
+          s4[m & 3] += __uint_as_float(static_cast<uint32_t>(hv) << 16);
+        }
+        zk += (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->zsync);
+      if (!warp_wait(&bars->zsync, ph, abort_flag)) break;
+      // Denominator: q^+ . z_prev + masked row sum of D.
+      float dz = 0.f;
+#pragma unroll
+      for (int k4 = 0; k4 < 32; ++k4) {
+        const float4 z4 = *reinterpret_cast<const float4*>(zs + 4 * k4);
+        dz = fmaf(bf16lo(qa[2 * k4]), z4.x, dz);
+        dz = fmaf(bf16hi(qa[2 * k4]), z4.y, dz);
+        dz = fmaf(bf16lo(qa[2 * k4 + 1]), z4.z, dz);
+        dz = fmaf(bf16hi(qa[2 * k4 + 1]), z4.w, dz);
+      }
+      if (!warp_wait(&bars->dready, ph, abort_flag)) break;
+      tc_fence_after();
+      float dintra = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t r[32];
+        tmem_ld_x32(t_nd + 32 * j, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) dintra += (32 * j + e <= row) ? __uint_as_float(r[e]) : 0.f;
+      }
+      const float hinv = 1.0f / (dz + dintra + p.eps);
+      // RoPE of Q^+ and K^+ in place.
+      const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
+      uint32_t pt = 0, ph_ = 0, pw = 0;
+      if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph_, pw);
+      {
+        uint32_t a[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) a[e] = qa[e];
+        rotate_row<DT, DH>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+#pragma unroll
+        for (int ck = 0; ck < 16; ++ck)
+          sts128(row_chunk(sbase + OFF_Q, row, ck), make_uint4(a[4 * ck], a[4 * ck + 1], a[4 * ck + 2], a[4 * ck + 3]));
+#pragma unroll
+        for (int ck = 0; ck < 16; ++ck) {
+          const uint4 rk = lds128(row_chunk(sbase + OFF_K, row, ck));
+          a[4 * ck] = rk.x;
+          a[4 * ck + 1] = rk.y;
+          a[4 * ck + 2] = rk.z;
+          a[4 * ck + 3] = rk.w;
+        }
+        rotate_row<DT, DH>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+#pragma unroll
+        for (int ck = 0; ck < 16; ++ck)
+          sts128(row_chunk(sbase + OFF_K, row, ck), make_uint4(a[4 * ck], a[4 * ck + 1], a[4 * ck + 2], a[4 * ck + 3]));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->rot);
+      // Causal mask on P (m <= n), back to TMEM as the bf16 A operand of P V.
+      if (!warp_wait(&bars->pready, ph, abort_flag)) break;
+      tc_fence_after();
+      {
+        uint32_t pb[64];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t r[32];
+          tmem_ld_x32(t_p + 32 * j, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int m0 = 32 * j + 2 * e;
+            const float p0 = m0 <= row ? __uint_as_float(r[2 * e]) : 0.f;
+            const float p1 = m0 + 1 <= row ? __uint_as_float(r[2 * e + 1]) : 0.f;
+            pb[16 * j + e] = pack_bf16(p0, p1);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tmem_st_x16(t_p + 16 * j, &pb[16 * j]);
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->pw);
+      // O = num / den * sigmoid(g), in place over G; then the new state's bf16 image.
+      if (!warp_wait(&bars->numready, ph, abort_flag)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t r[32];
+        tmem_ld_x32(t_nd + 32 * j, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t ag = row_chunk(sbase + OFF_G, row, 4 * j + e);
+          const uint4 gr = lds128(ag);
+          const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
+          uint32_t ov[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float o0 = __uint_as_float(r[8 * e + 2 * q]) * hinv * sigmoid_tanh(bf16lo(gw[q]));
+            const float o1 = __uint_as_float(r[8 * e + 2 * q + 1]) * hinv * sigmoid_tanh(bf16hi(gw[q]));
+            ov[q] = pack_bf16(o0, o1);
+          }
+          sts128(ag, make_uint4(ov[0], ov[1], ov[2], ov[3]));
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t r[32];
+        tmem_ld_x32(t_s + 32 * j, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          sts128(row_chunk(sbase + OFF_S, row, 4 * j + e),
+                 make_uint4(pack_bf16(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
+                            pack_bf16(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
+                            pack_bf16(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
+                            pack_bf16(__uint_as_float(r[8 * e + 6]), __uint_as_float(r[8 * e + 7]))));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->out);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 4) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace ca
+}  // namespace la

@@ -14,6 +14,7 @@
 #include "sm100.cuh"
 #include "state_tc.cuh"
 #include "apply_tc.cuh"
+#include "causal_tc.cuh"
 #include "simt.cuh"
 
 namespace {
@@ -32,7 +33,7 @@ int validate(const la_problem* p) {
   if (!p) return LA_ERR_NULL;
   if (p->B < 0 || p->H < 0 || p->T < 0 || p->Hh < 0 || p->W < 0 || p->block_frames < 0) return LA_ERR_SHAPE;
   if (p->dtype != LA_BF16 && p->dtype != LA_F32) return LA_ERR_UNSUPPORTED;
-  if ((p->flags & ~LA_FLAG_FORCE_SIMT) != 0u) return LA_ERR_UNSUPPORTED;
+  if ((p->flags & ~(LA_FLAG_FORCE_SIMT | LA_FLAG_TOKEN_CAUSAL)) != 0u) return LA_ERR_UNSUPPORTED;
   if (!is_pow2_dim(p->d)) return LA_ERR_UNSUPPORTED;
   if (p->dt < 0 || p->dh < 0 || p->dw < 0 || (p->dt & 1) || (p->dh & 1) || (p->dw & 1) ||
       p->dt + p->dh + p->dw != p->d)
@@ -125,7 +126,7 @@ struct PlanSet {
   Plan ps;            // state reduction
   Plan pa;            // apply
   int64_t units;      // B*H*nblk
-  size_t off_partial, off_states, off_img, off_zimg, off_tab, off_tab2, total;
+  size_t off_partial, off_states, off_img, off_zimg, off_tab, off_tab2, off_start, total;
   int64_t tab_entries;
 };
 
@@ -158,6 +159,8 @@ PlanSet make_plans(const la_problem& q, int sm_count) {
   off = align256(off + size_t(s.tab_entries) * 8);
   s.off_tab2 = off;  // the same entries in the apply kernel's layout (standard band split only)
   off = align256(off + (standard_bands(q) ? size_t(s.tab_entries) * 8 : 0));
+  s.off_start = off;  // token-causal: state carried into each CTA's range (tensor-core path)
+  off = align256(off + (s.tc ? size_t(s.ps.grid) * size_t(D * D + D) * 4 : 0));
   s.total = off;
   return s;
 }
@@ -492,6 +495,69 @@ int la_block_step(const la_problem* p, const void* Q, const void* K, const void*
   return LA_OK;
 }
 
+static int tokencausal_common(const la_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                              void* O, void* ws, size_t ws_bytes, cudaStream_t stream, cudaEvent_t* marks = nullptr,
+                              int nmarks = 0) {
+  static_assert(la::st::TILE == la::ca::TILE, "the causal kernel walks the state kernel's tile ranges");
+  int rc;
+  if (p->block_frames != 0) return LA_ERR_SHAPE;
+  const bool has_tok = elems(*p) > 0;
+  if ((rc = check_ptr(Q, has_tok)) || (rc = check_ptr(K, has_tok)) || (rc = check_ptr(V, has_tok)) ||
+      (rc = check_ptr(G, has_tok)) || (rc = check_ptr(O, has_tok)))
+    return rc;
+  if (p->dtype != LA_BF16 || p->d != 128 || (p->flags & LA_FLAG_FORCE_SIMT)) return LA_ERR_UNSUPPORTED;
+  if (!has_tok) {
+    g_last_launches = 0;
+    return LA_OK;
+  }
+  int sm = 0;
+  if ((rc = current_sm_count(&sm))) return rc;
+  const PlanSet s = make_plans(*p, sm);
+  if ((rc = check_ws(s, ws, ws_bytes))) return rc;
+  int nl = 0;
+  auto mark = [&](int i) {
+    if (i < nmarks && marks && marks[i]) cudaEventRecord(marks[i], stream);
+  };
+  mark(0);
+  if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
+  mark(nl);
+  // Per-segment state sums (the state kernel's partial slots), then each CTA's carried state.
+  if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
+  mark(nl);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* start = reinterpret_cast<float*>(w + s.off_start);
+  const int64_t threads = int64_t(s.ps.grid) * ((128 * 128 + 128) / 8);
+  if (launch_k(la::cmb::start_kernel, unsigned((threads + la::cmb::THREADS - 1) / la::cmb::THREADS),
+               la::cmb::THREADS, 0, stream, true, s.ps, reinterpret_cast<const float*>(w + s.off_partial), start))
+    return LA_ERR_CUDA;
+  ++nl;
+  mark(nl);
+  CUtensorMap tq, tk, tv, tg, to;
+  if (!make_tmap(&tq, Q, s.ps.BH, s.ps.N) || !make_tmap(&tk, K, s.ps.BH, s.ps.N) ||
+      !make_tmap(&tv, V, s.ps.BH, s.ps.N) || !make_tmap(&tg, G, s.ps.BH, s.ps.N) ||
+      !make_tmap(&to, O, s.ps.BH, s.ps.N))
+    return LA_ERR_CUDA;
+  auto kern = standard_bands(*p) ? la::ca::causal_tc_kernel<32, 48> : la::ca::causal_tc_kernel<-1, -1>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::ca::SMEM_BYTES) != cudaSuccess)
+    return LA_ERR_CUDA;
+  const Rope rope = make_rope(*p);
+  if (launch_k(kern, unsigned(s.ps.grid), la::ca::THREADS, la::ca::SMEM_BYTES, stream, true, tq, tk, tv, tg, to,
+               s.ps, rope, static_cast<const float*>(start), reinterpret_cast<const float2*>(w + s.off_tab),
+               reinterpret_cast<const float4*>(w + s.off_tab2)))
+    return LA_ERR_CUDA;
+  ++nl;
+  mark(nl);
+  g_last_launches = nl;
+  return LA_OK;
+}
+
+int la_forward_tokencausal(const la_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                           void* O, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  return tokencausal_common(p, Q, K, V, G, O, ws, ws_bytes, stream);
+}
+
 int la_state_scan(const la_problem* p, float* S, float* z, cudaStream_t stream) {
   int rc = validate(p);
   if (rc) return rc;
@@ -648,6 +714,10 @@ int la_forward_marked(const la_problem* p, const la_gates* gates, const void* Q,
   if (rc) return rc;
   if (nmarks < 0 || (nmarks > 0 && !marks)) return LA_ERR_NULL;
   if (p->block_frames == 0 && (S_incl || z_incl)) return LA_ERR_SHAPE;
+  if (p->flags & LA_FLAG_TOKEN_CAUSAL) {
+    if (gates || S_incl || z_incl) return LA_ERR_UNSUPPORTED;
+    return tokencausal_common(p, Q, K, V, G, O, ws, ws_bytes, stream, marks, nmarks);
+  }
   Gates gt;
   if ((rc = read_gates(gates, &gt))) return rc;
   return forward_common(p, Q, K, V, G, O, S_incl, z_incl, ws, ws_bytes, stream, marks, nmarks, gt);

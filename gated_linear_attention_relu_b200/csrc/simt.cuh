@@ -360,6 +360,44 @@ combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, fl
   }
 }
 
+// Token-causal: the state each CTA's first unit carries into the CTA's tile range, i.e. the sum,
+// in CTA order, of that unit's partial states from the CTAs before it (zero when the unit starts
+// in the CTA itself).  One thread per (CTA, group of 8 consecutive elements of [S | z]).
+__global__ void __launch_bounds__(THREADS)
+start_kernel(const Plan p, const float* __restrict__ partial, float* __restrict__ start) {
+  pdl_trigger();
+  pdl_wait();
+  const int D = p.d;
+  const int groups = (D * D + D) / 8;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
+  const int64_t c = idx / groups;
+  if (c >= p.grid) return;
+  const int e0 = static_cast<int>(idx - c * groups) * 8;
+  const int64_t slot_floats = static_cast<int64_t>(D) * D + static_cast<int64_t>(p.zparts) * D;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  const int64_t g0 = cta_start(p, c);
+  if (g0 < cta_start(p, c + 1)) {
+    const int64_t u = unit_of_tile(p, g0);
+    int64_t first = 0, count = 0;
+    unit_tiles(p, u, &first, &count);
+    for (int64_t cc = cta_of(p, first); cc < c; ++cc) {
+      const int64_t k = u - unit_of_tile(p, cta_start(p, cc));
+      const float* src = partial + (cc * p.maxseg + k) * slot_floats;
+      for (int zp = 0; zp < (e0 < D * D ? 1 : p.zparts); ++zp) {
+        const float4* s4 = reinterpret_cast<const float4*>(e0 < D * D ? src + e0 : src + D * D + zp * D + (e0 - D * D));
+        const float4 a = s4[0], b = s4[1];
+        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+      }
+    }
+  }
+  float4* d4 = reinterpret_cast<float4*>(start + c * (static_cast<int64_t>(D) * D + D) + e0);
+  d4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  d4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
 // In-place inclusive prefix over blocks of [B*H][nblk][D*D] and [B*H][nblk][D].
 __global__ void __launch_bounds__(THREADS)
 scan_kernel(int64_t BH, int64_t nblk, int D, float* S, float* z) {

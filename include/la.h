@@ -66,7 +66,8 @@ typedef enum {
 typedef enum { LA_BF16 = 0, LA_F32 = 1 } la_dtype;
 
 /* la_problem.flags */
-#define LA_FLAG_FORCE_SIMT 1u /* use the CUDA-core kernels even where tcgen05 kernels exist */
+#define LA_FLAG_FORCE_SIMT 1u   /* use the CUDA-core kernels even where tcgen05 kernels exist */
+#define LA_FLAG_TOKEN_CAUSAL 2u /* la_forward_marked: the token-causal operator (block_frames 0) */
 
 typedef struct {
   int64_t B, H;          /* batch and heads */
@@ -142,6 +143,16 @@ int la_forward_blockcausal(const la_problem* p, const void* Q, const void* K, co
                            const void* G, void* O, float* S_incl, float* z_incl,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Token-causal operator (the causal form of SANA-Video Sec. 3.4 taken token by token): token n
+ * of a head reads the states of tokens 0..n in the flattened order n = (t*Hh + h)*W + w:
+ *   O_n = (phi(Q_n) S_{<=n}) / (ReLU(Q_n) . z_{<=n} + eps) * sigmoid(G_n),
+ *   S_{<=n} = sum_{m<=n} phi(K_m)^T V_m,  z_{<=n} = sum_{m<=n} ReLU(K_m).
+ * p->block_frames must be 0.  Tensor-core path only in this version: bf16, d = 128, no
+ * LA_FLAG_FORCE_SIMT; anything else returns LA_ERR_UNSUPPORTED.  Q, K, V, G, O: [B,H,N,d]. */
+int la_forward_tokencausal(const la_problem* p, const void* Q, const void* K, const void* V,
+                           const void* G, void* O, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
 /* Optional terms of the full gated form (SANA-Video 2.0, Sec. 2, Eq. (1)):
  *   S = sum_n beta_n phi(K_n)^T V_n            (write gate; z keeps the un-gated ReLU(K_n):
  *                                               Eq. (1)'s denominator has no beta)
@@ -165,7 +176,8 @@ int la_forward_gated(const la_problem* p, const la_gates* gates, const void* Q, 
                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* The whole operator (bidirectional if p->block_frames == 0, else block-causal, with the
- * same arguments as la_forward_gated; gates may be NULL) with timing marks: records marks[0]
+ * same arguments as la_forward_gated; gates may be NULL; token-causal, as la_forward_tokencausal,
+ * when p->flags has LA_FLAG_TOKEN_CAUSAL, with gates, S_incl and z_incl NULL) with timing marks: records marks[0]
  * on `stream` before the first kernel and marks[i] right after the i-th kernel it queues, for
  * every i < nmarks.  The events are created and owned by the caller.  Used to time the
  * individual kernels of one forward pass with CUDA events. */

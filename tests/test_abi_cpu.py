@@ -104,3 +104,13 @@ def test_state_update_rejects_block_causal_problems_before_cuda():
     assert lib.la_state_update(ctypes.byref(cp), 16, 16, 16, 16, 16, 1 << 30, None) == 2
     cp = la.Problem(B=1, H=2, T=3, Hh=4, W=5, t0=4).c()
     assert lib.la_state_update(ctypes.byref(cp), None, 16, 16, 16, 16, 1 << 30, None) == 1
+
+
+def test_tokencausal_rejects_unsupported_problems_before_cuda():
+    lib = la.load()
+    for kw, status in ((dict(dtype="f32"), 5), (dict(d=64, bands=(16, 24, 24)), 5), (dict(force_simt=True), 5),
+                       (dict(block_frames=1), 2)):
+        args = dict(B=1, H=2, T=3, Hh=4, W=5)
+        args.update(kw)
+        cp = la.Problem(**args).c()
+        assert lib.la_forward_tokencausal(ctypes.byref(cp), 16, 16, 16, 16, 16, 16, 1 << 30, None) == status
