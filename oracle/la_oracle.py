@@ -43,7 +43,7 @@ __all__ = [
     "band_frequencies", "grid_positions", "relu", "sigmoid", "rope3d",
     "head_state", "head_apply", "forward_positions", "forward_bidir",
     "block_of_tokens", "block_states", "forward_blockcausal", "forward_brute", "rms_norm",
-    "tokencausal_rows", "forward_tokencausal",
+    "tokencausal_rows", "forward_tokencausal", "rope3d_transpose", "head_backward", "backward_bidir",
 ]
 
 
@@ -288,3 +288,67 @@ def forward_tokencausal(Q, K, V, G, grid, bands, base=10000.0, eps=1e-6):
     for u in range(B * H):
         O[u] = tokencausal_rows(q[u], k[u], v[u], g[u], pos, bands, base, eps)
     return O.reshape(B, H, N, d)
+
+
+# ----------------------------------------------------------------- gradients (bidirectional form)
+
+def rope3d_transpose(x: np.ndarray, pos: np.ndarray, bands, base: float) -> np.ndarray:
+    """The transpose of the RoPE map at each position (rotation by the opposite angle):
+    (x0, x1) -> (x0 cos a + x1 sin a, -x0 sin a + x1 cos a)."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    o = 0
+    for axis, D in enumerate(bands):
+        if D == 0:
+            continue
+        theta = band_frequencies(D, base)
+        ang = pos[:, axis:axis + 1].astype(np.float64) * theta[None, :]
+        c, s_ = np.cos(ang), np.sin(ang)
+        x0, x1 = x[:, o:o + D:2], x[:, o + 1:o + D:2]
+        out[:, o:o + D:2] = x0 * c + x1 * s_
+        out[:, o + 1:o + D:2] = -x0 * s_ + x1 * c
+        o += D
+    return out
+
+
+def head_backward(q, k, v, g, do, pos, bands, base, eps):
+    """Gradients of the bidirectional mixer of one head with respect to q, k, v, g, given the
+    output gradient ``do``.  With phi = RoPE(ReLU), S = sum phi(k)^T v, z = sum ReLU(k),
+    num = phi(q) S, den = ReLU(q).z + eps, y = num / den, o = y * sigmoid(g), the chain rule
+    gives, per token n (ReLU'(x) taken as [x > 0]):
+      dg = do * y * s (1 - s),  dy = do * s,  dnum = dy / den,  dden = -(dy . y) / den
+      dS = sum_n phi(q_n)^T dnum_n,  dz = sum_n dden_n ReLU(q_n)
+      dq = [q > 0] * (RoPE^T(dnum S^T) + dden z)
+      dv = phi(k) dS,  dk = [k > 0] * (RoPE^T(v dS^T) + dz)."""
+    q, k, v, g, do = (np.asarray(a, dtype=np.float64) for a in (q, k, v, g, do))
+    qp, kp = relu(q), relu(k)
+    qr, kr = rope3d(qp, pos, bands, base), rope3d(kp, pos, bands, base)
+    S = kr.T @ v
+    z = kp.sum(axis=0)
+    num = qr @ S
+    den = qp @ z + float(eps)
+    y = num / den[:, None]
+    sg = sigmoid(g)
+    dg = do * y * sg * (1.0 - sg)
+    dy = do * sg
+    dnum = dy / den[:, None]
+    dden = -np.sum(dy * y, axis=1) / den
+    dS = qr.T @ dnum
+    dz = qp.T @ dden
+    dq = (q > 0) * (rope3d_transpose(dnum @ S.T, pos, bands, base) + dden[:, None] * z[None, :])
+    dv = kr @ dS
+    dk = (k > 0) * (rope3d_transpose(v @ dS.T, pos, bands, base) + dz[None, :])
+    return dq, dk, dv, dg
+
+
+def backward_bidir(Q, K, V, G, dO, grid, bands, base=10000.0, eps=1e-6):
+    """Gradients (dQ, dK, dV, dG) of the bidirectional mixer over [B, H, N, d] inputs."""
+    T, Hh, W = grid
+    pos = grid_positions(T, Hh, W)
+    B, H, N, d = np.shape(Q)
+    q, k, v, g, do = _heads(Q), _heads(K), _heads(V), _heads(G), _heads(dO)
+    outs = [np.empty((B * H, N, d)) for _ in range(4)]
+    for u in range(B * H):
+        for o, r in zip(outs, head_backward(q[u], k[u], v[u], g[u], do[u], pos, bands, base, eps)):
+            o[u] = r
+    return tuple(o.reshape(B, H, N, d) for o in outs)

@@ -479,3 +479,47 @@ def test_tokencausal_first_last_and_causality():
     O2 = orc.forward_tokencausal(Q, K2, V2, G, (T, Hh, W), bands)[0, 0]
     assert np.array_equal(O2[:j], O[:j])
     assert not np.allclose(O2[j:], O[j:])
+
+
+# ----------------------------------------------------------------- gradients
+
+def _loss(q, k, v, g, do, pos, bands):
+    return float(np.sum(orc.forward_positions(q, k, v, g, pos, bands, 10000.0, 1e-6) * do))
+
+
+def test_backward_matches_central_differences():
+    """The oracle's gradients against central finite differences of the forward oracle (fp64):
+    d/dx sum(O * dO) for every input element of a small head."""
+    rng = np.random.default_rng(41)
+    T, Hh, W, d, bands = 2, 2, 3, 8, (2, 2, 4)
+    N = T * Hh * W
+    pos = orc.grid_positions(T, Hh, W)
+    q, k, v, g, do = (rng.standard_normal((N, d)) for _ in range(5))
+    # keep every entry away from the ReLU kink so the differences see a smooth function
+    for x in (q, k):
+        x[np.abs(x) < 0.05] = 0.3
+    grads = orc.head_backward(q, k, v, g, do, pos, bands, 10000.0, 1e-6)
+    h = 1e-6
+    for which, grad in enumerate(grads):
+        args = [q, k, v, g]
+        fd = np.empty_like(args[which])
+        for idx in np.ndindex(*fd.shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            fd[idx] = (_loss(*plus, do, pos, bands) - _loss(*minus, do, pos, bands)) / (2 * h)
+        assert np.allclose(grad, fd, rtol=1e-6, atol=1e-7), which
+
+
+def test_rope_transpose_is_the_inverse_rotation():
+    rng = np.random.default_rng(43)
+    pos = orc.grid_positions(3, 4, 5)
+    x = rng.standard_normal((len(pos), 16))
+    bands = (4, 6, 6)
+    assert np.allclose(orc.rope3d_transpose(orc.rope3d(x, pos, bands, 10000.0), pos, bands, 10000.0), x,
+                       rtol=1e-13, atol=1e-14)
+    y = rng.standard_normal(x.shape)
+    # <R x, y> = <x, R^T y> row by row
+    assert np.allclose(np.sum(orc.rope3d(x, pos, bands, 10000.0) * y, axis=1),
+                       np.sum(x * orc.rope3d_transpose(y, pos, bands, 10000.0), axis=1), rtol=1e-12)
