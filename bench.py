@@ -47,6 +47,8 @@ def parse():
                     help="full gated form: write gate beta [B,H,N] and RMSNorm before the output gate")
     ap.add_argument("--causal", action="store_true",
                     help="token-causal operator (token n reads tokens 0..n) on a bidirectional workload's shape")
+    ap.add_argument("--backward", action="store_true",
+                    help="gradients of the bidirectional operator (dQ, dK, dV, dG from dO)")
     ap.add_argument("--stream", action="store_true",
                     help="block-causal workloads: one la_block_step call per block on a carried cache, "
                          "as a block-autoregressive generator runs")
@@ -242,6 +244,11 @@ def main():
     if args.stream and w.block_frames <= 0:
         raise SystemExit("--stream needs a block-causal workload")
 
+    if args.backward:
+        if w.block_frames > 0 or args.gated or args.causal or args.stream:
+            raise SystemExit("--backward takes a bidirectional workload and no other mode")
+        dO = wl.generate_grad(w, dev, seed=w.seed + 11 + 1000 * rank)
+        grads = tuple(torch.empty_like(Q) for _ in range(4))
     if args.stream:
         # One block per call pair, on contiguous per-block tensors cut out before timing (a
         # generator produces each block's tensors as it goes).
@@ -265,6 +272,11 @@ def main():
                 la.block_step(pb, qb, kb, vb, gb, S_c, z_c, O=ob, ws=ws_s)
                 n += la.last_launch_count()
             counter["launches"] = n
+    elif args.backward:
+        counter = {"launches": 6}
+
+        def forward_plain():
+            la.backward_bidir(p, Q, K, V, G, dO, grads=grads, ws=ws)
     elif args.causal:
         if w.block_frames > 0 or args.gated:
             raise SystemExit("--causal takes a bidirectional workload and no --gated")
@@ -287,7 +299,8 @@ def main():
     for row in evs:
         for e in row:
             e.record(stream)
-    if not args.stream:
+    whole_step = args.stream or args.backward  # no per-kernel events for these
+    if not whole_step:
         for _ in range(max(3, args.warmup)):
             la.forward_marked(p, Q, K, V, G, O, ws, evs[0], S_incl, z_incl, **gates)
         launches_per_step = la.last_launch_count()
@@ -297,7 +310,7 @@ def main():
     for _ in range(max(3, args.warmup)):
         forward_plain()
     torch.cuda.synchronize()
-    if args.stream:
+    if whole_step:
         launches_per_step = counter["launches"]
 
     # Timed region (the headline): K steps of the public forward call, bracketed by a barrier and
@@ -321,7 +334,7 @@ def main():
     # per-kernel durations and the dominant kernel's roofline come from here.  (An event between
     # two kernels keeps the second from starting early, so these steps run a little longer.)
     marked_ms = None
-    if not args.stream:
+    if not whole_step:
         ldist.barrier(dev)
         torch.cuda.synchronize()
         m_start, m_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -339,13 +352,17 @@ def main():
     peak, peak_kind = measured_hbm()
     value = world * th * args.steps / (t_max * 1e-3)
     ms_per_step = t_max / args.steps
-    # bytes_min: Q, K, V, G read once and O written once (+ the write gate when gated).
+    # bytes_min: Q, K, V, G read once and O written once (+ the write gate when gated); the
+    # backward pass reads Q, K, V, G, dO and writes dQ, dK, dV, dG.
     min_bytes = w.min_bytes + (th * elem if args.gated else 0)
+    if args.backward:
+        min_bytes = 9 * th * w.d * elem
     roof_all = min_bytes / (ms_per_step * 1e-3) / 1e9
 
-    if args.stream:
-        # No events can sit inside la_state_update / la_apply, so the roofline is the whole step's.
-        kernels, dominant, alg, achieved, traffic = {}, "whole step (per-block calls)", min_bytes, roof_all, None
+    if whole_step:
+        # No events sit between these kernels, so the roofline is the whole step's.
+        kernels, alg, achieved, traffic = {}, min_bytes, roof_all, None
+        dominant = "whole step (per-block calls)" if args.stream else "whole step (6 kernels)"
     else:
         # Per-kernel durations inside the timed steps of the second region.
         tc = not args.simt and w.d == 128 and w.dtype == "bf16"
@@ -378,6 +395,8 @@ def main():
     config = config_of(w, world)
     if args.gated:
         config["gated"] = "write gate beta [B,H,N] + RMSNorm (gamma [d]) before the output gate"
+    if args.backward:
+        config["mode"] = "backward: dQ, dK, dV, dG from dO (recomputes the forward state)"
     if args.causal:
         config["mode"] = "token-causal (token n reads tokens 0..n; K and V are read by both passes)"
     if args.stream:
@@ -399,7 +418,7 @@ def main():
         "clocks": clk.summary(),
     }
 
-    if not args.no_e2e and not args.stream:
+    if not args.no_e2e and not whole_step:
         line["e2e"] = e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates, causal=args.causal)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, times = oracle_sample(w, args.cpu_seconds)

@@ -27,7 +27,7 @@ EXPORTS = [
     "la_workspace_bytes", "la_workspace_bytes_for", "la_state_reduce", "la_state_scan", "la_apply",
     "la_forward_bidir", "la_forward_blockcausal", "la_status_string", "la_device_error",
     "la_last_launch_count", "la_forward_marked", "la_selftest_host", "la_forward_bidir_static",
-    "la_state_update", "la_forward_gated", "la_block_step", "la_forward_tokencausal",
+    "la_state_update", "la_forward_gated", "la_block_step", "la_forward_tokencausal", "la_backward_bidir",
 ]
 
 
@@ -82,6 +82,7 @@ def load(path: Optional[str] = None):
         "la_state_update": (ctypes.c_int, [P, vp, vp, vp, vp, vp, sz, vp]),
         "la_block_step": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_tokencausal": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "la_backward_bidir": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_gated": (ctypes.c_int, [P, ctypes.POINTER(LaGates), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_apply": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_bidir": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -353,6 +354,24 @@ def forward_tokencausal(p: Problem, Q, K, V, G, O=None, ws=None, stream=None):
     _check(lib.la_forward_tokencausal(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(O), _ptr(ws),
                                       nbytes, _stream(stream)), "la_forward_tokencausal")
     return O
+
+
+def backward_bidir(p: Problem, Q, K, V, G, dO, grads=None, ws=None, stream=None):
+    """Gradients (dQ, dK, dV, dG) of the bidirectional operator given the output gradient dO."""
+    import torch
+
+    lib = load()
+    if grads is None:
+        grads = tuple(torch.empty_like(Q) for _ in range(4))
+    dQ, dK, dV, dG = grads
+    if ws is None:
+        ws, nbytes = workspace(p, Q.device)
+    else:
+        nbytes = ws.numel()
+    cp = p.c()
+    _check(lib.la_backward_bidir(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(dO), _ptr(dQ), _ptr(dK),
+                                 _ptr(dV), _ptr(dG), _ptr(ws), nbytes, _stream(stream)), "la_backward_bidir")
+    return dQ, dK, dV, dG
 
 
 def forward(p: Problem, Q, K, V, G, **kw):

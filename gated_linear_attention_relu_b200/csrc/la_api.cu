@@ -15,6 +15,7 @@
 #include "state_tc.cuh"
 #include "apply_tc.cuh"
 #include "causal_tc.cuh"
+#include "bwd_tc.cuh"
 #include "simt.cuh"
 
 namespace {
@@ -144,7 +145,8 @@ PlanSet make_plans(const la_problem& q, int sm_count) {
   }
   const int64_t D = q.d;
   s.units = s.ps.BH * s.ps.nblk;
-  const size_t slot_bytes = size_t(D * D + int64_t(s.ps.zparts) * D) * 4;
+  // (the backward kernel writes up to bw::ZPARTS dz rows per slot)
+  const size_t slot_bytes = size_t(D * D + int64_t(s.tc ? std::max(s.ps.zparts, la::bw::ZPARTS) : s.ps.zparts) * D) * 4;
   size_t off = 0;
   s.off_partial = off;
   off = align256(off + size_t(s.ps.grid) * size_t(s.ps.maxseg) * slot_bytes);
@@ -556,6 +558,71 @@ int la_forward_tokencausal(const la_problem* p, const void* Q, const void* K, co
   int rc = validate(p);
   if (rc) return rc;
   return tokencausal_common(p, Q, K, V, G, O, ws, ws_bytes, stream);
+}
+
+int la_backward_bidir(const la_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                      const void* dO, void* dQ, void* dK, void* dV, void* dG, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
+  static_assert(la::st::TILE == la::bw::TILE, "the backward kernels walk the state kernel's tile ranges");
+  int rc = validate(p);
+  if (rc) return rc;
+  if (p->block_frames != 0) return LA_ERR_SHAPE;
+  const bool has_tok = elems(*p) > 0;
+  const void* ins[5] = {Q, K, V, G, dO};
+  void* outs[4] = {dQ, dK, dV, dG};
+  for (const void* x : ins)
+    if ((rc = check_ptr(x, has_tok))) return rc;
+  for (void* x : outs)
+    if ((rc = check_ptr(x, has_tok))) return rc;
+  if (p->dtype != LA_BF16 || p->d != 128 || (p->flags & LA_FLAG_FORCE_SIMT)) return LA_ERR_UNSUPPORTED;
+  if (!has_tok) {
+    g_last_launches = 0;
+    return LA_OK;
+  }
+  int sm = 0;
+  if ((rc = current_sm_count(&sm))) return rc;
+  const PlanSet s = make_plans(*p, sm);
+  if ((rc = check_ws(s, ws, ws_bytes))) return rc;
+  int nl = 0;
+  // Forward state (S, z) and its operand image, as for the forward pass.
+  if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
+  if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
+  if ((rc = launch_combine(s, *p, ws, nullptr, nullptr, nullptr, nullptr, true, stream, &nl))) return rc;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const Rope rope = make_rope(*p);
+  const bool sb = standard_bands(*p);
+  CUtensorMap tq, tg, tdo, tdq, tdg, tk, tv, tdk, tdv;
+  if (!make_tmap(&tq, Q, s.ps.BH, s.ps.N) || !make_tmap(&tg, G, s.ps.BH, s.ps.N) ||
+      !make_tmap(&tdo, dO, s.ps.BH, s.ps.N) || !make_tmap(&tdq, dQ, s.ps.BH, s.ps.N) ||
+      !make_tmap(&tdg, dG, s.ps.BH, s.ps.N) || !make_tmap(&tk, K, s.ps.BH, s.ps.N) ||
+      !make_tmap(&tv, V, s.ps.BH, s.ps.N) || !make_tmap(&tdk, dK, s.ps.BH, s.ps.N) ||
+      !make_tmap(&tdv, dV, s.ps.BH, s.ps.N))
+    return LA_ERR_CUDA;
+  // Q side: dQ, dG and the partial sums of dS, dz.
+  auto kq = sb ? la::bw::bwdq_tc_kernel<32, 48> : la::bw::bwdq_tc_kernel<-1, -1>;
+  if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, la::bw::SMEM_Q) != cudaSuccess)
+    return LA_ERR_CUDA;
+  if (launch_k(kq, unsigned(s.ps.grid), la::bw::THREADS, la::bw::SMEM_Q, stream, true, tq, tg, tdo, tdq, tdg, s.ps,
+               rope, static_cast<const uint8_t*>(w + s.off_img), reinterpret_cast<const float*>(w + s.off_zimg),
+               reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2),
+               reinterpret_cast<float*>(w + s.off_partial)))
+    return LA_ERR_CUDA;
+  ++nl;
+  // dS, dz summed in fixed order into the operand image (reusing the state image's space).
+  PlanSet s2 = s;
+  s2.ps.zparts = la::bw::ZPARTS;
+  if ((rc = launch_combine(s2, *p, ws, nullptr, nullptr, nullptr, nullptr, true, stream, &nl))) return rc;
+  // K side: dK, dV.
+  auto kk = sb ? la::bw::bwdk_tc_kernel<32, 48> : la::bw::bwdk_tc_kernel<-1, -1>;
+  if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, la::bw::SMEM_K) != cudaSuccess)
+    return LA_ERR_CUDA;
+  if (launch_k(kk, unsigned(s.ps.grid), la::bw::THREADS, la::bw::SMEM_K, stream, true, tk, tv, tdk, tdv, s.ps, rope,
+               static_cast<const uint8_t*>(w + s.off_img), reinterpret_cast<const float*>(w + s.off_zimg),
+               reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2)))
+    return LA_ERR_CUDA;
+  ++nl;
+  g_last_launches = nl;
+  return LA_OK;
 }
 
 int la_state_scan(const la_problem* p, float* S, float* z, cudaStream_t stream) {

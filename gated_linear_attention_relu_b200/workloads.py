@@ -161,6 +161,18 @@ def generate_gates(w: Workload, device="cpu", seed: Optional[int] = None):
     return beta.to(_torch_dtype(w.dtype)).contiguous(), gamma.contiguous()
 
 
+
+def generate_grad(w: Workload, device="cpu", seed: Optional[int] = None):
+    """An output gradient dO [B, H, N, d] for workload ``w``: N(0, 1) rounded to ``w.dtype``, seeded
+    with ``w.seed + 11`` (or ``seed``), independent of ``generate``."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed((w.seed + 11) if seed is None else seed)
+    x = torch.randn((w.B, w.H, w.N, w.d), generator=g, device=device, dtype=torch.float32)
+    return x.to(_torch_dtype(w.dtype)).contiguous()
+
+
 def custom(name: str, B: int, H: int, T: int, Hh: int, W: int, d: int = 128,
            bands: Optional[Tuple[int, int, int]] = None, dtype: str = "bf16", seed: int = 7,
            qkv_scale: Optional[float] = None, k_shift: float = 0.0, block_frames: int = 0,

@@ -153,6 +153,19 @@ int la_forward_tokencausal(const la_problem* p, const void* Q, const void* K, co
                            const void* G, void* O, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream);
 
+/* Gradients of the bidirectional operator (la_forward_bidir) for training: given the output
+ * gradient dO, writes dQ, dK, dV, dG (same layout and dtype as the inputs).  With
+ * s = sigmoid(G), y = num / den the pre-gate output and ReLU'(x) = [x > 0]:
+ *   dG = dO y s (1 - s),  dnum = dO s / den,  dden = -(dO s . y) / den,
+ *   dS = sum_n phi(Q_n)^T dnum_n,  dz = sum_n dden_n ReLU(Q_n),
+ *   dQ = [Q > 0] (RoPE^T(dnum S^T) + dden z),  dV = phi(K) dS,  dK = [K > 0] (RoPE^T(V dS^T) + dz)
+ * (the chain rule through SANA-Video 2.0, Eq. (1)).  p->block_frames must be 0.  Tensor-core
+ * path only in this version: bf16, d = 128, no LA_FLAG_FORCE_SIMT; else LA_ERR_UNSUPPORTED.
+ * Recomputes the forward state; queues 6 kernels. */
+int la_backward_bidir(const la_problem* p, const void* Q, const void* K, const void* V,
+                      const void* G, const void* dO, void* dQ, void* dK, void* dV, void* dG,
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Optional terms of the full gated form (SANA-Video 2.0, Sec. 2, Eq. (1)):
  *   S = sum_n beta_n phi(K_n)^T V_n            (write gate; z keeps the un-gated ReLU(K_n):
  *                                               Eq. (1)'s denominator has no beta)

@@ -114,3 +114,12 @@ def test_tokencausal_rejects_unsupported_problems_before_cuda():
         args.update(kw)
         cp = la.Problem(**args).c()
         assert lib.la_forward_tokencausal(ctypes.byref(cp), 16, 16, 16, 16, 16, 16, 1 << 30, None) == status
+
+
+def test_backward_rejects_unsupported_problems_before_cuda():
+    lib = la.load()
+    for kw, status in ((dict(dtype="f32"), 5), (dict(d=32, bands=(8, 12, 12)), 5), (dict(block_frames=1), 2)):
+        args = dict(B=1, H=2, T=3, Hh=4, W=5)
+        args.update(kw)
+        cp = la.Problem(**args).c()
+        assert lib.la_backward_bidir(ctypes.byref(cp), *([16] * 9), 16, 1 << 30, None) == status
