@@ -294,7 +294,7 @@ def main():
 
     # Marker events around each kernel of each timed step; recorded once here so their CUDA
     # handles exist before the timed region.
-    nmark = 5
+    nmark = 6
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nmark)] for _ in range(args.steps)]
     for row in evs:
         for e in row:
@@ -368,6 +368,8 @@ def main():
         tc = not args.simt and w.d == 128 and w.dtype == "bf16"
         if args.causal:
             names = ["rope_table_kernel", "state_tc_kernel", "start_kernel", "causal_tc_kernel"]
+        elif tc and w.nblk > 1:
+            names = ["rope_table_kernel", "state_tc_kernel", "blocksum_kernel", "prefix_kernel", "apply_tc_kernel"]
         elif tc:
             names = ["rope_table_kernel", "state_tc_kernel", "combine_kernel", "apply_tc_kernel"]
         else:

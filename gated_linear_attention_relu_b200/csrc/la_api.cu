@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <functional>
 #include <mutex>
 
 #include <cuda.h>
@@ -314,8 +315,10 @@ int launch_state(const PlanSet& s, const la_problem& q, const void* K, const voi
   return launched_ok();
 }
 
+// `after` (optional) is called with the launch count after each kernel this queues (timing marks).
 int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk, float* z_blk, float* S_inc,
-                   float* z_inc, bool img, cudaStream_t st, int* nl, bool accumulate = false) {
+                   float* z_inc, bool img, cudaStream_t st, int* nl, bool accumulate = false,
+                   const std::function<void(int)>& after = nullptr) {
   const int64_t groups = (int64_t(s.ps.d) * s.ps.d + s.ps.d) / 8;
   const int64_t threads = s.ps.BH * groups;
   if (threads == 0 || s.ps.nblk == 0) return LA_OK;
@@ -325,12 +328,35 @@ int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk
   float* zim = img ? reinterpret_cast<float*>(w + s.off_zimg) : nullptr;
   (void)q;
   const int64_t cblocks = (threads + la::cmb::THREADS - 1) / la::cmb::THREADS;
+  // Block-causal, tensor-core path (several blocks, no accumulation): per-block sums of all units
+  // in parallel, then the prefix over blocks.  The per-block states go to the caller's S_blk if it
+  // wants them, else to the workspace's state area (on this path the inclusive states go only to
+  // the caller's buffer and the operand image, never to that area, so nothing aliases).
+  if (s.tc && s.ps.nblk > 1 && !accumulate) {
+    float* sb = S_blk ? S_blk : reinterpret_cast<float*>(w + s.off_states);
+    float* zb = S_blk ? z_blk : reinterpret_cast<float*>(w + s.off_states) + s.units * q.d * q.d;
+    const int64_t t1 = s.units * groups;
+    if (launch_k(la::cmb::blocksum_kernel, unsigned((t1 + la::cmb::THREADS - 1) / la::cmb::THREADS),
+                 la::cmb::THREADS, 0, st, s.tc && s.ps.total > 0, s.ps, partial, sb, zb))
+      return LA_ERR_CUDA;
+    ++*nl;
+    if (after) after(*nl);
+    if (S_inc || im) {
+      if (launch_k(la::cmb::prefix_kernel, unsigned(cblocks), la::cmb::THREADS, 0, st, true, s.ps,
+                   static_cast<const float*>(sb), static_cast<const float*>(zb), S_inc, z_inc, im, zim))
+        return LA_ERR_CUDA;
+      ++*nl;
+      if (after) after(*nl);
+    }
+    return LA_OK;
+  }
   // After the tensor-core state kernel (if it ran) the combine kernel may launch early; it waits
   // for that kernel before its first read.
   if (launch_k(la::cmb::combine_kernel, unsigned(cblocks), la::cmb::THREADS, 0, st, s.tc && s.ps.total > 0,
                s.ps, partial, S_blk, z_blk, S_inc, z_inc, im, zim, accumulate ? 1 : 0))
     return LA_ERR_CUDA;
   ++*nl;
+  if (after) after(*nl);
   return launched_ok();
 }
 
@@ -720,11 +746,9 @@ static int forward_common(const la_problem* p, const void* Q, const void* K, con
   const int b0 = nl;
   if ((rc = launch_state(s, *p, K, V, ws, stream, &nl, gt.beta))) return rc;
   if (nl != b0) mark(nl);
-  const int before = nl;
   if ((rc = launch_combine(s, *p, ws, nullptr, nullptr, need_fp32 ? st_S : nullptr, need_fp32 ? st_z : nullptr,
-                           s.tc, stream, &nl)))
+                           s.tc, stream, &nl, false, mark)))
     return rc;
-  if (nl != before) mark(nl);
   if (has_tok) {
     const int b2 = nl;
     if ((rc = launch_apply(s, *p, Q, G, st_S, st_z, O, ws, stream, &nl, gt))) return rc;

@@ -360,6 +360,71 @@ combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, fl
   }
 }
 
+// Block-causal combine, first pass: the state of every (head, block) unit alone, summed over its
+// CTAs' partial slots in increasing CTA order.  One thread per (unit, group of 8 consecutive
+// elements of [S | z]), so all units run in parallel.
+__global__ void __launch_bounds__(THREADS)
+blocksum_kernel(const Plan p, const float* __restrict__ partial, float* __restrict__ S_blk, float* __restrict__ z_blk) {
+  pdl_trigger();
+  pdl_wait();
+  const int D = p.d;
+  const int groups = (D * D + D) / 8;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
+  const int64_t u = idx / groups;
+  if (u >= p.BH * p.nblk) return;
+  const int e0 = static_cast<int>(idx - u * groups) * 8;
+  const int64_t slot_floats = static_cast<int64_t>(D) * D + static_cast<int64_t>(p.zparts) * D;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  int64_t first = 0, count = 0;
+  if (p.total > 0) unit_tiles(p, u, &first, &count);
+  if (count > 0) {
+    const int64_t c0 = cta_of(p, first), c1 = cta_of(p, first + count - 1);
+    for (int64_t cc = c0; cc <= c1; ++cc) {
+      const int64_t k = u - unit_of_tile(p, cta_start(p, cc));
+      const float* src = partial + (cc * p.maxseg + k) * slot_floats;
+      for (int zp = 0; zp < (e0 < D * D ? 1 : p.zparts); ++zp) {
+        const float4* s4 = reinterpret_cast<const float4*>(e0 < D * D ? src + e0 : src + D * D + zp * D + (e0 - D * D));
+        const float4 a = s4[0], b = s4[1];
+        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+      }
+    }
+  }
+  store8(S_blk, z_blk, u, D, e0, acc);
+}
+
+// Block-causal combine, second pass: inclusive prefix over the blocks of every head, from the
+// per-block states of the first pass; writes the inclusive states and/or the operand image.
+// One thread per (head, group of 8 elements); the loads of different blocks are independent, so
+// they overlap.
+__global__ void __launch_bounds__(THREADS)
+prefix_kernel(const Plan p, const float* __restrict__ S_blk, const float* __restrict__ z_blk, float* S_inc,
+              float* z_inc, uint8_t* img, float* zimg) {
+  pdl_trigger();
+  pdl_wait();
+  const int D = p.d;
+  const int groups = (D * D + D) / 8;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
+  const int64_t bh = idx / groups;
+  if (bh >= p.BH) return;
+  const int e0 = static_cast<int>(idx - bh * groups) * 8;
+  float run[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) run[e] = 0.f;
+#pragma unroll 4
+  for (int64_t blk = 0; blk < p.nblk; ++blk) {
+    const int64_t u = bh * p.nblk + blk;
+    const float* src = (e0 < D * D) ? S_blk + u * D * D + e0 : z_blk + u * D + (e0 - D * D);
+    const float4 a = reinterpret_cast<const float4*>(src)[0], b = reinterpret_cast<const float4*>(src)[1];
+    run[0] += a.x; run[1] += a.y; run[2] += a.z; run[3] += a.w;
+    run[4] += b.x; run[5] += b.y; run[6] += b.z; run[7] += b.w;
+    if (S_inc) store8(S_inc, z_inc, u, D, e0, run);
+    if (img) write_image(img, zimg, u, D, e0, run);
+  }
+}
+
 // Token-causal: the state each CTA's first unit carries into the CTA's tile range, i.e. the sum,
 // in CTA order, of that unit's partial states from the CTAs before it (zero when the unit starts
 // in the CTA itself).  One thread per (CTA, group of 8 consecutive elements of [S | z]).
