@@ -68,7 +68,7 @@ constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/tru
 // 65536 / THREADS); the control warpgroup shrinks to REGS_CTRL and the math groups grow to
 // REGS_MATH, never asking for more than the launch granted.
 constexpr uint32_t REGS_LAUNCH = (65536 / THREADS) / 8 * 8;
-constexpr uint32_t REGS_CTRL = 24;  // the single-lane control loops need few registers
+constexpr uint32_t REGS_CTRL = 56;  // the single-lane control loops (the MMA issuer keeps per-group state)
 constexpr uint32_t REGS_MATH_FIT = ((THREADS * REGS_LAUNCH - 128 * REGS_CTRL) / (128 * MATH_WGS)) / 8 * 8;
 constexpr uint32_t REGS_MATH = REGS_MATH_FIT > 232 ? 232 : REGS_MATH_FIT;
 constexpr bool SPLIT_REGS = true;
@@ -294,30 +294,72 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      for (int64_t g = g0; g < g1; ++g) {
-        const int64_t i = g - g0;
-        const int64_t u = unit_of_tile(p, g);
-        const int64_t ku = u - u_first;
-        const int b = static_cast<int>(ku % NSB);
-        const int m = static_cast<int>(i % NWG);
-        const uint32_t kph = static_cast<uint32_t>((i / NWG) & 1);  // parity of the group's k-th tile
-        if (!mbar_wait(&bars->accempty[m], kph ^ 1u, abort_flag)) break;
-        if (!mbar_wait(&bars->aready[m], kph, abort_flag)) break;
-        if (!mbar_wait(&bars->sfull[b], static_cast<uint32_t>((ku / NSB) & 1), abort_flag)) break;
-        tc_fence_after();
-        const uint32_t acc = tmem + static_cast<uint32_t>(m) * GROUP_COLS + ACC_COL;
-        const uint32_t at = tmem + static_cast<uint32_t>(m) * GROUP_COLS + A_COL;
-        const uint32_t sa = sbase + OFF_S + b * BUF;
+      // The math groups are served independently, each in its own tile order, so a group that is
+      // ahead never waits behind the other group's tile.  A state buffer is freed after the last
+      // of its unit's tiles in this CTA's range has been issued (by either group).
+      int64_t next[NWG];
+      uint32_t kdone[NWG];
+      for (int mm = 0; mm < NWG; ++mm) {
+        next[mm] = g0 + mm;
+        kdone[mm] = 0;
+      }
+      int64_t buf_unit[NSB], buf_issued[NSB];
+      for (int bb = 0; bb < NSB; ++bb) {
+        buf_unit[bb] = -1;
+        buf_issued[bb] = 0;
+      }
+      uint64_t t_progress = globaltimer_ns();
+      uint32_t idle = 0;
+      bool ok = true;
+      while (ok) {
+        bool pending = false, progressed = false;
+        for (int mm = 0; mm < NWG; ++mm) {
+          const int64_t g = next[mm];
+          if (g >= g1) continue;
+          pending = true;
+          const int64_t u = unit_of_tile(p, g);
+          const int64_t ku = u - u_first;
+          const int b = static_cast<int>(ku % NSB);
+          const uint32_t kph = kdone[mm] & 1u;
+          if (!mbar_test_wait(&bars->accempty[mm], kph ^ 1u) || !mbar_test_wait(&bars->aready[mm], kph) ||
+              !mbar_test_wait(&bars->sfull[b], static_cast<uint32_t>((ku / NSB) & 1)))
+            continue;
+          tc_fence_after();
+          const uint32_t acc = tmem + static_cast<uint32_t>(mm) * GROUP_COLS + ACC_COL;
+          const uint32_t at = tmem + static_cast<uint32_t>(mm) * GROUP_COLS + A_COL;
+          const uint32_t sa = sbase + OFF_S + b * BUF;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // K step kk: A columns 8kk .. 8kk+7 (16 bf16), B rows 16kk .. 16kk+15 (two 8-row groups).
-          const uint64_t bd = smem_desc_sw128(sa + kk * 2048, HALF, 1024);
-          mma_bf16_ts(acc, at + 8 * kk, bd, IDESC, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // K step kk: A columns 8kk .. 8kk+7 (16 bf16), B rows 16kk .. 16kk+15 (two 8-row groups).
+            const uint64_t bd = smem_desc_sw128(sa + kk * 2048, HALF, 1024);
+            mma_bf16_ts(acc, at + 8 * kk, bd, IDESC, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars->accfull[mm]);
+          mma_commit(&bars->afree[mm]);
+          if (buf_unit[b] != u) {
+            buf_unit[b] = u;
+            buf_issued[b] = 0;
+          }
+          int64_t first = 0, count = 0;
+          unit_tiles(p, u, &first, &count);
+          const int64_t in_range = (first + count < g1 ? first + count : g1) - (first > g0 ? first : g0);
+          if (++buf_issued[b] == in_range) mma_commit(&bars->sfree[b]);
+          next[mm] += NWG;
+          ++kdone[mm];
+          progressed = true;
         }
-        mma_commit(&bars->accfull[m]);
-        mma_commit(&bars->afree[m]);
-        const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != u);
-        if (last) mma_commit(&bars->sfree[b]);
+        if (!pending) break;
+        if (progressed) {
+          t_progress = globaltimer_ns();
+          idle = 0;
+        } else if ((++idle & 255u) == 0u) {
+          if (*abort_flag) break;
+          if (globaltimer_ns() - t_progress > LA_WAIT_LIMIT_NS) {
+            *abort_flag = 1;
+            atomicOr(&g_la_error, ERR_WAIT_TIMEOUT);
+            ok = false;
+          }
+        }
       }
       mma_commit(&bars->final_);
       mbar_wait_drain(&bars->final_, 0);
