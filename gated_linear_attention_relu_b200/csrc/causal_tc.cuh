@@ -18,8 +18,9 @@
 // image of the carried state in shared memory (rewritten after every chunk).
 //
 // Warps: 0-3 own the chunk's rows (thread = token = TMEM lane); warp 4 issues the TMA copies and
-// the MMAs.  One chunk at a time (each phase waits for the previous one): this first version
-// favours clarity over overlap.
+// the MMAs.  The phases of a chunk run in sequence; the next chunk's tiles are loaded as soon as
+// their buffers are free (Q and K once the products reading them are done, V after P V, G after
+// this chunk's O has been stored), so their latency overlaps the end of the chunk.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -124,37 +125,30 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tma_prefetch_desc(&tmG);
       tma_prefetch_desc(&tmO);
       int64_t prev_unit = -1;
-      int64_t issued = 0;
-      TileInfo tprev{};
-      bool ok = true;
-      for (int64_t g = g0; g < g1 && ok; ++g) {
+      int64_t issued = 0;  // chunks whose loads have been armed on `full`
+      auto load2 = [&](uint32_t off, const CUtensorMap* tm, const TileInfo& t) {
+        const int32_t n0 = static_cast<int32_t>(t.n0), bh = static_cast<int32_t>(t.bh);
+        tma_load_3d(smem + off, tm, 0, n0, bh, &bars->full);
+        tma_load_3d(smem + off + HALF, tm, 64, n0, bh, &bars->full);
+      };
+      if (g0 < g1) {
+        const TileInfo t0 = tile_info(p, g0);
+        mbar_arrive_expect_tx(&bars->full, 4 * BUF);
+        load2(OFF_Q, &tmQ, t0);
+        load2(OFF_K, &tmK, t0);
+        load2(OFF_V, &tmV, t0);
+        load2(OFF_G, &tmG, t0);
+        issued = 1;
+      }
+      for (int64_t g = g0; g < g1; ++g) {
         const int64_t i = g - g0;
         const uint32_t ph = static_cast<uint32_t>(i & 1);
         const TileInfo ti = tile_info(p, g);
         const bool first = ti.unit != prev_unit;
         const bool zero_start = first && !(g == g0 && has_start);
         prev_unit = ti.unit;
-        if (i > 0) {
-          // The previous chunk is finished: store its O (staged over G), then reuse the buffers.
-          if (!mbar_wait(&bars->out, static_cast<uint32_t>((i - 1) & 1), abort_flag)) break;
-          const int32_t pn0 = static_cast<int32_t>(tprev.n0), pbh = static_cast<int32_t>(tprev.bh);
-          tma_store_3d(&tmO, smem + OFF_G, 0, pn0, pbh);
-          tma_store_3d(&tmO, smem + OFF_G + HALF, 64, pn0, pbh);
-          bulk_commit_group();
-          bulk_wait_group_read0();
-        }
-        tprev = ti;
-        mbar_arrive_expect_tx(&bars->full, 4 * BUF);
-        const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
-        tma_load_3d(smem + OFF_Q, &tmQ, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + OFF_Q + HALF, &tmQ, 64, n0, bh, &bars->full);
-        tma_load_3d(smem + OFF_K, &tmK, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + OFF_K + HALF, &tmK, 64, n0, bh, &bars->full);
-        tma_load_3d(smem + OFF_V, &tmV, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + OFF_V + HALF, &tmV, 64, n0, bh, &bars->full);
-        tma_load_3d(smem + OFF_G, &tmG, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + OFF_G + HALF, &tmG, 64, n0, bh, &bars->full);
-        ++issued;
+        const bool has_next = g + 1 < g1;
+        const TileInfo tn = has_next ? tile_info(p, g + 1) : ti;
         // D = Q^+ K^+^T
         if (!mbar_wait(&bars->relu, ph, abort_flag)) break;
         tc_fence_after();
@@ -179,6 +173,15 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           mma_bf16(tmem + COL_S, desc_mn(sbase + OFF_K, kk), desc_mn(sbase + OFF_V, kk), IDESC_KV,
                    (kk > 0 || !zero_start) ? 1u : 0u);
         mma_commit(&bars->pready);
+        // Those products were the last readers of Q and K: the next chunk's Q and K can land
+        // while this chunk's P V product and epilogue run.
+        if (has_next) {
+          if (!mbar_wait(&bars->pready, ph, abort_flag)) break;
+          mbar_arrive_expect_tx(&bars->full, 4 * BUF);
+          load2(OFF_Q, &tmQ, tn);
+          load2(OFF_K, &tmK, tn);
+          ++issued;
+        }
         // num += (P o M) V
         if (!mbar_wait(&bars->pw, ph, abort_flag)) break;
         tc_fence_after();
@@ -187,14 +190,20 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           mma_bf16_ts(tmem + COL_ND, tmem + COL_P + 8u * kk, desc_mn(sbase + OFF_V, kk), IDESC_QS,
                       (kk > 0 || !zero_start) ? 1u : 0u);
         mma_commit(&bars->numready);
-      }
-      // Store the last chunk's O.
-      if (issued > 0 && !*abort_flag &&
-          mbar_wait(&bars->out, static_cast<uint32_t>((issued - 1) & 1), abort_flag)) {
-        const int32_t pn0 = static_cast<int32_t>(tprev.n0), pbh = static_cast<int32_t>(tprev.bh);
-        tma_store_3d(&tmO, smem + OFF_G, 0, pn0, pbh);
-        tma_store_3d(&tmO, smem + OFF_G + HALF, 64, pn0, pbh);
-        bulk_commit_group();
+        if (has_next) {
+          if (!mbar_wait(&bars->numready, ph, abort_flag)) break;
+          load2(OFF_V, &tmV, tn);
+        }
+        // O of this chunk (staged over G) out, then the next chunk's G in.
+        if (!mbar_wait(&bars->out, ph, abort_flag)) break;
+        {
+          const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
+          tma_store_3d(&tmO, smem + OFF_G, 0, n0, bh);
+          tma_store_3d(&tmO, smem + OFF_G + HALF, 64, n0, bh);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        if (has_next) load2(OFF_G, &tmG, tn);
       }
       bulk_wait_group0();
       if (*abort_flag && issued > 0) mbar_wait_drain(&bars->full, static_cast<uint32_t>((issued - 1) & 1));
