@@ -136,8 +136,12 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def oracle_sample(w, seconds, steps=None, warmup=0):
-    """Time the fp64 oracle on one head of the workload (all its tokens): token*heads/s."""
+def oracle_sample(w, seconds, steps=None, warmup=0, mode="forward"):
+    """Time the fp64 oracle on one head of the workload (all its tokens): token*heads/s.
+
+    ``mode`` picks the oracle of what the GPU run measures: "forward" (bidirectional or
+    block-causal, as the workload says), "gated" (write gate and RMSNorm), "causal"
+    (token-causal) or "backward" (gradients of the bidirectional form)."""
     import numpy as np
 
     import oracle as orc
@@ -146,9 +150,24 @@ def oracle_sample(w, seconds, steps=None, warmup=0):
     one = w.with_(B=1, H=1)
     Q, K, V, G = (t.float().numpy().astype(np.float64)[0, 0] for t in wl.generate(one, "cpu"))
     pos = orc.grid_positions(w.T, w.Hh, w.W)
+    if mode == "gated":
+        beta, gamma = (t.float().numpy().astype(np.float64) for t in wl.generate_gates(one, "cpu"))
+        beta = beta[0, 0]
+    if mode == "backward":
+        dO = wl.generate_grad(one, "cpu").float().numpy().astype(np.float64)[0, 0]
+    # The token-causal oracle walks rows one by one in Python: time it on a fixed sample of rows
+    # (it still carries the state over every token).
+    rows = np.sort(np.random.default_rng(0).choice(w.N, size=min(w.N, 2000), replace=False)) \
+        if mode == "causal" else None
 
     def run():
-        if w.block_frames > 0:
+        if mode == "causal":
+            orc.tokencausal_rows(Q, K, V, G, pos, w.bands, w.rope_base, w.eps, rows=rows)
+        elif mode == "backward":
+            orc.head_backward(Q, K, V, G, dO, pos, w.bands, w.rope_base, w.eps)
+        elif mode == "gated":
+            orc.forward_positions(Q, K, V, G, pos, w.bands, w.rope_base, w.eps, beta=beta, rms=(gamma, 1e-6))
+        elif w.block_frames > 0:
             Sb, zb = orc.block_states(K, V, pos, w.bands, w.rope_base, w.block_frames)
             Si, zi = np.cumsum(Sb, 0), np.cumsum(zb, 0)
             blk = orc.block_of_tokens(pos, w.block_frames)
@@ -178,7 +197,8 @@ def oracle_sample(w, seconds, steps=None, warmup=0):
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
         pass
-    value = w.N * len(times) / sum(times)
+    per_run = len(rows) if rows is not None else w.N
+    value = per_run * len(times) / sum(times)
     return value, threads, times
 
 
@@ -423,10 +443,11 @@ def main():
     if not args.no_e2e and not whole_step:
         line["e2e"] = e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates, causal=args.causal)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, times = oracle_sample(w, args.cpu_seconds)
+        mode = "causal" if args.causal else ("backward" if args.backward else ("gated" if args.gated else "forward"))
+        v, cores, times = oracle_sample(w, args.cpu_seconds, mode=mode)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"one head of {w.name} (all {w.N} tokens), {len(times)} runs, "
-                                          f"fp64 numpy oracle"}
+                                "sample": f"one head of {w.name} ({'2000 sampled outputs' if mode == 'causal' else f'all {w.N} tokens'}), "
+                                          f"{len(times)} runs, fp64 numpy oracle ({mode})"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     ldist.finalize()
