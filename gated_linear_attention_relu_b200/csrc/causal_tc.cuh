@@ -17,8 +17,8 @@
 // P o M goes back to TMEM as bf16 and is the A operand of the P V product; S_prev is the bf16
 // image of the carried state in shared memory (rewritten after every chunk).
 //
-// Warps: 0-3 own the chunk's rows (thread = token = TMEM lane); warp 4 issues the TMA copies and
-// the MMAs.  The phases of a chunk run in sequence; the next chunk's tiles are loaded as soon as
+// Warps: 0-7 own the chunk's rows, two per row (channel halves; thread = token = TMEM lane, warp
+// w reaching lanes 32 (w mod 4) ..); warp 8 issues the TMA copies and the MMAs.  The phases of a chunk run in sequence; the next chunk's tiles are loaded as soon as
 // their buffers are free (Q and K once the products reading them are done, V after P V, G after
 // this chunk's O has been stored), so their latency overlaps the end of the chunk.
 #pragma once
@@ -33,12 +33,16 @@ using namespace la::tile;
 
 constexpr int TILE = 128;
 constexpr int D = 128;
-constexpr int THREADS = 160;
+constexpr int MATH_WARPS = 8;  // two per TMEM lane quarter: channel halves of a row
+constexpr int CTRL_WARP = MATH_WARPS;
+constexpr int THREADS = 32 * (MATH_WARPS + 1);
 constexpr uint32_t HALF = 128 * 128;
 constexpr uint32_t BUF = 2 * HALF;
 constexpr uint32_t OFF_Q = 0, OFF_K = BUF, OFF_V = 2 * BUF, OFF_G = 3 * BUF, OFF_S = 4 * BUF;
-constexpr uint32_t OFF_Z = 5 * BUF;  // z of the tokens before the chunk, [128] fp32
-constexpr uint32_t OFF_BAR = OFF_Z + 512;
+constexpr uint32_t OFF_Z = 5 * BUF;            // z of the tokens before the chunk, [128] fp32
+constexpr uint32_t OFF_ZP = OFF_Z + 512;       // the chunk's K^+ column sums per row half, [2][128]
+constexpr uint32_t OFF_DX = OFF_ZP + 1024;     // partial denominators, [2 slots][2 halves][128]
+constexpr uint32_t OFF_BAR = OFF_DX + 2048;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S = 0, COL_ND = 128, COL_P = 256;  // carried S; D then num; P (then bf16 P)
@@ -57,7 +61,9 @@ struct Bars {
   uint64_t pready;    // MMA: num (inter), P and the S update done
   uint64_t pw;        // math: masked P written to TMEM as bf16 (4 warps)
   uint64_t numready;  // MMA: num += P V done
-  uint64_t out;       // math: O staged over G, S image rewritten (4 warps)
+  uint64_t out;       // math: O staged over G, S image rewritten (8 warps)
+  uint64_t denx[4];   // the two warps holding the halves of rows 32q .. 32q+31 (2 arrivals);
+                      // two phases per chunk: the denominator swap (even), the P handoff (odd)
   uint64_t final_;
   uint32_t tmem_base;
   int abort_flag;
@@ -93,20 +99,21 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->full, 1);
-    mbar_init(&bars->relu, 4);
-    mbar_init(&bars->zsync1, 4);
-    mbar_init(&bars->zsync, 4);
+    mbar_init(&bars->relu, MATH_WARPS);
+    mbar_init(&bars->zsync1, MATH_WARPS);
+    mbar_init(&bars->zsync, MATH_WARPS);
     mbar_init(&bars->dready, 1);
-    mbar_init(&bars->rot, 4);
+    mbar_init(&bars->rot, MATH_WARPS);
     mbar_init(&bars->pready, 1);
-    mbar_init(&bars->pw, 4);
+    mbar_init(&bars->pw, MATH_WARPS);
     mbar_init(&bars->numready, 1);
-    mbar_init(&bars->out, 4);
+    mbar_init(&bars->out, MATH_WARPS);
+    for (int q = 0; q < 4; ++q) mbar_init(&bars->denx[q], 2);
     mbar_init(&bars->final_, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == CTRL_WARP) {
     tmem_alloc(&bars->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
@@ -116,7 +123,7 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const uint32_t tmem = bars->tmem_base;
   pdl_trigger();
 
-  if (warp == 4) {
+  if (warp == CTRL_WARP) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA + MMA issue
       tma_prefetch_desc(&tmQ);
@@ -211,25 +218,31 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_wait_drain(&bars->final_, 0);
     }
   } else {
-    // ------------------------------------------------------------ rows (warps 0-3)
-    const int row = threadIdx.x;  // token row of the chunk = TMEM lane; also channel k for z and S
-    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t t_s = tmem + COL_S + lane_bits, t_nd = tmem + COL_ND + lane_bits, t_p = tmem + COL_P + lane_bits;
-    float zk = 0.f;  // z of channel `row` over the tokens before the chunk
+    // ------------------------------------------------------------ rows (warps 0-7)
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int row = quarter * 32 + lane;  // token row of the chunk = TMEM lane; also channel k for z and S
+    const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t t_s = tmem + COL_S + lane_bits + 64u * hf, t_nd = tmem + COL_ND + lane_bits + 64u * hf;
+    const uint32_t t_p = tmem + COL_P + lane_bits;
+    float* zp = reinterpret_cast<float*>(smem + OFF_ZP);
+    float* dx = reinterpret_cast<float*>(smem + OFF_DX);
+    uint64_t* denx = &bars->denx[quarter];
+    float zk = 0.f;  // (hf == 0) z of channel `row` over the tokens before the chunk
     pdl_wait();      // the start states and the cos/sin tables come from the kernels before
     if (g0 < g1 && has_start) {
-      // Carried state at the segment start: fp32 row `row` of S into TMEM, its bf16 image, z.
+      // Carried state at the segment start: this half of fp32 row `row` of S into TMEM, its bf16
+      // image, and z.
       const float* src = start + c * (D * D + D);
       uint32_t r[32];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 2; ++j) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(src[row * D + 32 * j + e]);
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(src[row * D + 64 * hf + 32 * j + e]);
         tmem_st_x16(t_s + 32 * j, &r[0]);
         tmem_st_x16(t_s + 32 * j + 16, &r[16]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int ck = 4 * j + e;
+          const int ck = 8 * hf + 4 * j + e;
           sts128(row_chunk(sbase + OFF_S, row, ck),
                  make_uint4(pack_bf16(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
                             pack_bf16(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
@@ -239,7 +252,7 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       tmem_st_wait();
       fence_proxy_async_smem();
-      zk = src[D * D + row];
+      if (hf == 0) zk = src[D * D + row];
     }
     int64_t prev_unit = -1;
     for (int64_t g = g0; g < g1; ++g) {
@@ -249,17 +262,18 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if (ti.unit != prev_unit && !(g == g0 && has_start)) zk = 0.f;  // a head starting in this CTA
       prev_unit = ti.unit;
       if (!warp_wait(&bars->full, ph, abort_flag)) break;
-      // ReLU of Q and K in place; q^+ kept in registers.
-      uint32_t qa[64];
+      // ReLU of this half of the Q and K rows in place; q^+ kept in registers.
+      uint32_t qa[32];
 #pragma unroll
-      for (int ck = 0; ck < 16; ++ck) {
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const int ck = 8 * hf + c8;
         const uint32_t aq = row_chunk(sbase + OFF_Q, row, ck);
         const uint4 rq = lds128(aq);
-        qa[4 * ck] = relu_bf16x2(rq.x);
-        qa[4 * ck + 1] = relu_bf16x2(rq.y);
-        qa[4 * ck + 2] = relu_bf16x2(rq.z);
-        qa[4 * ck + 3] = relu_bf16x2(rq.w);
-        sts128(aq, make_uint4(qa[4 * ck], qa[4 * ck + 1], qa[4 * ck + 2], qa[4 * ck + 3]));
+        qa[4 * c8] = relu_bf16x2(rq.x);
+        qa[4 * c8 + 1] = relu_bf16x2(rq.y);
+        qa[4 * c8 + 2] = relu_bf16x2(rq.z);
+        qa[4 * c8 + 3] = relu_bf16x2(rq.w);
+        sts128(aq, make_uint4(qa[4 * c8], qa[4 * c8 + 1], qa[4 * c8 + 2], qa[4 * c8 + 3]));
         const uint32_t ak = row_chunk(sbase + OFF_K, row, ck);
         const uint4 rk = lds128(ak);
         sts128(ak, make_uint4(relu_bf16x2(rk.x), relu_bf16x2(rk.y), relu_bf16x2(rk.z), relu_bf16x2(rk.w)));
@@ -270,9 +284,9 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         mbar_arrive(&bars->relu);
         mbar_arrive(&bars->zsync1);
       }
-      // z before the chunk, published for every row's denominator; then this chunk's K^+ column
-      // (thread `row` sums channel `row` over the chunk's rows, once every row is ReLU'd).
-      zs[row] = zk;
+      // z before the chunk, published for every row's denominator (hf 0); then this chunk's K^+
+      // column `row` over this half's 64 rows, once every row is ReLU'd.
+      if (hf == 0) zs[row] = zk;
       if (!warp_wait(&bars->zsync1, ph, abort_flag)) break;
       {
         const int kc = row;  // channel
@@ -280,106 +294,130 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const uint32_t cchunk = static_cast<uint32_t>((kc & 63) >> 3), cbyte = static_cast<uint32_t>(kc & 7) * 2u;
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-        for (int m = 0; m < TILE; ++m) {
+        for (int mm = 0; mm < 64; ++mm) {
+          const int m = 64 * hf + mm;
           uint16_t hv;
           asm volatile("ld.shared.u16 %0, [%1];"
                        : "=h"(hv)
                        : "r"(kbase + static_cast<uint32_t>(m) * 128u + ((cchunk ^ static_cast<uint32_t>(m & 7)) << 4) +
                              cbyte));
-          s4[m & 3] += __uint_as_float(static_cast<uint32_t>(hv) << 16);
+          s4[mm & 3] += __uint_as_float(static_cast<uint32_t>(hv) << 16);
         }
-        zk += (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        zp[hf * 128 + row] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->zsync);
       if (!warp_wait(&bars->zsync, ph, abort_flag)) break;
-      // Denominator: q^+ . z_prev + masked row sum of D.
-      float dz = 0.f;
+      if (hf == 0) zk += zp[row] + zp[128 + row];
+      // This half's share of the denominator: q^+ . z_prev over its channels plus the masked row
+      // sum of D over its columns; the two halves of the row add theirs.
+      float dpart = 0.f;
 #pragma unroll
-      for (int k4 = 0; k4 < 32; ++k4) {
-        const float4 z4 = *reinterpret_cast<const float4*>(zs + 4 * k4);
-        dz = fmaf(bf16lo(qa[2 * k4]), z4.x, dz);
-        dz = fmaf(bf16hi(qa[2 * k4]), z4.y, dz);
-        dz = fmaf(bf16lo(qa[2 * k4 + 1]), z4.z, dz);
-        dz = fmaf(bf16hi(qa[2 * k4 + 1]), z4.w, dz);
+      for (int k4 = 0; k4 < 16; ++k4) {
+        const float4 z4 = *reinterpret_cast<const float4*>(zs + 64 * hf + 4 * k4);
+        dpart = fmaf(bf16lo(qa[2 * k4]), z4.x, dpart);
+        dpart = fmaf(bf16hi(qa[2 * k4]), z4.y, dpart);
+        dpart = fmaf(bf16lo(qa[2 * k4 + 1]), z4.z, dpart);
+        dpart = fmaf(bf16hi(qa[2 * k4 + 1]), z4.w, dpart);
       }
       if (!warp_wait(&bars->dready, ph, abort_flag)) break;
       tc_fence_after();
-      float dintra = 0.f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 2; ++j) {
         uint32_t r[32];
         tmem_ld_x32(t_nd + 32 * j, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) dintra += (32 * j + e <= row) ? __uint_as_float(r[e]) : 0.f;
+        for (int e = 0; e < 32; ++e) dpart += (64 * hf + 32 * j + e <= row) ? __uint_as_float(r[e]) : 0.f;
       }
-      const float hinv = 1.0f / (dz + dintra + p.eps);
-      // RoPE of Q^+ and K^+ in place.
+      {
+        float* slot = dx + static_cast<int>(i & 1) * 256;
+        slot[hf * 128 + row] = dpart;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(denx);
+        if (!warp_wait(denx, 0u, abort_flag)) break;
+        const float other = slot[(hf ^ 1) * 128 + row];
+        dpart = hf == 0 ? dpart + other : other + dpart;
+      }
+      const float hinv = 1.0f / (dpart + p.eps);
+      // RoPE of this half of Q^+ and K^+ in place.
       const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
       uint32_t pt = 0, ph_ = 0, pw = 0;
       if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph_, pw);
       {
-        uint32_t a[64];
+        uint32_t a[32];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) a[e] = qa[e];
-        rotate_row<DT, DH>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        for (int e = 0; e < 32; ++e) a[e] = qa[e];
+        if (hf == 0)
+          rotate_half<DT, DH, 0>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        else
+          rotate_half<DT, DH, 1>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
 #pragma unroll
-        for (int ck = 0; ck < 16; ++ck)
-          sts128(row_chunk(sbase + OFF_Q, row, ck), make_uint4(a[4 * ck], a[4 * ck + 1], a[4 * ck + 2], a[4 * ck + 3]));
+        for (int c8 = 0; c8 < 8; ++c8)
+          sts128(row_chunk(sbase + OFF_Q, row, 8 * hf + c8), make_uint4(a[4 * c8], a[4 * c8 + 1], a[4 * c8 + 2], a[4 * c8 + 3]));
 #pragma unroll
-        for (int ck = 0; ck < 16; ++ck) {
-          const uint4 rk = lds128(row_chunk(sbase + OFF_K, row, ck));
-          a[4 * ck] = rk.x;
-          a[4 * ck + 1] = rk.y;
-          a[4 * ck + 2] = rk.z;
-          a[4 * ck + 3] = rk.w;
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const uint4 rk = lds128(row_chunk(sbase + OFF_K, row, 8 * hf + c8));
+          a[4 * c8] = rk.x;
+          a[4 * c8 + 1] = rk.y;
+          a[4 * c8 + 2] = rk.z;
+          a[4 * c8 + 3] = rk.w;
         }
-        rotate_row<DT, DH>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        if (hf == 0)
+          rotate_half<DT, DH, 0>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        else
+          rotate_half<DT, DH, 1>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
 #pragma unroll
-        for (int ck = 0; ck < 16; ++ck)
-          sts128(row_chunk(sbase + OFF_K, row, ck), make_uint4(a[4 * ck], a[4 * ck + 1], a[4 * ck + 2], a[4 * ck + 3]));
+        for (int c8 = 0; c8 < 8; ++c8)
+          sts128(row_chunk(sbase + OFF_K, row, 8 * hf + c8), make_uint4(a[4 * c8], a[4 * c8 + 1], a[4 * c8 + 2], a[4 * c8 + 3]));
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->rot);
-      // Causal mask on P (m <= n), back to TMEM as the bf16 A operand of P V.
+      // Causal mask on this half of P (columns m in [64 hf, 64 hf + 64), kept where m <= n), back
+      // to TMEM as bf16 (the A operand of P V: columns 32 hf .. 32 hf + 31).
       if (!warp_wait(&bars->pready, ph, abort_flag)) break;
       tc_fence_after();
       {
-        uint32_t pb[64];
+        uint32_t pb[32];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 2; ++j) {
           uint32_t r[32];
-          tmem_ld_x32(t_p + 32 * j, r);
+          tmem_ld_x32(t_p + 64u * hf + 32 * j, r);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const int m0 = 32 * j + 2 * e;
+            const int m0 = 64 * hf + 32 * j + 2 * e;
             const float p0 = m0 <= row ? __uint_as_float(r[2 * e]) : 0.f;
             const float p1 = m0 + 1 <= row ? __uint_as_float(r[2 * e + 1]) : 0.f;
             pb[16 * j + e] = pack_bf16(p0, p1);
           }
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) tmem_st_x16(t_p + 16 * j, &pb[16 * j]);
+        // Half 1 writes bf16 columns 32-63, which half 0 reads as fp32: the pair meets once more
+        // (the odd phase of its barrier) before either writes.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(denx);
+        if (!warp_wait(denx, 1u, abort_flag)) break;
+        tmem_st_x16(t_p + 32u * hf, &pb[0]);
+        tmem_st_x16(t_p + 32u * hf + 16, &pb[16]);
         tmem_st_wait();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->pw);
-      // O = num / den * sigmoid(g), in place over G; then the new state's bf16 image.
+      // O = num / den * sigmoid(g) for this half, in place over G; then this half of the new
+      // state's bf16 image.
       if (!warp_wait(&bars->numready, ph, abort_flag)) break;
       tc_fence_after();
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 2; ++j) {
         uint32_t r[32];
         tmem_ld_x32(t_nd + 32 * j, r);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint32_t ag = row_chunk(sbase + OFF_G, row, 4 * j + e);
+          const uint32_t ag = row_chunk(sbase + OFF_G, row, 8 * hf + 4 * j + e);
           const uint4 gr = lds128(ag);
           const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
           uint32_t ov[4];
@@ -393,13 +431,13 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 2; ++j) {
         uint32_t r[32];
         tmem_ld_x32(t_s + 32 * j, r);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          sts128(row_chunk(sbase + OFF_S, row, 4 * j + e),
+          sts128(row_chunk(sbase + OFF_S, row, 8 * hf + 4 * j + e),
                  make_uint4(pack_bf16(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
                             pack_bf16(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
                             pack_bf16(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
@@ -415,7 +453,7 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) tmem_dealloc(tmem, TMEM_COLS);
+  if (warp == CTRL_WARP) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 }  // namespace ca

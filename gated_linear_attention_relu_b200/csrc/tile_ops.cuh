@@ -69,6 +69,46 @@ __device__ __forceinline__ void rotate_row(uint32_t (&a)[64], const float2* __re
   }
 }
 
+// In place over half a row (channels [64 HF, 64 HF + 64) as 32 bf16 pairs, already ReLU'd):
+// a <- RoPE(a) at grid position (pt, ph, pw).
+template <int DT, int DH, int HF>
+__device__ __forceinline__ void rotate_half(uint32_t (&a)[32], const float2* __restrict__ tab,
+                                            const float4* __restrict__ tab2, const Rope& rope, const Plan& p,
+                                            int pt, int ph, int pw) {
+  if constexpr (DT >= 0 && DH >= 0) {
+    constexpr int DW = 128 - DT - DH;
+    static_assert(DT % 4 == 0 && DH % 4 == 0 && DW % 4 == 0, "bands of whole 16-byte entries");
+    const float4* bt = tab2 + pt * (DT / 4);
+    const float4* bh = tab2 + rope.tab_off_h / 2 + ph * (DH / 4);
+    const float4* bw = tab2 + rope.tab_off_w / 2 + pw;
+    const int W = static_cast<int>(p.W);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int pi = 32 * HF + 2 * j;
+      const int bnd = band_of<DT, DH>(pi, rope);
+      const int e = pair_in_band<DT, DH>(pi, rope) / 2;
+      const float4 cs = __ldg(bnd == 0 ? bt + e : (bnd == 1 ? bh + e : bw + e * W));
+      const float x0 = bf16lo(a[2 * j]), x1 = bf16hi(a[2 * j]);
+      const float y0 = bf16lo(a[2 * j + 1]), y1 = bf16hi(a[2 * j + 1]);
+      a[2 * j] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+      a[2 * j + 1] = pack_bf16(y0 * cs.z - y1 * cs.w, y0 * cs.w + y1 * cs.z);
+    }
+  } else {
+    const int ext[3] = {static_cast<int>(p.T), static_cast<int>(p.Hh), static_cast<int>(p.W)};
+    const int off[3] = {0, static_cast<int>(rope.tab_off_h), static_cast<int>(rope.tab_off_w)};
+    const int pos[3] = {pt, ph, pw};
+#pragma unroll 4
+    for (int j = 0; j < 32; ++j) {
+      const int pi = 32 * HF + j;
+      const int bnd = band_of<DT, DH>(pi, rope);
+      const int loc = pair_in_band<DT, DH>(pi, rope);
+      const float2 cs = __ldg(tab + off[bnd] + loc * ext[bnd] + pos[bnd]);
+      const float x0 = bf16lo(a[j]), x1 = bf16hi(a[j]);
+      a[j] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+    }
+  }
+}
+
 // In place over one row of 128 fp32 values: x <- RoPE^T(x) (rotation by the opposite angle) at grid
 // position (pt, ph, pw): (x0, x1) -> (x0 c + x1 s, -x0 s + x1 c).
 template <int DT, int DH>
