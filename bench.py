@@ -209,8 +209,10 @@ def run_reference(args):
     from gated_linear_attention_relu_b200 import workloads as wl
 
     w = wl.WORKLOADS[args.workload]
-    value, cores, times = oracle_sample(w, 0, steps=max(1, args.steps), warmup=max(0, args.warmup))
-    sample = f"one head of {w.name} (all {w.N} tokens), fp64 numpy oracle, per step"
+    mode = "causal" if args.causal else ("backward" if args.backward else ("gated" if args.gated else "forward"))
+    value, cores, times = oracle_sample(w, 0, steps=max(1, args.steps), warmup=max(0, args.warmup), mode=mode)
+    sample = (f"one head of {w.name} ({'2000 sampled outputs' if mode == 'causal' else f'all {w.N} tokens'}), "
+              f"fp64 numpy oracle ({mode}), per step"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": len(times), "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
