@@ -212,7 +212,7 @@ def run_reference(args):
     mode = "causal" if args.causal else ("backward" if args.backward else ("gated" if args.gated else "forward"))
     value, cores, times = oracle_sample(w, 0, steps=max(1, args.steps), warmup=max(0, args.warmup), mode=mode)
     sample = (f"one head of {w.name} ({'2000 sampled outputs' if mode == 'causal' else f'all {w.N} tokens'}), "
-              f"fp64 numpy oracle ({mode}), per step"
+              f"fp64 numpy oracle ({mode}), per step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": len(times), "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
