@@ -211,7 +211,7 @@ def run_reference(args):
     w = wl.WORKLOADS[args.workload]
     mode = "causal" if args.causal else ("backward" if args.backward else ("gated" if args.gated else "forward"))
     value, cores, times = oracle_sample(w, 0, steps=max(1, args.steps), warmup=max(0, args.warmup), mode=mode)
-    sample = (f"one head of {w.name} ({'2000 sampled outputs' if mode == 'causal' else f'all {w.N} tokens'}), "
+    sample = (f"one head of {w.name} ({f'{min(w.N, 2000)} sampled outputs' if mode == 'causal' else f'all {w.N} tokens'}), "
               f"fp64 numpy oracle ({mode}), per step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
@@ -448,7 +448,7 @@ def main():
         mode = "causal" if args.causal else ("backward" if args.backward else ("gated" if args.gated else "forward"))
         v, cores, times = oracle_sample(w, args.cpu_seconds, mode=mode)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"one head of {w.name} ({'2000 sampled outputs' if mode == 'causal' else f'all {w.N} tokens'}), "
+                                "sample": f"one head of {w.name} ({f'{min(w.N, 2000)} sampled outputs' if mode == 'causal' else f'all {w.N} tokens'}), "
                                           f"{len(times)} runs, fp64 numpy oracle ({mode})"}
     if rank == 0:
         print(json.dumps(line), flush=True)
