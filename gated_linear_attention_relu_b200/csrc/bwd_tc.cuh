@@ -10,7 +10,9 @@
 //   dv = phi(k) dS,  dk = [k > 0] (RoPE^T(v dS^T) + dz)
 //
 // Two kernels, both walking the same persistent tile ranges as the forward state kernel, one
-// 128-token tile at a time (warps 0-3: thread = token = TMEM lane; warp 4: TMA and MMA issue):
+// 128-token tile at a time (warps 0-7: two per row, by channel halves; thread = token = TMEM lane;
+// warp 8: TMA and MMA issue).  Outputs are staged in buffers of their own, so the next tile's
+// inputs load as soon as the products reading them are done:
 //   bwdq_tc_kernel: num = phi(Q) S and dphi(q) = dnum S^T (the state's bf16 image serves as S,
 //     read N-major, and as S^T, read K-major), dS += phi(Q)^T dnum (TMEM accumulator drained to
 //     the CTA's partial slot at the end of each unit, like the state kernel); dQ, dG out.
@@ -28,25 +30,31 @@ using namespace la::tile;
 
 constexpr int TILE = 128;
 constexpr int D = 128;
-constexpr int THREADS = 160;
+constexpr int MATH_WARPS = 8;
+constexpr int CTRL_WARP = MATH_WARPS;
+constexpr int THREADS = 32 * (MATH_WARPS + 1);
 constexpr uint32_t BUF = 2 * HALF;
-constexpr int ZPARTS = 4;  // dz partial rows per slot: one per math warp
+constexpr int ZPARTS = 4;  // dz partial rows per slot: one per lane quarter (the halves fill
+                           // disjoint channels of a row)
 constexpr uint32_t IDESC_QS = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/true);   // X S
 constexpr uint32_t IDESC_QST = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/false); // X S^T
 constexpr uint32_t IDESC_TD = idesc_bf16_f32(128, 128, /*a_mn=*/true, /*b_mn=*/true);    // X^T Y
 
-// ---- bwdq smem: Q (-> phi(Q) -> dQ), G (-> dG), dO (-> dnum), S image
-constexpr uint32_t QO_Q = 0, QO_G = BUF, QO_DO = 2 * BUF, QO_S = 3 * BUF, QO_BAR = 4 * BUF;
+// ---- bwdq smem: Q (-> phi(Q)), G (-> dG), dO (-> dnum), S image, dQ staging, exchanges
+constexpr uint32_t QO_Q = 0, QO_G = BUF, QO_DO = 2 * BUF, QO_S = 3 * BUF, QO_DQ = 4 * BUF;
+constexpr uint32_t QO_X = 5 * BUF;  // [2 values][2 halves][128] fp32: partial den, partial dy.y
+constexpr uint32_t QO_BAR = QO_X + 2048;
 constexpr uint32_t SMEM_Q = QO_BAR + 256 + 1024;
 constexpr uint32_t QCOL_NUM = 0, QCOL_DPQ = 128, QCOL_DS = 256;
-// ---- bwdk smem: K (-> phi(K) -> dK), V (-> dV), dS image
-constexpr uint32_t KO_K = 0, KO_V = BUF, KO_S = 2 * BUF, KO_BAR = 3 * BUF;
+// ---- bwdk smem: K (-> phi(K)), V, dS image, dK and dV staging
+constexpr uint32_t KO_K = 0, KO_V = BUF, KO_S = 2 * BUF, KO_DK = 3 * BUF, KO_DV = 4 * BUF, KO_BAR = 5 * BUF;
 constexpr uint32_t SMEM_K = KO_BAR + 256 + 1024;
 constexpr uint32_t KCOL_DV = 0, KCOL_DPK = 128;
 static_assert(SMEM_Q <= 232448 && SMEM_K <= 232448, "shared memory budget");
 
 struct BarsQ {
   uint64_t full, rot, numready, dn, dpqready, out, final_;
+  uint64_t pair[4];  // the two warps of rows 32q .. 32q+31: two meetings per tile (den, then dy.y)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -67,18 +75,6 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
   return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
 }
 
-// Pulls 128 fp32 columns of the calling thread's TMEM lane.
-__device__ __forceinline__ void pull128(uint32_t taddr, float (&x)[128]) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    uint32_t r[32];
-    tmem_ld_x32(taddr + 32 * j, r);
-    tmem_ld_wait();
-#pragma unroll
-    for (int e = 0; e < 32; ++e) x[32 * j + e] = __uint_as_float(r[e]);
-  }
-}
-
 template <int DT, int DH>
 __global__ void __launch_bounds__(THREADS, 1)
 bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
@@ -89,6 +85,7 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   BarsQ* bars = reinterpret_cast<BarsQ*>(smem + QO_BAR);
+  float* xch = reinterpret_cast<float*>(smem + QO_X);
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -101,16 +98,17 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->full, 1);
-    mbar_init(&bars->rot, 4);
+    mbar_init(&bars->rot, MATH_WARPS);
     mbar_init(&bars->numready, 1);
-    mbar_init(&bars->dn, 4);
+    mbar_init(&bars->dn, MATH_WARPS);
     mbar_init(&bars->dpqready, 1);
-    mbar_init(&bars->out, 4);
+    mbar_init(&bars->out, MATH_WARPS);
     mbar_init(&bars->final_, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], 2);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == CTRL_WARP) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -123,38 +121,33 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // partial slots the combine kernel before read: wait for them first.
   pdl_wait();
 
-  if (warp == 4) {
+  if (warp == CTRL_WARP) {
     if (lane == 0) {
-      int64_t prev_unit = -1;
+      auto load2 = [&](uint32_t off, const CUtensorMap* tm, const TileInfo& t) {
+        const int32_t n0 = static_cast<int32_t>(t.n0), bh = static_cast<int32_t>(t.bh);
+        tma_load_3d(smem + off, tm, 0, n0, bh, &bars->full);
+        tma_load_3d(smem + off + HALF, tm, 64, n0, bh, &bars->full);
+      };
       int64_t issued = 0;
-      TileInfo tprev{};
+      if (g0 < g1) {
+        const TileInfo t0 = tile_info(p, g0);
+        mbar_arrive_expect_tx(&bars->full, 4 * BUF);
+        bulk_load(smem + QO_S, simg + t0.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
+        load2(QO_Q, &tmQ, t0);
+        load2(QO_G, &tmG, t0);
+        load2(QO_DO, &tmDO, t0);
+        issued = 1;
+      }
+      int64_t prev_unit = -1;
       for (int64_t g = g0; g < g1; ++g) {
         const int64_t i = g - g0;
         const uint32_t ph = static_cast<uint32_t>(i & 1);
         const TileInfo ti = tile_info(p, g);
         const bool first = ti.unit != prev_unit;
         prev_unit = ti.unit;
-        if (i > 0) {
-          if (!mbar_wait(&bars->out, static_cast<uint32_t>((i - 1) & 1), abort_flag)) break;
-          const int32_t pn0 = static_cast<int32_t>(tprev.n0), pbh = static_cast<int32_t>(tprev.bh);
-          tma_store_3d(&tmDQ, smem + QO_Q, 0, pn0, pbh);
-          tma_store_3d(&tmDQ, smem + QO_Q + HALF, 64, pn0, pbh);
-          tma_store_3d(&tmDG, smem + QO_G, 0, pn0, pbh);
-          tma_store_3d(&tmDG, smem + QO_G + HALF, 64, pn0, pbh);
-          bulk_commit_group();
-          bulk_wait_group_read0();
-        }
-        tprev = ti;
-        mbar_arrive_expect_tx(&bars->full, 3 * BUF + (first ? BUF : 0u));
-        if (first) bulk_load(smem + QO_S, simg + ti.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
-        const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
-        tma_load_3d(smem + QO_Q, &tmQ, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + QO_Q + HALF, &tmQ, 64, n0, bh, &bars->full);
-        tma_load_3d(smem + QO_G, &tmG, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + QO_G + HALF, &tmG, 64, n0, bh, &bars->full);
-        tma_load_3d(smem + QO_DO, &tmDO, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + QO_DO + HALF, &tmDO, 64, n0, bh, &bars->full);
-        ++issued;
+        const bool has_next = g + 1 < g1;
+        const TileInfo tn = has_next ? tile_info(p, g + 1) : ti;
+        const bool next_new_unit = has_next && tn.unit != ti.unit;
         // num = phi(Q) S
         if (!mbar_wait(&bars->rot, ph, abort_flag)) break;
         tc_fence_after();
@@ -173,15 +166,28 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           mma_bf16(tmem + QCOL_DS, desc_mn(sbase + QO_Q, kk), desc_mn(sbase + QO_DO, kk), IDESC_TD,
                    (kk > 0 || !first) ? 1u : 0u);
         mma_commit(&bars->dpqready);
-      }
-      if (issued > 0 && !*abort_flag &&
-          mbar_wait(&bars->out, static_cast<uint32_t>((issued - 1) & 1), abort_flag)) {
-        const int32_t pn0 = static_cast<int32_t>(tprev.n0), pbh = static_cast<int32_t>(tprev.bh);
-        tma_store_3d(&tmDQ, smem + QO_Q, 0, pn0, pbh);
-        tma_store_3d(&tmDQ, smem + QO_Q + HALF, 64, pn0, pbh);
-        tma_store_3d(&tmDG, smem + QO_G, 0, pn0, pbh);
-        tma_store_3d(&tmDG, smem + QO_G + HALF, 64, pn0, pbh);
-        bulk_commit_group();
+        // Q, dO and the state image were last read by the products just done: the next tile's
+        // land while this tile's dq epilogue runs.  (G holds this tile's dG until it is stored.)
+        if (has_next) {
+          if (!mbar_wait(&bars->dpqready, ph, abort_flag)) break;
+          mbar_arrive_expect_tx(&bars->full, 3 * BUF + (next_new_unit ? BUF : 0u));
+          if (next_new_unit) bulk_load(smem + QO_S, simg + tn.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
+          load2(QO_Q, &tmQ, tn);
+          load2(QO_DO, &tmDO, tn);
+          ++issued;
+        }
+        // dQ (staged) and dG (over G) of this tile out; then the next tile's G.
+        if (!mbar_wait(&bars->out, ph, abort_flag)) break;
+        {
+          const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
+          tma_store_3d(&tmDQ, smem + QO_DQ, 0, n0, bh);
+          tma_store_3d(&tmDQ, smem + QO_DQ + HALF, 64, n0, bh);
+          tma_store_3d(&tmDG, smem + QO_G, 0, n0, bh);
+          tma_store_3d(&tmDG, smem + QO_G + HALF, 64, n0, bh);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        if (has_next) load2(QO_G, &tmG, tn);
       }
       bulk_wait_group0();
       if (*abort_flag && issued > 0) mbar_wait_drain(&bars->full, static_cast<uint32_t>((issued - 1) & 1));
@@ -189,76 +195,96 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_wait_drain(&bars->final_, 0);
     }
   } else {
-    const int row = threadIdx.x;
-    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
-    float dzacc[4] = {0.f, 0.f, 0.f, 0.f};  // dz of channels 4*lane .. 4*lane+3 over this warp's rows
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+    uint64_t* pr = &bars->pair[quarter];
+    float dzacc[2] = {0.f, 0.f};  // dz of channels 64 hf + 2 lane, +1 over this warp's rows
     for (int64_t g = g0; g < g1; ++g) {
       const int64_t i = g - g0;
       const uint32_t ph = static_cast<uint32_t>(i & 1);
       const TileInfo ti = tile_info(p, g);
       const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != ti.unit);
       if (!warp_wait(&bars->full, ph, abort_flag)) break;
-      // q^+ kept packed; phi(q) written in place (the A operand of num and of the dS update).
-      uint32_t qa[64];
+      // q^+ of this half kept packed; phi(q) written in place.
+      uint32_t qa[32];
 #pragma unroll
-      for (int ck = 0; ck < 16; ++ck) {
-        const uint4 rq = lds128(row_chunk(sbase + QO_Q, row, ck));
-        qa[4 * ck] = relu_bf16x2(rq.x);
-        qa[4 * ck + 1] = relu_bf16x2(rq.y);
-        qa[4 * ck + 2] = relu_bf16x2(rq.z);
-        qa[4 * ck + 3] = relu_bf16x2(rq.w);
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const uint4 rq = lds128(row_chunk(sbase + QO_Q, row, 8 * hf + c8));
+        qa[4 * c8] = relu_bf16x2(rq.x);
+        qa[4 * c8 + 1] = relu_bf16x2(rq.y);
+        qa[4 * c8 + 2] = relu_bf16x2(rq.z);
+        qa[4 * c8 + 3] = relu_bf16x2(rq.w);
       }
       const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
       uint32_t pt = 0, ph_ = 0, pw = 0;
       if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph_, pw);
       {
-        uint32_t a[64];
+        uint32_t a[32];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) a[e] = qa[e];
-        rotate_row<DT, DH>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        for (int e = 0; e < 32; ++e) a[e] = qa[e];
+        if (hf == 0)
+          rotate_half<DT, DH, 0>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        else
+          rotate_half<DT, DH, 1>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
 #pragma unroll
-        for (int ck = 0; ck < 16; ++ck)
-          sts128(row_chunk(sbase + QO_Q, row, ck), make_uint4(a[4 * ck], a[4 * ck + 1], a[4 * ck + 2], a[4 * ck + 3]));
+        for (int c8 = 0; c8 < 8; ++c8)
+          sts128(row_chunk(sbase + QO_Q, row, 8 * hf + c8), make_uint4(a[4 * c8], a[4 * c8 + 1], a[4 * c8 + 2], a[4 * c8 + 3]));
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->rot);
-      // den = q^+ . z + eps
-      const float* zg = zimg + ti.unit * D;
-      float den = 0.f;
+      // den = q^+ . z + eps: each half's share, then the pair adds them.
+      const float* zg = zimg + ti.unit * D + 64 * hf;
+      float dpart = 0.f;
 #pragma unroll
-      for (int k4 = 0; k4 < 32; ++k4) {
+      for (int k4 = 0; k4 < 16; ++k4) {
         const float4 z4 = __ldg(reinterpret_cast<const float4*>(zg + 4 * k4));
-        den = fmaf(bf16lo(qa[2 * k4]), z4.x, den);
-        den = fmaf(bf16hi(qa[2 * k4]), z4.y, den);
-        den = fmaf(bf16lo(qa[2 * k4 + 1]), z4.z, den);
-        den = fmaf(bf16hi(qa[2 * k4 + 1]), z4.w, den);
+        dpart = fmaf(bf16lo(qa[2 * k4]), z4.x, dpart);
+        dpart = fmaf(bf16hi(qa[2 * k4]), z4.y, dpart);
+        dpart = fmaf(bf16lo(qa[2 * k4 + 1]), z4.z, dpart);
+        dpart = fmaf(bf16hi(qa[2 * k4 + 1]), z4.w, dpart);
       }
-      den += p.eps;
+      xch[hf * 128 + row] = dpart;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pr);
+      if (!warp_wait(pr, 0u, abort_flag)) break;
+      const float dother = xch[(hf ^ 1) * 128 + row];
+      const float den = (hf == 0 ? dpart + dother : dother + dpart) + p.eps;
       const float rden = 1.0f / den;
-      // num -> y; with G and dO: dG (over G), dnum (over dO), dden.
+      // num -> y; with G and dO: dG (staged), dnum (over dO), this half's dy . y.
       if (!warp_wait(&bars->numready, ph, abort_flag)) break;
       tc_fence_after();
-      float x[128];
-      pull128(tmem + QCOL_NUM + lane_bits, x);  // num
+      float x[64];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        uint32_t r[32];
+        tmem_ld_x32(tmem + QCOL_NUM + lane_bits + 64u * hf + 32 * j, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[32 * j + e] = __uint_as_float(r[e]);
+      }
       float dyy = 0.f;
 #pragma unroll
-      for (int ck = 0; ck < 16; ++ck) {
-        const uint32_t ag = row_chunk(sbase + QO_G, row, ck), ad = row_chunk(sbase + QO_DO, row, ck);
-        const uint4 gr = lds128(ag), dr = lds128(ad);
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const int ck = 8 * hf + c8;
+        const uint32_t ag = row_chunk(sbase + QO_G, row, ck);
+        const uint4 gr = lds128(ag);
+        const uint32_t ad = row_chunk(sbase + QO_DO, row, ck);
+        const uint4 dr = lds128(ad);
         const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w}, dw[4] = {dr.x, dr.y, dr.z, dr.w};
         float dg8[8], dy8[8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int e = 8 * ck + 2 * q + h;
+            const int e = 8 * c8 + 2 * q + h;
             const float gv = h ? bf16hi(gw[q]) : bf16lo(gw[q]);
             const float dov = h ? bf16hi(dw[q]) : bf16lo(dw[q]);
             const float y = x[e] * rden;
-            const float s = sigmoid_f(gv);
-            dg8[2 * q + h] = dov * y * s * (1.f - s);
-            const float dy = dov * s;
+            const float sg = sigmoid_f(gv);
+            dg8[2 * q + h] = dov * y * sg * (1.f - sg);
+            const float dy = dov * sg;
             dy8[2 * q + h] = dy * rden;  // dnum
             dyy = fmaf(dy, y, dyy);
           }
@@ -266,22 +292,28 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         sts128(ag, pack8(dg8));
         sts128(ad, pack8(dy8));
       }
-      const float dden = -dyy * rden;
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->dn);
-      // dz over this warp's rows: every lane ends with channels 4*lane .. 4*lane+3 (a butterfly
-      // that halves the channel range per step; each sum is formed once, lower lane first).
+      xch[256 + hf * 128 + row] = dyy;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pr);
+      if (!warp_wait(pr, 1u, abort_flag)) break;
+      const float yother = xch[256 + (hf ^ 1) * 128 + row];
+      const float dden = -(hf == 0 ? dyy + yother : yother + dyy) * rden;
+      // dz over this warp's 32 rows for this half's 64 channels: lane L ends with channels
+      // 64 hf + 2L, 64 hf + 2L + 1 (a butterfly that halves the range per step, each sum formed
+      // once, lower lane first).
       {
-        float v[128];
+        float v[64];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
+        for (int e = 0; e < 32; ++e) {
           v[2 * e] = dden * bf16lo(qa[e]);
           v[2 * e + 1] = dden * bf16hi(qa[e]);
         }
 #pragma unroll
-        for (int off = 16, size = 128; off >= 1; off >>= 1, size >>= 1) {
+        for (int off = 16, size = 64; off >= 1; off >>= 1, size >>= 1) {
           const bool up = (lane & off) != 0;
 #pragma unroll
           for (int e = 0; e < size / 2; ++e) {
@@ -291,38 +323,55 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             v[e] = up ? other + keep : keep + other;
           }
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dzacc[e] += v[e];
+        dzacc[0] += v[0];
+        dzacc[1] += v[1];
       }
-      // dq = [q > 0] (RoPE^T(dnum S^T) + dden z), over phi(Q) (the MMAs are done with it).
+      // dq = [q > 0] (RoPE^T(dnum S^T) + dden z) for this half, into the dQ staging buffer.
       if (!warp_wait(&bars->dpqready, ph, abort_flag)) break;
       tc_fence_after();
-      pull128(tmem + QCOL_DPQ + lane_bits, x);
-      rotate_row_t<DT, DH>(x, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
 #pragma unroll
-      for (int ck = 0; ck < 16; ++ck) {
-        const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * ck));
-        const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * ck + 4));
+      for (int j = 0; j < 2; ++j) {
+        uint32_t r[32];
+        tmem_ld_x32(tmem + QCOL_DPQ + lane_bits + 64u * hf + 32 * j, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[32 * j + e] = __uint_as_float(r[e]);
+      }
+      if (hf == 0)
+        rotate_half_t<DT, DH, 0>(x, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+      else
+        rotate_half_t<DT, DH, 1>(x, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c8));
+        const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c8 + 4));
         const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
         float o8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const uint32_t w = qa[4 * ck + e / 2];
+          const uint32_t w = qa[4 * c8 + e / 2];
           const float qv = (e & 1) ? bf16hi(w) : bf16lo(w);
-          o8[e] = qv > 0.f ? x[8 * ck + e] + dden * zz[e] : 0.f;
+          o8[e] = qv > 0.f ? x[8 * c8 + e] + dden * zz[e] : 0.f;
         }
-        sts128(row_chunk(sbase + QO_Q, row, ck), pack8(o8));
+        sts128(row_chunk(sbase + QO_DQ, row, 8 * hf + c8), pack8(o8));
       }
       if (last) {
-        // dS of this unit (TMEM lane = channel k of phi(Q)) and dz -> the CTA's partial slot.
-        pull128(tmem + QCOL_DS + lane_bits, x);
+        // dS of this unit (TMEM lane = channel k of phi(Q); this half's 64 columns) and dz -> the
+        // CTA's partial slot.
         float* dst = partial + (c * p.maxseg + (ti.unit - u_first)) * slot_floats;
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          reinterpret_cast<float4*>(dst + row * D)[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
-        reinterpret_cast<float4*>(dst + D * D + warp * D)[lane] = make_float4(dzacc[0], dzacc[1], dzacc[2], dzacc[3]);
+        for (int j = 0; j < 2; ++j) {
+          uint32_t r[32];
+          tmem_ld_x32(tmem + QCOL_DS + lane_bits + 64u * hf + 32 * j, r);
+          tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dzacc[e] = 0.f;
+          for (int e = 0; e < 8; ++e)
+            reinterpret_cast<float4*>(dst + row * D + 64 * hf + 32 * j)[e] =
+                make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
+                            __uint_as_float(r[4 * e + 3]));
+        }
+        reinterpret_cast<float2*>(dst + D * D + quarter * D + 64 * hf)[lane] = make_float2(dzacc[0], dzacc[1]);
+        dzacc[0] = dzacc[1] = 0.f;
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -334,7 +383,7 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) tmem_dealloc(tmem, 512);
+  if (warp == CTRL_WARP) tmem_dealloc(tmem, 512);
 }
 
 template <int DT, int DH>
@@ -356,14 +405,14 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->full, 1);
-    mbar_init(&bars->rot, 4);
+    mbar_init(&bars->rot, MATH_WARPS);
     mbar_init(&bars->ready, 1);
-    mbar_init(&bars->out, 4);
+    mbar_init(&bars->out, MATH_WARPS);
     mbar_init(&bars->final_, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == CTRL_WARP) {
     tmem_alloc(&bars->tmem_base, 256);
     tmem_relinquish();
   }
@@ -374,36 +423,29 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   pdl_trigger();
   pdl_wait();
 
-  if (warp == 4) {
+  if (warp == CTRL_WARP) {
     if (lane == 0) {
-      int64_t prev_unit = -1;
+      auto load2 = [&](uint32_t off, const CUtensorMap* tm, const TileInfo& t) {
+        const int32_t n0 = static_cast<int32_t>(t.n0), bh = static_cast<int32_t>(t.bh);
+        tma_load_3d(smem + off, tm, 0, n0, bh, &bars->full);
+        tma_load_3d(smem + off + HALF, tm, 64, n0, bh, &bars->full);
+      };
       int64_t issued = 0;
-      TileInfo tprev{};
+      if (g0 < g1) {
+        const TileInfo t0 = tile_info(p, g0);
+        mbar_arrive_expect_tx(&bars->full, 3 * BUF);
+        bulk_load(smem + KO_S, dsimg + t0.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
+        load2(KO_K, &tmK, t0);
+        load2(KO_V, &tmV, t0);
+        issued = 1;
+      }
       for (int64_t g = g0; g < g1; ++g) {
         const int64_t i = g - g0;
         const uint32_t ph = static_cast<uint32_t>(i & 1);
         const TileInfo ti = tile_info(p, g);
-        const bool first = ti.unit != prev_unit;
-        prev_unit = ti.unit;
-        if (i > 0) {
-          if (!mbar_wait(&bars->out, static_cast<uint32_t>((i - 1) & 1), abort_flag)) break;
-          const int32_t pn0 = static_cast<int32_t>(tprev.n0), pbh = static_cast<int32_t>(tprev.bh);
-          tma_store_3d(&tmDK, smem + KO_K, 0, pn0, pbh);
-          tma_store_3d(&tmDK, smem + KO_K + HALF, 64, pn0, pbh);
-          tma_store_3d(&tmDV, smem + KO_V, 0, pn0, pbh);
-          tma_store_3d(&tmDV, smem + KO_V + HALF, 64, pn0, pbh);
-          bulk_commit_group();
-          bulk_wait_group_read0();
-        }
-        tprev = ti;
-        mbar_arrive_expect_tx(&bars->full, 2 * BUF + (first ? BUF : 0u));
-        if (first) bulk_load(smem + KO_S, dsimg + ti.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
-        const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
-        tma_load_3d(smem + KO_K, &tmK, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + KO_K + HALF, &tmK, 64, n0, bh, &bars->full);
-        tma_load_3d(smem + KO_V, &tmV, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + KO_V + HALF, &tmV, 64, n0, bh, &bars->full);
-        ++issued;
+        const bool has_next = g + 1 < g1;
+        const TileInfo tn = has_next ? tile_info(p, g + 1) : ti;
+        const bool next_new_unit = has_next && tn.unit != ti.unit;
         if (!mbar_wait(&bars->rot, ph, abort_flag)) break;
         tc_fence_after();
         // dV = phi(K) dS;  dphi(k) = V dS^T
@@ -414,15 +456,25 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + KCOL_DPK, desc_k(sbase + KO_V, kk), desc_k(sbase + KO_S, kk), IDESC_QST, kk > 0 ? 1u : 0u);
         mma_commit(&bars->ready);
-      }
-      if (issued > 0 && !*abort_flag &&
-          mbar_wait(&bars->out, static_cast<uint32_t>((issued - 1) & 1), abort_flag)) {
-        const int32_t pn0 = static_cast<int32_t>(tprev.n0), pbh = static_cast<int32_t>(tprev.bh);
-        tma_store_3d(&tmDK, smem + KO_K, 0, pn0, pbh);
-        tma_store_3d(&tmDK, smem + KO_K + HALF, 64, pn0, pbh);
-        tma_store_3d(&tmDV, smem + KO_V, 0, pn0, pbh);
-        tma_store_3d(&tmDV, smem + KO_V + HALF, 64, pn0, pbh);
-        bulk_commit_group();
+        // The products were the last readers of K, V and the dS image: the next tile's land now.
+        if (has_next) {
+          if (!mbar_wait(&bars->ready, ph, abort_flag)) break;
+          mbar_arrive_expect_tx(&bars->full, 2 * BUF + (next_new_unit ? BUF : 0u));
+          if (next_new_unit) bulk_load(smem + KO_S, dsimg + tn.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
+          load2(KO_K, &tmK, tn);
+          load2(KO_V, &tmV, tn);
+          ++issued;
+        }
+        if (!mbar_wait(&bars->out, ph, abort_flag)) break;
+        {
+          const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
+          tma_store_3d(&tmDK, smem + KO_DK, 0, n0, bh);
+          tma_store_3d(&tmDK, smem + KO_DK + HALF, 64, n0, bh);
+          tma_store_3d(&tmDV, smem + KO_DV, 0, n0, bh);
+          tma_store_3d(&tmDV, smem + KO_DV + HALF, 64, n0, bh);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
       }
       bulk_wait_group0();
       if (*abort_flag && issued > 0) mbar_wait_drain(&bars->full, static_cast<uint32_t>((issued - 1) & 1));
@@ -430,59 +482,80 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       mbar_wait_drain(&bars->final_, 0);
     }
   } else {
-    const int row = threadIdx.x;
-    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
     for (int64_t g = g0; g < g1; ++g) {
       const int64_t i = g - g0;
       const uint32_t ph = static_cast<uint32_t>(i & 1);
       const TileInfo ti = tile_info(p, g);
       if (!warp_wait(&bars->full, ph, abort_flag)) break;
-      uint32_t ka[64];
+      uint32_t ka[32];
 #pragma unroll
-      for (int ck = 0; ck < 16; ++ck) {
-        const uint4 rk = lds128(row_chunk(sbase + KO_K, row, ck));
-        ka[4 * ck] = rk.x;
-        ka[4 * ck + 1] = rk.y;
-        ka[4 * ck + 2] = rk.z;
-        ka[4 * ck + 3] = rk.w;
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const uint4 rk = lds128(row_chunk(sbase + KO_K, row, 8 * hf + c8));
+        ka[4 * c8] = rk.x;
+        ka[4 * c8 + 1] = rk.y;
+        ka[4 * c8 + 2] = rk.z;
+        ka[4 * c8 + 3] = rk.w;
       }
       const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
       uint32_t pt = 0, ph_ = 0, pw = 0;
       if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph_, pw);
       {
-        uint32_t a[64];
+        uint32_t a[32];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) a[e] = relu_bf16x2(ka[e]);
-        rotate_row<DT, DH>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        for (int e = 0; e < 32; ++e) a[e] = relu_bf16x2(ka[e]);
+        if (hf == 0)
+          rotate_half<DT, DH, 0>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        else
+          rotate_half<DT, DH, 1>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
 #pragma unroll
-        for (int ck = 0; ck < 16; ++ck)
-          sts128(row_chunk(sbase + KO_K, row, ck), make_uint4(a[4 * ck], a[4 * ck + 1], a[4 * ck + 2], a[4 * ck + 3]));
+        for (int c8 = 0; c8 < 8; ++c8)
+          sts128(row_chunk(sbase + KO_K, row, 8 * hf + c8), make_uint4(a[4 * c8], a[4 * c8 + 1], a[4 * c8 + 2], a[4 * c8 + 3]));
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->rot);
       if (!warp_wait(&bars->ready, ph, abort_flag)) break;
       tc_fence_after();
-      float x[128];
-      pull128(tmem + KCOL_DV + lane_bits, x);
+      float x[64];
 #pragma unroll
-      for (int ck = 0; ck < 16; ++ck) sts128(row_chunk(sbase + KO_V, row, ck), pack8(&x[8 * ck]));
-      pull128(tmem + KCOL_DPK + lane_bits, x);
-      rotate_row_t<DT, DH>(x, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
-      const float* zg = dzimg + ti.unit * D;
+      for (int j = 0; j < 2; ++j) {
+        uint32_t r[32];
+        tmem_ld_x32(tmem + KCOL_DV + lane_bits + 64u * hf + 32 * j, r);
+        tmem_ld_wait();
 #pragma unroll
-      for (int ck = 0; ck < 16; ++ck) {
-        const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * ck));
-        const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * ck + 4));
+        for (int e = 0; e < 32; ++e) x[32 * j + e] = __uint_as_float(r[e]);
+      }
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) sts128(row_chunk(sbase + KO_DV, row, 8 * hf + c8), pack8(&x[8 * c8]));
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        uint32_t r[32];
+        tmem_ld_x32(tmem + KCOL_DPK + lane_bits + 64u * hf + 32 * j, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[32 * j + e] = __uint_as_float(r[e]);
+      }
+      if (hf == 0)
+        rotate_half_t<DT, DH, 0>(x, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+      else
+        rotate_half_t<DT, DH, 1>(x, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+      const float* zg = dzimg + ti.unit * D + 64 * hf;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c8));
+        const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c8 + 4));
         const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
         float o8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const uint32_t w = ka[4 * ck + e / 2];
+          const uint32_t w = ka[4 * c8 + e / 2];
           const float kv = (e & 1) ? bf16hi(w) : bf16lo(w);
-          o8[e] = kv > 0.f ? x[8 * ck + e] + zz[e] : 0.f;
+          o8[e] = kv > 0.f ? x[8 * c8 + e] + zz[e] : 0.f;
         }
-        sts128(row_chunk(sbase + KO_K, row, ck), pack8(o8));
+        sts128(row_chunk(sbase + KO_DK, row, 8 * hf + c8), pack8(o8));
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -494,7 +567,7 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) tmem_dealloc(tmem, 256);
+  if (warp == CTRL_WARP) tmem_dealloc(tmem, 256);
 }
 
 }  // namespace bw

@@ -148,5 +148,44 @@ __device__ __forceinline__ void rotate_row_t(float (&x)[128], const float2* __re
   }
 }
 
+// In place over half a row of fp32 values (channels [64 HF, 64 HF + 64)): x <- RoPE^T(x).
+template <int DT, int DH, int HF>
+__device__ __forceinline__ void rotate_half_t(float (&x)[64], const float2* __restrict__ tab,
+                                              const float4* __restrict__ tab2, const Rope& rope, const Plan& p,
+                                              int pt, int ph, int pw) {
+  if constexpr (DT >= 0 && DH >= 0) {
+    const float4* bt = tab2 + pt * (DT / 4);
+    const float4* bh = tab2 + rope.tab_off_h / 2 + ph * (DH / 4);
+    const float4* bw = tab2 + rope.tab_off_w / 2 + pw;
+    const int W = static_cast<int>(p.W);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int pi = 32 * HF + 2 * j;
+      const int bnd = band_of<DT, DH>(pi, rope);
+      const int e = pair_in_band<DT, DH>(pi, rope) / 2;
+      const float4 cs = __ldg(bnd == 0 ? bt + e : (bnd == 1 ? bh + e : bw + e * W));
+      const float x0 = x[4 * j], x1 = x[4 * j + 1], y0 = x[4 * j + 2], y1 = x[4 * j + 3];
+      x[4 * j] = x0 * cs.x + x1 * cs.y;
+      x[4 * j + 1] = x1 * cs.x - x0 * cs.y;
+      x[4 * j + 2] = y0 * cs.z + y1 * cs.w;
+      x[4 * j + 3] = y1 * cs.z - y0 * cs.w;
+    }
+  } else {
+    const int ext[3] = {static_cast<int>(p.T), static_cast<int>(p.Hh), static_cast<int>(p.W)};
+    const int off[3] = {0, static_cast<int>(rope.tab_off_h), static_cast<int>(rope.tab_off_w)};
+    const int pos[3] = {pt, ph, pw};
+#pragma unroll 4
+    for (int j = 0; j < 32; ++j) {
+      const int pi = 32 * HF + j;
+      const int bnd = band_of<DT, DH>(pi, rope);
+      const int loc = pair_in_band<DT, DH>(pi, rope);
+      const float2 cs = __ldg(tab + off[bnd] + loc * ext[bnd] + pos[bnd]);
+      const float x0 = x[2 * j], x1 = x[2 * j + 1];
+      x[2 * j] = x0 * cs.x + x1 * cs.y;
+      x[2 * j + 1] = x1 * cs.x - x0 * cs.y;
+    }
+  }
+}
+
 }  // namespace tile
 }  // namespace la
