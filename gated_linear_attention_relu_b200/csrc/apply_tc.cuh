@@ -352,7 +352,11 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (progressed) {
           t_progress = globaltimer_ns();
           idle = 0;
-        } else if ((++idle & 255u) == 0u) {
+          continue;
+        }
+        // Nothing ready: back off briefly instead of spinning on the issue slots the math warps use.
+        __nanosleep(32);
+        if ((++idle & 255u) == 0u) {
           if (*abort_flag) break;
           if (globaltimer_ns() - t_progress > LA_WAIT_LIMIT_NS) {
             *abort_flag = 1;
