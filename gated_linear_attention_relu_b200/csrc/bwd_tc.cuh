@@ -10,9 +10,10 @@
 //   dv = phi(k) dS,  dk = [k > 0] (RoPE^T(v dS^T) + dz)
 //
 // Two kernels, both walking the same persistent tile ranges as the forward state kernel, one
-// 128-token tile at a time (warps 0-7: two per row, by channel halves; thread = token = TMEM lane;
-// warp 8: TMA and MMA issue).  Outputs are staged in buffers of their own, so the next tile's
-// inputs load as soon as the products reading them are done:
+// 128-token tile at a time (warps 0-15: four per row, by channel quarters; thread = token = TMEM
+// lane; warp 16: TMA and MMA issue).  Outputs are staged in buffers of their own, so the next
+// tile's inputs load as soon as the products reading them are done; the input read last (G in
+// the first kernel, V in the second) lands on a barrier of its own, waited for only by its reader:
 //   bwdq_tc_kernel: num = phi(Q) S and dphi(q) = dnum S^T (the state's bf16 image serves as S,
 //     read N-major, and as S^T, read K-major), dS += phi(Q)^T dnum (TMEM accumulator drained to
 //     the CTA's partial slot at the end of each unit, like the state kernel); dQ, dG out.
@@ -30,20 +31,21 @@ using namespace la::tile;
 
 constexpr int TILE = 128;
 constexpr int D = 128;
-constexpr int MATH_WARPS = 8;
+constexpr int MATH_WARPS = 16;  // four per TMEM lane quarter: channel quarters of a row
+constexpr int PARTS = MATH_WARPS / 4;
 constexpr int CTRL_WARP = MATH_WARPS;
 constexpr int THREADS = 32 * (MATH_WARPS + 1);
 constexpr uint32_t BUF = 2 * HALF;
-constexpr int ZPARTS = 4;  // dz partial rows per slot: one per lane quarter (the halves fill
-                           // disjoint channels of a row)
+constexpr int ZPARTS = 4;  // dz partial rows per slot: one per lane quarter (the channel quarters
+                           // fill disjoint channels of a row)
 constexpr uint32_t IDESC_QS = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/true);   // X S
 constexpr uint32_t IDESC_QST = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/false); // X S^T
 constexpr uint32_t IDESC_TD = idesc_bf16_f32(128, 128, /*a_mn=*/true, /*b_mn=*/true);    // X^T Y
 
 // ---- bwdq smem: Q (-> phi(Q)), G (-> dG), dO (-> dnum), S image, dQ staging, exchanges
 constexpr uint32_t QO_Q = 0, QO_G = BUF, QO_DO = 2 * BUF, QO_S = 3 * BUF, QO_DQ = 4 * BUF;
-constexpr uint32_t QO_X = 5 * BUF;  // [2 values][2 halves][128] fp32: partial den, partial dy.y
-constexpr uint32_t QO_BAR = QO_X + 2048;
+constexpr uint32_t QO_X = 5 * BUF;  // [2 values][4 parts][128] fp32: partial den, partial dy.y
+constexpr uint32_t QO_BAR = QO_X + 2 * PARTS * 512;
 constexpr uint32_t SMEM_Q = QO_BAR + 256 + 1024;
 constexpr uint32_t QCOL_NUM = 0, QCOL_DPQ = 128, QCOL_DS = 256;
 // ---- bwdk smem: K (-> phi(K)), V, dS image, dK and dV staging
@@ -53,13 +55,17 @@ constexpr uint32_t KCOL_DV = 0, KCOL_DPK = 128;
 static_assert(SMEM_Q <= 232448 && SMEM_K <= 232448, "shared memory budget");
 
 struct BarsQ {
-  uint64_t full, rot, numready, dn, dpqready, out, final_;
-  uint64_t pair[4];  // the two warps of rows 32q .. 32q+31: two meetings per tile (den, then dy.y)
+  uint64_t full;    // Q, dO (and the state image at a unit's first tile) landed
+  uint64_t full_g;  // G landed
+  uint64_t rot, numready, dn, dpqready, out, final_;
+  uint64_t pair[4];  // the four warps of rows 32q .. 32q+31: two meetings per tile (den, then dy.y)
   uint32_t tmem_base;
   int abort_flag;
 };
 struct BarsK {
-  uint64_t full, rot, ready, out, final_;
+  uint64_t full;    // K (and the dS image at a unit's first tile) landed
+  uint64_t full_v;  // V landed
+  uint64_t rot, ready, out, final_;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -98,13 +104,14 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->full, 1);
+    mbar_init(&bars->full_g, 1);
     mbar_init(&bars->rot, MATH_WARPS);
     mbar_init(&bars->numready, 1);
     mbar_init(&bars->dn, MATH_WARPS);
     mbar_init(&bars->dpqready, 1);
     mbar_init(&bars->out, MATH_WARPS);
     mbar_init(&bars->final_, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], 2);
+    for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], PARTS);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -123,20 +130,21 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (warp == CTRL_WARP) {
     if (lane == 0) {
-      auto load2 = [&](uint32_t off, const CUtensorMap* tm, const TileInfo& t) {
+      auto load2 = [&](uint32_t off, const CUtensorMap* tm, const TileInfo& t, uint64_t* bar) {
         const int32_t n0 = static_cast<int32_t>(t.n0), bh = static_cast<int32_t>(t.bh);
-        tma_load_3d(smem + off, tm, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + off + HALF, tm, 64, n0, bh, &bars->full);
+        tma_load_3d(smem + off, tm, 0, n0, bh, bar);
+        tma_load_3d(smem + off + HALF, tm, 64, n0, bh, bar);
       };
-      int64_t issued = 0;
+      int64_t issued = 0, issued_g = 0;
       if (g0 < g1) {
         const TileInfo t0 = tile_info(p, g0);
-        mbar_arrive_expect_tx(&bars->full, 4 * BUF);
+        mbar_arrive_expect_tx(&bars->full, 3 * BUF);
         bulk_load(smem + QO_S, simg + t0.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
-        load2(QO_Q, &tmQ, t0);
-        load2(QO_G, &tmG, t0);
-        load2(QO_DO, &tmDO, t0);
-        issued = 1;
+        load2(QO_Q, &tmQ, t0, &bars->full);
+        load2(QO_DO, &tmDO, t0, &bars->full);
+        mbar_arrive_expect_tx(&bars->full_g, BUF);
+        load2(QO_G, &tmG, t0, &bars->full_g);
+        issued = issued_g = 1;
       }
       int64_t prev_unit = -1;
       for (int64_t g = g0; g < g1; ++g) {
@@ -170,10 +178,10 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // land while this tile's dq epilogue runs.  (G holds this tile's dG until it is stored.)
         if (has_next) {
           if (!mbar_wait(&bars->dpqready, ph, abort_flag)) break;
-          mbar_arrive_expect_tx(&bars->full, 3 * BUF + (next_new_unit ? BUF : 0u));
+          mbar_arrive_expect_tx(&bars->full, 2 * BUF + (next_new_unit ? BUF : 0u));
           if (next_new_unit) bulk_load(smem + QO_S, simg + tn.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
-          load2(QO_Q, &tmQ, tn);
-          load2(QO_DO, &tmDO, tn);
+          load2(QO_Q, &tmQ, tn, &bars->full);
+          load2(QO_DO, &tmDO, tn, &bars->full);
           ++issued;
         }
         // dQ (staged) and dG (over G) of this tile out; then the next tile's G.
@@ -187,87 +195,97 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           bulk_commit_group();
           bulk_wait_group_read0();
         }
-        if (has_next) load2(QO_G, &tmG, tn);
+        if (has_next) {
+          mbar_arrive_expect_tx(&bars->full_g, BUF);
+          load2(QO_G, &tmG, tn, &bars->full_g);
+          ++issued_g;
+        }
       }
       bulk_wait_group0();
-      if (*abort_flag && issued > 0) mbar_wait_drain(&bars->full, static_cast<uint32_t>((issued - 1) & 1));
+      if (*abort_flag) {
+        if (issued > 0) mbar_wait_drain(&bars->full, static_cast<uint32_t>((issued - 1) & 1));
+        if (issued_g > 0) mbar_wait_drain(&bars->full_g, static_cast<uint32_t>((issued_g - 1) & 1));
+      }
       mma_commit(&bars->final_);
       mbar_wait_drain(&bars->final_, 0);
     }
   } else {
-    const int quarter = warp & 3, hf = warp >> 2;
+    const int quarter = warp & 3, part = warp >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+    const int cpart = 32 * part;  // this warp's channels
     uint64_t* pr = &bars->pair[quarter];
-    float dzacc[2] = {0.f, 0.f};  // dz of channels 64 hf + 2 lane, +1 over this warp's rows
+    float dzacc = 0.f;  // dz of channel 32 part + lane over this warp's rows
     for (int64_t g = g0; g < g1; ++g) {
       const int64_t i = g - g0;
       const uint32_t ph = static_cast<uint32_t>(i & 1);
       const TileInfo ti = tile_info(p, g);
       const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != ti.unit);
       if (!warp_wait(&bars->full, ph, abort_flag)) break;
-      // q^+ of this half kept packed; phi(q) written in place.
-      uint32_t qa[32];
+      // q^+ of this quarter kept packed; phi(q) written in place.
+      uint32_t qa[16];
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const uint4 rq = lds128(row_chunk(sbase + QO_Q, row, 8 * hf + c8));
-        qa[4 * c8] = relu_bf16x2(rq.x);
-        qa[4 * c8 + 1] = relu_bf16x2(rq.y);
-        qa[4 * c8 + 2] = relu_bf16x2(rq.z);
-        qa[4 * c8 + 3] = relu_bf16x2(rq.w);
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const uint4 rq = lds128(row_chunk(sbase + QO_Q, row, 4 * part + c4));
+        qa[4 * c4] = relu_bf16x2(rq.x);
+        qa[4 * c4 + 1] = relu_bf16x2(rq.y);
+        qa[4 * c4 + 2] = relu_bf16x2(rq.z);
+        qa[4 * c4 + 3] = relu_bf16x2(rq.w);
       }
       const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
       uint32_t pt = 0, ph_ = 0, pw = 0;
       if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph_, pw);
+      const int ipt = static_cast<int>(pt), iph = static_cast<int>(ph_), ipw = static_cast<int>(pw);
       {
-        uint32_t a[32];
+        uint32_t a[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) a[e] = qa[e];
-        if (hf == 0)
-          rotate_half<DT, DH, 0>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
-        else
-          rotate_half<DT, DH, 1>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        for (int e = 0; e < 16; ++e) a[e] = qa[e];
+        switch (part) {
+          case 0: rotate_span<DT, DH, 0, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 1: rotate_span<DT, DH, 16, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 2: rotate_span<DT, DH, 32, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+          default: rotate_span<DT, DH, 48, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+        }
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8)
-          sts128(row_chunk(sbase + QO_Q, row, 8 * hf + c8), make_uint4(a[4 * c8], a[4 * c8 + 1], a[4 * c8 + 2], a[4 * c8 + 3]));
+        for (int c4 = 0; c4 < 4; ++c4)
+          sts128(row_chunk(sbase + QO_Q, row, 4 * part + c4), make_uint4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->rot);
-      // den = q^+ . z + eps: each half's share, then the pair adds them.
-      const float* zg = zimg + ti.unit * D + 64 * hf;
+      // den = q^+ . z + eps: each quarter's share, then the four add them in a fixed order.
+      const float* zg = zimg + ti.unit * D + cpart;
       float dpart = 0.f;
 #pragma unroll
-      for (int k4 = 0; k4 < 16; ++k4) {
+      for (int k4 = 0; k4 < 8; ++k4) {
         const float4 z4 = __ldg(reinterpret_cast<const float4*>(zg + 4 * k4));
         dpart = fmaf(bf16lo(qa[2 * k4]), z4.x, dpart);
         dpart = fmaf(bf16hi(qa[2 * k4]), z4.y, dpart);
         dpart = fmaf(bf16lo(qa[2 * k4 + 1]), z4.z, dpart);
         dpart = fmaf(bf16hi(qa[2 * k4 + 1]), z4.w, dpart);
       }
-      xch[hf * 128 + row] = dpart;
+      xch[part * 128 + row] = dpart;
       __syncwarp();
       if (lane == 0) mbar_arrive(pr);
       if (!warp_wait(pr, 0u, abort_flag)) break;
-      const float dother = xch[(hf ^ 1) * 128 + row];
-      const float den = (hf == 0 ? dpart + dother : dother + dpart) + p.eps;
+      const float den = ((xch[row] + xch[128 + row]) + (xch[256 + row] + xch[384 + row])) + p.eps;
       const float rden = 1.0f / den;
-      // num -> y; with G and dO: dG (staged), dnum (over dO), this half's dy . y.
+      // num -> y; with G and dO: dG (over G), dnum (over dO), this quarter's dy . y.
       if (!warp_wait(&bars->numready, ph, abort_flag)) break;
+      if (!warp_wait(&bars->full_g, ph, abort_flag)) break;
       tc_fence_after();
-      float x[64];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      float x[32];
+      {
         uint32_t r[32];
-        tmem_ld_x32(tmem + QCOL_NUM + lane_bits + 64u * hf + 32 * j, r);
+        tmem_ld_x32(tmem + QCOL_NUM + lane_bits + static_cast<uint32_t>(cpart), r);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[32 * j + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
       }
       float dyy = 0.f;
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const int ck = 8 * hf + c8;
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const int ck = 4 * part + c4;
         const uint32_t ag = row_chunk(sbase + QO_G, row, ck);
         const uint4 gr = lds128(ag);
         const uint32_t ad = row_chunk(sbase + QO_DO, row, ck);
@@ -278,7 +296,7 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int q = 0; q < 4; ++q) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int e = 8 * c8 + 2 * q + h;
+            const int e = 8 * c4 + 2 * q + h;
             const float gv = h ? bf16hi(gw[q]) : bf16lo(gw[q]);
             const float dov = h ? bf16hi(dw[q]) : bf16lo(dw[q]);
             const float y = x[e] * rden;
@@ -296,24 +314,24 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->dn);
-      xch[256 + hf * 128 + row] = dyy;
+      xch[PARTS * 128 + part * 128 + row] = dyy;
       __syncwarp();
       if (lane == 0) mbar_arrive(pr);
       if (!warp_wait(pr, 1u, abort_flag)) break;
-      const float yother = xch[256 + (hf ^ 1) * 128 + row];
-      const float dden = -(hf == 0 ? dyy + yother : yother + dyy) * rden;
-      // dz over this warp's 32 rows for this half's 64 channels: lane L ends with channels
-      // 64 hf + 2L, 64 hf + 2L + 1 (a butterfly that halves the range per step, each sum formed
-      // once, lower lane first).
+      const float* yx = xch + PARTS * 128;
+      const float dden = -((yx[row] + yx[128 + row]) + (yx[256 + row] + yx[384 + row])) * rden;
+      // dz over this warp's 32 rows for this quarter's 32 channels: lane L ends with channel
+      // 32 part + L (a butterfly that halves the range per step, each sum formed once, lower
+      // lane first).
       {
-        float v[64];
+        float v[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < 16; ++e) {
           v[2 * e] = dden * bf16lo(qa[e]);
           v[2 * e + 1] = dden * bf16hi(qa[e]);
         }
 #pragma unroll
-        for (int off = 16, size = 64; off >= 1; off >>= 1, size >>= 1) {
+        for (int off = 16, size = 32; off >= 1; off >>= 1, size >>= 1) {
           const bool up = (lane & off) != 0;
 #pragma unroll
           for (int e = 0; e < size / 2; ++e) {
@@ -323,55 +341,52 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             v[e] = up ? other + keep : keep + other;
           }
         }
-        dzacc[0] += v[0];
-        dzacc[1] += v[1];
+        dzacc += v[0];
       }
-      // dq = [q > 0] (RoPE^T(dnum S^T) + dden z) for this half, into the dQ staging buffer.
+      // dq = [q > 0] (RoPE^T(dnum S^T) + dden z) for this quarter, into the dQ staging buffer.
       if (!warp_wait(&bars->dpqready, ph, abort_flag)) break;
       tc_fence_after();
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      {
         uint32_t r[32];
-        tmem_ld_x32(tmem + QCOL_DPQ + lane_bits + 64u * hf + 32 * j, r);
+        tmem_ld_x32(tmem + QCOL_DPQ + lane_bits + static_cast<uint32_t>(cpart), r);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[32 * j + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
       }
-      if (hf == 0)
-        rotate_half_t<DT, DH, 0>(x, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
-      else
-        rotate_half_t<DT, DH, 1>(x, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+      switch (part) {
+        case 0: rotate_span_t<DT, DH, 0, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+        case 1: rotate_span_t<DT, DH, 16, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+        case 2: rotate_span_t<DT, DH, 32, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+        default: rotate_span_t<DT, DH, 48, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+      }
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c8));
-        const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c8 + 4));
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4));
+        const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4 + 4));
         const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
         float o8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const uint32_t w = qa[4 * c8 + e / 2];
+          const uint32_t w = qa[4 * c4 + e / 2];
           const float qv = (e & 1) ? bf16hi(w) : bf16lo(w);
-          o8[e] = qv > 0.f ? x[8 * c8 + e] + dden * zz[e] : 0.f;
+          o8[e] = qv > 0.f ? x[8 * c4 + e] + dden * zz[e] : 0.f;
         }
-        sts128(row_chunk(sbase + QO_DQ, row, 8 * hf + c8), pack8(o8));
+        sts128(row_chunk(sbase + QO_DQ, row, 4 * part + c4), pack8(o8));
       }
       if (last) {
-        // dS of this unit (TMEM lane = channel k of phi(Q); this half's 64 columns) and dz -> the
-        // CTA's partial slot.
+        // dS of this unit (TMEM lane = channel k of phi(Q); this quarter's 32 columns) and dz ->
+        // the CTA's partial slot.
         float* dst = partial + (c * p.maxseg + (ti.unit - u_first)) * slot_floats;
+        uint32_t r[32];
+        tmem_ld_x32(tmem + QCOL_DS + lane_bits + static_cast<uint32_t>(cpart), r);
+        tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          uint32_t r[32];
-          tmem_ld_x32(tmem + QCOL_DS + lane_bits + 64u * hf + 32 * j, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            reinterpret_cast<float4*>(dst + row * D + 64 * hf + 32 * j)[e] =
-                make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
-                            __uint_as_float(r[4 * e + 3]));
-        }
-        reinterpret_cast<float2*>(dst + D * D + quarter * D + 64 * hf)[lane] = make_float2(dzacc[0], dzacc[1]);
-        dzacc[0] = dzacc[1] = 0.f;
+        for (int e = 0; e < 8; ++e)
+          reinterpret_cast<float4*>(dst + row * D + cpart)[e] =
+              make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
+                          __uint_as_float(r[4 * e + 3]));
+        dst[D * D + quarter * D + cpart + lane] = dzacc;
+        dzacc = 0.f;
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -405,6 +420,7 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->full, 1);
+    mbar_init(&bars->full_v, 1);
     mbar_init(&bars->rot, MATH_WARPS);
     mbar_init(&bars->ready, 1);
     mbar_init(&bars->out, MATH_WARPS);
@@ -425,19 +441,20 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 
   if (warp == CTRL_WARP) {
     if (lane == 0) {
-      auto load2 = [&](uint32_t off, const CUtensorMap* tm, const TileInfo& t) {
+      auto load2 = [&](uint32_t off, const CUtensorMap* tm, const TileInfo& t, uint64_t* bar) {
         const int32_t n0 = static_cast<int32_t>(t.n0), bh = static_cast<int32_t>(t.bh);
-        tma_load_3d(smem + off, tm, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + off + HALF, tm, 64, n0, bh, &bars->full);
+        tma_load_3d(smem + off, tm, 0, n0, bh, bar);
+        tma_load_3d(smem + off + HALF, tm, 64, n0, bh, bar);
       };
-      int64_t issued = 0;
+      int64_t issued = 0, issued_v = 0;
       if (g0 < g1) {
         const TileInfo t0 = tile_info(p, g0);
-        mbar_arrive_expect_tx(&bars->full, 3 * BUF);
+        mbar_arrive_expect_tx(&bars->full, 2 * BUF);
         bulk_load(smem + KO_S, dsimg + t0.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
-        load2(KO_K, &tmK, t0);
-        load2(KO_V, &tmV, t0);
-        issued = 1;
+        load2(KO_K, &tmK, t0, &bars->full);
+        mbar_arrive_expect_tx(&bars->full_v, BUF);
+        load2(KO_V, &tmV, t0, &bars->full_v);
+        issued = issued_v = 1;
       }
       for (int64_t g = g0; g < g1; ++g) {
         const int64_t i = g - g0;
@@ -452,6 +469,8 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + KCOL_DV, desc_k(sbase + KO_K, kk), desc_mn(sbase + KO_S, kk), IDESC_QS, kk > 0 ? 1u : 0u);
+        if (!mbar_wait(&bars->full_v, ph, abort_flag)) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + KCOL_DPK, desc_k(sbase + KO_V, kk), desc_k(sbase + KO_S, kk), IDESC_QST, kk > 0 ? 1u : 0u);
@@ -459,11 +478,13 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         // The products were the last readers of K, V and the dS image: the next tile's land now.
         if (has_next) {
           if (!mbar_wait(&bars->ready, ph, abort_flag)) break;
-          mbar_arrive_expect_tx(&bars->full, 2 * BUF + (next_new_unit ? BUF : 0u));
+          mbar_arrive_expect_tx(&bars->full, BUF + (next_new_unit ? BUF : 0u));
           if (next_new_unit) bulk_load(smem + KO_S, dsimg + tn.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
-          load2(KO_K, &tmK, tn);
-          load2(KO_V, &tmV, tn);
+          load2(KO_K, &tmK, tn, &bars->full);
+          mbar_arrive_expect_tx(&bars->full_v, BUF);
+          load2(KO_V, &tmV, tn, &bars->full_v);
           ++issued;
+          ++issued_v;
         }
         if (!mbar_wait(&bars->out, ph, abort_flag)) break;
         {
@@ -477,85 +498,92 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         }
       }
       bulk_wait_group0();
-      if (*abort_flag && issued > 0) mbar_wait_drain(&bars->full, static_cast<uint32_t>((issued - 1) & 1));
+      if (*abort_flag) {
+        if (issued > 0) mbar_wait_drain(&bars->full, static_cast<uint32_t>((issued - 1) & 1));
+        if (issued_v > 0) mbar_wait_drain(&bars->full_v, static_cast<uint32_t>((issued_v - 1) & 1));
+      }
       mma_commit(&bars->final_);
       mbar_wait_drain(&bars->final_, 0);
     }
   } else {
-    const int quarter = warp & 3, hf = warp >> 2;
+    const int quarter = warp & 3, part = warp >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+    const int cpart = 32 * part;  // this warp's channels
     for (int64_t g = g0; g < g1; ++g) {
       const int64_t i = g - g0;
       const uint32_t ph = static_cast<uint32_t>(i & 1);
       const TileInfo ti = tile_info(p, g);
       if (!warp_wait(&bars->full, ph, abort_flag)) break;
-      uint32_t ka[32];
+      uint32_t ka[16];
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const uint4 rk = lds128(row_chunk(sbase + KO_K, row, 8 * hf + c8));
-        ka[4 * c8] = rk.x;
-        ka[4 * c8 + 1] = rk.y;
-        ka[4 * c8 + 2] = rk.z;
-        ka[4 * c8 + 3] = rk.w;
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const uint4 rk = lds128(row_chunk(sbase + KO_K, row, 4 * part + c4));
+        ka[4 * c4] = rk.x;
+        ka[4 * c4 + 1] = rk.y;
+        ka[4 * c4 + 2] = rk.z;
+        ka[4 * c4 + 3] = rk.w;
       }
       const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
       uint32_t pt = 0, ph_ = 0, pw = 0;
       if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph_, pw);
+      const int ipt = static_cast<int>(pt), iph = static_cast<int>(ph_), ipw = static_cast<int>(pw);
       {
-        uint32_t a[32];
+        uint32_t a[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) a[e] = relu_bf16x2(ka[e]);
-        if (hf == 0)
-          rotate_half<DT, DH, 0>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
-        else
-          rotate_half<DT, DH, 1>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        for (int e = 0; e < 16; ++e) a[e] = relu_bf16x2(ka[e]);
+        switch (part) {
+          case 0: rotate_span<DT, DH, 0, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 1: rotate_span<DT, DH, 16, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 2: rotate_span<DT, DH, 32, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+          default: rotate_span<DT, DH, 48, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+        }
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8)
-          sts128(row_chunk(sbase + KO_K, row, 8 * hf + c8), make_uint4(a[4 * c8], a[4 * c8 + 1], a[4 * c8 + 2], a[4 * c8 + 3]));
+        for (int c4 = 0; c4 < 4; ++c4)
+          sts128(row_chunk(sbase + KO_K, row, 4 * part + c4), make_uint4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->rot);
       if (!warp_wait(&bars->ready, ph, abort_flag)) break;
       tc_fence_after();
-      float x[64];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      float x[32];
+      {
         uint32_t r[32];
-        tmem_ld_x32(tmem + KCOL_DV + lane_bits + 64u * hf + 32 * j, r);
+        tmem_ld_x32(tmem + KCOL_DV + lane_bits + static_cast<uint32_t>(cpart), r);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[32 * j + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
       }
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) sts128(row_chunk(sbase + KO_DV, row, 8 * hf + c8), pack8(&x[8 * c8]));
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      for (int c4 = 0; c4 < 4; ++c4) sts128(row_chunk(sbase + KO_DV, row, 4 * part + c4), pack8(&x[8 * c4]));
+      {
         uint32_t r[32];
-        tmem_ld_x32(tmem + KCOL_DPK + lane_bits + 64u * hf + 32 * j, r);
+        tmem_ld_x32(tmem + KCOL_DPK + lane_bits + static_cast<uint32_t>(cpart), r);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[32 * j + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
       }
-      if (hf == 0)
-        rotate_half_t<DT, DH, 0>(x, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
-      else
-        rotate_half_t<DT, DH, 1>(x, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
-      const float* zg = dzimg + ti.unit * D + 64 * hf;
+      switch (part) {
+        case 0: rotate_span_t<DT, DH, 0, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+        case 1: rotate_span_t<DT, DH, 16, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+        case 2: rotate_span_t<DT, DH, 32, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+        default: rotate_span_t<DT, DH, 48, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+      }
+      const float* zg = dzimg + ti.unit * D + cpart;
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c8));
-        const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c8 + 4));
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4));
+        const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4 + 4));
         const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
         float o8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const uint32_t w = ka[4 * c8 + e / 2];
+          const uint32_t w = ka[4 * c4 + e / 2];
           const float kv = (e & 1) ? bf16hi(w) : bf16lo(w);
-          o8[e] = kv > 0.f ? x[8 * c8 + e] + zz[e] : 0.f;
+          o8[e] = kv > 0.f ? x[8 * c4 + e] + zz[e] : 0.f;
         }
-        sts128(row_chunk(sbase + KO_DK, row, 8 * hf + c8), pack8(o8));
+        sts128(row_chunk(sbase + KO_DK, row, 4 * part + c4), pack8(o8));
       }
       fence_proxy_async_smem();
       tc_fence_before();

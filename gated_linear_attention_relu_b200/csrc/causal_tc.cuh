@@ -17,10 +17,12 @@
 // P o M goes back to TMEM as bf16 and is the A operand of the P V product; S_prev is the bf16
 // image of the carried state in shared memory (rewritten after every chunk).
 //
-// Warps: 0-7 own the chunk's rows, two per row (channel halves; thread = token = TMEM lane, warp
-// w reaching lanes 32 (w mod 4) ..); warp 8 issues the TMA copies and the MMAs.  The phases of a chunk run in sequence; the next chunk's tiles are loaded as soon as
-// their buffers are free (Q and K once the products reading them are done, V after P V, G after
-// this chunk's O has been stored), so their latency overlaps the end of the chunk.
+// Warps: 0-15 own the chunk's rows, four per row (channel quarters; thread = token = TMEM lane,
+// warp w reaching lanes 32 (w mod 4) ..); warp 16 issues the TMA copies and the MMAs.  The phases
+// of a chunk run in sequence; the next chunk's tiles are loaded as soon as their buffers are free
+// (Q and K once the products reading them are done, V after P V, G after this chunk's O has been
+// stored), each pair on its own barrier and waited for only by its first reader (Q and K: the
+// ReLU pass; V: the state update; G: the epilogue), so their latency overlaps the chunk's work.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -33,26 +35,30 @@ using namespace la::tile;
 
 constexpr int TILE = 128;
 constexpr int D = 128;
-constexpr int MATH_WARPS = 8;  // two per TMEM lane quarter: channel halves of a row
+constexpr int MATH_WARPS = 16;  // four per TMEM lane quarter: channel quarters of a row
+constexpr int PARTS = MATH_WARPS / 4;
 constexpr int CTRL_WARP = MATH_WARPS;
 constexpr int THREADS = 32 * (MATH_WARPS + 1);
 constexpr uint32_t HALF = 128 * 128;
 constexpr uint32_t BUF = 2 * HALF;
 constexpr uint32_t OFF_Q = 0, OFF_K = BUF, OFF_V = 2 * BUF, OFF_G = 3 * BUF, OFF_S = 4 * BUF;
-constexpr uint32_t OFF_Z = 5 * BUF;            // z of the tokens before the chunk, [128] fp32
-constexpr uint32_t OFF_ZP = OFF_Z + 512;       // the chunk's K^+ column sums per row half, [2][128]
-constexpr uint32_t OFF_DX = OFF_ZP + 1024;     // partial denominators, [2 slots][2 halves][128]
-constexpr uint32_t OFF_BAR = OFF_DX + 2048;
+constexpr uint32_t OFF_Z = 5 * BUF;              // z of the tokens before the chunk, [128] fp32
+constexpr uint32_t OFF_ZP = OFF_Z + 512;         // the chunk's K^+ column sums per row quarter, [4][128]
+constexpr uint32_t OFF_DX = OFF_ZP + 4 * 512;    // partial denominators, [2 slots][4 parts][128]
+constexpr uint32_t OFF_BAR = OFF_DX + 2 * 4 * 512;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_S = 0, COL_ND = 128, COL_P = 256;  // carried S; D then num; P (then bf16 P)
+// carried S; D then num; P (fp32); the masked P as bf16 (the A operand of P V)
+constexpr uint32_t COL_S = 0, COL_ND = 128, COL_P = 256, COL_PB = 384;
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/false);
 constexpr uint32_t IDESC_QS = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/true);
 constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, /*a_mn=*/true, /*b_mn=*/true);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 struct Bars {
-  uint64_t full;      // Q, K, V, G of the chunk landed
+  uint64_t full_qk;   // Q and K of the chunk landed
+  uint64_t full_v;    // V landed
+  uint64_t full_g;    // G landed
   uint64_t relu;      // math: Q^+ and K^+ written in place (4 warps)
   uint64_t zsync1;    // math: every row's K^+ written (4 warps), before the column reads
   uint64_t zsync;     // math: z published and K^+ columns read (4 warps)
@@ -62,8 +68,7 @@ struct Bars {
   uint64_t pw;        // math: masked P written to TMEM as bf16 (4 warps)
   uint64_t numready;  // MMA: num += P V done
   uint64_t out;       // math: O staged over G, S image rewritten (8 warps)
-  uint64_t denx[4];   // the two warps holding the halves of rows 32q .. 32q+31 (2 arrivals);
-                      // two phases per chunk: the denominator swap (even), the P handoff (odd)
+  uint64_t denx[4];   // the four warps holding the quarters of rows 32q .. 32q+31 (4 arrivals)
   uint64_t final_;
   uint32_t tmem_base;
   int abort_flag;
@@ -98,7 +103,9 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   }
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->full, 1);
+    mbar_init(&bars->full_qk, 1);
+    mbar_init(&bars->full_v, 1);
+    mbar_init(&bars->full_g, 1);
     mbar_init(&bars->relu, MATH_WARPS);
     mbar_init(&bars->zsync1, MATH_WARPS);
     mbar_init(&bars->zsync, MATH_WARPS);
@@ -108,7 +115,7 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     mbar_init(&bars->pw, MATH_WARPS);
     mbar_init(&bars->numready, 1);
     mbar_init(&bars->out, MATH_WARPS);
-    for (int q = 0; q < 4; ++q) mbar_init(&bars->denx[q], 2);
+    for (int q = 0; q < 4; ++q) mbar_init(&bars->denx[q], PARTS);
     mbar_init(&bars->final_, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -132,20 +139,23 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tma_prefetch_desc(&tmG);
       tma_prefetch_desc(&tmO);
       int64_t prev_unit = -1;
-      int64_t issued = 0;  // chunks whose loads have been armed on `full`
-      auto load2 = [&](uint32_t off, const CUtensorMap* tm, const TileInfo& t) {
+      // chunks whose loads have been armed on full_qk, full_v, full_g
+      int64_t issued_qk = 0, issued_v = 0, issued_g = 0;
+      auto load2 = [&](uint32_t off, const CUtensorMap* tm, const TileInfo& t, uint64_t* bar) {
         const int32_t n0 = static_cast<int32_t>(t.n0), bh = static_cast<int32_t>(t.bh);
-        tma_load_3d(smem + off, tm, 0, n0, bh, &bars->full);
-        tma_load_3d(smem + off + HALF, tm, 64, n0, bh, &bars->full);
+        tma_load_3d(smem + off, tm, 0, n0, bh, bar);
+        tma_load_3d(smem + off + HALF, tm, 64, n0, bh, bar);
       };
       if (g0 < g1) {
         const TileInfo t0 = tile_info(p, g0);
-        mbar_arrive_expect_tx(&bars->full, 4 * BUF);
-        load2(OFF_Q, &tmQ, t0);
-        load2(OFF_K, &tmK, t0);
-        load2(OFF_V, &tmV, t0);
-        load2(OFF_G, &tmG, t0);
-        issued = 1;
+        mbar_arrive_expect_tx(&bars->full_qk, 2 * BUF);
+        load2(OFF_Q, &tmQ, t0, &bars->full_qk);
+        load2(OFF_K, &tmK, t0, &bars->full_qk);
+        mbar_arrive_expect_tx(&bars->full_v, BUF);
+        load2(OFF_V, &tmV, t0, &bars->full_v);
+        mbar_arrive_expect_tx(&bars->full_g, BUF);
+        load2(OFF_G, &tmG, t0, &bars->full_g);
+        issued_qk = issued_v = issued_g = 1;
       }
       for (int64_t g = g0; g < g1; ++g) {
         const int64_t i = g - g0;
@@ -175,6 +185,8 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + COL_P, desc_k(sbase + OFF_Q, kk), desc_k(sbase + OFF_K, kk), IDESC_QK, kk > 0 ? 1u : 0u);
+        if (!mbar_wait(&bars->full_v, ph, abort_flag)) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + COL_S, desc_mn(sbase + OFF_K, kk), desc_mn(sbase + OFF_V, kk), IDESC_KV,
@@ -184,22 +196,24 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         // while this chunk's P V product and epilogue run.
         if (has_next) {
           if (!mbar_wait(&bars->pready, ph, abort_flag)) break;
-          mbar_arrive_expect_tx(&bars->full, 4 * BUF);
-          load2(OFF_Q, &tmQ, tn);
-          load2(OFF_K, &tmK, tn);
-          ++issued;
+          mbar_arrive_expect_tx(&bars->full_qk, 2 * BUF);
+          load2(OFF_Q, &tmQ, tn, &bars->full_qk);
+          load2(OFF_K, &tmK, tn, &bars->full_qk);
+          ++issued_qk;
         }
         // num += (P o M) V
         if (!mbar_wait(&bars->pw, ph, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + COL_ND, tmem + COL_P + 8u * kk, desc_mn(sbase + OFF_V, kk), IDESC_QS,
+          mma_bf16_ts(tmem + COL_ND, tmem + COL_PB + 8u * kk, desc_mn(sbase + OFF_V, kk), IDESC_QS,
                       (kk > 0 || !zero_start) ? 1u : 0u);
         mma_commit(&bars->numready);
         if (has_next) {
           if (!mbar_wait(&bars->numready, ph, abort_flag)) break;
-          load2(OFF_V, &tmV, tn);
+          mbar_arrive_expect_tx(&bars->full_v, BUF);
+          load2(OFF_V, &tmV, tn, &bars->full_v);
+          ++issued_v;
         }
         // O of this chunk (staged over G) out, then the next chunk's G in.
         if (!mbar_wait(&bars->out, ph, abort_flag)) break;
@@ -210,49 +224,53 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           bulk_commit_group();
           bulk_wait_group_read0();
         }
-        if (has_next) load2(OFF_G, &tmG, tn);
+        if (has_next) {
+          mbar_arrive_expect_tx(&bars->full_g, BUF);
+          load2(OFF_G, &tmG, tn, &bars->full_g);
+          ++issued_g;
+        }
       }
       bulk_wait_group0();
-      if (*abort_flag && issued > 0) mbar_wait_drain(&bars->full, static_cast<uint32_t>((issued - 1) & 1));
+      if (*abort_flag) {
+        if (issued_qk > 0) mbar_wait_drain(&bars->full_qk, static_cast<uint32_t>((issued_qk - 1) & 1));
+        if (issued_v > 0) mbar_wait_drain(&bars->full_v, static_cast<uint32_t>((issued_v - 1) & 1));
+        if (issued_g > 0) mbar_wait_drain(&bars->full_g, static_cast<uint32_t>((issued_g - 1) & 1));
+      }
       mma_commit(&bars->final_);
       mbar_wait_drain(&bars->final_, 0);
     }
   } else {
-    // ------------------------------------------------------------ rows (warps 0-7)
-    const int quarter = warp & 3, hf = warp >> 2;
+    // ------------------------------------------------------------ rows (warps 0-15)
+    const int quarter = warp & 3, part = warp >> 2;
     const int row = quarter * 32 + lane;  // token row of the chunk = TMEM lane; also channel k for z and S
     const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t t_s = tmem + COL_S + lane_bits + 64u * hf, t_nd = tmem + COL_ND + lane_bits + 64u * hf;
-    const uint32_t t_p = tmem + COL_P + lane_bits;
+    const uint32_t cpart = 32u * static_cast<uint32_t>(part);  // this warp's channels (and P columns)
+    const uint32_t t_s = tmem + COL_S + lane_bits + cpart, t_nd = tmem + COL_ND + lane_bits + cpart;
+    const uint32_t t_p = tmem + COL_P + lane_bits + cpart, t_pb = tmem + COL_PB + lane_bits + cpart / 2;
     float* zp = reinterpret_cast<float*>(smem + OFF_ZP);
     float* dx = reinterpret_cast<float*>(smem + OFF_DX);
     uint64_t* denx = &bars->denx[quarter];
-    float zk = 0.f;  // (hf == 0) z of channel `row` over the tokens before the chunk
+    float zk = 0.f;  // (part 0) z of channel `row` over the tokens before the chunk
     pdl_wait();      // the start states and the cos/sin tables come from the kernels before
     if (g0 < g1 && has_start) {
-      // Carried state at the segment start: this half of fp32 row `row` of S into TMEM, its bf16
-      // image, and z.
+      // Carried state at the segment start: this quarter of fp32 row `row` of S into TMEM, its
+      // bf16 image, and z.
       const float* src = start + c * (D * D + D);
       uint32_t r[32];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(src[row * D + cpart + e]);
+      tmem_st_x16(t_s, &r[0]);
+      tmem_st_x16(t_s + 16, &r[16]);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(src[row * D + 64 * hf + 32 * j + e]);
-        tmem_st_x16(t_s + 32 * j, &r[0]);
-        tmem_st_x16(t_s + 32 * j + 16, &r[16]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int ck = 8 * hf + 4 * j + e;
-          sts128(row_chunk(sbase + OFF_S, row, ck),
-                 make_uint4(pack_bf16(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
-                            pack_bf16(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
-                            pack_bf16(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
-                            pack_bf16(__uint_as_float(r[8 * e + 6]), __uint_as_float(r[8 * e + 7]))));
-        }
-      }
+      for (int e = 0; e < 4; ++e)
+        sts128(row_chunk(sbase + OFF_S, row, 4 * part + e),
+               make_uint4(pack_bf16(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
+                          pack_bf16(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
+                          pack_bf16(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
+                          pack_bf16(__uint_as_float(r[8 * e + 6]), __uint_as_float(r[8 * e + 7]))));
       tmem_st_wait();
       fence_proxy_async_smem();
-      if (hf == 0) zk = src[D * D + row];
+      if (part == 0) zk = src[D * D + row];
     }
     int64_t prev_unit = -1;
     for (int64_t g = g0; g < g1; ++g) {
@@ -261,19 +279,19 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const TileInfo ti = tile_info(p, g);
       if (ti.unit != prev_unit && !(g == g0 && has_start)) zk = 0.f;  // a head starting in this CTA
       prev_unit = ti.unit;
-      if (!warp_wait(&bars->full, ph, abort_flag)) break;
-      // ReLU of this half of the Q and K rows in place; q^+ kept in registers.
-      uint32_t qa[32];
+      if (!warp_wait(&bars->full_qk, ph, abort_flag)) break;
+      // ReLU of this quarter of the Q and K rows in place; q^+ kept in registers.
+      uint32_t qa[16];
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const int ck = 8 * hf + c8;
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const int ck = 4 * part + c4;
         const uint32_t aq = row_chunk(sbase + OFF_Q, row, ck);
         const uint4 rq = lds128(aq);
-        qa[4 * c8] = relu_bf16x2(rq.x);
-        qa[4 * c8 + 1] = relu_bf16x2(rq.y);
-        qa[4 * c8 + 2] = relu_bf16x2(rq.z);
-        qa[4 * c8 + 3] = relu_bf16x2(rq.w);
-        sts128(aq, make_uint4(qa[4 * c8], qa[4 * c8 + 1], qa[4 * c8 + 2], qa[4 * c8 + 3]));
+        qa[4 * c4] = relu_bf16x2(rq.x);
+        qa[4 * c4 + 1] = relu_bf16x2(rq.y);
+        qa[4 * c4 + 2] = relu_bf16x2(rq.z);
+        qa[4 * c4 + 3] = relu_bf16x2(rq.w);
+        sts128(aq, make_uint4(qa[4 * c4], qa[4 * c4 + 1], qa[4 * c4 + 2], qa[4 * c4 + 3]));
         const uint32_t ak = row_chunk(sbase + OFF_K, row, ck);
         const uint4 rk = lds128(ak);
         sts128(ak, make_uint4(relu_bf16x2(rk.x), relu_bf16x2(rk.y), relu_bf16x2(rk.z), relu_bf16x2(rk.w)));
@@ -284,9 +302,9 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         mbar_arrive(&bars->relu);
         mbar_arrive(&bars->zsync1);
       }
-      // z before the chunk, published for every row's denominator (hf 0); then this chunk's K^+
-      // column `row` over this half's 64 rows, once every row is ReLU'd.
-      if (hf == 0) zs[row] = zk;
+      // z before the chunk, published for every row's denominator (part 0); then this chunk's K^+
+      // column `row` over the rows of this quarter, once every row is ReLU'd.
+      if (part == 0) zs[row] = zk;
       if (!warp_wait(&bars->zsync1, ph, abort_flag)) break;
       {
         const int kc = row;  // channel
@@ -294,8 +312,8 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const uint32_t cchunk = static_cast<uint32_t>((kc & 63) >> 3), cbyte = static_cast<uint32_t>(kc & 7) * 2u;
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-        for (int mm = 0; mm < 64; ++mm) {
-          const int m = 64 * hf + mm;
+        for (int mm = 0; mm < 32; ++mm) {
+          const int m = 32 * part + mm;
           uint16_t hv;
           asm volatile("ld.shared.u16 %0, [%1];"
                        : "=h"(hv)
@@ -303,18 +321,18 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                              cbyte));
           s4[mm & 3] += __uint_as_float(static_cast<uint32_t>(hv) << 16);
         }
-        zp[hf * 128 + row] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        zp[part * 128 + row] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->zsync);
       if (!warp_wait(&bars->zsync, ph, abort_flag)) break;
-      if (hf == 0) zk += zp[row] + zp[128 + row];
-      // This half's share of the denominator: q^+ . z_prev over its channels plus the masked row
-      // sum of D over its columns; the two halves of the row add theirs.
+      if (part == 0) zk += ((zp[row] + zp[128 + row]) + (zp[256 + row] + zp[384 + row]));
+      // This quarter's share of the denominator: q^+ . z_prev over its channels plus the masked
+      // row sum of D over its columns; the four quarters of the row add theirs.
       float dpart = 0.f;
 #pragma unroll
-      for (int k4 = 0; k4 < 16; ++k4) {
-        const float4 z4 = *reinterpret_cast<const float4*>(zs + 64 * hf + 4 * k4);
+      for (int k4 = 0; k4 < 8; ++k4) {
+        const float4 z4 = *reinterpret_cast<const float4*>(zs + cpart + 4 * k4);
         dpart = fmaf(bf16lo(qa[2 * k4]), z4.x, dpart);
         dpart = fmaf(bf16hi(qa[2 * k4]), z4.y, dpart);
         dpart = fmaf(bf16lo(qa[2 * k4 + 1]), z4.z, dpart);
@@ -322,102 +340,95 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
       if (!warp_wait(&bars->dready, ph, abort_flag)) break;
       tc_fence_after();
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      {
         uint32_t r[32];
-        tmem_ld_x32(t_nd + 32 * j, r);
+        tmem_ld_x32(t_nd, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) dpart += (64 * hf + 32 * j + e <= row) ? __uint_as_float(r[e]) : 0.f;
+        for (int e = 0; e < 32; ++e) dpart += (static_cast<int>(cpart) + e <= row) ? __uint_as_float(r[e]) : 0.f;
       }
+      float den;
       {
-        float* slot = dx + static_cast<int>(i & 1) * 256;
-        slot[hf * 128 + row] = dpart;
+        float* slot = dx + static_cast<int>(i & 1) * (PARTS * 128);
+        slot[part * 128 + row] = dpart;
         __syncwarp();
         if (lane == 0) mbar_arrive(denx);
-        if (!warp_wait(denx, 0u, abort_flag)) break;
-        const float other = slot[(hf ^ 1) * 128 + row];
-        dpart = hf == 0 ? dpart + other : other + dpart;
+        if (!warp_wait(denx, ph, abort_flag)) break;
+        den = (slot[row] + slot[128 + row]) + (slot[256 + row] + slot[384 + row]);
       }
-      const float hinv = 1.0f / (dpart + p.eps);
-      // RoPE of this half of Q^+ and K^+ in place.
+      const float hinv = 1.0f / (den + p.eps);
+      // RoPE of this quarter of Q^+ and K^+ in place.
       const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
       uint32_t pt = 0, ph_ = 0, pw = 0;
       if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph_, pw);
       {
-        uint32_t a[32];
+        auto rot = [&](uint32_t (&a)[16]) {
+          const int ipt = static_cast<int>(pt), iph = static_cast<int>(ph_), ipw = static_cast<int>(pw);
+          switch (part) {
+            case 0: rotate_span<DT, DH, 0, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+            case 1: rotate_span<DT, DH, 16, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+            case 2: rotate_span<DT, DH, 32, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+            default: rotate_span<DT, DH, 48, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+          }
+        };
+        uint32_t a[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) a[e] = qa[e];
-        if (hf == 0)
-          rotate_half<DT, DH, 0>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
-        else
-          rotate_half<DT, DH, 1>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        for (int e = 0; e < 16; ++e) a[e] = qa[e];
+        rot(a);
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8)
-          sts128(row_chunk(sbase + OFF_Q, row, 8 * hf + c8), make_uint4(a[4 * c8], a[4 * c8 + 1], a[4 * c8 + 2], a[4 * c8 + 3]));
+        for (int c4 = 0; c4 < 4; ++c4)
+          sts128(row_chunk(sbase + OFF_Q, row, 4 * part + c4), make_uint4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          const uint4 rk = lds128(row_chunk(sbase + OFF_K, row, 8 * hf + c8));
-          a[4 * c8] = rk.x;
-          a[4 * c8 + 1] = rk.y;
-          a[4 * c8 + 2] = rk.z;
-          a[4 * c8 + 3] = rk.w;
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const uint4 rk = lds128(row_chunk(sbase + OFF_K, row, 4 * part + c4));
+          a[4 * c4] = rk.x;
+          a[4 * c4 + 1] = rk.y;
+          a[4 * c4 + 2] = rk.z;
+          a[4 * c4 + 3] = rk.w;
         }
-        if (hf == 0)
-          rotate_half<DT, DH, 0>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
-        else
-          rotate_half<DT, DH, 1>(a, tab, tab2, rope, p, static_cast<int>(pt), static_cast<int>(ph_), static_cast<int>(pw));
+        rot(a);
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8)
-          sts128(row_chunk(sbase + OFF_K, row, 8 * hf + c8), make_uint4(a[4 * c8], a[4 * c8 + 1], a[4 * c8 + 2], a[4 * c8 + 3]));
+        for (int c4 = 0; c4 < 4; ++c4)
+          sts128(row_chunk(sbase + OFF_K, row, 4 * part + c4), make_uint4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->rot);
-      // Causal mask on this half of P (columns m in [64 hf, 64 hf + 64), kept where m <= n), back
-      // to TMEM as bf16 (the A operand of P V: columns 32 hf .. 32 hf + 31).
+      // Causal mask on this quarter of P (columns m in [32 part, 32 part + 32), kept where m <= n),
+      // written as bf16 to the A operand of P V (columns 16 part .. 16 part + 15 of that region).
       if (!warp_wait(&bars->pready, ph, abort_flag)) break;
       tc_fence_after();
       {
-        uint32_t pb[32];
+        uint32_t pb[16];
+        uint32_t r[32];
+        tmem_ld_x32(t_p, r);
+        tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          uint32_t r[32];
-          tmem_ld_x32(t_p + 64u * hf + 32 * j, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int m0 = 64 * hf + 32 * j + 2 * e;
-            const float p0 = m0 <= row ? __uint_as_float(r[2 * e]) : 0.f;
-            const float p1 = m0 + 1 <= row ? __uint_as_float(r[2 * e + 1]) : 0.f;
-            pb[16 * j + e] = pack_bf16(p0, p1);
-          }
+        for (int e = 0; e < 16; ++e) {
+          const int m0 = static_cast<int>(cpart) + 2 * e;
+          const float p0 = m0 <= row ? __uint_as_float(r[2 * e]) : 0.f;
+          const float p1 = m0 + 1 <= row ? __uint_as_float(r[2 * e + 1]) : 0.f;
+          pb[e] = pack_bf16(p0, p1);
         }
-        // Half 1 writes bf16 columns 32-63, which half 0 reads as fp32: the pair meets once more
-        // (the odd phase of its barrier) before either writes.
-        __syncwarp();
-        if (lane == 0) mbar_arrive(denx);
-        if (!warp_wait(denx, 1u, abort_flag)) break;
-        tmem_st_x16(t_p + 32u * hf, &pb[0]);
-        tmem_st_x16(t_p + 32u * hf + 16, &pb[16]);
+        tmem_st_x16(t_pb, &pb[0]);
         tmem_st_wait();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->pw);
-      // O = num / den * sigmoid(g) for this half, in place over G; then this half of the new
+      // O = num / den * sigmoid(g) for this quarter, in place over G; then this quarter of the new
       // state's bf16 image.
       if (!warp_wait(&bars->numready, ph, abort_flag)) break;
+      if (!warp_wait(&bars->full_g, ph, abort_flag)) break;
       tc_fence_after();
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      {
         uint32_t r[32];
-        tmem_ld_x32(t_nd + 32 * j, r);
+        tmem_ld_x32(t_nd, r);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint32_t ag = row_chunk(sbase + OFF_G, row, 8 * hf + 4 * j + e);
+          const uint32_t ag = row_chunk(sbase + OFF_G, row, 4 * part + e);
           const uint4 gr = lds128(ag);
           const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
           uint32_t ov[4];
@@ -430,14 +441,13 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           sts128(ag, make_uint4(ov[0], ov[1], ov[2], ov[3]));
         }
       }
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      {
         uint32_t r[32];
-        tmem_ld_x32(t_s + 32 * j, r);
+        tmem_ld_x32(t_s, r);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          sts128(row_chunk(sbase + OFF_S, row, 8 * hf + 4 * j + e),
+          sts128(row_chunk(sbase + OFF_S, row, 4 * part + e),
                  make_uint4(pack_bf16(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
                             pack_bf16(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
                             pack_bf16(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),

@@ -69,12 +69,14 @@ __device__ __forceinline__ void rotate_row(uint32_t (&a)[64], const float2* __re
   }
 }
 
-// In place over half a row (channels [64 HF, 64 HF + 64) as 32 bf16 pairs, already ReLU'd):
-// a <- RoPE(a) at grid position (pt, ph, pw).
-template <int DT, int DH, int HF>
-__device__ __forceinline__ void rotate_half(uint32_t (&a)[32], const float2* __restrict__ tab,
+// In place over the NP bf16 pairs of a row starting at pair P0 (channels [2 P0, 2 P0 + 2 NP),
+// already ReLU'd): a <- RoPE(a) at grid position (pt, ph, pw).  P0 and NP are even, so the span
+// covers whole 16-byte table entries.
+template <int DT, int DH, int P0, int NP>
+__device__ __forceinline__ void rotate_span(uint32_t (&a)[NP], const float2* __restrict__ tab,
                                             const float4* __restrict__ tab2, const Rope& rope, const Plan& p,
                                             int pt, int ph, int pw) {
+  static_assert(P0 % 2 == 0 && NP % 2 == 0, "spans of whole table entries");
   if constexpr (DT >= 0 && DH >= 0) {
     constexpr int DW = 128 - DT - DH;
     static_assert(DT % 4 == 0 && DH % 4 == 0 && DW % 4 == 0, "bands of whole 16-byte entries");
@@ -83,8 +85,8 @@ __device__ __forceinline__ void rotate_half(uint32_t (&a)[32], const float2* __r
     const float4* bw = tab2 + rope.tab_off_w / 2 + pw;
     const int W = static_cast<int>(p.W);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int pi = 32 * HF + 2 * j;
+    for (int j = 0; j < NP / 2; ++j) {
+      const int pi = P0 + 2 * j;
       const int bnd = band_of<DT, DH>(pi, rope);
       const int e = pair_in_band<DT, DH>(pi, rope) / 2;
       const float4 cs = __ldg(bnd == 0 ? bt + e : (bnd == 1 ? bh + e : bw + e * W));
@@ -98,8 +100,8 @@ __device__ __forceinline__ void rotate_half(uint32_t (&a)[32], const float2* __r
     const int off[3] = {0, static_cast<int>(rope.tab_off_h), static_cast<int>(rope.tab_off_w)};
     const int pos[3] = {pt, ph, pw};
 #pragma unroll 4
-    for (int j = 0; j < 32; ++j) {
-      const int pi = 32 * HF + j;
+    for (int j = 0; j < NP; ++j) {
+      const int pi = P0 + j;
       const int bnd = band_of<DT, DH>(pi, rope);
       const int loc = pair_in_band<DT, DH>(pi, rope);
       const float2 cs = __ldg(tab + off[bnd] + loc * ext[bnd] + pos[bnd]);
@@ -107,6 +109,14 @@ __device__ __forceinline__ void rotate_half(uint32_t (&a)[32], const float2* __r
       a[j] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
     }
   }
+}
+
+// Half a row (channels [64 HF, 64 HF + 64) as 32 bf16 pairs).
+template <int DT, int DH, int HF>
+__device__ __forceinline__ void rotate_half(uint32_t (&a)[32], const float2* __restrict__ tab,
+                                            const float4* __restrict__ tab2, const Rope& rope, const Plan& p,
+                                            int pt, int ph, int pw) {
+  rotate_span<DT, DH, 32 * HF, 32>(a, tab, tab2, rope, p, pt, ph, pw);
 }
 
 // In place over one row of 128 fp32 values: x <- RoPE^T(x) (rotation by the opposite angle) at grid
@@ -148,19 +158,21 @@ __device__ __forceinline__ void rotate_row_t(float (&x)[128], const float2* __re
   }
 }
 
-// In place over half a row of fp32 values (channels [64 HF, 64 HF + 64)): x <- RoPE^T(x).
-template <int DT, int DH, int HF>
-__device__ __forceinline__ void rotate_half_t(float (&x)[64], const float2* __restrict__ tab,
+// In place over the fp32 values of NP pairs starting at pair P0 (channels [2 P0, 2 P0 + 2 NP)):
+// x <- RoPE^T(x).  P0 and NP are even.
+template <int DT, int DH, int P0, int NP>
+__device__ __forceinline__ void rotate_span_t(float (&x)[2 * NP], const float2* __restrict__ tab,
                                               const float4* __restrict__ tab2, const Rope& rope, const Plan& p,
                                               int pt, int ph, int pw) {
+  static_assert(P0 % 2 == 0 && NP % 2 == 0, "spans of whole table entries");
   if constexpr (DT >= 0 && DH >= 0) {
     const float4* bt = tab2 + pt * (DT / 4);
     const float4* bh = tab2 + rope.tab_off_h / 2 + ph * (DH / 4);
     const float4* bw = tab2 + rope.tab_off_w / 2 + pw;
     const int W = static_cast<int>(p.W);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int pi = 32 * HF + 2 * j;
+    for (int j = 0; j < NP / 2; ++j) {
+      const int pi = P0 + 2 * j;
       const int bnd = band_of<DT, DH>(pi, rope);
       const int e = pair_in_band<DT, DH>(pi, rope) / 2;
       const float4 cs = __ldg(bnd == 0 ? bt + e : (bnd == 1 ? bh + e : bw + e * W));
@@ -175,8 +187,8 @@ __device__ __forceinline__ void rotate_half_t(float (&x)[64], const float2* __re
     const int off[3] = {0, static_cast<int>(rope.tab_off_h), static_cast<int>(rope.tab_off_w)};
     const int pos[3] = {pt, ph, pw};
 #pragma unroll 4
-    for (int j = 0; j < 32; ++j) {
-      const int pi = 32 * HF + j;
+    for (int j = 0; j < NP; ++j) {
+      const int pi = P0 + j;
       const int bnd = band_of<DT, DH>(pi, rope);
       const int loc = pair_in_band<DT, DH>(pi, rope);
       const float2 cs = __ldg(tab + off[bnd] + loc * ext[bnd] + pos[bnd]);
@@ -185,6 +197,14 @@ __device__ __forceinline__ void rotate_half_t(float (&x)[64], const float2* __re
       x[2 * j + 1] = x1 * cs.x - x0 * cs.y;
     }
   }
+}
+
+// Half a row of fp32 values (channels [64 HF, 64 HF + 64)).
+template <int DT, int DH, int HF>
+__device__ __forceinline__ void rotate_half_t(float (&x)[64], const float2* __restrict__ tab,
+                                              const float4* __restrict__ tab2, const Rope& rope, const Plan& p,
+                                              int pt, int ph, int pw) {
+  rotate_span_t<DT, DH, 32 * HF, 32>(x, tab, tab2, rope, p, pt, ph, pw);
 }
 
 }  // namespace tile
