@@ -9,20 +9,25 @@
 // Chunkwise form.  The tiles of every head are split into contiguous segments, one per
 // persistent CTA (the same split as the state kernel's, whose per-segment sums the start
 // kernel prefix-sums into each CTA's starting state).  A CTA walks its 128-token chunks in order
-// carrying S (fp32, in TMEM) and z (fp32, channel k in thread k); for chunk c with rows n, m:
-//   D   = Q^+ K^+^T                     (tensor cores; masked row sums -> intra-chunk denominator)
-//   num = phi(Q) S_prev + (P o M) V,    P = phi(Q) phi(K)^T, M_nm = [m <= n]
-//   den = q_n^+ . z_prev + sum_{m<=n} D_nm + eps
-//   S  += phi(K)^T V,  z += column sums of K^+
-// P o M goes back to TMEM as bf16 and is the A operand of the P V product; S_prev is the bf16
-// image of the carried state in shared memory (rewritten after every chunk).
+// carrying S (fp32, in TMEM) and z (fp32, in shared memory); for chunk c with rows n, m:
+//   C   = M K^+,                        M_nm = [m <= n]  (C_n = sum_{m<=n} k_m^+ over the chunk)
+//   num = phi(Q) S_prev + (P o M) V,    P = phi(Q) phi(K)^T
+//   den = q_n^+ . (z_prev + C_n) + eps
+//   S  += phi(K)^T V,  z += C_127 (the chunk's last row: its column sums of K^+)
+// M is a constant bf16 operand in TMEM, so C is one product of the same form as (P o M) V; P o M
+// goes back to TMEM as bf16 and is the A operand of that product; S_prev is the bf16 image of
+// the carried state in shared memory (rewritten after every chunk).
 //
 // Warps: 0-15 own the chunk's rows, four per row (channel quarters; thread = token = TMEM lane,
-// warp w reaching lanes 32 (w mod 4) ..); warp 16 issues the TMA copies and the MMAs.  The phases
-// of a chunk run in sequence; the next chunk's tiles are loaded as soon as their buffers are free
-// (Q and K once the products reading them are done, V after P V, G after this chunk's O has been
-// stored), each pair on its own barrier and waited for only by its first reader (Q and K: the
-// ReLU pass; V: the state update; G: the epilogue), so their latency overlaps the chunk's work.
+// warp w reaching lanes 32 (w mod 4) ..); warp 16 issues the TMA copies and the MMAs.  Only K^+
+// goes back to shared memory before the first product; the rotation of Q runs while C is
+// computed (into the columns P takes later), phi(Q) S_prev starts as soon as phi(Q) is written,
+// K is rotated from registers, and the mask of P starts once P alone is done (the state update
+// runs under it).  The next chunk's tiles are loaded as soon as their
+// buffers are free (Q and K once the products reading them are done, V after P V, G after this
+// chunk's O has been stored), each on its own barrier and waited for only by its first reader
+// (Q and K: the ReLU pass; V: the state update; G: the epilogue), so their latency overlaps the
+// chunk's work.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -42,14 +47,15 @@ constexpr int THREADS = 32 * (MATH_WARPS + 1);
 constexpr uint32_t HALF = 128 * 128;
 constexpr uint32_t BUF = 2 * HALF;
 constexpr uint32_t OFF_Q = 0, OFF_K = BUF, OFF_V = 2 * BUF, OFF_G = 3 * BUF, OFF_S = 4 * BUF;
-constexpr uint32_t OFF_Z = 5 * BUF;              // z of the tokens before the chunk, [128] fp32
-constexpr uint32_t OFF_ZP = OFF_Z + 512;         // the chunk's K^+ column sums per row quarter, [4][128]
-constexpr uint32_t OFF_DX = OFF_ZP + 4 * 512;    // partial denominators, [2 slots][4 parts][128]
+constexpr uint32_t OFF_Z = 5 * BUF;              // z of the tokens before the chunk, [2 slots][128] fp32
+constexpr uint32_t OFF_ZC = OFF_Z + 1024;        // the chunk's column sums of K^+, [128] fp32
+constexpr uint32_t OFF_DX = OFF_ZC + 512;        // partial denominators, [2 slots][4 parts][128]
 constexpr uint32_t OFF_BAR = OFF_DX + 2 * 4 * 512;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
-// carried S; D then num; P (fp32); the masked P as bf16 (the A operand of P V)
-constexpr uint32_t COL_S = 0, COL_ND = 128, COL_P = 256, COL_PB = 384;
+// carried S; num; C then P (fp32); the masked P as bf16 (the A operand of P V); the mask M as
+// bf16 (the A operand of C)
+constexpr uint32_t COL_S = 0, COL_ND = 128, COL_P = 256, COL_PB = 384, COL_M = 448;
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/false);
 constexpr uint32_t IDESC_QS = idesc_bf16_f32(128, 128, /*a_mn=*/false, /*b_mn=*/true);
 constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, 128, /*a_mn=*/true, /*b_mn=*/true);
@@ -59,12 +65,13 @@ struct Bars {
   uint64_t full_qk;   // Q and K of the chunk landed
   uint64_t full_v;    // V landed
   uint64_t full_g;    // G landed
-  uint64_t relu;      // math: Q^+ and K^+ written in place (4 warps)
-  uint64_t zsync1;    // math: every row's K^+ written (4 warps), before the column reads
-  uint64_t zsync;     // math: z published and K^+ columns read (4 warps)
-  uint64_t dready;    // MMA: D = Q^+ K^+^T done (and its operand reads)
-  uint64_t rot;       // math: phi(Q), phi(K) written in place (4 warps)
-  uint64_t pready;    // MMA: num (inter), P and the S update done
+  uint64_t relu;      // math: K^+ written in place (and, before the first chunk, M into TMEM)
+  uint64_t qready;    // math: phi(Q) written in place
+  uint64_t zready;    // math: z before chunk i published in slot i mod 2 (phase i; 16 warps)
+  uint64_t dready;    // MMA: C = M K^+ done (and its operand reads)
+  uint64_t rot;       // math: phi(K) written in place, C read
+  uint64_t pdone;     // MMA: P done (num = phi(Q) S_prev too)
+  uint64_t pready;    // MMA: the S update done too (the last reader of Q and K)
   uint64_t pw;        // math: masked P written to TMEM as bf16 (4 warps)
   uint64_t numready;  // MMA: num += P V done
   uint64_t out;       // math: O staged over G, S image rewritten (8 warps)
@@ -107,8 +114,9 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     mbar_init(&bars->full_v, 1);
     mbar_init(&bars->full_g, 1);
     mbar_init(&bars->relu, MATH_WARPS);
-    mbar_init(&bars->zsync1, MATH_WARPS);
-    mbar_init(&bars->zsync, MATH_WARPS);
+    mbar_init(&bars->qready, MATH_WARPS);
+    mbar_init(&bars->zready, MATH_WARPS);
+    mbar_init(&bars->pdone, 1);
     mbar_init(&bars->dready, 1);
     mbar_init(&bars->rot, MATH_WARPS);
     mbar_init(&bars->pready, 1);
@@ -166,15 +174,15 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         prev_unit = ti.unit;
         const bool has_next = g + 1 < g1;
         const TileInfo tn = has_next ? tile_info(p, g + 1) : ti;
-        // D = Q^+ K^+^T
+        // C = M K^+ (into the P columns)
         if (!mbar_wait(&bars->relu, ph, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + COL_ND, desc_k(sbase + OFF_Q, kk), desc_k(sbase + OFF_K, kk), IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(tmem + COL_P, tmem + COL_M + 8u * kk, desc_mn(sbase + OFF_K, kk), IDESC_QS, kk > 0 ? 1u : 0u);
         mma_commit(&bars->dready);
-        // num = phi(Q) S_prev;  P = phi(Q) phi(K)^T;  S += phi(K)^T V
-        if (!mbar_wait(&bars->rot, ph, abort_flag)) break;
+        // num = phi(Q) S_prev
+        if (!mbar_wait(&bars->qready, ph, abort_flag)) break;
         tc_fence_after();
         if (!zero_start) {
 #pragma unroll
@@ -182,9 +190,13 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             mma_bf16(tmem + COL_ND, desc_k(sbase + OFF_Q, kk), desc_mn(sbase + OFF_S, kk), IDESC_QS,
                      kk > 0 ? 1u : 0u);
         }
+        // P = phi(Q) phi(K)^T over C (read by then);  S += phi(K)^T V
+        if (!mbar_wait(&bars->rot, ph, abort_flag)) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + COL_P, desc_k(sbase + OFF_Q, kk), desc_k(sbase + OFF_K, kk), IDESC_QK, kk > 0 ? 1u : 0u);
+        mma_commit(&bars->pdone);
         if (!mbar_wait(&bars->full_v, ph, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
@@ -242,16 +254,26 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   } else {
     // ------------------------------------------------------------ rows (warps 0-15)
     const int quarter = warp & 3, part = warp >> 2;
-    const int row = quarter * 32 + lane;  // token row of the chunk = TMEM lane; also channel k for z and S
+    const int row = quarter * 32 + lane;  // token row of the chunk = TMEM lane
     const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t cpart = 32u * static_cast<uint32_t>(part);  // this warp's channels (and P columns)
     const uint32_t t_s = tmem + COL_S + lane_bits + cpart, t_nd = tmem + COL_ND + lane_bits + cpart;
     const uint32_t t_p = tmem + COL_P + lane_bits + cpart, t_pb = tmem + COL_PB + lane_bits + cpart / 2;
-    float* zp = reinterpret_cast<float*>(smem + OFF_ZP);
+    float* zc = reinterpret_cast<float*>(smem + OFF_ZC);
     float* dx = reinterpret_cast<float*>(smem + OFF_DX);
     uint64_t* denx = &bars->denx[quarter];
-    float zk = 0.f;  // (part 0) z of channel `row` over the tokens before the chunk
-    pdl_wait();      // the start states and the cos/sin tables come from the kernels before
+    // The mask M: row `row`, this quarter's columns m = cpart .. cpart + 31 as bf16 pairs.
+    {
+      uint32_t mk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int m0 = static_cast<int>(cpart) + 2 * e;
+        mk[e] = (m0 <= row ? 0x3F80u : 0u) | (m0 + 1 <= row ? 0x3F800000u : 0u);
+      }
+      tmem_st_x16(tmem + COL_M + lane_bits + cpart / 2, mk);
+      tmem_st_wait();
+    }
+    pdl_wait();  // the start states and the cos/sin tables come from the kernels before
     if (g0 < g1 && has_start) {
       // Carried state at the segment start: this quarter of fp32 row `row` of S into TMEM, its
       // bf16 image, and z.
@@ -270,107 +292,53 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                           pack_bf16(__uint_as_float(r[8 * e + 6]), __uint_as_float(r[8 * e + 7]))));
       tmem_st_wait();
       fence_proxy_async_smem();
-      if (part == 0) zk = src[D * D + row];
     }
-    int64_t prev_unit = -1;
+    // z before the first chunk (slot 0, phase 0 of zready).
+    if (part == 0) zs[row] = (g0 < g1 && has_start) ? start[c * (D * D + D) + D * D + row] : 0.f;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->zready);
     for (int64_t g = g0; g < g1; ++g) {
       const int64_t i = g - g0;
       const uint32_t ph = static_cast<uint32_t>(i & 1);
       const TileInfo ti = tile_info(p, g);
-      if (ti.unit != prev_unit && !(g == g0 && has_start)) zk = 0.f;  // a head starting in this CTA
-      prev_unit = ti.unit;
+      // Does the next chunk start a head (then its z starts from zero)?
+      const bool next_new = g + 1 < g1 && unit_of_tile(p, g + 1) != ti.unit;
       if (!warp_wait(&bars->full_qk, ph, abort_flag)) break;
-      // ReLU of this quarter of the Q and K rows in place; q^+ kept in registers.
-      uint32_t qa[16];
+      // ReLU of this quarter of the Q and K rows; K^+ back in place, both kept in registers.
+      uint32_t qa[16], ka[16];
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
-        const int ck = 4 * part + c4;
-        const uint32_t aq = row_chunk(sbase + OFF_Q, row, ck);
-        const uint4 rq = lds128(aq);
+        const uint4 rq = lds128(row_chunk(sbase + OFF_Q, row, 4 * part + c4));
         qa[4 * c4] = relu_bf16x2(rq.x);
         qa[4 * c4 + 1] = relu_bf16x2(rq.y);
         qa[4 * c4 + 2] = relu_bf16x2(rq.z);
         qa[4 * c4 + 3] = relu_bf16x2(rq.w);
-        sts128(aq, make_uint4(qa[4 * c4], qa[4 * c4 + 1], qa[4 * c4 + 2], qa[4 * c4 + 3]));
-        const uint32_t ak = row_chunk(sbase + OFF_K, row, ck);
+        const uint32_t ak = row_chunk(sbase + OFF_K, row, 4 * part + c4);
         const uint4 rk = lds128(ak);
-        sts128(ak, make_uint4(relu_bf16x2(rk.x), relu_bf16x2(rk.y), relu_bf16x2(rk.z), relu_bf16x2(rk.w)));
+        ka[4 * c4] = relu_bf16x2(rk.x);
+        ka[4 * c4 + 1] = relu_bf16x2(rk.y);
+        ka[4 * c4 + 2] = relu_bf16x2(rk.z);
+        ka[4 * c4 + 3] = relu_bf16x2(rk.w);
+        sts128(ak, make_uint4(ka[4 * c4], ka[4 * c4 + 1], ka[4 * c4 + 2], ka[4 * c4 + 3]));
       }
       fence_proxy_async_smem();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bars->relu);
-        mbar_arrive(&bars->zsync1);
-      }
-      // z before the chunk, published for every row's denominator (part 0); then this chunk's K^+
-      // column `row` over the rows of this quarter, once every row is ReLU'd.
-      if (part == 0) zs[row] = zk;
-      if (!warp_wait(&bars->zsync1, ph, abort_flag)) break;
-      {
-        const int kc = row;  // channel
-        const uint32_t kbase = sbase + OFF_K + static_cast<uint32_t>(kc >> 6) * HALF;
-        const uint32_t cchunk = static_cast<uint32_t>((kc & 63) >> 3), cbyte = static_cast<uint32_t>(kc & 7) * 2u;
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int mm = 0; mm < 32; ++mm) {
-          const int m = 32 * part + mm;
-          uint16_t hv;
-          asm volatile("ld.shared.u16 %0, [%1];"
-                       : "=h"(hv)
-                       : "r"(kbase + static_cast<uint32_t>(m) * 128u + ((cchunk ^ static_cast<uint32_t>(m & 7)) << 4) +
-                             cbyte));
-          s4[mm & 3] += __uint_as_float(static_cast<uint32_t>(hv) << 16);
-        }
-        zp[part * 128 + row] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->zsync);
-      if (!warp_wait(&bars->zsync, ph, abort_flag)) break;
-      if (part == 0) zk += ((zp[row] + zp[128 + row]) + (zp[256 + row] + zp[384 + row]));
-      // This quarter's share of the denominator: q^+ . z_prev over its channels plus the masked
-      // row sum of D over its columns; the four quarters of the row add theirs.
-      float dpart = 0.f;
-#pragma unroll
-      for (int k4 = 0; k4 < 8; ++k4) {
-        const float4 z4 = *reinterpret_cast<const float4*>(zs + cpart + 4 * k4);
-        dpart = fmaf(bf16lo(qa[2 * k4]), z4.x, dpart);
-        dpart = fmaf(bf16hi(qa[2 * k4]), z4.y, dpart);
-        dpart = fmaf(bf16lo(qa[2 * k4 + 1]), z4.z, dpart);
-        dpart = fmaf(bf16hi(qa[2 * k4 + 1]), z4.w, dpart);
-      }
-      if (!warp_wait(&bars->dready, ph, abort_flag)) break;
-      tc_fence_after();
-      {
-        uint32_t r[32];
-        tmem_ld_x32(t_nd, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) dpart += (static_cast<int>(cpart) + e <= row) ? __uint_as_float(r[e]) : 0.f;
-      }
-      float den;
-      {
-        float* slot = dx + static_cast<int>(i & 1) * (PARTS * 128);
-        slot[part * 128 + row] = dpart;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(denx);
-        if (!warp_wait(denx, ph, abort_flag)) break;
-        den = (slot[row] + slot[128 + row]) + (slot[256 + row] + slot[384 + row]);
-      }
-      const float hinv = 1.0f / (den + p.eps);
-      // RoPE of this quarter of Q^+ and K^+ in place.
+      if (lane == 0) mbar_arrive(&bars->relu);
+      // RoPE of this quarter of Q^+ over Q (no product reads Q before phi(Q)), while C runs.
       const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
       uint32_t pt = 0, ph_ = 0, pw = 0;
       if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph_, pw);
+      auto rot = [&](uint32_t (&a)[16]) {
+        const int ipt = static_cast<int>(pt), iph = static_cast<int>(ph_), ipw = static_cast<int>(pw);
+        switch (part) {
+          case 0: rotate_span<DT, DH, 0, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 1: rotate_span<DT, DH, 16, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 2: rotate_span<DT, DH, 32, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+          default: rotate_span<DT, DH, 48, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
+        }
+      };
       {
-        auto rot = [&](uint32_t (&a)[16]) {
-          const int ipt = static_cast<int>(pt), iph = static_cast<int>(ph_), ipw = static_cast<int>(pw);
-          switch (part) {
-            case 0: rotate_span<DT, DH, 0, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
-            case 1: rotate_span<DT, DH, 16, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
-            case 2: rotate_span<DT, DH, 32, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
-            default: rotate_span<DT, DH, 48, 16>(a, tab, tab2, rope, p, ipt, iph, ipw); break;
-          }
-        };
         uint32_t a[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) a[e] = qa[e];
@@ -378,26 +346,68 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4)
           sts128(row_chunk(sbase + OFF_Q, row, 4 * part + c4), make_uint4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const uint4 rk = lds128(row_chunk(sbase + OFF_K, row, 4 * part + c4));
-          a[4 * c4] = rk.x;
-          a[4 * c4 + 1] = rk.y;
-          a[4 * c4 + 2] = rk.z;
-          a[4 * c4 + 3] = rk.w;
-        }
-        rot(a);
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-          sts128(row_chunk(sbase + OFF_K, row, 4 * part + c4), make_uint4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->qready);
+      // This quarter's share of the denominator, q^+ . (z_prev + C_n) over its channels; the
+      // last row's C is the chunk's column sums, which advance z for the next chunk.
+      float dpart;
+      if (!warp_wait(&bars->zready, ph, abort_flag)) break;
+      {
+        const float* zcur = zs + (i & 1) * 128;
+        if (!warp_wait(&bars->dready, ph, abort_flag)) break;
+        tc_fence_after();
+        uint32_t r[32];
+        tmem_ld_x32(t_p, r);
+        tmem_ld_wait();
+        float d4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 z4 = *reinterpret_cast<const float4*>(zcur + cpart + 4 * k4);
+          d4[0] = fmaf(bf16lo(qa[2 * k4]), z4.x + __uint_as_float(r[4 * k4]), d4[0]);
+          d4[1] = fmaf(bf16hi(qa[2 * k4]), z4.y + __uint_as_float(r[4 * k4 + 1]), d4[1]);
+          d4[2] = fmaf(bf16lo(qa[2 * k4 + 1]), z4.z + __uint_as_float(r[4 * k4 + 2]), d4[2]);
+          d4[3] = fmaf(bf16hi(qa[2 * k4 + 1]), z4.w + __uint_as_float(r[4 * k4 + 3]), d4[3]);
+        }
+        dpart = (d4[0] + d4[1]) + (d4[2] + d4[3]);
+        if (quarter == 3) {
+          if (lane == 31) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              *reinterpret_cast<float4*>(zc + cpart + 4 * e) =
+                  make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
+                              __uint_as_float(r[4 * e + 3]));
+          }
+          __syncwarp();
+          const int k = static_cast<int>(cpart) + lane;
+          zs[((i + 1) & 1) * 128 + k] = next_new ? 0.f : zcur[k] + zc[k];
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->zready);
+      // RoPE of this quarter of K^+ over K^+ (C, its last reader, is done).
+      rot(ka);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4)
+        sts128(row_chunk(sbase + OFF_K, row, 4 * part + c4), make_uint4(ka[4 * c4], ka[4 * c4 + 1], ka[4 * c4 + 2], ka[4 * c4 + 3]));
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->rot);
+      float hinv;
+      {
+        float* slot = dx + static_cast<int>(i & 1) * (PARTS * 128);
+        slot[part * 128 + row] = dpart;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(denx);
+        if (!warp_wait(denx, ph, abort_flag)) break;
+        const float den = (slot[row] + slot[128 + row]) + (slot[256 + row] + slot[384 + row]);
+        hinv = 1.0f / (den + p.eps);
+      }
       // Causal mask on this quarter of P (columns m in [32 part, 32 part + 32), kept where m <= n),
       // written as bf16 to the A operand of P V (columns 16 part .. 16 part + 15 of that region).
-      if (!warp_wait(&bars->pready, ph, abort_flag)) break;
+      if (!warp_wait(&bars->pdone, ph, abort_flag)) break;
       tc_fence_after();
       {
         uint32_t pb[16];
