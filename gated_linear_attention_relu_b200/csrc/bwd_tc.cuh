@@ -57,7 +57,10 @@ static_assert(SMEM_Q <= 232448 && SMEM_K <= 232448, "shared memory budget");
 struct BarsQ {
   uint64_t full;    // Q, dO (and the state image at a unit's first tile) landed
   uint64_t full_g;  // G landed
-  uint64_t rot, numready, dn, dpqready, out, final_;
+  uint64_t rot, numready, dn;
+  uint64_t dpqready;  // MMA: dphi(q) = dnum S^T done
+  uint64_t dsdone;    // MMA: dS += phi(Q)^T dnum done too (the last reader of Q, dO, the state image)
+  uint64_t out, final_;
   uint64_t pair[4];  // the four warps of rows 32q .. 32q+31: two meetings per tile (den, then dy.y)
   uint32_t tmem_base;
   int abort_flag;
@@ -65,7 +68,10 @@ struct BarsQ {
 struct BarsK {
   uint64_t full;    // K (and the dS image at a unit's first tile) landed
   uint64_t full_v;  // V landed
-  uint64_t rot, ready, out, final_;
+  uint64_t rot;
+  uint64_t dvready;  // MMA: dV = phi(K) dS done
+  uint64_t ready;    // MMA: dphi(k) = V dS^T done too (the last reader of K, V, the dS image)
+  uint64_t out, final_;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -109,6 +115,7 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     mbar_init(&bars->numready, 1);
     mbar_init(&bars->dn, MATH_WARPS);
     mbar_init(&bars->dpqready, 1);
+    mbar_init(&bars->dsdone, 1);
     mbar_init(&bars->out, MATH_WARPS);
     mbar_init(&bars->final_, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], PARTS);
@@ -169,15 +176,16 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + QCOL_DPQ, desc_k(sbase + QO_DO, kk), desc_k(sbase + QO_S, kk), IDESC_QST, kk > 0 ? 1u : 0u);
+        mma_commit(&bars->dpqready);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + QCOL_DS, desc_mn(sbase + QO_Q, kk), desc_mn(sbase + QO_DO, kk), IDESC_TD,
                    (kk > 0 || !first) ? 1u : 0u);
-        mma_commit(&bars->dpqready);
+        mma_commit(&bars->dsdone);
         // Q, dO and the state image were last read by the products just done: the next tile's
         // land while this tile's dq epilogue runs.  (G holds this tile's dG until it is stored.)
         if (has_next) {
-          if (!mbar_wait(&bars->dpqready, ph, abort_flag)) break;
+          if (!mbar_wait(&bars->dsdone, ph, abort_flag)) break;
           mbar_arrive_expect_tx(&bars->full, 2 * BUF + (next_new_unit ? BUF : 0u));
           if (next_new_unit) bulk_load(smem + QO_S, simg + tn.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
           load2(QO_Q, &tmQ, tn, &bars->full);
@@ -274,41 +282,45 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!warp_wait(&bars->numready, ph, abort_flag)) break;
       if (!warp_wait(&bars->full_g, ph, abort_flag)) break;
       tc_fence_after();
-      float x[32];
-      {
-        uint32_t r[32];
-        tmem_ld_x32(tmem + QCOL_NUM + lane_bits + static_cast<uint32_t>(cpart), r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
-      }
       float dyy = 0.f;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        const int ck = 4 * part + c4;
-        const uint32_t ag = row_chunk(sbase + QO_G, row, ck);
-        const uint4 gr = lds128(ag);
-        const uint32_t ad = row_chunk(sbase + QO_DO, row, ck);
-        const uint4 dr = lds128(ad);
-        const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w}, dw[4] = {dr.x, dr.y, dr.z, dr.w};
-        float dg8[8], dy8[8];
+      for (int hh = 0; hh < 2; ++hh) {
+        // num of 16 channels at a time (fewer live registers)
+        float x[16];
+        {
+          uint32_t r[16];
+          tmem_ld_x16(tmem + QCOL_NUM + lane_bits + static_cast<uint32_t>(cpart) + 16u * static_cast<uint32_t>(hh), r);
+          tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int e = 8 * c4 + 2 * q + h;
-            const float gv = h ? bf16hi(gw[q]) : bf16lo(gw[q]);
-            const float dov = h ? bf16hi(dw[q]) : bf16lo(dw[q]);
-            const float y = x[e] * rden;
-            const float sg = sigmoid_f(gv);
-            dg8[2 * q + h] = dov * y * sg * (1.f - sg);
-            const float dy = dov * sg;
-            dy8[2 * q + h] = dy * rden;  // dnum
-            dyy = fmaf(dy, y, dyy);
-          }
+          for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(r[e]);
         }
-        sts128(ag, pack8(dg8));
-        sts128(ad, pack8(dy8));
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int ck = 4 * part + 2 * hh + cc;
+          const uint32_t ag = row_chunk(sbase + QO_G, row, ck);
+          const uint4 gr = lds128(ag);
+          const uint32_t ad = row_chunk(sbase + QO_DO, row, ck);
+          const uint4 dr = lds128(ad);
+          const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w}, dw[4] = {dr.x, dr.y, dr.z, dr.w};
+          float dg8[8], dy8[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int e = 8 * cc + 2 * q + h;
+              const float gv = h ? bf16hi(gw[q]) : bf16lo(gw[q]);
+              const float dov = h ? bf16hi(dw[q]) : bf16lo(dw[q]);
+              const float y = x[e] * rden;
+              const float sg = sigmoid_f(gv);
+              dg8[2 * q + h] = dov * y * sg * (1.f - sg);
+              const float dy = dov * sg;
+              dy8[2 * q + h] = dy * rden;  // dnum
+              dyy = fmaf(dy, y, dyy);
+            }
+          }
+          sts128(ag, pack8(dg8));
+          sts128(ad, pack8(dy8));
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -346,36 +358,48 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // dq = [q > 0] (RoPE^T(dnum S^T) + dden z) for this quarter, into the dQ staging buffer.
       if (!warp_wait(&bars->dpqready, ph, abort_flag)) break;
       tc_fence_after();
-      {
-        uint32_t r[32];
-        tmem_ld_x32(tmem + QCOL_DPQ + lane_bits + static_cast<uint32_t>(cpart), r);
-        tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
-      }
-      switch (part) {
-        case 0: rotate_span_t<DT, DH, 0, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
-        case 1: rotate_span_t<DT, DH, 16, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
-        case 2: rotate_span_t<DT, DH, 32, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
-        default: rotate_span_t<DT, DH, 48, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
-      }
+      for (int hh = 0; hh < 2; ++hh) {
+        // 16 channels at a time (fewer live registers)
+        float x[16];
+        {
+          uint32_t r[16];
+          tmem_ld_x16(tmem + QCOL_DPQ + lane_bits + static_cast<uint32_t>(cpart) + 16u * static_cast<uint32_t>(hh), r);
+          tmem_ld_wait();
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4));
-        const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4 + 4));
-        const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-        float o8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint32_t w = qa[4 * c4 + e / 2];
-          const float qv = (e & 1) ? bf16hi(w) : bf16lo(w);
-          o8[e] = qv > 0.f ? x[8 * c4 + e] + dden * zz[e] : 0.f;
+          for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(r[e]);
         }
-        sts128(row_chunk(sbase + QO_DQ, row, 4 * part + c4), pack8(o8));
+        switch (2 * part + hh) {
+          case 0: rotate_span_t<DT, DH, 0, 8>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 1: rotate_span_t<DT, DH, 8, 8>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 2: rotate_span_t<DT, DH, 16, 8>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 3: rotate_span_t<DT, DH, 24, 8>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 4: rotate_span_t<DT, DH, 32, 8>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 5: rotate_span_t<DT, DH, 40, 8>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 6: rotate_span_t<DT, DH, 48, 8>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+          default: rotate_span_t<DT, DH, 56, 8>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
+        }
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c4 = 2 * hh + cc;
+          const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4));
+          const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4 + 4));
+          const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+          float o8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t w = qa[4 * c4 + e / 2];
+            const float qv = (e & 1) ? bf16hi(w) : bf16lo(w);
+            o8[e] = qv > 0.f ? x[8 * cc + e] + dden * zz[e] : 0.f;
+          }
+          sts128(row_chunk(sbase + QO_DQ, row, 4 * part + c4), pack8(o8));
+        }
       }
       if (last) {
         // dS of this unit (TMEM lane = channel k of phi(Q); this quarter's 32 columns) and dz ->
         // the CTA's partial slot.
+        if (!warp_wait(&bars->dsdone, ph, abort_flag)) break;
+        tc_fence_after();
         float* dst = partial + (c * p.maxseg + (ti.unit - u_first)) * slot_floats;
         uint32_t r[32];
         tmem_ld_x32(tmem + QCOL_DS + lane_bits + static_cast<uint32_t>(cpart), r);
@@ -422,6 +446,7 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     mbar_init(&bars->full, 1);
     mbar_init(&bars->full_v, 1);
     mbar_init(&bars->rot, MATH_WARPS);
+    mbar_init(&bars->dvready, 1);
     mbar_init(&bars->ready, 1);
     mbar_init(&bars->out, MATH_WARPS);
     mbar_init(&bars->final_, 1);
@@ -469,6 +494,7 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + KCOL_DV, desc_k(sbase + KO_K, kk), desc_mn(sbase + KO_S, kk), IDESC_QS, kk > 0 ? 1u : 0u);
+        mma_commit(&bars->dvready);
         if (!mbar_wait(&bars->full_v, ph, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
@@ -545,7 +571,7 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->rot);
-      if (!warp_wait(&bars->ready, ph, abort_flag)) break;
+      if (!warp_wait(&bars->dvready, ph, abort_flag)) break;
       tc_fence_after();
       float x[32];
       {
@@ -557,33 +583,45 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       }
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) sts128(row_chunk(sbase + KO_DV, row, 4 * part + c4), pack8(&x[8 * c4]));
-      {
-        uint32_t r[32];
-        tmem_ld_x32(tmem + KCOL_DPK + lane_bits + static_cast<uint32_t>(cpart), r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
-      }
-      switch (part) {
-        case 0: rotate_span_t<DT, DH, 0, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
-        case 1: rotate_span_t<DT, DH, 16, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
-        case 2: rotate_span_t<DT, DH, 32, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
-        default: rotate_span_t<DT, DH, 48, 16>(x, tab, tab2, rope, p, ipt, iph, ipw); break;
-      }
+      if (!warp_wait(&bars->ready, ph, abort_flag)) break;
+      tc_fence_after();
       const float* zg = dzimg + ti.unit * D + cpart;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4));
-        const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4 + 4));
-        const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-        float o8[8];
+      for (int hh = 0; hh < 2; ++hh) {
+        // 16 channels at a time (fewer live registers)
+        float y[16];
+        {
+          uint32_t r[16];
+          tmem_ld_x16(tmem + KCOL_DPK + lane_bits + static_cast<uint32_t>(cpart) + 16u * static_cast<uint32_t>(hh), r);
+          tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint32_t w = ka[4 * c4 + e / 2];
-          const float kv = (e & 1) ? bf16hi(w) : bf16lo(w);
-          o8[e] = kv > 0.f ? x[8 * c4 + e] + zz[e] : 0.f;
+          for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(r[e]);
         }
-        sts128(row_chunk(sbase + KO_DK, row, 4 * part + c4), pack8(o8));
+        switch (2 * part + hh) {
+          case 0: rotate_span_t<DT, DH, 0, 8>(y, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 1: rotate_span_t<DT, DH, 8, 8>(y, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 2: rotate_span_t<DT, DH, 16, 8>(y, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 3: rotate_span_t<DT, DH, 24, 8>(y, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 4: rotate_span_t<DT, DH, 32, 8>(y, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 5: rotate_span_t<DT, DH, 40, 8>(y, tab, tab2, rope, p, ipt, iph, ipw); break;
+          case 6: rotate_span_t<DT, DH, 48, 8>(y, tab, tab2, rope, p, ipt, iph, ipw); break;
+          default: rotate_span_t<DT, DH, 56, 8>(y, tab, tab2, rope, p, ipt, iph, ipw); break;
+        }
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c4 = 2 * hh + cc;
+          const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4));
+          const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4 + 4));
+          const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+          float o8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t w = ka[4 * c4 + e / 2];
+            const float kv = (e & 1) ? bf16hi(w) : bf16lo(w);
+            o8[e] = kv > 0.f ? y[8 * cc + e] + zz[e] : 0.f;
+          }
+          sts128(row_chunk(sbase + KO_DK, row, 4 * part + c4), pack8(o8));
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();

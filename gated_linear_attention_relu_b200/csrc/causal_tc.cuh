@@ -427,8 +427,23 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->pw);
-      // O = num / den * sigmoid(g) for this quarter, in place over G; then this quarter of the new
-      // state's bf16 image.
+      // This quarter of the updated state's bf16 image, while P V runs (phi(Q) S_prev, the old
+      // image's reader, finished before P).
+      if (!warp_wait(&bars->pready, ph, abort_flag)) break;
+      tc_fence_after();
+      {
+        uint32_t r[32];
+        tmem_ld_x32(t_s, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          sts128(row_chunk(sbase + OFF_S, row, 4 * part + e),
+                 make_uint4(pack_bf16(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
+                            pack_bf16(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
+                            pack_bf16(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
+                            pack_bf16(__uint_as_float(r[8 * e + 6]), __uint_as_float(r[8 * e + 7]))));
+      }
+      // O = num / den * sigmoid(g) for this quarter, in place over G.
       if (!warp_wait(&bars->numready, ph, abort_flag)) break;
       if (!warp_wait(&bars->full_g, ph, abort_flag)) break;
       tc_fence_after();
@@ -450,18 +465,6 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           }
           sts128(ag, make_uint4(ov[0], ov[1], ov[2], ov[3]));
         }
-      }
-      {
-        uint32_t r[32];
-        tmem_ld_x32(t_s, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          sts128(row_chunk(sbase + OFF_S, row, 4 * part + e),
-                 make_uint4(pack_bf16(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
-                            pack_bf16(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
-                            pack_bf16(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
-                            pack_bf16(__uint_as_float(r[8 * e + 6]), __uint_as_float(r[8 * e + 7]))));
       }
       fence_proxy_async_smem();
       tc_fence_before();
