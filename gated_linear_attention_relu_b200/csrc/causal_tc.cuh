@@ -22,12 +22,12 @@
 // warp w reaching lanes 32 (w mod 4) ..); warp 16 issues the TMA copies and the MMAs.  Only K^+
 // goes back to shared memory before the first product; the rotation of Q runs while C is
 // computed (into the columns P takes later), phi(Q) S_prev starts as soon as phi(Q) is written,
-// K is rotated from registers, and the mask of P starts once P alone is done (the state update
-// runs under it).  The next chunk's tiles are loaded as soon as their
-// buffers are free (Q and K once the products reading them are done, V after P V, G after this
-// chunk's O has been stored), each on its own barrier and waited for only by its first reader
-// (Q and K: the ReLU pass; V: the state update; G: the epilogue), so their latency overlaps the
-// chunk's work.
+// K is rotated from registers, the mask of P starts once P alone is done (the state update runs
+// under it), and the new state image is written while P V runs.  The next chunk's tiles are
+// loaded as soon as their buffers are free (Q and K once the products reading them are done, V
+// after P V, G after this chunk's O has been stored), each on its own barrier and waited for only
+// by its first reader (Q and K: the ReLU pass; V: the state update; G: the epilogue), so their
+// latency overlaps the chunk's work.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
