@@ -45,21 +45,25 @@ constexpr uint32_t IDESC_TD = idesc_bf16_f32(128, 128, /*a_mn=*/true, /*b_mn=*/t
 // ---- bwdq smem: Q (-> phi(Q)), G (-> dG), dO (-> dnum), S image, dQ staging, exchanges
 constexpr uint32_t QO_Q = 0, QO_G = BUF, QO_DO = 2 * BUF, QO_S = 3 * BUF, QO_DQ = 4 * BUF;
 constexpr uint32_t QO_X = 5 * BUF;  // [2 values][4 parts][128] fp32: partial den, partial dy.y
-constexpr uint32_t QO_BAR = QO_X + 2 * PARTS * 512;
+constexpr uint32_t QO_Z = QO_X + 2 * PARTS * 512;  // z of the unit, [2 slots by unit parity][128] fp32
+constexpr uint32_t QO_BAR = QO_Z + 1024;
 constexpr uint32_t SMEM_Q = QO_BAR + 256 + 1024;
 constexpr uint32_t QCOL_NUM = 0, QCOL_DPQ = 128, QCOL_DS = 256;
 // ---- bwdk smem: K (-> phi(K)), V, dS image, dK and dV staging
-constexpr uint32_t KO_K = 0, KO_V = BUF, KO_S = 2 * BUF, KO_DK = 3 * BUF, KO_DV = 4 * BUF, KO_BAR = 5 * BUF;
+constexpr uint32_t KO_K = 0, KO_V = BUF, KO_S = 2 * BUF, KO_DK = 3 * BUF, KO_DV = 4 * BUF;
+constexpr uint32_t KO_Z = 5 * BUF;  // dz of the unit, [2 slots by unit parity][128] fp32
+constexpr uint32_t KO_BAR = KO_Z + 1024;
 constexpr uint32_t SMEM_K = KO_BAR + 256 + 1024;
 constexpr uint32_t KCOL_DV = 0, KCOL_DPK = 128;
 static_assert(SMEM_Q <= 232448 && SMEM_K <= 232448, "shared memory budget");
 
 struct BarsQ {
-  uint64_t full;    // Q, dO (and the state image at a unit's first tile) landed
-  uint64_t full_g;  // G landed
+  uint64_t full;     // Q (and the state image and z at a unit's first tile) landed
+  uint64_t full_do;  // dO landed
+  uint64_t full_g;   // G landed
   uint64_t rot, numready, dn;
-  uint64_t dpqready;  // MMA: dphi(q) = dnum S^T done
-  uint64_t dsdone;    // MMA: dS += phi(Q)^T dnum done too (the last reader of Q, dO, the state image)
+  uint64_t qfree;     // MMA: dS += phi(Q)^T dnum done (the last reader of Q)
+  uint64_t dpqready;  // MMA: dphi(q) = dnum S^T done too (the last reader of dnum, the state image)
   uint64_t out, final_;
   uint64_t pair[4];  // the four warps of rows 32q .. 32q+31: two meetings per tile (den, then dy.y)
   uint32_t tmem_base;
@@ -77,10 +81,10 @@ struct BarsK {
 };
 static_assert(sizeof(BarsQ) <= 256 && sizeof(BarsK) <= 256, "barrier block too large");
 
-__device__ __forceinline__ float sigmoid_f(float g) {
+__device__ __forceinline__ float tanh_f(float x) {
   float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(0.5f * g));
-  return 0.5f + 0.5f * y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ uint4 pack8(const float* x) {
@@ -110,12 +114,13 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->full, 1);
+    mbar_init(&bars->full_do, 1);
     mbar_init(&bars->full_g, 1);
     mbar_init(&bars->rot, MATH_WARPS);
     mbar_init(&bars->numready, 1);
     mbar_init(&bars->dn, MATH_WARPS);
+    mbar_init(&bars->qfree, 1);
     mbar_init(&bars->dpqready, 1);
-    mbar_init(&bars->dsdone, 1);
     mbar_init(&bars->out, MATH_WARPS);
     mbar_init(&bars->final_, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], PARTS);
@@ -142,16 +147,19 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tma_load_3d(smem + off, tm, 0, n0, bh, bar);
         tma_load_3d(smem + off + HALF, tm, 64, n0, bh, bar);
       };
-      int64_t issued = 0, issued_g = 0;
+      int64_t issued = 0, issued_do = 0, issued_g = 0;
+      int64_t zslot = 0;  // z slot of the unit being loaded (unit parity within the CTA)
       if (g0 < g1) {
         const TileInfo t0 = tile_info(p, g0);
-        mbar_arrive_expect_tx(&bars->full, 3 * BUF);
+        mbar_arrive_expect_tx(&bars->full, 2 * BUF + 512);
         bulk_load(smem + QO_S, simg + t0.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
+        bulk_load(smem + QO_Z, zimg + t0.unit * D, 512, &bars->full);
         load2(QO_Q, &tmQ, t0, &bars->full);
-        load2(QO_DO, &tmDO, t0, &bars->full);
+        mbar_arrive_expect_tx(&bars->full_do, BUF);
+        load2(QO_DO, &tmDO, t0, &bars->full_do);
         mbar_arrive_expect_tx(&bars->full_g, BUF);
         load2(QO_G, &tmG, t0, &bars->full_g);
-        issued = issued_g = 1;
+        issued = issued_do = issued_g = 1;
       }
       int64_t prev_unit = -1;
       for (int64_t g = g0; g < g1; ++g) {
@@ -170,38 +178,49 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + QCOL_NUM, desc_k(sbase + QO_Q, kk), desc_mn(sbase + QO_S, kk), IDESC_QS, kk > 0 ? 1u : 0u);
         mma_commit(&bars->numready);
-        // dphi(q) = dnum S^T;  dS += phi(Q)^T dnum
+        // dS += phi(Q)^T dnum (frees Q first);  dphi(q) = dnum S^T
         if (!mbar_wait(&bars->dn, ph, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + QCOL_DPQ, desc_k(sbase + QO_DO, kk), desc_k(sbase + QO_S, kk), IDESC_QST, kk > 0 ? 1u : 0u);
-        mma_commit(&bars->dpqready);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + QCOL_DS, desc_mn(sbase + QO_Q, kk), desc_mn(sbase + QO_DO, kk), IDESC_TD,
                    (kk > 0 || !first) ? 1u : 0u);
-        mma_commit(&bars->dsdone);
-        // Q, dO and the state image were last read by the products just done: the next tile's
-        // land while this tile's dq epilogue runs.  (G holds this tile's dG until it is stored.)
+        mma_commit(&bars->qfree);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + QCOL_DPQ, desc_k(sbase + QO_DO, kk), desc_k(sbase + QO_S, kk), IDESC_QST, kk > 0 ? 1u : 0u);
+        bulk_wait_group_read0();  // the previous tile's dQ has left the staging buffer the epilogue reuses
+        mma_commit(&bars->dpqready);
+        // The next tile's Q once dS has read this one (and, at a new unit, the state image and z
+        // once dphi(q) has read the image); its dO once dphi(q) has read dnum.  (G holds this
+        // tile's dG until it is stored.)
         if (has_next) {
-          if (!mbar_wait(&bars->dsdone, ph, abort_flag)) break;
-          mbar_arrive_expect_tx(&bars->full, 2 * BUF + (next_new_unit ? BUF : 0u));
-          if (next_new_unit) bulk_load(smem + QO_S, simg + tn.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
+          if (!mbar_wait(next_new_unit ? &bars->dpqready : &bars->qfree, ph, abort_flag)) break;
+          mbar_arrive_expect_tx(&bars->full, BUF + (next_new_unit ? BUF + 512u : 0u));
+          if (next_new_unit) {
+            zslot ^= 1;
+            bulk_load(smem + QO_S, simg + tn.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
+            bulk_load(smem + QO_Z + 512u * static_cast<uint32_t>(zslot), zimg + tn.unit * D, 512, &bars->full);
+          }
           load2(QO_Q, &tmQ, tn, &bars->full);
-          load2(QO_DO, &tmDO, tn, &bars->full);
           ++issued;
+          if (!mbar_wait(&bars->dpqready, ph, abort_flag)) break;
+          mbar_arrive_expect_tx(&bars->full_do, BUF);
+          load2(QO_DO, &tmDO, tn, &bars->full_do);
+          ++issued_do;
         }
-        // dQ (staged) and dG (over G) of this tile out; then the next tile's G.
+        // dG (over G) and dQ (staged) of this tile out, as two groups; the next tile's G once dG
+        // has been read out (dQ's read is waited for before the next dq epilogue may start).
         if (!mbar_wait(&bars->out, ph, abort_flag)) break;
         {
           const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
-          tma_store_3d(&tmDQ, smem + QO_DQ, 0, n0, bh);
-          tma_store_3d(&tmDQ, smem + QO_DQ + HALF, 64, n0, bh);
           tma_store_3d(&tmDG, smem + QO_G, 0, n0, bh);
           tma_store_3d(&tmDG, smem + QO_G + HALF, 64, n0, bh);
           bulk_commit_group();
-          bulk_wait_group_read0();
+          tma_store_3d(&tmDQ, smem + QO_DQ, 0, n0, bh);
+          tma_store_3d(&tmDQ, smem + QO_DQ + HALF, 64, n0, bh);
+          bulk_commit_group();
+          bulk_wait_group_read1();
         }
         if (has_next) {
           mbar_arrive_expect_tx(&bars->full_g, BUF);
@@ -212,6 +231,7 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bulk_wait_group0();
       if (*abort_flag) {
         if (issued > 0) mbar_wait_drain(&bars->full, static_cast<uint32_t>((issued - 1) & 1));
+        if (issued_do > 0) mbar_wait_drain(&bars->full_do, static_cast<uint32_t>((issued_do - 1) & 1));
         if (issued_g > 0) mbar_wait_drain(&bars->full_g, static_cast<uint32_t>((issued_g - 1) & 1));
       }
       mma_commit(&bars->final_);
@@ -224,11 +244,15 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int cpart = 32 * part;  // this warp's channels
     uint64_t* pr = &bars->pair[quarter];
     float dzacc = 0.f;  // dz of channel 32 part + lane over this warp's rows
+    int zslot = 0;      // z slot of the current unit
+    int64_t prev_unit = -1;
     for (int64_t g = g0; g < g1; ++g) {
       const int64_t i = g - g0;
       const uint32_t ph = static_cast<uint32_t>(i & 1);
       const TileInfo ti = tile_info(p, g);
       const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != ti.unit);
+      if (prev_unit >= 0 && ti.unit != prev_unit) zslot ^= 1;
+      prev_unit = ti.unit;
       if (!warp_wait(&bars->full, ph, abort_flag)) break;
       // q^+ of this quarter kept packed; phi(q) written in place.
       uint32_t qa[16];
@@ -262,11 +286,11 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->rot);
       // den = q^+ . z + eps: each quarter's share, then the four add them in a fixed order.
-      const float* zg = zimg + ti.unit * D + cpart;
+      const float* zg = reinterpret_cast<const float*>(smem + QO_Z) + zslot * D + cpart;
       float dpart = 0.f;
 #pragma unroll
       for (int k4 = 0; k4 < 8; ++k4) {
-        const float4 z4 = __ldg(reinterpret_cast<const float4*>(zg + 4 * k4));
+        const float4 z4 = *reinterpret_cast<const float4*>(zg + 4 * k4);
         dpart = fmaf(bf16lo(qa[2 * k4]), z4.x, dpart);
         dpart = fmaf(bf16hi(qa[2 * k4]), z4.y, dpart);
         dpart = fmaf(bf16lo(qa[2 * k4 + 1]), z4.z, dpart);
@@ -281,19 +305,18 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // num -> y; with G and dO: dG (over G), dnum (over dO), this quarter's dy . y.
       if (!warp_wait(&bars->numready, ph, abort_flag)) break;
       if (!warp_wait(&bars->full_g, ph, abort_flag)) break;
+      if (!warp_wait(&bars->full_do, ph, abort_flag)) break;
       tc_fence_after();
-      float dyy = 0.f;
+      // Channel pairs in packed fp32 (sigmoid(g) = 1/2 + tanh(g/2)/2, with g/2 exact in bf16):
+      //   y = num / den, dy = dO s, dG = dy y (1 - s), dnum = dy / den, dy . y accumulated.
+      const uint64_t rden2 = pk(rden, rden), half2 = pk(0.5f, 0.5f), mhalf2 = pk(-0.5f, -0.5f);
+      uint64_t dyy2 = 0;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         // num of 16 channels at a time (fewer live registers)
-        float x[16];
-        {
-          uint32_t r[16];
-          tmem_ld_x16(tmem + QCOL_NUM + lane_bits + static_cast<uint32_t>(cpart) + 16u * static_cast<uint32_t>(hh), r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(r[e]);
-        }
+        uint32_t r[16];
+        tmem_ld_x16(tmem + QCOL_NUM + lane_bits + static_cast<uint32_t>(cpart) + 16u * static_cast<uint32_t>(hh), r);
+        tmem_ld_wait();
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int ck = 4 * part + 2 * hh + cc;
@@ -302,25 +325,29 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const uint32_t ad = row_chunk(sbase + QO_DO, row, ck);
           const uint4 dr = lds128(ad);
           const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w}, dw[4] = {dr.x, dr.y, dr.z, dr.w};
-          float dg8[8], dy8[8];
+          uint32_t dgw[4], dnw[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int e = 8 * cc + 2 * q + h;
-              const float gv = h ? bf16hi(gw[q]) : bf16lo(gw[q]);
-              const float dov = h ? bf16hi(dw[q]) : bf16lo(dw[q]);
-              const float y = x[e] * rden;
-              const float sg = sigmoid_f(gv);
-              dg8[2 * q + h] = dov * y * sg * (1.f - sg);
-              const float dy = dov * sg;
-              dy8[2 * q + h] = dy * rden;  // dnum
-              dyy = fmaf(dy, y, dyy);
-            }
+            const int e = 8 * cc + 2 * q;
+            const uint32_t gh = half_bf16x2(gw[q]);
+            const uint64_t t2 = pk(tanh_f(bf16lo(gh)), tanh_f(bf16hi(gh)));
+            const uint64_t sg2 = fma2(t2, half2, half2), om2 = fma2(t2, mhalf2, half2);
+            const uint64_t y2 = mul2(pk(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), rden2);
+            const uint64_t dy2 = mul2(pk(bf16lo(dw[q]), bf16hi(dw[q])), sg2);
+            const float2 dg = upk(mul2(mul2(dy2, y2), om2));
+            const float2 dn = upk(mul2(dy2, rden2));
+            dyy2 = fma2(dy2, y2, dyy2);
+            dgw[q] = pack_bf16(dg.x, dg.y);
+            dnw[q] = pack_bf16(dn.x, dn.y);
           }
-          sts128(ag, pack8(dg8));
-          sts128(ad, pack8(dy8));
+          sts128(ag, make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]));
+          sts128(ad, make_uint4(dnw[0], dnw[1], dnw[2], dnw[3]));
         }
+      }
+      float dyy;
+      {
+        const float2 d = upk(dyy2);
+        dyy = d.x + d.y;
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -382,8 +409,8 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c4 = 2 * hh + cc;
-          const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4));
-          const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4 + 4));
+          const float4 za = *reinterpret_cast<const float4*>(zg + 8 * c4);
+          const float4 zb = *reinterpret_cast<const float4*>(zg + 8 * c4 + 4);
           const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
           float o8[8];
 #pragma unroll
@@ -398,7 +425,7 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (last) {
         // dS of this unit (TMEM lane = channel k of phi(Q); this quarter's 32 columns) and dz ->
         // the CTA's partial slot.
-        if (!warp_wait(&bars->dsdone, ph, abort_flag)) break;
+        if (!warp_wait(&bars->qfree, ph, abort_flag)) break;
         tc_fence_after();
         float* dst = partial + (c * p.maxseg + (ti.unit - u_first)) * slot_floats;
         uint32_t r[32];
@@ -472,10 +499,12 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         tma_load_3d(smem + off + HALF, tm, 64, n0, bh, bar);
       };
       int64_t issued = 0, issued_v = 0;
+      int64_t zslot = 0;  // dz slot of the unit being loaded (unit parity within the CTA)
       if (g0 < g1) {
         const TileInfo t0 = tile_info(p, g0);
-        mbar_arrive_expect_tx(&bars->full, 2 * BUF);
+        mbar_arrive_expect_tx(&bars->full, 2 * BUF + 512);
         bulk_load(smem + KO_S, dsimg + t0.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
+        bulk_load(smem + KO_Z, dzimg + t0.unit * D, 512, &bars->full);
         load2(KO_K, &tmK, t0, &bars->full);
         mbar_arrive_expect_tx(&bars->full_v, BUF);
         load2(KO_V, &tmV, t0, &bars->full_v);
@@ -494,33 +523,41 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + KCOL_DV, desc_k(sbase + KO_K, kk), desc_mn(sbase + KO_S, kk), IDESC_QS, kk > 0 ? 1u : 0u);
+        bulk_wait_group_read1();  // the previous tile's dV has left its staging buffer
         mma_commit(&bars->dvready);
         if (!mbar_wait(&bars->full_v, ph, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + KCOL_DPK, desc_k(sbase + KO_V, kk), desc_k(sbase + KO_S, kk), IDESC_QST, kk > 0 ? 1u : 0u);
+        bulk_wait_group_read0();  // and its dK
         mma_commit(&bars->ready);
         // The products were the last readers of K, V and the dS image: the next tile's land now.
         if (has_next) {
           if (!mbar_wait(&bars->ready, ph, abort_flag)) break;
-          mbar_arrive_expect_tx(&bars->full, BUF + (next_new_unit ? BUF : 0u));
-          if (next_new_unit) bulk_load(smem + KO_S, dsimg + tn.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
+          mbar_arrive_expect_tx(&bars->full, BUF + (next_new_unit ? BUF + 512u : 0u));
+          if (next_new_unit) {
+            zslot ^= 1;
+            bulk_load(smem + KO_S, dsimg + tn.unit * static_cast<int64_t>(BUF), BUF, &bars->full);
+            bulk_load(smem + KO_Z + 512u * static_cast<uint32_t>(zslot), dzimg + tn.unit * D, 512, &bars->full);
+          }
           load2(KO_K, &tmK, tn, &bars->full);
           mbar_arrive_expect_tx(&bars->full_v, BUF);
           load2(KO_V, &tmV, tn, &bars->full_v);
           ++issued;
           ++issued_v;
         }
+        // dV and dK of this tile out, as two groups; their reads are waited for before the next
+        // tile's products are committed to the epilogues that rewrite the staging buffers.
         if (!mbar_wait(&bars->out, ph, abort_flag)) break;
         {
           const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
-          tma_store_3d(&tmDK, smem + KO_DK, 0, n0, bh);
-          tma_store_3d(&tmDK, smem + KO_DK + HALF, 64, n0, bh);
           tma_store_3d(&tmDV, smem + KO_DV, 0, n0, bh);
           tma_store_3d(&tmDV, smem + KO_DV + HALF, 64, n0, bh);
           bulk_commit_group();
-          bulk_wait_group_read0();
+          tma_store_3d(&tmDK, smem + KO_DK, 0, n0, bh);
+          tma_store_3d(&tmDK, smem + KO_DK + HALF, 64, n0, bh);
+          bulk_commit_group();
         }
       }
       bulk_wait_group0();
@@ -536,10 +573,14 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     const int row = quarter * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
     const int cpart = 32 * part;  // this warp's channels
+    int zslot = 0;                // dz slot of the current unit
+    int64_t prev_unit = -1;
     for (int64_t g = g0; g < g1; ++g) {
       const int64_t i = g - g0;
       const uint32_t ph = static_cast<uint32_t>(i & 1);
       const TileInfo ti = tile_info(p, g);
+      if (prev_unit >= 0 && ti.unit != prev_unit) zslot ^= 1;
+      prev_unit = ti.unit;
       if (!warp_wait(&bars->full, ph, abort_flag)) break;
       uint32_t ka[16];
 #pragma unroll
@@ -585,7 +626,7 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       for (int c4 = 0; c4 < 4; ++c4) sts128(row_chunk(sbase + KO_DV, row, 4 * part + c4), pack8(&x[8 * c4]));
       if (!warp_wait(&bars->ready, ph, abort_flag)) break;
       tc_fence_after();
-      const float* zg = dzimg + ti.unit * D + cpart;
+      const float* zg = reinterpret_cast<const float*>(smem + KO_Z) + zslot * D + cpart;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         // 16 channels at a time (fewer live registers)
@@ -610,8 +651,8 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c4 = 2 * hh + cc;
-          const float4 za = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4));
-          const float4 zb = __ldg(reinterpret_cast<const float4*>(zg + 8 * c4 + 4));
+          const float4 za = *reinterpret_cast<const float4*>(zg + 8 * c4);
+          const float4 zb = *reinterpret_cast<const float4*>(zg + 8 * c4 + 4);
           const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
           float o8[8];
 #pragma unroll
