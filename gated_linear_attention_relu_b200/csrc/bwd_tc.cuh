@@ -12,8 +12,10 @@
 // Two kernels, both walking the same persistent tile ranges as the forward state kernel, one
 // 128-token tile at a time (warps 0-15: four per row, by channel quarters; thread = token = TMEM
 // lane; warp 16: TMA and MMA issue).  Outputs are staged in buffers of their own, so the next
-// tile's inputs load as soon as the products reading them are done; the input read last (G in
-// the first kernel, V in the second) lands on a barrier of its own, waited for only by its reader:
+// tile's inputs load as soon as the products reading them are done; every input lands on a
+// barrier of its own, waited for only by its first reader (the first kernel: Q with the state
+// image and z, then dO, then G; the second: K with the dS image and dz, then V), and the two
+// products of a tile are committed apart so each epilogue waits only for the one it reads:
 //   bwdq_tc_kernel: num = phi(Q) S and dphi(q) = dnum S^T (the state's bf16 image serves as S,
 //     read N-major, and as S^T, read K-major), dS += phi(Q)^T dnum (TMEM accumulator drained to
 //     the CTA's partial slot at the end of each unit, like the state kernel); dQ, dG out.
