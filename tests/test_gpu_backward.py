@@ -17,6 +17,10 @@ CASES = [
     wl.custom("bw_split", B=1, H=2, T=8, Hh=10, W=40),               # 25 tiles per head over many CTAs
     wl.custom("bw_sparse", B=1, H=2, T=4, Hh=7, W=23, k_shift=-0.5, qkv_scale=1.0),
     wl.custom("bw_bands", B=1, H=2, T=3, Hh=6, W=20, bands=(0, 64, 64)),
+    wl.custom("bw_many_heads", B=1, H=160, T=1, Hh=2, W=64),        # one-tile heads, 12 CTAs hold two
+    # 74 tiles per head (ragged), 3 per CTA: four CTAs end one head and start the next, so the
+    # state image and z (two slots by unit parity) change inside a CTA
+    wl.custom("bw_cross", B=1, H=6, T=14, Hh=11, W=61),
 ]
 NAMES = ("dQ", "dK", "dV", "dG")
 

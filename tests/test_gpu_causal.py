@@ -23,6 +23,9 @@ CASES = [
     wl.custom("tc_single", B=1, H=2, T=1, Hh=1, W=1),
     wl.custom("tc_sparse", B=1, H=2, T=4, Hh=7, W=23, k_shift=-0.5, qkv_scale=1.0),
     wl.custom("tc_bands", B=1, H=2, T=3, Hh=6, W=20, bands=(0, 64, 64)),
+    # 74 tiles per head (ragged), 3 per CTA: four CTAs carry one head's start state into its
+    # ragged last tile and then begin the next head with z and S from zero
+    wl.custom("tc_cross", B=1, H=6, T=14, Hh=11, W=61),
 ]
 
 
