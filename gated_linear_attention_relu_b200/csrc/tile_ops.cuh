@@ -1,6 +1,7 @@
 // tile_ops.cuh -- shared pieces of the single-stage tensor-core kernels (token-causal, backward):
 // operand descriptors and row addressing of a 128 x 128 bf16 tile in the canonical 128B-swizzled
-// layout (two 64-channel halves of 128 rows x 128 B, as TMA writes it), and the RoPE of one row.
+// layout (two 64-channel halves of 128 rows x 128 B, as TMA writes it), and the RoPE of a span of a
+// row and its transpose.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -29,44 +30,6 @@ __device__ __forceinline__ float sigmoid_tanh(float g) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(0.5f * g));
   return 0.5f + 0.5f * y;
-}
-
-// In place over one row (64 bf16 pairs, already ReLU'd): a <- RoPE(a) at grid position (pt, ph, pw).
-template <int DT, int DH>
-__device__ __forceinline__ void rotate_row(uint32_t (&a)[64], const float2* __restrict__ tab,
-                                           const float4* __restrict__ tab2, const Rope& rope, const Plan& p,
-                                           int pt, int ph, int pw) {
-  if constexpr (DT >= 0 && DH >= 0) {
-    constexpr int DW = 128 - DT - DH;
-    static_assert(DT % 4 == 0 && DH % 4 == 0 && DW % 4 == 0, "bands of whole 16-byte entries");
-    const float4* bt = tab2 + pt * (DT / 4);
-    const float4* bh = tab2 + rope.tab_off_h / 2 + ph * (DH / 4);
-    const float4* bw = tab2 + rope.tab_off_w / 2 + pw;
-    const int W = static_cast<int>(p.W);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int pi = 2 * j;
-      const int bnd = band_of<DT, DH>(pi, rope);
-      const int e = pair_in_band<DT, DH>(pi, rope) / 2;
-      const float4 cs = __ldg(bnd == 0 ? bt + e : (bnd == 1 ? bh + e : bw + e * W));
-      const float x0 = bf16lo(a[pi]), x1 = bf16hi(a[pi]);
-      const float y0 = bf16lo(a[pi + 1]), y1 = bf16hi(a[pi + 1]);
-      a[pi] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
-      a[pi + 1] = pack_bf16(y0 * cs.z - y1 * cs.w, y0 * cs.w + y1 * cs.z);
-    }
-  } else {
-    const int ext[3] = {static_cast<int>(p.T), static_cast<int>(p.Hh), static_cast<int>(p.W)};
-    const int off[3] = {0, static_cast<int>(rope.tab_off_h), static_cast<int>(rope.tab_off_w)};
-    const int pos[3] = {pt, ph, pw};
-#pragma unroll 4
-    for (int pi = 0; pi < 64; ++pi) {
-      const int bnd = band_of<DT, DH>(pi, rope);
-      const int loc = pair_in_band<DT, DH>(pi, rope);
-      const float2 cs = __ldg(tab + off[bnd] + loc * ext[bnd] + pos[bnd]);
-      const float x0 = bf16lo(a[pi]), x1 = bf16hi(a[pi]);
-      a[pi] = pack_bf16(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
-    }
-  }
 }
 
 // In place over the NP bf16 pairs of a row starting at pair P0 (channels [2 P0, 2 P0 + 2 NP),
@@ -111,53 +74,6 @@ __device__ __forceinline__ void rotate_span(uint32_t (&a)[NP], const float2* __r
   }
 }
 
-// Half a row (channels [64 HF, 64 HF + 64) as 32 bf16 pairs).
-template <int DT, int DH, int HF>
-__device__ __forceinline__ void rotate_half(uint32_t (&a)[32], const float2* __restrict__ tab,
-                                            const float4* __restrict__ tab2, const Rope& rope, const Plan& p,
-                                            int pt, int ph, int pw) {
-  rotate_span<DT, DH, 32 * HF, 32>(a, tab, tab2, rope, p, pt, ph, pw);
-}
-
-// In place over one row of 128 fp32 values: x <- RoPE^T(x) (rotation by the opposite angle) at grid
-// position (pt, ph, pw): (x0, x1) -> (x0 c + x1 s, -x0 s + x1 c).
-template <int DT, int DH>
-__device__ __forceinline__ void rotate_row_t(float (&x)[128], const float2* __restrict__ tab,
-                                             const float4* __restrict__ tab2, const Rope& rope, const Plan& p,
-                                             int pt, int ph, int pw) {
-  if constexpr (DT >= 0 && DH >= 0) {
-    const float4* bt = tab2 + pt * (DT / 4);
-    const float4* bh = tab2 + rope.tab_off_h / 2 + ph * (DH / 4);
-    const float4* bw = tab2 + rope.tab_off_w / 2 + pw;
-    const int W = static_cast<int>(p.W);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int pi = 2 * j;
-      const int bnd = band_of<DT, DH>(pi, rope);
-      const int e = pair_in_band<DT, DH>(pi, rope) / 2;
-      const float4 cs = __ldg(bnd == 0 ? bt + e : (bnd == 1 ? bh + e : bw + e * W));
-      const float x0 = x[2 * pi], x1 = x[2 * pi + 1], y0 = x[2 * pi + 2], y1 = x[2 * pi + 3];
-      x[2 * pi] = x0 * cs.x + x1 * cs.y;
-      x[2 * pi + 1] = x1 * cs.x - x0 * cs.y;
-      x[2 * pi + 2] = y0 * cs.z + y1 * cs.w;
-      x[2 * pi + 3] = y1 * cs.z - y0 * cs.w;
-    }
-  } else {
-    const int ext[3] = {static_cast<int>(p.T), static_cast<int>(p.Hh), static_cast<int>(p.W)};
-    const int off[3] = {0, static_cast<int>(rope.tab_off_h), static_cast<int>(rope.tab_off_w)};
-    const int pos[3] = {pt, ph, pw};
-#pragma unroll 4
-    for (int pi = 0; pi < 64; ++pi) {
-      const int bnd = band_of<DT, DH>(pi, rope);
-      const int loc = pair_in_band<DT, DH>(pi, rope);
-      const float2 cs = __ldg(tab + off[bnd] + loc * ext[bnd] + pos[bnd]);
-      const float x0 = x[2 * pi], x1 = x[2 * pi + 1];
-      x[2 * pi] = x0 * cs.x + x1 * cs.y;
-      x[2 * pi + 1] = x1 * cs.x - x0 * cs.y;
-    }
-  }
-}
-
 // In place over the fp32 values of NP pairs starting at pair P0 (channels [2 P0, 2 P0 + 2 NP)):
 // x <- RoPE^T(x).  P0 and NP are even.
 template <int DT, int DH, int P0, int NP>
@@ -197,14 +113,6 @@ __device__ __forceinline__ void rotate_span_t(float (&x)[2 * NP], const float2* 
       x[2 * j + 1] = x1 * cs.x - x0 * cs.y;
     }
   }
-}
-
-// Half a row of fp32 values (channels [64 HF, 64 HF + 64)).
-template <int DT, int DH, int HF>
-__device__ __forceinline__ void rotate_half_t(float (&x)[64], const float2* __restrict__ tab,
-                                              const float4* __restrict__ tab2, const Rope& rope, const Plan& p,
-                                              int pt, int ph, int pw) {
-  rotate_span_t<DT, DH, 32 * HF, 32>(x, tab, tab2, rope, p, pt, ph, pw);
 }
 
 }  // namespace tile
