@@ -442,8 +442,9 @@ def main():
         "clocks": clk.summary(),
     }
 
-    if not args.no_e2e and not whole_step:
-        line["e2e"] = e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates, causal=args.causal)
+    if not args.no_e2e and not args.stream:
+        line["e2e"] = e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates, causal=args.causal,
+                          dO=dO if args.backward else None, grads=grads if args.backward else None)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         mode = "causal" if args.causal else ("backward" if args.backward else ("gated" if args.gated else "forward"))
         v, cores, times = oracle_sample(w, args.cpu_seconds, mode=mode)
@@ -456,22 +457,42 @@ def main():
     return 0
 
 
-def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None, causal=False):
+def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None, causal=False, dO=None, grads=None):
     """Same metric through the public API with the inputs in pinned host memory: every step
-    copies Q, K, V, G (and the write gate when gated) host->device, runs the operator and copies
-    O device->host.  Steps are pipelined the way a caller streaming batches would run them: two
-    device copies of the inputs and of O, the host->device copies on one stream, the operator on
-    the current stream and the device->host copy on a third, so step k+1's inputs and step k-1's
-    output cross the host link while step k computes (each copy engine works one direction)."""
+    copies the step's inputs host->device (Q, K, V, G, and the write gate when gated, or dO for
+    the backward pass), runs the operator and copies its outputs (O, or dQ, dK, dV, dG)
+    device->host.  Steps are pipelined the way a caller streaming batches would run them: two
+    device copies of the inputs and of the outputs, the host->device copies on one stream, the
+    operator on the current stream and the device->host copies on a third, so step k+1's inputs
+    and step k-1's outputs cross the host link while step k computes (each copy engine works one
+    direction)."""
     import torch
 
     gates = gates or {}
-    names = ["Q", "K", "V", "G"] + (["beta"] if "beta" in gates else [])
-    srcs0 = [Q, K, V, G] + ([gates["beta"]] if "beta" in gates else [])
+    if dO is not None:
+        srcs0, outs0 = [Q, K, V, G, dO], list(grads)
+
+        def run(d, o):
+            la.backward_bidir(p, d[0], d[1], d[2], d[3], d[4], grads=tuple(o), ws=ws)
+    else:
+        srcs0 = [Q, K, V, G] + ([gates["beta"]] if "beta" in gates else [])
+        outs0 = [O]
+
+        def run(d, o):
+            if gates:
+                g = dict(gates)
+                if len(d) > 4:
+                    g["beta"] = d[4]
+                la.forward_gated(p, d[0], d[1], d[2], d[3], O=o[0], ws=ws, **g)
+            elif causal:
+                la.forward_tokencausal(p, d[0], d[1], d[2], d[3], O=o[0], ws=ws)
+            else:
+                la.forward(p, d[0], d[1], d[2], d[3], O=o[0], ws=ws)
+
     hosts = [t.cpu().pin_memory() for t in srcs0]
     dsets = [srcs0, [torch.empty_like(t) for t in srcs0]]
-    outs = [O, torch.empty_like(O)]
-    ohost = [torch.empty(O.shape, dtype=O.dtype).pin_memory() for _ in range(2)]
+    osets = [outs0, [torch.empty_like(t) for t in outs0]]
+    ohost = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs0] for _ in range(2)]
     steps = max(3, min(args.steps, 10))
     cur = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
@@ -482,29 +503,21 @@ def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None, causal
 
     def step(k):
         j = k & 1
-        d = dsets[j]
         with torch.cuda.stream(s_in):
             if used[j]:
                 s_in.wait_event(ev_done[j])  # the operator of step k-2 has read this input set
-            for hsrc, dst in zip(hosts, d):
+            for hsrc, dst in zip(hosts, dsets[j]):
                 dst.copy_(hsrc, non_blocking=True)
             ev_in[j].record(s_in)
         cur.wait_event(ev_in[j])
         if used[j]:
-            cur.wait_event(ev_out[j])  # step k-2's O has left this buffer
-        kw = dict(zip(names[4:], d[4:]))
-        if gates:
-            g = dict(gates)
-            g.update(kw)
-            la.forward_gated(p, d[0], d[1], d[2], d[3], O=outs[j], ws=ws, **g)
-        elif causal:
-            la.forward_tokencausal(p, d[0], d[1], d[2], d[3], O=outs[j], ws=ws)
-        else:
-            la.forward(p, d[0], d[1], d[2], d[3], O=outs[j], ws=ws)
+            cur.wait_event(ev_out[j])  # step k-2's outputs have left these buffers
+        run(dsets[j], osets[j])
         ev_done[j].record(cur)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_done[j])
-            ohost[j].copy_(outs[j], non_blocking=True)
+            for hdst, src in zip(ohost[j], osets[j]):
+                hdst.copy_(src, non_blocking=True)
             ev_out[j].record(s_out)
         used[j] = True
 
@@ -525,9 +538,10 @@ def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None, causal
     t = ldist.max_over_ranks(s.elapsed_time(e), dev)
     th = w.B * w.H * w.N
     h2d = sum(x.numel() * x.element_size() for x in srcs0)
+    d2h = sum(x.numel() * x.element_size() for x in outs0)
     return {"value": world * th * steps / (t * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": O.numel() * O.element_size(), "steps": steps,
-            "pipelined": "two input and output buffers; copies in, operator and copy out on three streams"}
+            "d2h_bytes_per_step": d2h, "steps": steps,
+            "pipelined": "two input and output buffers; copies in, operator and copies out on three streams"}
 
 
 if __name__ == "__main__":
