@@ -44,6 +44,7 @@ __all__ = [
     "head_state", "head_apply", "forward_positions", "forward_bidir",
     "block_of_tokens", "block_states", "forward_blockcausal", "forward_brute", "rms_norm",
     "tokencausal_rows", "forward_tokencausal", "rope3d_transpose", "head_backward", "backward_bidir",
+    "head_backward_gated", "backward_gated",
 ]
 
 
@@ -244,37 +245,31 @@ def forward_brute(q, k, v, g, pos, bands, base, eps, visible=None, beta=None, rm
     return out
 
 
-def tokencausal_rows(q, k, v, g, pos, bands, base, eps, rows=None, chunk=1024):
+def tokencausal_rows(q, k, v, g, pos, bands, base, eps, rows=None):
     """Token-causal output of one head at the listed token indices (all when None):
     o_n = (RoPE(q_n^+) S_{<=n}) / (q_n^+ . z_{<=n} + eps) * sigmoid(g_n), with
     S_{<=n} = sum_{m<=n} RoPE(k_m^+)^T v_m and z_{<=n} = sum_{m<=n} k_m^+.
 
-    Walks the tokens in order, carrying (S, z) across chunks of ``chunk`` tokens; inside a chunk
-    the rows up to n are summed explicitly."""
+    A running prefix sum: the tokens are walked in order and, before row n is evaluated, the
+    tokens since the previous requested row (up to n itself) are added to (S, z)."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     g = np.asarray(g, dtype=np.float64)
     N, d = q.shape
-    want = np.arange(N) if rows is None else np.sort(np.asarray(rows))
-    out = {}
+    order = np.arange(N) if rows is None else np.unique(np.asarray(rows))
+    kp = relu(k)
+    kr = rope3d(kp, pos, bands, base)
     S = np.zeros((d, d))
     z = np.zeros(d)
-    for c0 in range(0, N, chunk):
-        c1 = min(N, c0 + chunk)
-        kp = relu(k[c0:c1])
-        kr = rope3d(kp, pos[c0:c1], bands, base)
-        sel = want[(want >= c0) & (want < c1)]
-        if len(sel):
-            qp = relu(q[sel])
-            qr = rope3d(qp, pos[sel], bands, base)
-            for i, n in enumerate(sel):
-                j = n - c0 + 1  # rows c0..n of this chunk
-                num = qr[i] @ S + (kr[:j] @ qr[i]) @ v[c0:c0 + j]
-                den = qp[i] @ z + (kp[:j] @ qp[i]).sum() + float(eps)
-                out[int(n)] = num / den * sigmoid(g[n])
-        S = S + kr.T @ v[c0:c1]
-        z = z + kp.sum(axis=0)
+    done = 0  # tokens 0 .. done-1 are in (S, z)
+    out = {}
+    for n in order:
+        n = int(n)
+        S = S + kr[done:n + 1].T @ v[done:n + 1]
+        z = z + kp[done:n + 1].sum(axis=0)
+        done = n + 1
+        out[n] = head_apply(q[n:n + 1], g[n:n + 1], S, z, pos[n:n + 1], bands, base, eps)[0]
     return np.array([out[int(n)] for n in (np.arange(N) if rows is None else np.asarray(rows))])
 
 
@@ -339,6 +334,105 @@ def head_backward(q, k, v, g, do, pos, bands, base, eps):
     dv = kr @ dS
     dk = (k > 0) * (rope3d_transpose(v @ dS.T, pos, bands, base) + dz[None, :])
     return dq, dk, dv, dg
+
+
+def head_backward_gated(q, k, v, g, do, pos, bands, base, eps, block_frames=0, beta=None, rms=None):
+    """Gradients of one head of the operator in its full form: block-causal when block_frames > 0
+    (token n reads the summed states of the blocks up to its own), write gate beta per token on the
+    state, RMSNorm (rms = (gamma, norm_eps)) before the output gate.  Returns dq, dk, dv, dg, dbeta
+    (None without beta) and dgamma (None without RMSNorm or with gamma None).
+
+    Forward, per token n in block b(n) (one block in the bidirectional form):
+      S_b = sum_{m: b(m) <= b} beta_m phi(k_m)^T v_m,  z_b = sum_{m: b(m) <= b} ReLU(k_m),
+      y_n = (phi(q_n) S_{b(n)}) / (ReLU(q_n) . z_{b(n)} + eps),
+      u_n = y_n / r_n * gamma with r_n = sqrt(mean(y_n^2) + norm_eps)   (u = y without RMSNorm),
+      o_n = u_n * sigmoid(g_n).
+    Chain rule:
+      dg = do u s (1 - s),  du = do s,  dgamma = sum_n du_n y_n / r_n,
+      dy = (dyh - yh (yh . dyh) / d) / r with yh = y / r and dyh = du gamma   (dy = du without),
+      dnum = dy / den,  dden = -(dy . y) / den,
+      dS_b = sum_{n in block b} phi(q_n)^T dnum_n,  dz_b = sum_{n in block b} dden_n ReLU(q_n),
+      and a key of block c feeds every S_b with b >= c, so it sees the suffix sums
+      dS^c = sum_{b >= c} dS_b,  dz^c = sum_{b >= c} dz_b:
+      dq = [q > 0] (RoPE^T(dnum S_{b(n)}^T) + dden z_{b(n)}),
+      dv_m = beta_m phi(k_m) dS^{b(m)},  dk_m = [k > 0] (RoPE^T(beta_m v_m dS^{b(m)T}) + dz^{b(m)}),
+      dbeta_m = phi(k_m) . (dS^{b(m)} v_m)."""
+    q, k, v, g, do = (np.asarray(a, dtype=np.float64) for a in (q, k, v, g, do))
+    N, d = q.shape
+    bt = np.ones(N) if beta is None else np.asarray(beta, dtype=np.float64)
+    blk = block_of_tokens(pos, block_frames) if block_frames > 0 else np.zeros(N, dtype=np.int64)
+    nblk = int(blk.max()) + 1 if N else 0
+    qp, kp = relu(q), relu(k)
+    qr, kr = rope3d(qp, pos, bands, base), rope3d(kp, pos, bands, base)
+    # inclusive states per block
+    S = np.zeros((nblk, d, d))
+    z = np.zeros((nblk, d))
+    for b in range(nblk):
+        sel = blk <= b
+        S[b] = (kr[sel] * bt[sel][:, None]).T @ v[sel]
+        z[b] = kp[sel].sum(axis=0)
+    Sn, zn = S[blk], z[blk]                      # the state each token reads
+    num = np.einsum("ni,nij->nj", qr, Sn)
+    den = np.einsum("ni,ni->n", qp, zn) + float(eps)
+    y = num / den[:, None]
+    sg = sigmoid(g)
+    if rms is not None:
+        gamma = np.ones(d) if rms[0] is None else np.asarray(rms[0], dtype=np.float64)
+        r = np.sqrt(np.mean(y * y, axis=1) + float(rms[1]))
+        yh = y / r[:, None]
+        u = yh * gamma
+    else:
+        u = y
+    dg = do * u * sg * (1.0 - sg)
+    du = do * sg
+    dgamma = None
+    if rms is not None:
+        if rms[0] is not None:
+            dgamma = np.sum(du * yh, axis=0)
+        dyh = du * gamma
+        dy = (dyh - yh * np.sum(yh * dyh, axis=1, keepdims=True) / d) / r[:, None]
+    else:
+        dy = du
+    dnum = dy / den[:, None]
+    dden = -np.sum(dy * y, axis=1) / den
+    dSb = np.zeros((nblk, d, d))
+    dzb = np.zeros((nblk, d))
+    for b in range(nblk):
+        sel = blk == b
+        dSb[b] = qr[sel].T @ dnum[sel]
+        dzb[b] = qp[sel].T @ dden[sel]
+    dSs = np.cumsum(dSb[::-1], axis=0)[::-1]     # suffix sums over blocks
+    dzs = np.cumsum(dzb[::-1], axis=0)[::-1]
+    dq = (q > 0) * (rope3d_transpose(np.einsum("nj,nij->ni", dnum, Sn), pos, bands, base) + dden[:, None] * zn)
+    P = np.einsum("nj,nij->ni", v, dSs[blk])     # v_m dS^T, row by row
+    dv = bt[:, None] * np.einsum("ni,nij->nj", kr, dSs[blk])
+    dk = (k > 0) * (rope3d_transpose(bt[:, None] * P, pos, bands, base) + dzs[blk])
+    dbeta = np.sum(kr * P, axis=1) if beta is not None else None
+    return dq, dk, dv, dg, dbeta, dgamma
+
+
+def backward_gated(Q, K, V, G, dO, grid, bands, base=10000.0, eps=1e-6, block_frames=0, beta=None, rms=None):
+    """head_backward_gated over [B, H, N, d] inputs (beta: [B, H, N]).  Returns dQ, dK, dV, dG,
+    dbeta ([B, H, N] or None) and dgamma ([d], summed over the heads, or None)."""
+    T, Hh, W = grid
+    pos = grid_positions(T, Hh, W)
+    B, H, N, d = np.shape(Q)
+    q, k, v, g, do = _heads(Q), _heads(K), _heads(V), _heads(G), _heads(dO)
+    bt = None if beta is None else np.asarray(beta, dtype=np.float64).reshape(B * H, N)
+    outs = [np.empty((B * H, N, d)) for _ in range(4)]
+    dbeta = None if beta is None else np.empty((B * H, N))
+    dgamma = None
+    for u in range(B * H):
+        r = head_backward_gated(q[u], k[u], v[u], g[u], do[u], pos, bands, base, eps, block_frames,
+                                None if bt is None else bt[u], rms)
+        for o, x in zip(outs, r[:4]):
+            o[u] = x
+        if dbeta is not None:
+            dbeta[u] = r[4]
+        if r[5] is not None:
+            dgamma = r[5] if dgamma is None else dgamma + r[5]
+    res = [o.reshape(B, H, N, d) for o in outs]
+    return (*res, None if dbeta is None else dbeta.reshape(B, H, N), dgamma)
 
 
 def backward_bidir(Q, K, V, G, dO, grid, bands, base=10000.0, eps=1e-6):

@@ -444,17 +444,17 @@ def test_rms_norm_invariances_and_placement():
 
 def test_tokencausal_linear_form_equals_masked_brute_form():
     rng = np.random.default_rng(31)
-    for T, Hh, W, d, bands, chunk in ((3, 2, 5, 16, (4, 6, 6), 7), (2, 3, 4, 8, (2, 2, 4), 1000)):
+    for T, Hh, W, d, bands in ((3, 2, 5, 16, (4, 6, 6)), (2, 3, 4, 8, (2, 2, 4))):
         N = T * Hh * W
         pos = orc.grid_positions(T, Hh, W)
         q, k, v, g = (rng.standard_normal((N, d)) for _ in range(4))
-        lin = orc.tokencausal_rows(q, k, v, g, pos, bands, 10000.0, 1e-6, chunk=chunk)
+        lin = orc.tokencausal_rows(q, k, v, g, pos, bands, 10000.0, 1e-6)
         mask = np.tril(np.ones((N, N), dtype=bool))
         bru = orc.forward_brute(q, k, v, g, pos, bands, 10000.0, 1e-6, visible=mask)
         assert np.allclose(lin, bru, rtol=1e-11, atol=1e-13)
         # sampled rows agree with the full evaluation
         rows = [0, 5, N - 1, 13]
-        assert np.allclose(orc.tokencausal_rows(q, k, v, g, pos, bands, 10000.0, 1e-6, rows=rows, chunk=4),
+        assert np.allclose(orc.tokencausal_rows(q, k, v, g, pos, bands, 10000.0, 1e-6, rows=rows),
                            lin[rows], rtol=1e-12)
 
 
@@ -523,3 +523,111 @@ def test_rope_transpose_is_the_inverse_rotation():
     # <R x, y> = <x, R^T y> row by row
     assert np.allclose(np.sum(orc.rope3d(x, pos, bands, 10000.0) * y, axis=1),
                        np.sum(x * orc.rope3d_transpose(y, pos, bands, 10000.0), axis=1), rtol=1e-12)
+
+
+def test_multihead_wrappers_take_each_head_separately():
+    # Two heads (B = 1, H = 2) through the [B, H, N, d] wrappers: each head's result is that of
+    # the masked brute form (token-causal) or the central differences pinned above (gradients)
+    # on that head alone, so a mix-up of heads or of the B/H order fails here.
+    rng = np.random.default_rng(47)
+    T, Hh, W, d, bands = 2, 2, 3, 8, (2, 2, 4)
+    N = T * Hh * W
+    pos = orc.grid_positions(T, Hh, W)
+    Q, K, V, G, dO = (rng.standard_normal((1, 2, N, d)) for _ in range(5))
+    Q[:, 1] *= 3.0  # make the heads differ in scale too
+    O = orc.forward_tokencausal(Q, K, V, G, (T, Hh, W), bands)
+    mask = np.tril(np.ones((N, N), dtype=bool))
+    for h in range(2):
+        bru = orc.forward_brute(Q[0, h], K[0, h], V[0, h], G[0, h], pos, bands, 10000.0, 1e-6, visible=mask)
+        assert np.allclose(O[0, h], bru, rtol=1e-11, atol=1e-13)
+    grads = orc.backward_bidir(Q, K, V, G, dO, (T, Hh, W), bands)
+    for h in range(2):
+        args = [Q[0, h].copy(), K[0, h].copy(), V[0, h].copy(), G[0, h].copy()]
+        for x in args[:2]:
+            x[np.abs(x) < 0.05] = 0.3
+        Qh, Kh = Q.copy(), K.copy()
+        Qh[0, h], Kh[0, h] = args[0], args[1]
+        gh = orc.backward_bidir(Qh, Kh, V, G, dO, (T, Hh, W), bands)
+        fd = _fd_grads(lambda a: _loss(*a, dO[0, h], pos, bands), args)
+        for which in range(4):
+            assert np.allclose(gh[which][0, h], fd[which], rtol=1e-6, atol=1e-7), (h, which)
+    assert grads[0].shape == Q.shape
+
+
+def _fd_grads(loss, args, h=1e-6):
+    """Central differences of loss(args) with respect to every element of every array in args."""
+    out = []
+    for which in range(len(args)):
+        fd = np.empty_like(args[which])
+        for idx in np.ndindex(*fd.shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            fd[idx] = (loss(plus) - loss(minus)) / (2 * h)
+        out.append(fd)
+    return out
+
+
+@pytest.mark.parametrize("block_frames,use_beta,use_rms", [
+    (1, False, False), (2, False, False), (0, True, False), (0, False, True), (2, True, True)])
+def test_gated_blockcausal_backward_matches_central_differences(block_frames, use_beta, use_rms):
+    """Gradients of the full form (block-causal states, write gate beta, RMSNorm with gamma) against
+    central differences of the forward oracle: d/dx sum(O * dO) for every element of q, k, v, g,
+    beta and gamma."""
+    rng = np.random.default_rng(53 + 7 * block_frames + 2 * use_beta + use_rms)
+    T, Hh, W, d, bands = 3, 2, 2, 8, (2, 2, 4)
+    N = T * Hh * W
+    pos = orc.grid_positions(T, Hh, W)
+    q, k, v, g, do = (rng.standard_normal((N, d)) for _ in range(5))
+    for x in (q, k):
+        x[np.abs(x) < 0.05] = 0.3
+    beta = rng.uniform(0.2, 1.5, N) if use_beta else None
+    gamma = rng.uniform(0.5, 1.5, d) if use_rms else None
+    rms = (gamma, 1e-3) if use_rms else None
+
+    def fwd(q_, k_, v_, g_, beta_, gamma_):
+        r = (gamma_, 1e-3) if use_rms else None
+        shape = (1, 1, N, d)
+        b4 = None if beta_ is None else beta_.reshape(1, 1, N)
+        if block_frames > 0:
+            return orc.forward_blockcausal(q_.reshape(shape), k_.reshape(shape), v_.reshape(shape),
+                                           g_.reshape(shape), (T, Hh, W), bands, block_frames=block_frames,
+                                           beta=b4, rms=r)[0, 0]
+        return orc.forward_positions(q_, k_, v_, g_, pos, bands, 10000.0, 1e-6, beta=beta_, rms=r)
+
+    args = [q, k, v, g] + ([beta] if use_beta else []) + ([gamma] if use_rms else [])
+
+    def loss(a):
+        it = iter(a[4:])
+        b_ = next(it) if use_beta else None
+        gm = next(it) if use_rms else None
+        return float(np.sum(fwd(a[0], a[1], a[2], a[3], b_, gm) * do))
+
+    dq, dk, dv, dg, dbeta, dgamma = orc.head_backward_gated(q, k, v, g, do, pos, bands, 10000.0, 1e-6,
+                                                            block_frames, beta, rms)
+    got = [dq, dk, dv, dg] + ([dbeta] if use_beta else []) + ([dgamma] if use_rms else [])
+    fd = _fd_grads(loss, args)
+    for i, (a, b) in enumerate(zip(got, fd)):
+        assert np.allclose(a, b, rtol=1e-6, atol=2e-7), i
+    assert (dbeta is None) == (not use_beta) and (dgamma is None) == (not use_rms)
+
+
+def test_gated_backward_reduces_to_the_plain_bidirectional_gradients():
+    rng = np.random.default_rng(59)
+    T, Hh, W, d, bands = 2, 3, 4, 16, (4, 6, 6)
+    N = T * Hh * W
+    pos = orc.grid_positions(T, Hh, W)
+    q, k, v, g, do = (rng.standard_normal((N, d)) for _ in range(5))
+    plain = orc.head_backward(q, k, v, g, do, pos, bands, 10000.0, 1e-6)
+    full = orc.head_backward_gated(q, k, v, g, do, pos, bands, 10000.0, 1e-6)
+    for a, b in zip(plain, full[:4]):
+        assert np.allclose(a, b, rtol=1e-12, atol=1e-14)
+    # one block covering every frame is the bidirectional form
+    one = orc.head_backward_gated(q, k, v, g, do, pos, bands, 10000.0, 1e-6, block_frames=T)
+    for a, b in zip(plain, one[:4]):
+        assert np.allclose(a, b, rtol=1e-12, atol=1e-14)
+    # beta = 1 gives the un-gated gradients and dbeta = phi(k) . (dS v)
+    ones = orc.head_backward_gated(q, k, v, g, do, pos, bands, 10000.0, 1e-6, beta=np.ones(N))
+    for a, b in zip(plain, ones[:4]):
+        assert np.allclose(a, b, rtol=1e-12, atol=1e-14)
