@@ -168,6 +168,10 @@ PlanSet make_plans(const la_problem& q, int sm_count) {
   return s;
 }
 
+// Bytes the non-token-causal paths use: everything before the token-causal start states, which
+// sit last in the layout and are read by no other path.
+size_t forward_bytes(const PlanSet& s) { return s.off_start; }
+
 Rope make_rope(const la_problem& q) {
   Rope r;
   std::memset(&r, 0, sizeof r);
@@ -420,9 +424,11 @@ int launch_apply(const PlanSet& s, const la_problem& q, const void* Q, const voi
   return launched_ok();
 }
 
-int check_ws(const PlanSet& s, const void* ws, size_t ws_bytes) {
-  if (s.total == 0) return LA_OK;
-  if (!ws || ws_bytes < s.total) return LA_ERR_WORKSPACE;
+// `need`: the bytes the calling path uses (the whole layout unless given).
+int check_ws(const PlanSet& s, const void* ws, size_t ws_bytes, size_t need = size_t(-1)) {
+  if (need == size_t(-1)) need = s.total;
+  if (need == 0) return LA_OK;
+  if (!ws || ws_bytes < need) return LA_ERR_WORKSPACE;
   if (!aligned16(ws)) return LA_ERR_ALIGN;
   return LA_OK;
 }
@@ -730,7 +736,7 @@ static int forward_common(const la_problem* p, const void* Q, const void* K, con
   int sm = 0;
   if ((rc = current_sm_count(&sm))) return rc;
   const PlanSet s = make_plans(*p, sm);
-  if ((rc = check_ws(s, ws, ws_bytes))) return rc;
+  if ((rc = check_ws(s, ws, ws_bytes, forward_bytes(s)))) return rc;
   uint8_t* w = static_cast<uint8_t*>(ws);
   float* st_S = S_incl ? S_incl : reinterpret_cast<float*>(w + s.off_states);
   float* st_z = z_incl ? z_incl : reinterpret_cast<float*>(w + s.off_states) + s.units * p->d * p->d;
@@ -873,10 +879,15 @@ int la_forward_bidir_static(const la_problem* p, const void* Q, const void* K, c
   int rc = validate(p);
   if (rc) return rc;
   if (p->block_frames != 0) return LA_ERR_SHAPE;
+  // Argument errors are reported before any CUDA call, as for every other entry point.
+  const bool has_tok = elems(*p) > 0;
+  if ((rc = check_ptr(Q, has_tok)) || (rc = check_ptr(K, has_tok)) || (rc = check_ptr(V, has_tok)) ||
+      (rc = check_ptr(G, has_tok)) || (rc = check_ptr(O, has_tok)))
+    return rc;
   int dev = 0, sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LA_ERR_CUDA;
   if ((rc = current_sm_count(&sm))) return rc;
-  if (make_plans(*p, sm).total > LA_STATIC_WORKSPACE_BYTES) return LA_ERR_WORKSPACE;
+  if (forward_bytes(make_plans(*p, sm)) > LA_STATIC_WORKSPACE_BYTES) return LA_ERR_WORKSPACE;
   void* ws = nullptr;
   if ((rc = static_workspace(dev, &ws))) return rc;
   return forward_common(p, Q, K, V, G, O, nullptr, nullptr, ws, LA_STATIC_WORKSPACE_BYTES, stream);

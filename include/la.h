@@ -212,9 +212,14 @@ int la_forward_marked(const la_problem* p, const la_gates* gates, const void* Q,
  *  - The scratch lives in every GPU that loads the library, until the process exits.
  *  - The first call on a device looks up the scratch's device address (a host-side query that
  *    allocates nothing); make that first call before any stream capture.
- *  - Problems whose workspace (la_workspace_bytes) exceeds LA_STATIC_WORKSPACE_BYTES are
- *    rejected with LA_ERR_WORKSPACE before anything is launched.  B = 1, H = 32 at the
- *    720p/5s and 720p/60s latent grids fits.
+ *  - It needs la_workspace_bytes() less the token-causal start states that sit last in that
+ *    layout (sm_count x (d*d + d) x 4 bytes on the tensor-core path), which only
+ *    la_forward_tokencausal reads.  Problems needing more than LA_STATIC_WORKSPACE_BYTES are
+ *    rejected with LA_ERR_WORKSPACE before anything is launched.  The need grows with the SM
+ *    count: B = 1, H = 32 at the 720p/5s or 720p/60s latent grid takes about 22 MiB on a
+ *    148-SM B200 and fits up to about 200 SMs.
+ *  - NULL or misaligned Q, K, V, G, O are reported (LA_ERR_NULL / LA_ERR_ALIGN) before any
+ *    CUDA call, as for la_forward_bidir.
  *  - All calls, on any stream, share the one scratch array, which keeps whatever the last call
  *    left in it.  Nothing in it needs clearing (each call writes every byte it later reads),
  *    but calls whose GPU work overlaps in time race on it: serialise them. */

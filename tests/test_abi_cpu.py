@@ -123,3 +123,25 @@ def test_backward_rejects_unsupported_problems_before_cuda():
         args.update(kw)
         cp = la.Problem(**args).c()
         assert lib.la_backward_bidir(ctypes.byref(cp), *([16] * 9), 16, 1 << 30, None) == status
+
+
+def test_static_entry_point_checks_pointers_before_cuda():
+    # A NULL or misaligned tensor is an argument error, reported before the device is queried,
+    # even for a problem far too large for the fixed scratch.
+    lib = la.load()
+    for p in (la.Problem(B=1, H=2, T=3, Hh=4, W=5), la.Problem(B=8, H=64, T=241, Hh=45, W=80)):
+        cp = p.c()
+        assert lib.la_forward_bidir_static(ctypes.byref(cp), None, 16, 16, 16, 16, None) == 1
+        assert lib.la_forward_bidir_static(ctypes.byref(cp), 16, 16, 16, 16, 24, None) == 4
+    cp = la.Problem(B=1, H=2, T=3, Hh=4, W=5, block_frames=1).c()
+    assert lib.la_forward_bidir_static(ctypes.byref(cp), 16, 16, 16, 16, 16, None) == 2
+
+
+@pytest.mark.parametrize("T", [21, 241])
+def test_static_scratch_fits_720p_on_a_b200(T):
+    # The allocation-free forward uses the workspace layout without its last region, the
+    # token-causal start states (one (d*d + d)-float state per CTA, i.e. per SM here).
+    p = la.Problem(B=1, H=32, T=T, Hh=45, W=80)
+    sm = 148
+    need = la.workspace_bytes(p, sm_count=sm) - sm * (128 * 128 + 128) * 4
+    assert 0 < need <= 32 << 20

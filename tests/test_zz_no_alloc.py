@@ -5,8 +5,10 @@ every allocation, or a service that fixes its memory at start-up), so they canno
 workspace la_forward_bidir needs.  la_forward_bidir_static uses the library's fixed device
 scratch instead.  This test calls it through the C ABI twice in a row, on two different problems
 (so the second call runs on scratch the first one left behind), and checks each output against
-la_forward_bidir with the tolerance the parity tests use.  It lives in a file of its own that
-pytest collects last.
+la_forward_bidir bit for bit (both run the same kernels on the same work split, with every
+reduction in a fixed order, so any difference means stale scratch was read), and the second one
+against the fp64 oracle as well, with the tolerance the parity tests use.  It lives in a file of
+its own that pytest collects last.
 """
 import ctypes
 
@@ -15,7 +17,8 @@ import torch
 
 import gated_linear_attention_relu_b200 as la
 from gated_linear_attention_relu_b200 import workloads as wl
-from la_test_util import TOL_BF16
+import oracle as orc
+from la_test_util import TOL_BF16, rel_err, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -38,9 +41,11 @@ def test_static_scratch_forward_matches_workspace_forward_twice():
         assert _static_call(p, Q, K, V, G, O) == 0
         torch.cuda.synchronize()
         assert la.device_error() == 0
-        scale = ref.float().abs().max().item()
-        err = (O.float() - ref.float()).abs().max().item()
-        assert err <= TOL_BF16 * scale, (w.name, err, scale)
+        assert torch.equal(O, ref), (w.name, (O.float() - ref.float()).abs().max().item())
+    # the second problem against the oracle too
+    o_ref = orc.forward_bidir(to64(Q), to64(K), to64(V), to64(G), (w.T, w.Hh, w.W), w.bands, w.rope_base, w.eps)
+    err = rel_err(to64(O), o_ref)
+    assert err <= TOL_BF16, (w.name, err)
 
 
 def test_static_scratch_rejects_problems_that_do_not_fit():
