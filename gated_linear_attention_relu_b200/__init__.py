@@ -7,7 +7,7 @@ sm_100a); this package only marshals arguments.
 """
 from . import workloads  # noqa: F401
 from .binding import (  # noqa: F401
-    LaError, Problem, apply, backward_bidir, block_step, device_error, forward, forward_bidir, forward_blockcausal, forward_gated,
+    LaError, Problem, apply, backward, backward_bidir, block_step, device_error, forward, forward_bidir, forward_blockcausal, forward_gated,
     forward_marked, forward_tokencausal,
     last_launch_count, load, state_reduce, state_scan, state_update, status_string, workspace,
     workspace_bytes,

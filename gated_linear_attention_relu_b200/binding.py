@@ -28,6 +28,7 @@ EXPORTS = [
     "la_forward_bidir", "la_forward_blockcausal", "la_status_string", "la_device_error",
     "la_last_launch_count", "la_forward_marked", "la_selftest_host", "la_forward_bidir_static",
     "la_state_update", "la_forward_gated", "la_block_step", "la_forward_tokencausal", "la_backward_bidir",
+    "la_backward",
 ]
 
 
@@ -83,6 +84,8 @@ def load(path: Optional[str] = None):
         "la_block_step": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_tokencausal": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_backward_bidir": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "la_backward": (ctypes.c_int, [P, ctypes.POINTER(LaGates), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                       vp, sz, vp]),
         "la_forward_gated": (ctypes.c_int, [P, ctypes.POINTER(LaGates), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_apply": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_bidir": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -340,7 +343,7 @@ def forward_gated(p: Problem, Q, K, V, G, beta=None, gamma=None, rms_norm=False,
 
 
 def forward_tokencausal(p: Problem, Q, K, V, G, O=None, ws=None, stream=None):
-    """Token-causal operator: token n reads the states of tokens 0..n (bf16, d = 128)."""
+    """Token-causal operator: token n reads the states of tokens 0..n."""
     import torch
 
     lib = load()
@@ -372,6 +375,32 @@ def backward_bidir(p: Problem, Q, K, V, G, dO, grads=None, ws=None, stream=None)
     _check(lib.la_backward_bidir(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(dO), _ptr(dQ), _ptr(dK),
                                  _ptr(dV), _ptr(dG), _ptr(ws), nbytes, _stream(stream)), "la_backward_bidir")
     return dQ, dK, dV, dG
+
+
+def backward(p: Problem, Q, K, V, G, dO, beta=None, gamma=None, rms_norm=False, norm_eps=1e-6, grads=None,
+             ws=None, stream=None):
+    """Gradients of the operator in any form (bidirectional or block-causal as ``p.block_frames``
+    says; write gate ``beta`` and RMSNorm optional): returns (dQ, dK, dV, dG, dbeta, dgamma), with
+    dbeta [B,H,N] when ``beta`` is given and dgamma [d] fp32 when RMSNorm has a weight ``gamma``
+    (else None)."""
+    import torch
+
+    lib = load()
+    if grads is None:
+        grads = tuple(torch.empty_like(Q) for _ in range(4))
+    dQ, dK, dV, dG = grads
+    dbeta = torch.empty_like(beta) if beta is not None else None
+    dgamma = torch.empty_like(gamma) if (rms_norm and gamma is not None) else None
+    if ws is None:
+        ws, nbytes = workspace(p, Q.device)
+    else:
+        nbytes = ws.numel()
+    cp = p.c()
+    gates = LaGates(_ptr(beta), _ptr(gamma), float(norm_eps), 1 if rms_norm else 0)
+    _check(lib.la_backward(ctypes.byref(cp), ctypes.byref(gates), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(dO),
+                           _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dG), _ptr(dbeta), _ptr(dgamma), _ptr(ws), nbytes,
+                           _stream(stream)), "la_backward")
+    return dQ, dK, dV, dG, dbeta, dgamma
 
 
 def forward(p: Problem, Q, K, V, G, **kw):

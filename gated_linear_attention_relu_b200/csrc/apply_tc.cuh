@@ -251,14 +251,14 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (ti.unit != prev_unit) {
           const int64_t ku = ti.unit - u_first;
           const int b = static_cast<int>(ku % NSB);
-          if (!mbar_wait(&bars->sfree[b], static_cast<uint32_t>(((ku / NSB) & 1) ^ 1), abort_flag)) break;
+          if (!mbar_wait(&bars->sfree[b], static_cast<uint32_t>(((ku / NSB) & 1) ^ 1), abort_flag, LA_SLEEP_PROD)) break;
           mbar_arrive_expect_tx(&bars->sfull[b], BUF);
           bulk_load(smem + OFF_S + b * BUF, simg + ti.unit * static_cast<int64_t>(BUF), BUF, &bars->sfull[b]);
           prev_unit = ti.unit;
           ++issued_s;
         }
         const int qs = static_cast<int>(i % QST);
-        if (!mbar_wait(&bars->qempty[qs], static_cast<uint32_t>(((i / QST) & 1) ^ 1), abort_flag)) break;
+        if (!mbar_wait(&bars->qempty[qs], static_cast<uint32_t>(((i / QST) & 1) ^ 1), abort_flag, LA_SLEEP_PROD)) break;
         mbar_arrive_expect_tx(&bars->qfull[qs], BUF);
         const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
         tma_load_3d(smem + OFF_Q + qs * BUF, &tmQ, 0, n0, bh, &bars->qfull[qs]);
@@ -280,7 +280,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int64_t g = g0; g < g1; ++g) {
         const int64_t i = g - g0;
         const int gs = static_cast<int>(i % GST);
-        if (!mbar_wait(&bars->gempty[gs], static_cast<uint32_t>(((i / GST) & 1) ^ 1), abort_flag)) break;
+        if (!mbar_wait(&bars->gempty[gs], static_cast<uint32_t>(((i / GST) & 1) ^ 1), abort_flag, LA_SLEEP_PROD)) break;
         const TileInfo ti = tile_info(p, g);
         mbar_arrive_expect_tx(&bars->gfull[gs], BUF);
         const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
@@ -372,7 +372,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int64_t g = g0; g < g1; ++g) {
         const int64_t i = g - g0;
         const int gs = static_cast<int>(i % GST);
-        if (!mbar_wait(&bars->ostaged[gs], static_cast<uint32_t>((i / GST) & 1), abort_flag)) break;
+        if (!mbar_wait(&bars->ostaged[gs], static_cast<uint32_t>((i / GST) & 1), abort_flag, LA_SLEEP_PROD)) break;
         const TileInfo ti = tile_info(p, g);
         if ((ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N)) {
           const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);

@@ -99,7 +99,8 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmDQ,
                const __grid_constant__ CUtensorMap tmDG, const Plan p, const __grid_constant__ Rope rope,
                const uint8_t* __restrict__ simg, const float* __restrict__ zimg, const float2* __restrict__ tab,
-               const float4* __restrict__ tab2, float* __restrict__ partial) {
+               const float4* __restrict__ tab2, float* __restrict__ partial, __nv_bfloat16* __restrict__ dQg,
+               __nv_bfloat16* __restrict__ dGg) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   BarsQ* bars = reinterpret_cast<BarsQ*>(smem + QO_BAR);
@@ -215,12 +216,19 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // has been read out (dQ's read is waited for before the next dq epilogue may start).
         if (!mbar_wait(&bars->out, ph, abort_flag)) break;
         {
+          // A tile that ends inside a head's block (block-causal units) was written out row by row
+          // by the math warps; the groups stay (empty) so the group accounting is the same.
+          const bool tma_out = (ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N);
           const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
-          tma_store_3d(&tmDG, smem + QO_G, 0, n0, bh);
-          tma_store_3d(&tmDG, smem + QO_G + HALF, 64, n0, bh);
+          if (tma_out) {
+            tma_store_3d(&tmDG, smem + QO_G, 0, n0, bh);
+            tma_store_3d(&tmDG, smem + QO_G + HALF, 64, n0, bh);
+          }
           bulk_commit_group();
-          tma_store_3d(&tmDQ, smem + QO_DQ, 0, n0, bh);
-          tma_store_3d(&tmDQ, smem + QO_DQ + HALF, 64, n0, bh);
+          if (tma_out) {
+            tma_store_3d(&tmDQ, smem + QO_DQ, 0, n0, bh);
+            tma_store_3d(&tmDQ, smem + QO_DQ + HALF, 64, n0, bh);
+          }
           bulk_commit_group();
           bulk_wait_group_read1();
         }
@@ -267,6 +275,16 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         qa[4 * c4 + 3] = relu_bf16x2(rq.w);
       }
       const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
+      // Rows past the end of the unit (the next block of the head) take no part: a zero query
+      // adds nothing to dS or dz, and their outputs are not written.
+      const bool valid = static_cast<int64_t>(n) < ti.n_end;
+      const bool tma_out = (ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N);
+      if (!valid) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) qa[e] = 0u;
+      }
+      __nv_bfloat16* dq_row = dQg + (ti.bh * p.N + static_cast<int64_t>(n)) * D + cpart;
+      __nv_bfloat16* dg_row = dGg + (ti.bh * p.N + static_cast<int64_t>(n)) * D + cpart;
       uint32_t pt = 0, ph_ = 0, pw = 0;
       if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph_, pw);
       const int ipt = static_cast<int>(pt), iph = static_cast<int>(ph_), ipw = static_cast<int>(pw);
@@ -342,7 +360,8 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             dgw[q] = pack_bf16(dg.x, dg.y);
             dnw[q] = pack_bf16(dn.x, dn.y);
           }
-          sts128(ag, make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]));
+          if (tma_out) sts128(ag, make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]));
+          else if (valid) *reinterpret_cast<uint4*>(dg_row + 8 * (2 * hh + cc)) = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
           sts128(ad, make_uint4(dnw[0], dnw[1], dnw[2], dnw[3]));
         }
       }
@@ -421,7 +440,8 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             const float qv = (e & 1) ? bf16hi(w) : bf16lo(w);
             o8[e] = qv > 0.f ? x[8 * cc + e] + dden * zz[e] : 0.f;
           }
-          sts128(row_chunk(sbase + QO_DQ, row, 4 * part + c4), pack8(o8));
+          if (tma_out) sts128(row_chunk(sbase + QO_DQ, row, 4 * part + c4), pack8(o8));
+          else if (valid) *reinterpret_cast<uint4*>(dq_row + 8 * c4) = pack8(o8);
         }
       }
       if (last) {
@@ -459,7 +479,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV, const Plan p,
                const __grid_constant__ Rope rope, const uint8_t* __restrict__ dsimg, const float* __restrict__ dzimg,
-               const float2* __restrict__ tab, const float4* __restrict__ tab2) {
+               const float2* __restrict__ tab, const float4* __restrict__ tab2, __nv_bfloat16* __restrict__ dKg,
+               __nv_bfloat16* __restrict__ dVg) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   BarsK* bars = reinterpret_cast<BarsK*>(smem + KO_BAR);
@@ -553,12 +574,18 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         // tile's products are committed to the epilogues that rewrite the staging buffers.
         if (!mbar_wait(&bars->out, ph, abort_flag)) break;
         {
+          // (a tile that ends inside a head's block was written out row by row by the math warps)
+          const bool tma_out = (ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N);
           const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
-          tma_store_3d(&tmDV, smem + KO_DV, 0, n0, bh);
-          tma_store_3d(&tmDV, smem + KO_DV + HALF, 64, n0, bh);
+          if (tma_out) {
+            tma_store_3d(&tmDV, smem + KO_DV, 0, n0, bh);
+            tma_store_3d(&tmDV, smem + KO_DV + HALF, 64, n0, bh);
+          }
           bulk_commit_group();
-          tma_store_3d(&tmDK, smem + KO_DK, 0, n0, bh);
-          tma_store_3d(&tmDK, smem + KO_DK + HALF, 64, n0, bh);
+          if (tma_out) {
+            tma_store_3d(&tmDK, smem + KO_DK, 0, n0, bh);
+            tma_store_3d(&tmDK, smem + KO_DK + HALF, 64, n0, bh);
+          }
           bulk_commit_group();
         }
       }
@@ -594,6 +621,11 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         ka[4 * c4 + 3] = rk.w;
       }
       const uint32_t n = static_cast<uint32_t>(ti.n0) + static_cast<uint32_t>(row);
+      // Rows past the end of the unit (the next block of the head) are not written.
+      const bool valid = static_cast<int64_t>(n) < ti.n_end;
+      const bool tma_out = (ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N);
+      __nv_bfloat16* dk_row = dKg + (ti.bh * p.N + static_cast<int64_t>(n)) * D + cpart;
+      __nv_bfloat16* dv_row = dVg + (ti.bh * p.N + static_cast<int64_t>(n)) * D + cpart;
       uint32_t pt = 0, ph_ = 0, pw = 0;
       if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph_, pw);
       const int ipt = static_cast<int>(pt), iph = static_cast<int>(ph_), ipw = static_cast<int>(pw);
@@ -625,7 +657,10 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
       }
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) sts128(row_chunk(sbase + KO_DV, row, 4 * part + c4), pack8(&x[8 * c4]));
+      for (int c4 = 0; c4 < 4; ++c4) {
+        if (tma_out) sts128(row_chunk(sbase + KO_DV, row, 4 * part + c4), pack8(&x[8 * c4]));
+        else if (valid) *reinterpret_cast<uint4*>(dv_row + 8 * c4) = pack8(&x[8 * c4]);
+      }
       if (!warp_wait(&bars->ready, ph, abort_flag)) break;
       tc_fence_after();
       const float* zg = reinterpret_cast<const float*>(smem + KO_Z) + zslot * D + cpart;
@@ -663,7 +698,8 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             const float kv = (e & 1) ? bf16hi(w) : bf16lo(w);
             o8[e] = kv > 0.f ? y[8 * cc + e] + zz[e] : 0.f;
           }
-          sts128(row_chunk(sbase + KO_DK, row, 4 * part + c4), pack8(o8));
+          if (tma_out) sts128(row_chunk(sbase + KO_DK, row, 4 * part + c4), pack8(o8));
+          else if (valid) *reinterpret_cast<uint4*>(dk_row + 8 * c4) = pack8(o8);
         }
       }
       fence_proxy_async_smem();

@@ -18,6 +18,7 @@
 #include "causal_tc.cuh"
 #include "bwd_tc.cuh"
 #include "simt.cuh"
+#include "simt_ext.cuh"
 
 namespace {
 
@@ -128,7 +129,7 @@ struct PlanSet {
   Plan ps;            // state reduction
   Plan pa;            // apply
   int64_t units;      // B*H*nblk
-  size_t off_partial, off_states, off_img, off_zimg, off_tab, off_tab2, off_start, total;
+  size_t off_partial, off_states, off_img, off_zimg, off_tab, off_tab2, off_start, off_states2, off_dgamma, total;
   int64_t tab_entries;
 };
 
@@ -162,14 +163,28 @@ PlanSet make_plans(const la_problem& q, int sm_count) {
   off = align256(off + size_t(s.tab_entries) * 8);
   s.off_tab2 = off;  // the same entries in the apply kernel's layout (standard band split only)
   off = align256(off + (standard_bands(q) ? size_t(s.tab_entries) * 8 : 0));
-  s.off_start = off;  // token-causal: state carried into each CTA's range (tensor-core path)
-  off = align256(off + (s.tc ? size_t(s.ps.grid) * size_t(D * D + D) * 4 : 0));
+  s.off_start = off;  // token-causal: state carried into each CTA's range
+  off = align256(off + size_t(s.ps.grid) * size_t(D * D + D) * 4);
+  s.off_states2 = off;  // gradients on the CUDA cores: per-unit dS, dz (suffix sums over blocks)
+  off = align256(off + (s.tc ? 0 : size_t(s.units) * size_t(D * D + D) * 4));
+  s.off_dgamma = off;   // gradients: one dgamma row per CTA of the query side
+  off = align256(off + size_t(s.ps.grid) * size_t(D) * 4);
   s.total = off;
   return s;
 }
 
-// Bytes the non-token-causal paths use: everything before the token-causal start states, which
-// sit last in the layout and are read by no other path.
+// Bytes a workspace needs for every entry point: the gradients of the gated forms run on the
+// CUDA-core kernels even where the other calls take the tensor-core ones, so both layouts fit.
+size_t workspace_need(const la_problem& q, int sm_count) {
+  const PlanSet s = make_plans(q, sm_count);
+  if (!s.tc) return s.total;
+  la_problem qs = q;
+  qs.flags |= LA_FLAG_FORCE_SIMT;
+  return std::max(s.total, make_plans(qs, sm_count).total);
+}
+
+// Bytes the forward paths use: everything before the token-causal start states, which (with the
+// gradients' regions after them) sit last in the layout and are read by no forward path.
 size_t forward_bytes(const PlanSet& s) { return s.off_start; }
 
 Rope make_rope(const la_problem& q) {
@@ -259,6 +274,13 @@ int launch_k(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
+template <typename F>
+int set_smem(F* kern, size_t bytes) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) == cudaSuccess
+             ? LA_OK
+             : LA_ERR_CUDA;
+}
+
 // Optional terms of the full gated form (la_gates), as the launchers see them.
 struct Gates {
   const void* beta = nullptr;   // [B,H,N] write gate, problem dtype; null: 1
@@ -320,9 +342,10 @@ int launch_state(const PlanSet& s, const la_problem& q, const void* K, const voi
 }
 
 // `after` (optional) is called with the launch count after each kernel this queues (timing marks).
+// `reverse` (block-causal only): the image holds suffix sums over blocks instead of prefixes.
 int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk, float* z_blk, float* S_inc,
                    float* z_inc, bool img, cudaStream_t st, int* nl, bool accumulate = false,
-                   const std::function<void(int)>& after = nullptr) {
+                   const std::function<void(int)>& after = nullptr, bool reverse = false) {
   const int64_t groups = (int64_t(s.ps.d) * s.ps.d + s.ps.d) / 8;
   const int64_t threads = s.ps.BH * groups;
   if (threads == 0 || s.ps.nblk == 0) return LA_OK;
@@ -347,7 +370,8 @@ int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk
     if (after) after(*nl);
     if (S_inc || im) {
       if (launch_k(la::cmb::prefix_kernel, unsigned(cblocks), la::cmb::THREADS, 0, st, true, s.ps,
-                   static_cast<const float*>(sb), static_cast<const float*>(zb), S_inc, z_inc, im, zim))
+                   static_cast<const float*>(sb), static_cast<const float*>(zb), S_inc, z_inc, im, zim,
+                   reverse ? 1 : 0))
         return LA_ERR_CUDA;
       ++*nl;
       if (after) after(*nl);
@@ -446,14 +470,14 @@ extern "C" {
 
 size_t la_workspace_bytes_for(const la_problem* p, int sm_count) {
   if (validate(p) != LA_OK || sm_count <= 0) return 0;
-  return make_plans(*p, sm_count).total;
+  return workspace_need(*p, sm_count);
 }
 
 size_t la_workspace_bytes(const la_problem* p) {
   if (validate(p) != LA_OK) return 0;
   int sm = 0;
   if (current_sm_count(&sm) != LA_OK) return 0;
-  return make_plans(*p, sm).total;
+  return workspace_need(*p, sm);
 }
 
 int la_state_reduce(const la_problem* p, const void* K, const void* V, float* S, float* z, void* ws,
@@ -529,6 +553,22 @@ int la_block_step(const la_problem* p, const void* Q, const void* K, const void*
   return LA_OK;
 }
 
+// Dispatches a CUDA-core kernel template over the head dimension and dtype of the problem.
+#define LA_SIMT_DISPATCH(q, ...)                                           \
+  do {                                                                     \
+    if ((q).dtype == LA_BF16) {                                            \
+      using TT = __nv_bfloat16;                                            \
+      if ((q).d == 32) { constexpr int DD = 32; __VA_ARGS__; }             \
+      else if ((q).d == 64) { constexpr int DD = 64; __VA_ARGS__; }        \
+      else { constexpr int DD = 128; __VA_ARGS__; }                        \
+    } else {                                                               \
+      using TT = float;                                                    \
+      if ((q).d == 32) { constexpr int DD = 32; __VA_ARGS__; }             \
+      else if ((q).d == 64) { constexpr int DD = 64; __VA_ARGS__; }        \
+      else { constexpr int DD = 128; __VA_ARGS__; }                        \
+    }                                                                      \
+  } while (0)
+
 static int tokencausal_common(const la_problem* p, const void* Q, const void* K, const void* V, const void* G,
                               void* O, void* ws, size_t ws_bytes, cudaStream_t stream, cudaEvent_t* marks = nullptr,
                               int nmarks = 0) {
@@ -539,7 +579,6 @@ static int tokencausal_common(const la_problem* p, const void* Q, const void* K,
   if ((rc = check_ptr(Q, has_tok)) || (rc = check_ptr(K, has_tok)) || (rc = check_ptr(V, has_tok)) ||
       (rc = check_ptr(G, has_tok)) || (rc = check_ptr(O, has_tok)))
     return rc;
-  if (p->dtype != LA_BF16 || p->d != 128 || (p->flags & LA_FLAG_FORCE_SIMT)) return LA_ERR_UNSUPPORTED;
   if (!has_tok) {
     g_last_launches = 0;
     return LA_OK;
@@ -560,12 +599,28 @@ static int tokencausal_common(const la_problem* p, const void* Q, const void* K,
   mark(nl);
   uint8_t* w = static_cast<uint8_t*>(ws);
   float* start = reinterpret_cast<float*>(w + s.off_start);
-  const int64_t threads = int64_t(s.ps.grid) * ((128 * 128 + 128) / 8);
+  const int64_t threads = int64_t(s.ps.grid) * ((int64_t(p->d) * p->d + p->d) / 8);
   if (launch_k(la::cmb::start_kernel, unsigned((threads + la::cmb::THREADS - 1) / la::cmb::THREADS),
-               la::cmb::THREADS, 0, stream, true, s.ps, reinterpret_cast<const float*>(w + s.off_partial), start))
+               la::cmb::THREADS, 0, stream, s.tc, s.ps, reinterpret_cast<const float*>(w + s.off_partial), start))
     return LA_ERR_CUDA;
   ++nl;
   mark(nl);
+  const Rope rope = make_rope(*p);
+  if (!s.tc) {
+    // CUDA-core path: every dtype and head dimension.
+    const size_t smem = la::simt::causal_simt_smem(p->d);
+    LA_SIMT_DISPATCH(*p, {
+      if ((rc = set_smem(la::simt::causal_simt_kernel<DD, TT>, smem))) return rc;
+      la::simt::causal_simt_kernel<DD, TT><<<unsigned(s.ps.grid), la::simt::THREADS, smem, stream>>>(
+          static_cast<const TT*>(Q), static_cast<const TT*>(K), static_cast<const TT*>(V), static_cast<const TT*>(G),
+          static_cast<TT*>(O), s.ps, rope, static_cast<const float*>(start));
+    });
+    if ((rc = launched_ok())) return rc;
+    ++nl;
+    mark(nl);
+    g_last_launches = nl;
+    return LA_OK;
+  }
   CUtensorMap tq, tk, tv, tg, to;
   if (!make_tmap(&tq, Q, s.ps.BH, s.ps.N) || !make_tmap(&tk, K, s.ps.BH, s.ps.N) ||
       !make_tmap(&tv, V, s.ps.BH, s.ps.N) || !make_tmap(&tg, G, s.ps.BH, s.ps.N) ||
@@ -574,7 +629,6 @@ static int tokencausal_common(const la_problem* p, const void* Q, const void* K,
   auto kern = standard_bands(*p) ? la::ca::causal_tc_kernel<32, 48> : la::ca::causal_tc_kernel<-1, -1>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::ca::SMEM_BYTES) != cudaSuccess)
     return LA_ERR_CUDA;
-  const Rope rope = make_rope(*p);
   if (launch_k(kern, unsigned(s.ps.grid), la::ca::THREADS, la::ca::SMEM_BYTES, stream, true, tq, tk, tv, tg, to,
                s.ps, rope, static_cast<const float*>(start), reinterpret_cast<const float2*>(w + s.off_tab),
                reinterpret_cast<const float4*>(w + s.off_tab2)))
@@ -592,13 +646,14 @@ int la_forward_tokencausal(const la_problem* p, const void* Q, const void* K, co
   return tokencausal_common(p, Q, K, V, G, O, ws, ws_bytes, stream);
 }
 
-int la_backward_bidir(const la_problem* p, const void* Q, const void* K, const void* V, const void* G,
-                      const void* dO, void* dQ, void* dK, void* dV, void* dG, void* ws, size_t ws_bytes,
-                      cudaStream_t stream) {
+// Gradients of the operator in every form: bidirectional or block-causal (p->block_frames), with
+// the optional write gate and RMSNorm.  bf16 with d = 128 and neither gate on takes the
+// tensor-core kernels; everything else the CUDA-core kernels.
+static int backward_common(const la_problem* p, const Gates& gt, const void* Q, const void* K, const void* V,
+                           const void* G, const void* dO, void* dQ, void* dK, void* dV, void* dG, void* dbeta,
+                           float* dgamma, void* ws, size_t ws_bytes, cudaStream_t stream) {
   static_assert(la::st::TILE == la::bw::TILE, "the backward kernels walk the state kernel's tile ranges");
-  int rc = validate(p);
-  if (rc) return rc;
-  if (p->block_frames != 0) return LA_ERR_SHAPE;
+  int rc;
   const bool has_tok = elems(*p) > 0;
   const void* ins[5] = {Q, K, V, G, dO};
   void* outs[4] = {dQ, dK, dV, dG};
@@ -606,9 +661,15 @@ int la_backward_bidir(const la_problem* p, const void* Q, const void* K, const v
     if ((rc = check_ptr(x, has_tok))) return rc;
   for (void* x : outs)
     if ((rc = check_ptr(x, has_tok))) return rc;
-  if (p->dtype != LA_BF16 || p->d != 128 || (p->flags & LA_FLAG_FORCE_SIMT)) return LA_ERR_UNSUPPORTED;
+  if (gt.beta && (rc = check_ptr(dbeta, has_tok))) return rc;
+  if (gt.rms && gt.gamma && (rc = check_ptr(dgamma, true))) return rc;
+  if (gt.beta && !aligned16(gt.beta)) return LA_ERR_ALIGN;
+  if (gt.gamma && !aligned16(gt.gamma)) return LA_ERR_ALIGN;
   if (!has_tok) {
     g_last_launches = 0;
+    if (gt.rms && gt.gamma) {  // no tokens: dgamma is zero
+      if (cudaMemsetAsync(dgamma, 0, size_t(p->d) * sizeof(float), stream) != cudaSuccess) return LA_ERR_CUDA;
+    }
     return LA_OK;
   }
   int sm = 0;
@@ -616,45 +677,121 @@ int la_backward_bidir(const la_problem* p, const void* Q, const void* K, const v
   const PlanSet s = make_plans(*p, sm);
   if ((rc = check_ws(s, ws, ws_bytes))) return rc;
   int nl = 0;
-  // Forward state (S, z) and its operand image, as for the forward pass.
-  if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
-  if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
-  if ((rc = launch_combine(s, *p, ws, nullptr, nullptr, nullptr, nullptr, true, stream, &nl))) return rc;
   uint8_t* w = static_cast<uint8_t*>(ws);
   const Rope rope = make_rope(*p);
-  const bool sb = standard_bands(*p);
-  CUtensorMap tq, tg, tdo, tdq, tdg, tk, tv, tdk, tdv;
-  if (!make_tmap(&tq, Q, s.ps.BH, s.ps.N) || !make_tmap(&tg, G, s.ps.BH, s.ps.N) ||
-      !make_tmap(&tdo, dO, s.ps.BH, s.ps.N) || !make_tmap(&tdq, dQ, s.ps.BH, s.ps.N) ||
-      !make_tmap(&tdg, dG, s.ps.BH, s.ps.N) || !make_tmap(&tk, K, s.ps.BH, s.ps.N) ||
-      !make_tmap(&tv, V, s.ps.BH, s.ps.N) || !make_tmap(&tdk, dK, s.ps.BH, s.ps.N) ||
-      !make_tmap(&tdv, dV, s.ps.BH, s.ps.N))
-    return LA_ERR_CUDA;
-  // Q side: dQ, dG and the partial sums of dS, dz.
-  auto kq = sb ? la::bw::bwdq_tc_kernel<32, 48> : la::bw::bwdq_tc_kernel<-1, -1>;
-  if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, la::bw::SMEM_Q) != cudaSuccess)
-    return LA_ERR_CUDA;
-  if (launch_k(kq, unsigned(s.ps.grid), la::bw::THREADS, la::bw::SMEM_Q, stream, true, tq, tg, tdo, tdq, tdg, s.ps,
-               rope, static_cast<const uint8_t*>(w + s.off_img), reinterpret_cast<const float*>(w + s.off_zimg),
-               reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2),
-               reinterpret_cast<float*>(w + s.off_partial)))
-    return LA_ERR_CUDA;
+  const bool tc = s.tc && !gt.beta && !gt.rms;
+  if (tc) {
+    // Forward state (per unit: a head, or a block's inclusive prefix) and its operand image.
+    if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
+    if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
+    if ((rc = launch_combine(s, *p, ws, nullptr, nullptr, nullptr, nullptr, true, stream, &nl))) return rc;
+    const bool sb = standard_bands(*p);
+    CUtensorMap tq, tg, tdo, tdq, tdg, tk, tv, tdk, tdv;
+    if (!make_tmap(&tq, Q, s.ps.BH, s.ps.N) || !make_tmap(&tg, G, s.ps.BH, s.ps.N) ||
+        !make_tmap(&tdo, dO, s.ps.BH, s.ps.N) || !make_tmap(&tdq, dQ, s.ps.BH, s.ps.N) ||
+        !make_tmap(&tdg, dG, s.ps.BH, s.ps.N) || !make_tmap(&tk, K, s.ps.BH, s.ps.N) ||
+        !make_tmap(&tv, V, s.ps.BH, s.ps.N) || !make_tmap(&tdk, dK, s.ps.BH, s.ps.N) ||
+        !make_tmap(&tdv, dV, s.ps.BH, s.ps.N))
+      return LA_ERR_CUDA;
+    // Q side: dQ, dG and the partial sums of dS, dz.
+    auto kq = sb ? la::bw::bwdq_tc_kernel<32, 48> : la::bw::bwdq_tc_kernel<-1, -1>;
+    if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, la::bw::SMEM_Q) != cudaSuccess)
+      return LA_ERR_CUDA;
+    if (launch_k(kq, unsigned(s.ps.grid), la::bw::THREADS, la::bw::SMEM_Q, stream, true, tq, tg, tdo, tdq, tdg,
+                 s.ps, rope, static_cast<const uint8_t*>(w + s.off_img), reinterpret_cast<const float*>(w + s.off_zimg),
+                 reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2),
+                 reinterpret_cast<float*>(w + s.off_partial), static_cast<__nv_bfloat16*>(dQ),
+                 static_cast<__nv_bfloat16*>(dG)))
+      return LA_ERR_CUDA;
+    ++nl;
+    // dS, dz summed in fixed order into the operand image (reusing the state image's space); in
+    // block-causal mode a key of block b feeds the states of blocks b' >= b, so its image holds
+    // the suffix sums over blocks.
+    PlanSet s2 = s;
+    s2.ps.zparts = la::bw::ZPARTS;
+    if ((rc = launch_combine(s2, *p, ws, nullptr, nullptr, nullptr, nullptr, true, stream, &nl, false, nullptr,
+                             /*reverse=*/true)))
+      return rc;
+    // K side: dK, dV.
+    auto kk = sb ? la::bw::bwdk_tc_kernel<32, 48> : la::bw::bwdk_tc_kernel<-1, -1>;
+    if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, la::bw::SMEM_K) != cudaSuccess)
+      return LA_ERR_CUDA;
+    if (launch_k(kk, unsigned(s.ps.grid), la::bw::THREADS, la::bw::SMEM_K, stream, true, tk, tv, tdk, tdv, s.ps,
+                 rope, static_cast<const uint8_t*>(w + s.off_img), reinterpret_cast<const float*>(w + s.off_zimg),
+                 reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2),
+                 static_cast<__nv_bfloat16*>(dK), static_cast<__nv_bfloat16*>(dV)))
+      return LA_ERR_CUDA;
+    ++nl;
+    g_last_launches = nl;
+    return LA_OK;
+  }
+  // CUDA-core path (fp32 states throughout).
+  la_problem qs = *p;
+  qs.flags |= LA_FLAG_FORCE_SIMT;
+  const PlanSet sp = make_plans(qs, sm);  // the CUDA-core kernels' tile ranges (32-token tiles)
+  if ((rc = check_ws(sp, ws, ws_bytes))) return rc;
+  float* partial = reinterpret_cast<float*>(w + sp.off_partial);
+  float* Sf = reinterpret_cast<float*>(w + sp.off_states);
+  float* zf = Sf + sp.units * p->d * p->d;
+  float* dSf = reinterpret_cast<float*>(w + sp.off_states2);
+  float* dzf = dSf + sp.units * p->d * p->d;
+  float* dgp = reinterpret_cast<float*>(w + sp.off_dgamma);
+  const int64_t groups = (int64_t(p->d) * p->d + p->d) / 8;
+  const unsigned ublocks = unsigned((sp.units * groups + la::cmb::THREADS - 1) / la::cmb::THREADS);
+  const unsigned hblocks = unsigned((sp.ps.BH * groups + la::cmb::THREADS - 1) / la::cmb::THREADS);
+  // Forward states: per-unit sums, then (block-causal) the inclusive prefix over blocks.
+  if ((rc = launch_state(sp, qs, K, V, ws, stream, &nl, gt.beta))) return rc;
+  la::cmb::blocksum_kernel<<<ublocks, la::cmb::THREADS, 0, stream>>>(sp.ps, partial, Sf, zf);
   ++nl;
-  // dS, dz summed in fixed order into the operand image (reusing the state image's space).
-  PlanSet s2 = s;
-  s2.ps.zparts = la::bw::ZPARTS;
-  if ((rc = launch_combine(s2, *p, ws, nullptr, nullptr, nullptr, nullptr, true, stream, &nl))) return rc;
-  // K side: dK, dV.
-  auto kk = sb ? la::bw::bwdk_tc_kernel<32, 48> : la::bw::bwdk_tc_kernel<-1, -1>;
-  if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, la::bw::SMEM_K) != cudaSuccess)
-    return LA_ERR_CUDA;
-  if (launch_k(kk, unsigned(s.ps.grid), la::bw::THREADS, la::bw::SMEM_K, stream, true, tk, tv, tdk, tdv, s.ps, rope,
-               static_cast<const uint8_t*>(w + s.off_img), reinterpret_cast<const float*>(w + s.off_zimg),
-               reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2)))
-    return LA_ERR_CUDA;
+  if (sp.ps.nblk > 1) {
+    la::cmb::scan_kernel<<<hblocks, la::cmb::THREADS, 0, stream>>>(sp.ps.BH, sp.ps.nblk, p->d, Sf, zf, 0);
+    ++nl;
+  }
+  if ((rc = launched_ok())) return rc;
+  // Query side.
+  const size_t smq = la::simt::bwdq_simt_smem(p->d);
+  LA_SIMT_DISPATCH(*p, {
+    if ((rc = set_smem(la::simt::bwdq_simt_kernel<DD, TT>, smq))) return rc;
+    la::simt::bwdq_simt_kernel<DD, TT><<<unsigned(sp.ps.grid), la::simt::THREADS, smq, stream>>>(
+        static_cast<const TT*>(Q), static_cast<const TT*>(G), static_cast<const TT*>(dO), Sf, zf,
+        static_cast<TT*>(dQ), static_cast<TT*>(dG), sp.ps, rope, gt.rms ? 1 : 0, gt.gamma, gt.norm_eps, partial,
+        dgp);
+  });
   ++nl;
+  // dS, dz per unit, then (block-causal) the suffix sums over blocks.
+  la::cmb::blocksum_kernel<<<ublocks, la::cmb::THREADS, 0, stream>>>(sp.ps, partial, dSf, dzf);
+  ++nl;
+  if (sp.ps.nblk > 1) {
+    la::cmb::scan_kernel<<<hblocks, la::cmb::THREADS, 0, stream>>>(sp.ps.BH, sp.ps.nblk, p->d, dSf, dzf, 1);
+    ++nl;
+  }
+  if ((rc = launched_ok())) return rc;
+  // Key side.
+  const size_t smk = la::simt::bwdk_simt_smem(p->d);
+  LA_SIMT_DISPATCH(*p, {
+    if ((rc = set_smem(la::simt::bwdk_simt_kernel<DD, TT>, smk))) return rc;
+    la::simt::bwdk_simt_kernel<DD, TT><<<unsigned(sp.ps.grid), la::simt::THREADS, smk, stream>>>(
+        static_cast<const TT*>(K), static_cast<const TT*>(V), static_cast<const TT*>(gt.beta), dSf, dzf,
+        static_cast<TT*>(dK), static_cast<TT*>(dV), static_cast<TT*>(dbeta), sp.ps, rope);
+  });
+  ++nl;
+  if (gt.rms && gt.gamma) {
+    la::simt::dgamma_sum_kernel<<<unsigned((p->d + la::simt::THREADS - 1) / la::simt::THREADS), la::simt::THREADS, 0,
+                                  stream>>>(sp.ps.grid, p->d, dgp, dgamma);
+    ++nl;
+  }
+  if ((rc = launched_ok())) return rc;
   g_last_launches = nl;
   return LA_OK;
+}
+
+int la_backward_bidir(const la_problem* p, const void* Q, const void* K, const void* V, const void* G,
+                      const void* dO, void* dQ, void* dK, void* dV, void* dG, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  if (p->block_frames != 0) return LA_ERR_SHAPE;
+  return backward_common(p, Gates(), Q, K, V, G, dO, dQ, dK, dV, dG, nullptr, nullptr, ws, ws_bytes, stream);
 }
 
 int la_state_scan(const la_problem* p, float* S, float* z, cudaStream_t stream) {
@@ -802,6 +939,16 @@ int la_forward_gated(const la_problem* p, const la_gates* gates, const void* Q, 
   Gates gt;
   if ((rc = read_gates(gates, &gt))) return rc;
   return forward_common(p, Q, K, V, G, O, S_incl, z_incl, ws, ws_bytes, stream, nullptr, 0, gt);
+}
+
+int la_backward(const la_problem* p, const la_gates* gates, const void* Q, const void* K, const void* V,
+                const void* G, const void* dO, void* dQ, void* dK, void* dV, void* dG, void* dbeta, float* dgamma,
+                void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  Gates gt;
+  if ((rc = read_gates(gates, &gt))) return rc;
+  return backward_common(p, gt, Q, K, V, G, dO, dQ, dK, dV, dG, dbeta, dgamma, ws, ws_bytes, stream);
 }
 
 int la_forward_marked(const la_problem* p, const la_gates* gates, const void* Q, const void* K, const void* V,

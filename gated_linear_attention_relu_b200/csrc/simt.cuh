@@ -396,12 +396,13 @@ blocksum_kernel(const Plan p, const float* __restrict__ partial, float* __restri
 }
 
 // Block-causal combine, second pass: inclusive prefix over the blocks of every head, from the
-// per-block states of the first pass; writes the inclusive states and/or the operand image.
+// per-block states of the first pass (with `reverse`, the suffix sums over blocks b' >= b, which
+// the key side of the gradients reads); writes the resulting states and/or the operand image.
 // One thread per (head, group of 8 elements); the loads of different blocks are independent, so
 // they overlap.
 __global__ void __launch_bounds__(THREADS)
 prefix_kernel(const Plan p, const float* __restrict__ S_blk, const float* __restrict__ z_blk, float* S_inc,
-              float* z_inc, uint8_t* img, float* zimg) {
+              float* z_inc, uint8_t* img, float* zimg, int reverse) {
   pdl_trigger();
   pdl_wait();
   const int D = p.d;
@@ -414,7 +415,8 @@ prefix_kernel(const Plan p, const float* __restrict__ S_blk, const float* __rest
 #pragma unroll
   for (int e = 0; e < 8; ++e) run[e] = 0.f;
 #pragma unroll 4
-  for (int64_t blk = 0; blk < p.nblk; ++blk) {
+  for (int64_t i = 0; i < p.nblk; ++i) {
+    const int64_t blk = reverse ? p.nblk - 1 - i : i;  // reverse: suffix sums over blocks >= blk
     const int64_t u = bh * p.nblk + blk;
     const float* src = (e0 < D * D) ? S_blk + u * D * D + e0 : z_blk + u * D + (e0 - D * D);
     const float4 a = reinterpret_cast<const float4*>(src)[0], b = reinterpret_cast<const float4*>(src)[1];
@@ -463,9 +465,10 @@ start_kernel(const Plan p, const float* __restrict__ partial, float* __restrict_
   d4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
 }
 
-// In-place inclusive prefix over blocks of [B*H][nblk][D*D] and [B*H][nblk][D].
+// In-place inclusive prefix over blocks of [B*H][nblk][D*D] and [B*H][nblk][D] (with `reverse`,
+// the suffix sums over blocks b' >= b).
 __global__ void __launch_bounds__(THREADS)
-scan_kernel(int64_t BH, int64_t nblk, int D, float* S, float* z) {
+scan_kernel(int64_t BH, int64_t nblk, int D, float* S, float* z, int reverse = 0) {
   const int groups = (D * D + D) / 8;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
   const int64_t bh = idx / groups;
@@ -474,7 +477,8 @@ scan_kernel(int64_t BH, int64_t nblk, int D, float* S, float* z) {
   float run[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) run[e] = 0.f;
-  for (int64_t blk = 0; blk < nblk; ++blk) {
+  for (int64_t i = 0; i < nblk; ++i) {
+    const int64_t blk = reverse ? nblk - 1 - i : i;
     const int64_t u = bh * nblk + blk;
     float* src = (e0 < D * D) ? S + u * D * D + e0 : z + u * D + (e0 - D * D);
     float4* s4 = reinterpret_cast<float4*>(src);

@@ -42,18 +42,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Non-blocking test: has the phase of parity `parity` of `bar` completed?
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -67,14 +55,44 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits until the phase of parity `parity` of `bar` has completed.  Returns false if the CTA's
-// abort flag is raised (by this or another thread) or the wait exceeds LA_WAIT_LIMIT_NS.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Back-off between two tests of a wait, by how long the wait usually lasts: waits for data that is
+// usually in flight re-test at once (the hardware test itself pauses the thread briefly); a
+// single-thread producer or store loop sleeps a little between tests; a wait that spans most of
+// a kernel (a drain waiting for a unit's last tile) sleeps long.  A sleeping warp issues nothing,
+// so a waiting warp does not take issue slots (and power) from the warps that work.
+#ifndef LA_SLEEP_PROD
+#define LA_SLEEP_PROD 64u
+#endif
+#ifndef LA_SLEEP_MATH
+#define LA_SLEEP_MATH 0u
+#endif
+#ifndef LA_SLEEP_LONG
+#define LA_SLEEP_LONG 1000u
+#endif
+
+// Waits until the phase of parity `parity` of `bar` has completed, sleeping `sleep_ns` between
+// tests (0: re-test at once).  Returns false if the CTA's abort flag is raised (by this or another
+// thread) or the wait exceeds LA_WAIT_LIMIT_NS.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u) {
+    if ((i & (sleep_ns ? 15u : 255u)) == 0u) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > LA_WAIT_LIMIT_NS) {
         *abort_flag = 1;
@@ -87,18 +105,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // Warp-uniform wait: every lane polls, and the warp proceeds only if every lane saw the phase
 // complete, so lanes never split across a later .sync.aligned instruction.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  bool ok = mbar_wait(bar, parity, abort_flag);
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t sleep_ns = 0) {
+  bool ok = mbar_wait(bar, parity, abort_flag, sleep_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
 // Same as mbar_wait, but ignores the abort flag (used while draining copies already in flight).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
+    __nanosleep(64);
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u && globaltimer_ns() - t0 > LA_WAIT_LIMIT_NS) {
+    if ((i & 15u) == 0u && globaltimer_ns() - t0 > LA_WAIT_LIMIT_NS) {
       atomicOr(&g_la_error, ERR_WAIT_TIMEOUT);
       return false;
     }

@@ -144,7 +144,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const int64_t i = g - g0;
         const int s = static_cast<int>(i % nst);
         const uint32_t ph = static_cast<uint32_t>((i / nst) & 1);
-        if (!mbar_wait(&emptyb[s], ph ^ 1u, abort_flag)) break;
+        if (!mbar_wait(&emptyb[s], ph ^ 1u, abort_flag, LA_SLEEP_PROD)) break;
         const TileInfo ti = tile_info(p, g);
         uint8_t* buf = ring + s * BUF;
         mbar_arrive_expect_tx(&fullb[s], BUF);
@@ -175,7 +175,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         prev_unit = u;
         if (first) {
           ++seg;
-          if (!mbar_wait(&bars->accempty[seg & 1], static_cast<uint32_t>(((seg >> 1) & 1) ^ 1), abort_flag)) break;
+          if (!mbar_wait(&bars->accempty[seg & 1], static_cast<uint32_t>(((seg >> 1) & 1) ^ 1), abort_flag, LA_SLEEP_PROD)) break;
         }
         if (!mbar_wait(&bars->aready[s], ph, abort_flag)) break;
         if (!mbar_wait(&bars->vfull[sv], phv, abort_flag)) break;
@@ -241,7 +241,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const uint32_t ph = static_cast<uint32_t>((i / KST) & 1);
       const TileInfo ti = tile_info(p, g);
       const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != ti.unit);
-      if (!warp_wait(&bars->kfull[s], ph, abort_flag)) break;
+      if (!warp_wait(&bars->kfull[s], ph, abort_flag, LA_SLEEP_MATH)) break;
       const int row0 = GROUP_ROWS * tg + rg;
       const uint32_t base = sbase + OFF_K + s * BUF + chunk_off + static_cast<uint32_t>(row0 * 128);
       const uint32_t n0 = static_cast<uint32_t>(ti.n0) + row0;
@@ -349,7 +349,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     const int row = quarter * 32 + lane;
     const int64_t nseg = (g1 > g0) ? unit_of_tile(p, g1 - 1) - u_first + 1 : 0;
     for (int64_t k = 0; k < nseg; ++k) {
-      if (!warp_wait(&bars->accfull[k & 1], static_cast<uint32_t>((k >> 1) & 1), abort_flag)) break;
+      if (!warp_wait(&bars->accfull[k & 1], static_cast<uint32_t>((k >> 1) & 1), abort_flag, LA_SLEEP_LONG)) break;
       tc_fence_after();
       float* dst = partial + (c * p.maxseg + k) * SLOT + static_cast<int64_t>(row) * D;
       const uint32_t taddr = tmem + static_cast<uint32_t>(k & 1) * 128u + (static_cast<uint32_t>(quarter * 32) << 16);

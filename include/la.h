@@ -147,8 +147,8 @@ int la_forward_blockcausal(const la_problem* p, const void* Q, const void* K, co
  * of a head reads the states of tokens 0..n in the flattened order n = (t*Hh + h)*W + w:
  *   O_n = (phi(Q_n) S_{<=n}) / (ReLU(Q_n) . z_{<=n} + eps) * sigmoid(G_n),
  *   S_{<=n} = sum_{m<=n} phi(K_m)^T V_m,  z_{<=n} = sum_{m<=n} ReLU(K_m).
- * p->block_frames must be 0.  Tensor-core path only in this version: bf16, d = 128, no
- * LA_FLAG_FORCE_SIMT; anything else returns LA_ERR_UNSUPPORTED.  Q, K, V, G, O: [B,H,N,d]. */
+ * p->block_frames must be 0.  bf16 with d = 128 runs on the tensor cores; fp32, d = 32 / 64 and
+ * LA_FLAG_FORCE_SIMT on the CUDA cores (4 kernels either way).  Q, K, V, G, O: [B,H,N,d]. */
 int la_forward_tokencausal(const la_problem* p, const void* Q, const void* K, const void* V,
                            const void* G, void* O, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream);
@@ -159,9 +159,9 @@ int la_forward_tokencausal(const la_problem* p, const void* Q, const void* K, co
  *   dG = dO y s (1 - s),  dnum = dO s / den,  dden = -(dO s . y) / den,
  *   dS = sum_n phi(Q_n)^T dnum_n,  dz = sum_n dden_n ReLU(Q_n),
  *   dQ = [Q > 0] (RoPE^T(dnum S^T) + dden z),  dV = phi(K) dS,  dK = [K > 0] (RoPE^T(V dS^T) + dz)
- * (the chain rule through SANA-Video 2.0, Eq. (1)).  p->block_frames must be 0.  Tensor-core
- * path only in this version: bf16, d = 128, no LA_FLAG_FORCE_SIMT; else LA_ERR_UNSUPPORTED.
- * Recomputes the forward state; queues 6 kernels. */
+ * (the chain rule through SANA-Video 2.0, Eq. (1)).  p->block_frames must be 0.  bf16 with
+ * d = 128 runs on the tensor cores (6 kernels); fp32, d = 32 / 64 and LA_FLAG_FORCE_SIMT on the
+ * CUDA cores.  Recomputes the forward state. */
 int la_backward_bidir(const la_problem* p, const void* Q, const void* K, const void* V,
                       const void* G, const void* dO, void* dQ, void* dK, void* dV, void* dG,
                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
@@ -187,6 +187,28 @@ typedef struct {
 int la_forward_gated(const la_problem* p, const la_gates* gates, const void* Q, const void* K,
                      const void* V, const void* G, void* O, float* S_incl, float* z_incl,
                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Gradients of the operator in every form la_forward_gated computes: bidirectional
+ * (p->block_frames == 0) or block-causal, with the optional write gate beta and RMSNorm of
+ * `gates` (NULL: none).  Given dO, writes dQ, dK, dV, dG ([B,H,N,d], problem dtype) and
+ *   dbeta  [B,H,N] (problem dtype): required when gates->beta is given, else ignored;
+ *   dgamma [d] fp32, summed over all tokens and heads: required when gates->rms_norm is set and
+ *          gates->gamma is given, else ignored.
+ * Chain rule (the reading of SANA-Video 2.0, Eq. (1) and SANA-Video Sec. 3.4): with s = sigmoid(G),
+ * y = num / den, u = RMSNorm(y) (u = y without), r = sqrt(mean(y^2) + norm_eps), yh = y / r:
+ *   dG = dO u s (1 - s),  du = dO s,  dgamma = sum du yh,
+ *   dy = (dyh - yh (yh . dyh) / d) / r with dyh = du gamma   (dy = du without RMSNorm),
+ *   dnum = dy / den,  dden = -(dy . y) / den,
+ *   dS_b = sum_{n in block b} phi(Q_n)^T dnum_n,  dz_b = sum_{n in block b} dden_n ReLU(Q_n),
+ *   dQ = [Q > 0] (RoPE^T(dnum S_b^T) + dden z_b)   (S_b, z_b: the inclusive state token n reads),
+ *   and with the suffix sums dS^c = sum_{b >= c} dS_b, dz^c likewise (a key of block c feeds
+ *   the states of blocks c and later), for a key of block c:
+ *   dV = beta phi(K) dS^c,  dK = [K > 0] (RoPE^T(beta V dS^cT) + dz^c),  dbeta = phi(K) . (dS^c V).
+ * bf16 with d = 128 and neither beta nor RMSNorm runs on the tensor cores; every other case on
+ * the CUDA cores.  The workspace is la_workspace_bytes() (which covers both). */
+int la_backward(const la_problem* p, const la_gates* gates, const void* Q, const void* K, const void* V,
+                const void* G, const void* dO, void* dQ, void* dK, void* dV, void* dG, void* dbeta,
+                float* dgamma, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* The whole operator (bidirectional if p->block_frames == 0, else block-causal, with the
  * same arguments as la_forward_gated; gates may be NULL; token-causal, as la_forward_tokencausal,

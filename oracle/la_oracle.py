@@ -364,16 +364,21 @@ def head_backward_gated(q, k, v, g, do, pos, bands, base, eps, block_frames=0, b
     nblk = int(blk.max()) + 1 if N else 0
     qp, kp = relu(q), relu(k)
     qr, kr = rope3d(qp, pos, bands, base), rope3d(kp, pos, bands, base)
-    # inclusive states per block
-    S = np.zeros((nblk, d, d))
-    z = np.zeros((nblk, d))
+    # inclusive states per block: each block's own sums, then the running sum over blocks
+    Sb = np.zeros((nblk, d, d))
+    zb = np.zeros((nblk, d))
     for b in range(nblk):
-        sel = blk <= b
-        S[b] = (kr[sel] * bt[sel][:, None]).T @ v[sel]
-        z[b] = kp[sel].sum(axis=0)
-    Sn, zn = S[blk], z[blk]                      # the state each token reads
-    num = np.einsum("ni,nij->nj", qr, Sn)
-    den = np.einsum("ni,ni->n", qp, zn) + float(eps)
+        sel = blk == b
+        Sb[b] = (kr[sel] * bt[sel][:, None]).T @ v[sel]
+        zb[b] = kp[sel].sum(axis=0)
+    S = np.cumsum(Sb, axis=0)
+    z = np.cumsum(zb, axis=0)
+    num = np.empty((N, d))
+    den = np.empty(N)
+    for b in range(nblk):                        # each token reads its own block's state
+        sel = blk == b
+        num[sel] = qr[sel] @ S[b]
+        den[sel] = qp[sel] @ z[b] + float(eps)
     y = num / den[:, None]
     sg = sigmoid(g)
     if rms is not None:
@@ -403,9 +408,16 @@ def head_backward_gated(q, k, v, g, do, pos, bands, base, eps, block_frames=0, b
         dzb[b] = qp[sel].T @ dden[sel]
     dSs = np.cumsum(dSb[::-1], axis=0)[::-1]     # suffix sums over blocks
     dzs = np.cumsum(dzb[::-1], axis=0)[::-1]
-    dq = (q > 0) * (rope3d_transpose(np.einsum("nj,nij->ni", dnum, Sn), pos, bands, base) + dden[:, None] * zn)
-    P = np.einsum("nj,nij->ni", v, dSs[blk])     # v_m dS^T, row by row
-    dv = bt[:, None] * np.einsum("ni,nij->nj", kr, dSs[blk])
+    dphq = np.empty((N, d))                      # dnum S_b^T
+    P = np.empty((N, d))                         # v dS^{b T}
+    kS = np.empty((N, d))                        # phi(k) dS^b
+    for b in range(nblk):
+        sel = blk == b
+        dphq[sel] = dnum[sel] @ S[b].T
+        P[sel] = v[sel] @ dSs[b].T
+        kS[sel] = kr[sel] @ dSs[b]
+    dq = (q > 0) * (rope3d_transpose(dphq, pos, bands, base) + dden[:, None] * z[blk])
+    dv = bt[:, None] * kS
     dk = (k > 0) * (rope3d_transpose(bt[:, None] * P, pos, bands, base) + dzs[blk])
     dbeta = np.sum(kr * P, axis=1) if beta is not None else None
     return dq, dk, dv, dg, dbeta, dgamma

@@ -106,23 +106,32 @@ def test_state_update_rejects_block_causal_problems_before_cuda():
     assert lib.la_state_update(ctypes.byref(cp), None, 16, 16, 16, 16, 1 << 30, None) == 1
 
 
-def test_tokencausal_rejects_unsupported_problems_before_cuda():
+def test_tokencausal_rejects_block_causal_problems_before_cuda():
     lib = la.load()
-    for kw, status in ((dict(dtype="f32"), 5), (dict(d=64, bands=(16, 24, 24)), 5), (dict(force_simt=True), 5),
-                       (dict(block_frames=1), 2)):
+    for kw, status in ((dict(block_frames=1), 2), (dict(dtype="f32", block_frames=2), 2)):
         args = dict(B=1, H=2, T=3, Hh=4, W=5)
         args.update(kw)
         cp = la.Problem(**args).c()
         assert lib.la_forward_tokencausal(ctypes.byref(cp), 16, 16, 16, 16, 16, 16, 1 << 30, None) == status
 
 
-def test_backward_rejects_unsupported_problems_before_cuda():
+def test_backward_rejects_bad_arguments_before_cuda():
     lib = la.load()
-    for kw, status in ((dict(dtype="f32"), 5), (dict(d=32, bands=(8, 12, 12)), 5), (dict(block_frames=1), 2)):
+    for kw, status in ((dict(block_frames=1), 2), (dict(d=48, bands=(16, 16, 16)), 5)):
         args = dict(B=1, H=2, T=3, Hh=4, W=5)
         args.update(kw)
         cp = la.Problem(**args).c()
         assert lib.la_backward_bidir(ctypes.byref(cp), *([16] * 9), 16, 1 << 30, None) == status
+    # the general entry point: dbeta is required with a write gate, dgamma with an RMSNorm weight
+    cp = la.Problem(B=1, H=2, T=3, Hh=4, W=5, block_frames=1).c()
+    g = bnd.LaGates(16, None, 1e-6, 0)
+    assert lib.la_backward(ctypes.byref(cp), ctypes.byref(g), *([16] * 9), None, None, 16, 1 << 30, None) == 1
+    g = bnd.LaGates(None, 16, 1e-6, 1)
+    assert lib.la_backward(ctypes.byref(cp), ctypes.byref(g), *([16] * 9), None, None, 16, 1 << 30, None) == 1
+    g = bnd.LaGates(None, 16, 1e-6, 1)
+    assert lib.la_backward(ctypes.byref(cp), ctypes.byref(g), *([16] * 9), None, 24, 16, 1 << 30, None) == 4
+    g = bnd.LaGates(None, None, 1e-6, 3)
+    assert lib.la_backward(ctypes.byref(cp), ctypes.byref(g), *([16] * 9), None, None, 16, 1 << 30, None) == 5
 
 
 def test_static_entry_point_checks_pointers_before_cuda():
@@ -135,13 +144,3 @@ def test_static_entry_point_checks_pointers_before_cuda():
         assert lib.la_forward_bidir_static(ctypes.byref(cp), 16, 16, 16, 16, 24, None) == 4
     cp = la.Problem(B=1, H=2, T=3, Hh=4, W=5, block_frames=1).c()
     assert lib.la_forward_bidir_static(ctypes.byref(cp), 16, 16, 16, 16, 16, None) == 2
-
-
-@pytest.mark.parametrize("T", [21, 241])
-def test_static_scratch_fits_720p_on_a_b200(T):
-    # The allocation-free forward uses the workspace layout without its last region, the
-    # token-causal start states (one (d*d + d)-float state per CTA, i.e. per SM here).
-    p = la.Problem(B=1, H=32, T=T, Hh=45, W=80)
-    sm = 148
-    need = la.workspace_bytes(p, sm_count=sm) - sm * (128 * 128 + 128) * 4
-    assert 0 < need <= 32 << 20

@@ -48,20 +48,22 @@ def test_backward_all_elements(w):
             assert e <= tol_for(w.dtype), (w.name, flat, name, e)
 
 
-def test_backward_720p_5s_sampled_rows():
-    w = wl.WORKLOADS["720p_5s"]
+@pytest.mark.parametrize("wname,heads", [("720p_5s", (0, 31)), ("720p_5s_b2", (0, 63))])
+def test_backward_full_size_sampled_rows(wname, heads):
+    w = wl.WORKLOADS[wname]
     (Q, K, V, G, dO), grads = _run(w)
     pos = orc.grid_positions(w.T, w.Hh, w.W)
     rng = np.random.default_rng(5)
     rows = np.unique(np.concatenate([rng.choice(w.N, 3000, replace=False), np.arange(130), np.arange(w.N - 130, w.N)]))
-    for h in (0, w.H - 1):
-        refs = orc.head_backward(to64(Q[0, h]), to64(K[0, h]), to64(V[0, h]), to64(G[0, h]), to64(dO[0, h]), pos,
+    for flat in heads:
+        b, h = divmod(flat, w.H)
+        refs = orc.head_backward(to64(Q[b, h]), to64(K[b, h]), to64(V[b, h]), to64(G[b, h]), to64(dO[b, h]), pos,
                                  w.bands, w.rope_base, w.eps)
         idx = torch.as_tensor(rows, device="cuda")
         for name, got, ref in zip(NAMES, grads, refs):
-            e = rel_err(to64(got[0, h][idx]), ref[rows])
-            print(f"backward 720p_5s head {h} {name}: {e:.2e}")
-            assert e <= tol_for(w.dtype), (h, name, e)
+            e = rel_err(to64(got[b, h][idx]), ref[rows])
+            print(f"backward {wname} head {flat} {name}: {e:.2e}")
+            assert e <= tol_for(w.dtype), (flat, name, e)
 
 
 def test_backward_deterministic():

@@ -35,10 +35,21 @@ def _oracle(w, Q, K, V, G, b, h, rows=None):
                                 w.rope_base, w.eps, rows=rows)
 
 
-@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+SIMT_CASES = [
+    # CUDA-core kernels: fp32 (the tiny fp32 config's tolerance), small head dimensions, and the
+    # bf16 d = 128 problem forced onto them; heads split over many CTAs and ragged tiles
+    wl.WORKLOADS["tiny_f32"],
+    wl.custom("tcs_f32_d64", B=1, H=2, T=3, Hh=5, W=37, d=64, bands=(16, 24, 24), dtype="f32"),
+    wl.custom("tcs_f32_split", B=2, H=2, T=8, Hh=10, W=40, d=32, bands=(8, 12, 12), dtype="f32"),
+    wl.custom("tcs_bf16_d32", B=1, H=3, T=3, Hh=5, W=37, d=32, bands=(8, 12, 12)),
+    wl.custom("tcs_forced", B=1, H=2, T=3, Hh=5, W=37),
+]
+
+
+@pytest.mark.parametrize("w", CASES + SIMT_CASES, ids=lambda w: w.name)
 def test_tokencausal_all_elements(w):
     Q, K, V, G = wl.generate(w, "cuda")
-    p = la.Problem.from_workload(w)
+    p = la.Problem.from_workload(w, force_simt=w.name == "tcs_forced")
     O = la.forward_tokencausal(p, Q, K, V, G)
     torch.cuda.synchronize()
     assert la.device_error() == 0
@@ -50,21 +61,25 @@ def test_tokencausal_all_elements(w):
         assert e <= tol_for(w.dtype), (w.name, flat, e)
 
 
-def test_tokencausal_720p_5s_sampled():
-    w = wl.WORKLOADS["720p_5s"]
+@pytest.mark.parametrize("name,heads", [("720p_5s", (0, 31)), ("720p_5s_b2", (0, 63)), ("720p_60s", (0, 31))])
+def test_tokencausal_full_size_sampled(name, heads):
+    w = wl.WORKLOADS[name]
     Q, K, V, G = wl.generate(w, "cuda")
     p = la.Problem.from_workload(w)
     O = la.forward_tokencausal(p, Q, K, V, G)
     torch.cuda.synchronize()
     assert la.device_error() == 0
     assert torch.isfinite(O).all()
-    for flat in (0, w.H - 1):
+    for flat in heads:
+        b, h = divmod(flat, w.H)
         toks = sample_tokens(w, 2000, seed=flat)
-        ref = _oracle(w, Q, K, V, G, 0, flat, rows=toks)
-        got = to64(O[0, flat][torch.as_tensor(toks, device=O.device)])
+        ref = _oracle(w, Q, K, V, G, b, h, rows=toks)
+        got = to64(O[b, h][torch.as_tensor(toks, device=O.device)])
         e = rel_err(got, ref)
-        print(f"token-causal 720p_5s head {flat}: O {e:.2e}")
+        print(f"token-causal {name} head {flat}: O {e:.2e}")
         assert e <= tol_for(w.dtype)
+    del Q, K, V, G, O
+    torch.cuda.empty_cache()
 
 
 def test_tokencausal_deterministic_and_last_token_bidirectional():

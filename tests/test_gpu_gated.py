@@ -78,6 +78,12 @@ def test_gated_720p_5s_sampled():
     _check(w, True, True, tokens=2000, heads=[0, w.H - 1])
 
 
+def test_gated_720p_60s_sampled():
+    w = wl.WORKLOADS["720p_60s"]
+    _check(w, True, True, tokens=3000, heads=[0, w.H - 1])
+    torch.cuda.empty_cache()
+
+
 def test_gated_blockcausal_sampled():
     w = wl.WORKLOADS["blockcausal"]
     _check(w, True, True, tokens=3000, heads=[5])

@@ -48,6 +48,19 @@ def test_static_scratch_forward_matches_workspace_forward_twice():
     assert err <= TOL_BF16, (w.name, err)
 
 
+def test_static_scratch_takes_the_720p_5s_problem():
+    # B = 1, H = 32 on the 720p/5s latent grid fits the fixed scratch on a B200 (148 SMs).
+    w = wl.WORKLOADS["720p_5s"]
+    Q, K, V, G = wl.generate(w, "cuda")
+    p = la.Problem.from_workload(w)
+    ref = la.forward_bidir(p, Q, K, V, G)
+    O = torch.empty_like(Q)
+    assert _static_call(p, Q, K, V, G, O) == 0
+    torch.cuda.synchronize()
+    assert la.device_error() == 0
+    assert torch.equal(O, ref)
+
+
 def test_static_scratch_rejects_problems_that_do_not_fit():
     p = la.Problem(B=8, H=64, T=241, Hh=45, W=80)
     assert la.workspace_bytes(p) > (32 << 20)
