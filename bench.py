@@ -48,7 +48,8 @@ def parse():
     ap.add_argument("--causal", action="store_true",
                     help="token-causal operator (token n reads tokens 0..n) on a bidirectional workload's shape")
     ap.add_argument("--backward", action="store_true",
-                    help="gradients of the bidirectional operator (dQ, dK, dV, dG from dO)")
+                    help="gradients (dQ, dK, dV, dG from dO; with --gated also dbeta, dgamma) of the "
+                         "workload's form, bidirectional or block-causal")
     ap.add_argument("--stream", action="store_true",
                     help="block-causal workloads: one la_block_step call per block on a carried cache, "
                          "as a block-autoregressive generator runs")
@@ -141,7 +142,8 @@ def oracle_sample(w, seconds, steps=None, warmup=0, mode="forward"):
 
     ``mode`` picks the oracle of what the GPU run measures: "forward" (bidirectional or
     block-causal, as the workload says), "gated" (write gate and RMSNorm), "causal"
-    (token-causal) or "backward" (gradients of the bidirectional form)."""
+    (token-causal), "backward" (gradients, bidirectional or block-causal) or "backward_gated"
+    (gradients of the gated form)."""
     import numpy as np
 
     import oracle as orc
@@ -150,10 +152,10 @@ def oracle_sample(w, seconds, steps=None, warmup=0, mode="forward"):
     one = w.with_(B=1, H=1)
     Q, K, V, G = (t.float().numpy().astype(np.float64)[0, 0] for t in wl.generate(one, "cpu"))
     pos = orc.grid_positions(w.T, w.Hh, w.W)
-    if mode == "gated":
+    if mode in ("gated", "backward_gated"):
         beta, gamma = (t.float().numpy().astype(np.float64) for t in wl.generate_gates(one, "cpu"))
         beta = beta[0, 0]
-    if mode == "backward":
+    if mode in ("backward", "backward_gated"):
         dO = wl.generate_grad(one, "cpu").float().numpy().astype(np.float64)[0, 0]
     # The token-causal oracle walks rows one by one in Python: time it on a fixed sample of rows
     # (it still carries the state over every token).
@@ -163,8 +165,12 @@ def oracle_sample(w, seconds, steps=None, warmup=0, mode="forward"):
     def run():
         if mode == "causal":
             orc.tokencausal_rows(Q, K, V, G, pos, w.bands, w.rope_base, w.eps, rows=rows)
-        elif mode == "backward":
+        elif mode == "backward" and w.block_frames <= 0:
             orc.head_backward(Q, K, V, G, dO, pos, w.bands, w.rope_base, w.eps)
+        elif mode in ("backward", "backward_gated"):
+            gated = mode == "backward_gated"
+            orc.head_backward_gated(Q, K, V, G, dO, pos, w.bands, w.rope_base, w.eps, block_frames=w.block_frames,
+                                    beta=beta if gated else None, rms=(gamma, 1e-6) if gated else None)
         elif mode == "gated":
             orc.forward_positions(Q, K, V, G, pos, w.bands, w.rope_base, w.eps, beta=beta, rms=(gamma, 1e-6))
         elif w.block_frames > 0:
@@ -210,6 +216,8 @@ def run_reference(args):
 
     w = wl.WORKLOADS[args.workload]
     mode = "causal" if args.causal else ("backward" if args.backward else ("gated" if args.gated else "forward"))
+    if args.backward and args.gated:
+        mode = "backward_gated"
     value, cores, times = oracle_sample(w, 0, steps=max(1, args.steps), warmup=max(0, args.warmup), mode=mode)
     sample = (f"one head of {w.name} ({f'{min(w.N, 2000)} sampled outputs' if mode == 'causal' else f'all {w.N} tokens'}), "
               f"fp64 numpy oracle ({mode}), per step")
@@ -267,8 +275,8 @@ def main():
         raise SystemExit("--stream needs a block-causal workload")
 
     if args.backward:
-        if w.block_frames > 0 or args.gated or args.causal or args.stream:
-            raise SystemExit("--backward takes a bidirectional workload and no other mode")
+        if args.causal or args.stream:
+            raise SystemExit("--backward takes no --causal or --stream")
         dO = wl.generate_grad(w, dev, seed=w.seed + 11 + 1000 * rank)
         grads = tuple(torch.empty_like(Q) for _ in range(4))
     if args.stream:
@@ -295,10 +303,11 @@ def main():
                 n += la.last_launch_count()
             counter["launches"] = n
     elif args.backward:
-        counter = {"launches": 6}
+        counter = {"launches": 0}
 
         def forward_plain():
-            la.backward_bidir(p, Q, K, V, G, dO, grads=grads, ws=ws)
+            la.backward(p, Q, K, V, G, dO, grads=grads, ws=ws, **gates)
+            counter["launches"] = la.last_launch_count()
     elif args.causal:
         if w.block_frames > 0 or args.gated:
             raise SystemExit("--causal takes a bidirectional workload and no --gated")
@@ -375,16 +384,16 @@ def main():
     value = world * th * args.steps / (t_max * 1e-3)
     ms_per_step = t_max / args.steps
     # bytes_min: Q, K, V, G read once and O written once (+ the write gate when gated); the
-    # backward pass reads Q, K, V, G, dO and writes dQ, dK, dV, dG.
+    # backward pass reads Q, K, V, G, dO and writes dQ, dK, dV, dG (+ reads beta, writes dbeta).
     min_bytes = w.min_bytes + (th * elem if args.gated else 0)
     if args.backward:
-        min_bytes = 9 * th * w.d * elem
+        min_bytes = 9 * th * w.d * elem + (2 * th * elem if args.gated else 0)
     roof_all = min_bytes / (ms_per_step * 1e-3) / 1e9
 
     if whole_step:
         # No events sit between these kernels, so the roofline is the whole step's.
         kernels, alg, achieved, traffic = {}, min_bytes, roof_all, None
-        dominant = "whole step (per-block calls)" if args.stream else "whole step (6 kernels)"
+        dominant = "whole step (per-block calls)" if args.stream else f"whole step ({launches_per_step} kernels)"
     else:
         # Per-kernel durations inside the timed steps of the second region.
         tc = not args.simt and w.d == 128 and w.dtype == "bf16"
@@ -420,7 +429,8 @@ def main():
     if args.gated:
         config["gated"] = "write gate beta [B,H,N] + RMSNorm (gamma [d]) before the output gate"
     if args.backward:
-        config["mode"] = "backward: dQ, dK, dV, dG from dO (recomputes the forward state)"
+        config["mode"] = ("backward: dQ, dK, dV, dG" + (", dbeta, dgamma" if args.gated else "") +
+                          " from dO (recomputes the forward state)")
     if args.causal:
         config["mode"] = "token-causal (token n reads tokens 0..n; K and V are read by both passes)"
     if args.stream:
@@ -447,6 +457,8 @@ def main():
                           dO=dO if args.backward else None, grads=grads if args.backward else None)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         mode = "causal" if args.causal else ("backward" if args.backward else ("gated" if args.gated else "forward"))
+        if args.backward and args.gated:
+            mode = "backward_gated"
         v, cores, times = oracle_sample(w, args.cpu_seconds, mode=mode)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": f"one head of {w.name} ({f'{min(w.N, 2000)} sampled outputs' if mode == 'causal' else f'all {w.N} tokens'}), "
@@ -470,10 +482,14 @@ def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None, causal
 
     gates = gates or {}
     if dO is not None:
-        srcs0, outs0 = [Q, K, V, G, dO], list(grads)
+        srcs0 = [Q, K, V, G, dO] + ([gates["beta"]] if "beta" in gates else [])
+        outs0 = list(grads)
 
         def run(d, o):
-            la.backward_bidir(p, d[0], d[1], d[2], d[3], d[4], grads=tuple(o), ws=ws)
+            g = dict(gates)
+            if len(d) > 5:
+                g["beta"] = d[5]
+            la.backward(p, d[0], d[1], d[2], d[3], d[4], grads=tuple(o), ws=ws, **g)
     else:
         srcs0 = [Q, K, V, G] + ([gates["beta"]] if "beta" in gates else [])
         outs0 = [O]

@@ -10,10 +10,12 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-@pytest.mark.parametrize("mode", [[], ["--gated"], ["--causal"], ["--backward"]], ids=lambda m: m[0][2:] if m else "forward")
+@pytest.mark.parametrize("mode", [[], ["--gated"], ["--causal"], ["--backward"], ["--backward", "--gated"]],
+                         ids=lambda m: "_".join(x[2:] for x in m) if m else "forward")
 def test_reference_arm_prints_one_json_line(mode):
-    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
-                          "tiny_f32", "--steps", "2", "--warmup", "0"] + mode,
+    wl_args = [] if "--workload" in mode else ["--workload", "tiny_f32"]
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "2", "--warmup", "0"] + wl_args + mode,
                          capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert out.returncode == 0, out.stderr
     lines = [l for l in out.stdout.splitlines() if l.strip()]
