@@ -452,7 +452,9 @@ def main():
         "clocks": clk.summary(),
     }
 
-    if not args.no_e2e and not args.stream:
+    if not args.no_e2e and args.stream:
+        line["e2e"] = e2e_stream(la, w, blocks, ws_s, S_c, z_c, dev, args, ldist, world)
+    elif not args.no_e2e:
         line["e2e"] = e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates, causal=args.causal,
                           dO=dO if args.backward else None, grads=grads if args.backward else None)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -467,6 +469,76 @@ def main():
         print(json.dumps(line), flush=True)
     ldist.finalize()
     return 0
+
+
+def e2e_stream(la, w, blocks, ws, S_c, z_c, dev, args, ldist, world):
+    """End to end for block-autoregressive generation through la_block_step: a step is one video.
+    Each block's Q, K, V, G come from pinned host memory (as a generator would hand them over) and
+    the block's O goes back to the host; block j+1's inputs cross the host link while block j
+    computes (two device buffer sets, copies in on one stream, the operator on the current stream,
+    copies out on a third)."""
+    import torch
+
+    hosts = [[t.cpu().pin_memory() for t in ins] for _, ins, _ in blocks]
+    ohost = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _, _, o in blocks]
+    # two device sets per block length (a last block may be shorter), contiguous [B, H, n, d]
+    sets = {}
+    for _, ins, o in blocks:
+        n = o.shape[2]
+        if n not in sets:
+            sets[n] = ([[torch.empty_like(t) for t in ins] for _ in range(2)], [torch.empty_like(o) for _ in range(2)])
+    cur = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
+    nb = len(blocks)
+
+    def video():
+        S_c.zero_()
+        z_c.zero_()
+        for j, (pb, _, o) in enumerate(blocks):
+            k = j & 1
+            dsets, osets = sets[o.shape[2]]
+            with torch.cuda.stream(s_in):
+                if used[k]:
+                    s_in.wait_event(ev_done[k])  # block j-2's operator has read set k
+                for hsrc, dst in zip(hosts[j], dsets[k]):
+                    dst.copy_(hsrc, non_blocking=True)
+                ev_in[k].record(s_in)
+            cur.wait_event(ev_in[k])
+            if used[k]:
+                cur.wait_event(ev_out[k])  # block j-2's output has left set k
+            d = dsets[k]
+            la.block_step(pb, d[0], d[1], d[2], d[3], S_c, z_c, O=osets[k], ws=ws)
+            ev_done[k].record(cur)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[k])
+                ohost[j].copy_(osets[k], non_blocking=True)
+                ev_out[k].record(s_out)
+            used[k] = True
+
+    video()
+    torch.cuda.synchronize()
+    ldist.barrier(dev)
+    steps = max(3, min(args.steps, 10))
+    st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st.record(cur)
+    s_in.wait_stream(cur)
+    s_out.wait_stream(cur)
+    for _ in range(steps):
+        video()
+    cur.wait_stream(s_in)
+    cur.wait_stream(s_out)
+    en.record(cur)
+    torch.cuda.synchronize()
+    t = ldist.max_over_ranks(st.elapsed_time(en), dev)
+    h2d = sum(x.numel() * x.element_size() for hb in hosts for x in hb)
+    d2h = sum(x.numel() * x.element_size() for x in ohost)
+    return {"value": world * w.B * w.H * w.N * steps / (t * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps,
+            "pipelined": f"{nb} la_block_step calls per video; block j+1 copied in while block j computes"}
 
 
 def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None, causal=False, dO=None, grads=None):

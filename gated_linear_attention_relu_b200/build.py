@@ -29,6 +29,19 @@ def command(out: str = LIB, extra=()) -> list:
             "-I", os.path.join(ROOT, "include"), "-I", CSRC, *extra, "-o", out, *SOURCES]
 
 
+def build_variant(out: str, defines=(), verbose: bool = False) -> str:
+    """Builds the library with extra preprocessor definitions (e.g. the checked build,
+    ``LA_CHECKED``, or the test-hooks build) into ``out``."""
+    cmd = command(out, extra=[f"-D{d}" for d in defines])
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        sys.stderr.write(r.stdout + r.stderr)
+        raise RuntimeError(f"nvcc failed building {out}")
+    return out
+
+
 def up_to_date(out: str = LIB) -> bool:
     if not os.path.exists(out):
         return False

@@ -248,6 +248,7 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int64_t g = g0; g < g1; ++g) {
         const int64_t i = g - g0;
         const TileInfo ti = tile_info(p, g);
+        in_bounds(ti.unit < p.BH * p.nblk && ti.bh < p.BH && ti.n0 < ti.n_end && ti.n_end <= p.N);
         if (ti.unit != prev_unit) {
           const int64_t ku = ti.unit - u_first;
           const int b = static_cast<int>(ku % NSB);
@@ -435,6 +436,8 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         uint32_t pt = 0, ph = 0, pw = 0;
         // Rows past the end of the head keep position 0 (their output is dropped).
         if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph, pw);
+        in_bounds(pt < static_cast<uint32_t>(p.T) && ph < static_cast<uint32_t>(p.Hh) &&
+                  pw < static_cast<uint32_t>(p.W));
         const float* zg = zimg + ti.unit * D + 64 * hf;
         const int ipt = static_cast<int>(pt), iph = static_cast<int>(ph), ipw = static_cast<int>(pw);
         const float dpart =

@@ -449,6 +449,7 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // the CTA's partial slot.
         if (!warp_wait(&bars->qfree, ph, abort_flag)) break;
         tc_fence_after();
+        if (!in_bounds(ti.unit - u_first < p.maxseg)) break;
         float* dst = partial + (c * p.maxseg + (ti.unit - u_first)) * slot_floats;
         uint32_t r[32];
         tmem_ld_x32(tmem + QCOL_DS + lane_bits + static_cast<uint32_t>(cpart), r);

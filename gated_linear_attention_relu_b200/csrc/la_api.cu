@@ -994,6 +994,15 @@ int la_device_error(cudaStream_t stream) {
 
 int la_last_launch_count(void) { return g_last_launches; }
 
+#ifdef LA_TEST_HOOKS
+// Hooks build only (not part of the regular library): from the next launch on, the state kernel
+// does not issue the K load of global tile `tile` (-1: load every tile), so the bounded waits for
+// it run out and the kernel winds down with the error word set.  Used to test that path.
+int la_test_skip_tile(long long tile) {
+  return cudaMemcpyToSymbol(la::g_la_skip_tile, &tile, sizeof tile) == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+#endif
+
 }  // extern "C"
 
 // Fixed scratch for callers that cannot allocate (la_forward_bidir_static).  In host code the

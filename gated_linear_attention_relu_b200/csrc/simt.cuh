@@ -109,7 +109,7 @@ state_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __r
       for (int r = 0; r < TS; ++r) zacc += kp[r][tid];
 
     const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != ti.unit);
-    if (last) {
+    if (last && in_bounds(ti.unit - u_first < p.maxseg)) {
       float* dst = partial + (c * p.maxseg + (ti.unit - u_first)) * slot_floats;
 #pragma unroll
       for (int i = 0; i < R; ++i)
@@ -336,6 +336,7 @@ combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, fl
 #pragma unroll 4
       for (int64_t cc = c0; cc <= c1; ++cc) {
         const int64_t k = u - unit_of_tile(p, cta_start(p, cc));
+        if (!in_bounds(k >= 0 && k < p.maxseg && cc < p.grid)) continue;
         const float* src = partial + (cc * p.maxseg + k) * slot_floats;
         if (e0 < D * D) {
           const float4* s4 = reinterpret_cast<const float4*>(src + e0);
@@ -383,6 +384,7 @@ blocksum_kernel(const Plan p, const float* __restrict__ partial, float* __restri
     const int64_t c0 = cta_of(p, first), c1 = cta_of(p, first + count - 1);
     for (int64_t cc = c0; cc <= c1; ++cc) {
       const int64_t k = u - unit_of_tile(p, cta_start(p, cc));
+      if (!in_bounds(k >= 0 && k < p.maxseg && cc < p.grid)) continue;
       const float* src = partial + (cc * p.maxseg + k) * slot_floats;
       for (int zp = 0; zp < (e0 < D * D ? 1 : p.zparts); ++zp) {
         const float4* s4 = reinterpret_cast<const float4*>(e0 < D * D ? src + e0 : src + D * D + zp * D + (e0 - D * D));
@@ -451,6 +453,7 @@ start_kernel(const Plan p, const float* __restrict__ partial, float* __restrict_
     unit_tiles(p, u, &first, &count);
     for (int64_t cc = cta_of(p, first); cc < c; ++cc) {
       const int64_t k = u - unit_of_tile(p, cta_start(p, cc));
+      if (!in_bounds(k >= 0 && k < p.maxseg)) continue;
       const float* src = partial + (cc * p.maxseg + k) * slot_floats;
       for (int zp = 0; zp < (e0 < D * D ? 1 : p.zparts); ++zp) {
         const float4* s4 = reinterpret_cast<const float4*>(e0 < D * D ? src + e0 : src + D * D + zp * D + (e0 - D * D));

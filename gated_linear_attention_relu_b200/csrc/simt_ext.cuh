@@ -376,7 +376,7 @@ bwdq_simt_kernel(const T* __restrict__ Q, const T* __restrict__ G, const T* __re
     if (tid < D)
       for (int r = 0; r < TS; ++r) dzacc = fmaf(dden[r], qp[r * LD + tid], dzacc);
     const bool last = (g + 1 == g1) || (unit_of_tile(p, g + 1) != ti.unit);
-    if (last) {
+    if (last && in_bounds(ti.unit - u_first < p.maxseg)) {
       float* dst = partial + (c * p.maxseg + (ti.unit - u_first)) * slot_floats;
 #pragma unroll
       for (int i = 0; i < R; ++i)

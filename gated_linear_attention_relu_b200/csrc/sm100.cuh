@@ -16,7 +16,28 @@ namespace la {
 // Per-device error word: bit 0 = an mbarrier wait timed out, bit 1 = bad shared-memory alignment.
 __device__ unsigned int g_la_error;
 
-enum : unsigned { ERR_WAIT_TIMEOUT = 1u, ERR_SMEM_ALIGN = 2u, ERR_TMEM = 4u };
+enum : unsigned { ERR_WAIT_TIMEOUT = 1u, ERR_SMEM_ALIGN = 2u, ERR_TMEM = 4u, ERR_BOUNDS = 8u };
+
+// Bounds checks of the checked build (LA_CHECKED): every index the kernels compute from the work
+// decomposition (tiles, units, partial slots, grid positions) is tested against its extent; a
+// failed test records ERR_BOUNDS in the error word and the access is skipped or clamped, so a
+// bookkeeping mistake shows up in la_device_error() instead of touching memory it should not.
+// Other builds compile the tests away.
+#ifdef LA_CHECKED
+__device__ __forceinline__ bool in_bounds(bool ok) {
+  if (!ok) atomicOr(&g_la_error, ERR_BOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(bool) { return true; }
+#endif
+
+// Test hook of the hooks build (LA_TEST_HOOKS): the state kernel never issues the K load of this
+// global tile, so the waits for it run out (bounded) and the kernel winds down with
+// ERR_WAIT_TIMEOUT set, as it would after any lost arrival.  -1: off.
+#ifdef LA_TEST_HOOKS
+__device__ long long g_la_skip_tile = -1;
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

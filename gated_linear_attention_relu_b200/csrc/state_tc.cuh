@@ -146,6 +146,10 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const uint32_t ph = static_cast<uint32_t>((i / nst) & 1);
         if (!mbar_wait(&emptyb[s], ph ^ 1u, abort_flag, LA_SLEEP_PROD)) break;
         const TileInfo ti = tile_info(p, g);
+        in_bounds(ti.bh < p.BH && ti.n0 < ti.n_end && ti.n_end <= p.N);
+#ifdef LA_TEST_HOOKS
+        if (is_k && g == g_la_skip_tile) continue;  // (counted as issued: the drain below waits for it)
+#endif
         uint8_t* buf = ring + s * BUF;
         mbar_arrive_expect_tx(&fullb[s], BUF);
         const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
@@ -250,6 +254,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       // the chunk's cos/sin, z, written back in place.
       const __nv_bfloat16* beta_h = BETA ? beta + ti.bh * p.N : nullptr;
       auto item = [&](uint32_t addr, uint32_t keep, uint32_t n, uint32_t pt, uint32_t ph_, uint32_t pw) {
+        in_bounds(n < N && pt < static_cast<uint32_t>(p.T) && ph_ < Hd && pw < Wd);
         const uint4 raw = lds128(addr);
         float2 cs[4];
         if constexpr (UNIFORM) {
@@ -333,8 +338,8 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
           zs[e] += __shfl_xor_sync(0xffffffffu, zs[e], 8);
           zs[e] += __shfl_xor_sync(0xffffffffu, zs[e], 16);
         }
-        if (lane < 4) {
-          const int64_t slot = c * p.maxseg + (ti.unit - u_first);
+        const int64_t slot = c * p.maxseg + (ti.unit - u_first);
+        if (lane < 4 && in_bounds(ti.unit - u_first < p.maxseg && slot < int64_t(p.grid) * p.maxseg)) {
           float4* zd = reinterpret_cast<float4*>(partial + slot * SLOT + D * D + tg * D + 8 * ck);
           zd[0] = make_float4(zs[0], zs[1], zs[2], zs[3]);
           zd[1] = make_float4(zs[4], zs[5], zs[6], zs[7]);
@@ -351,6 +356,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     for (int64_t k = 0; k < nseg; ++k) {
       if (!warp_wait(&bars->accfull[k & 1], static_cast<uint32_t>((k >> 1) & 1), abort_flag, LA_SLEEP_LONG)) break;
       tc_fence_after();
+      if (!in_bounds(k < p.maxseg)) break;
       float* dst = partial + (c * p.maxseg + k) * SLOT + static_cast<int64_t>(row) * D;
       const uint32_t taddr = tmem + static_cast<uint32_t>(k & 1) * 128u + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll
