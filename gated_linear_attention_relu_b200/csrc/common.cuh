@@ -61,6 +61,11 @@ struct Plan {
   int32_t zparts;          // partial z rows per slot (summed in order by the combine kernel)
   float eps;
   FastDiv fd_tph, fd_tfull, fd_HW, fd_W;  // tiles_per_head, tiles_full, Hh*W, W
+  // CTA ranges without 64-bit division: total = cta_q * grid + cta_r, so
+  // c * total / grid = c * cta_q + (c * cta_r) / grid, and c * cta_r < grid^2 < 2^31.
+  int64_t cta_q;
+  uint32_t cta_r;
+  FastDiv fd_grid;
 };
 
 // Rotation parameters of the d/2 channel pairs (at most 64 for d = 128).
@@ -126,11 +131,20 @@ __host__ __device__ inline int64_t unit_of_tile(const Plan& p, int64_t g) {
   return int64_t(bh) * p.nblk + blk;
 }
 
-__host__ __device__ inline int64_t cta_start(const Plan& p, int64_t c) { return c * p.total / p.grid; }
+// First tile of CTA c, floor(c * total / grid) (c <= grid < 46341, checked on the host).
+__host__ __device__ inline int64_t cta_start(const Plan& p, int64_t c) {
+  return c * p.cta_q + static_cast<int64_t>(fdiv(static_cast<uint32_t>(c) * p.cta_r, p.fd_grid));
+}
 
-// The CTA whose range holds tile g.
+// The CTA whose range holds tile g: the largest c with cta_start(c) <= g.  Estimated in double
+// precision (error well below one CTA), then settled exactly against cta_start.
 __host__ __device__ inline int64_t cta_of(const Plan& p, int64_t g) {
-  return ((g + 1) * static_cast<int64_t>(p.grid) - 1) / p.total;
+  int64_t c = static_cast<int64_t>(static_cast<double>(g) * static_cast<double>(p.grid) / static_cast<double>(p.total));
+  if (c >= p.grid) c = p.grid - 1;
+  if (c < 0) c = 0;
+  while (c + 1 < p.grid && cta_start(p, c + 1) <= g) ++c;
+  while (c > 0 && cta_start(p, c) > g) --c;
+  return c;
 }
 
 // Global tile range [first, first + count) of unit u.

@@ -68,6 +68,10 @@ int check_ptr(const void* ptr, bool needed) {
 
 // ------------------------------------------------------------------------------- planning
 void set_fastdiv(Plan& p) {
+  const int64_t g = p.grid > 0 ? p.grid : 1;
+  p.cta_q = p.total / g;
+  p.cta_r = static_cast<uint32_t>(p.total % g);
+  p.fd_grid = la::make_fastdiv(static_cast<uint32_t>(g));
   p.fd_tph = la::make_fastdiv(static_cast<uint32_t>(p.tiles_per_head > 0 ? p.tiles_per_head : 1));
   p.fd_tfull = la::make_fastdiv(static_cast<uint32_t>(p.tiles_full > 0 ? p.tiles_full : 1));
   p.fd_HW = la::make_fastdiv(static_cast<uint32_t>(p.HW > 0 ? p.HW : 1));
@@ -108,6 +112,8 @@ Plan build_plan(const la_problem& q, int64_t tile, int64_t grid_cap, int zparts)
   p.tiles_last = (last_len + tile - 1) / tile;
   p.tiles_per_head = (p.nblk - 1) * p.tiles_full + p.tiles_last;
   p.total = p.BH * p.tiles_per_head;
+  // (at most 46340 CTAs, so that the CTA-range arithmetic of common.cuh stays within 32 bits)
+  if (grid_cap > 46340) grid_cap = 46340;
   p.grid = static_cast<int32_t>(p.total < grid_cap ? p.total : grid_cap);
   set_fastdiv(p);
   int64_t maxseg = 0;
@@ -1067,11 +1073,29 @@ int la_selftest_host(void) {
       if (la::fdiv(n, f) != n / d) return 2;
     }
   }
+  // CTA ranges (32-bit arithmetic) against exact 64-bit division, and cta_of against its definition.
+  for (int trial = 0; trial < 4000; ++trial) {
+    x ^= x << 13; x ^= x >> 7; x ^= x << 17;
+    Plan p;
+    std::memset(&p, 0, sizeof p);
+    p.total = static_cast<int64_t>(x & 0x7fffffffu) + 1;
+    const int64_t gcap = trial % 3 == 0 ? 46340 : static_cast<int64_t>((x >> 33) % 1000) + 1;
+    p.grid = static_cast<int32_t>(p.total < gcap ? p.total : gcap);
+    set_fastdiv(p);
+    for (int k = 0; k < 8; ++k) {
+      x ^= x << 13; x ^= x >> 7; x ^= x << 17;
+      const int64_t c = static_cast<int64_t>(x % static_cast<uint64_t>(p.grid + 1));
+      if (la::cta_start(p, c) != c * p.total / p.grid) return 11;
+      const int64_t g = static_cast<int64_t>((x >> 20) % static_cast<uint64_t>(p.total));
+      const int64_t o = la::cta_of(p, g);
+      if (!(la::cta_start(p, o) <= g && g < la::cta_start(p, o + 1))) return 12;
+    }
+  }
   // Decomposition invariants on assorted problems and SM counts.
   struct Shape { int64_t B, H, T, Hh, W; int32_t bf; };
   const Shape shapes[] = {{1, 32, 21, 45, 80, 0}, {1, 32, 81, 45, 80, 3}, {3, 70, 1, 2, 64, 0},
                           {1, 2, 7, 6, 10, 2}, {2, 1, 3, 5, 30, 10}, {1, 1, 1, 1, 1, 0}, {1, 3, 6, 4, 33, 1}};
-  const int sms[] = {1, 7, 148, 1000};
+  const int sms[] = {1, 7, 148, 1000, 46340, 60000};
   for (const Shape& sh : shapes)
     for (int sm : sms)
       for (int64_t tile : {int64_t(32), int64_t(128)}) {
