@@ -46,15 +46,16 @@ constexpr uint32_t IDESC_TD = idesc_bf16_f32(128, 128, /*a_mn=*/true, /*b_mn=*/t
 
 // ---- bwdq smem: Q (-> phi(Q)), G (-> dG), dO (-> dnum), S image, dQ staging, exchanges
 constexpr uint32_t QO_Q = 0, QO_G = BUF, QO_DO = 2 * BUF, QO_S = 3 * BUF, QO_DQ = 4 * BUF;
-constexpr uint32_t QO_X = 5 * BUF;  // [2 values][4 parts][128] fp32: partial den, partial dy.y
-constexpr uint32_t QO_Z = QO_X + 2 * PARTS * 512;  // z of the unit, [2 slots by unit parity][128] fp32
+constexpr uint32_t QO_X = 5 * BUF;  // [3 values][4 parts][128] fp32: partial den, dy.y (RMSNorm: sum y^2, sum y du gamma)
+constexpr uint32_t QO_Z = QO_X + 3 * PARTS * 512;  // z of the unit, [2 slots by unit parity][128] fp32
 constexpr uint32_t QO_BAR = QO_Z + 1024;
 constexpr uint32_t SMEM_Q = QO_BAR + 256 + 1024;
 constexpr uint32_t QCOL_NUM = 0, QCOL_DPQ = 128, QCOL_DS = 256;
 // ---- bwdk smem: K (-> phi(K)), V, dS image, dK and dV staging
 constexpr uint32_t KO_K = 0, KO_V = BUF, KO_S = 2 * BUF, KO_DK = 3 * BUF, KO_DV = 4 * BUF;
 constexpr uint32_t KO_Z = 5 * BUF;  // dz of the unit, [2 slots by unit parity][128] fp32
-constexpr uint32_t KO_BAR = KO_Z + 1024;
+constexpr uint32_t KO_X = KO_Z + 1024;  // [2 slots by tile parity][4 parts][128] fp32: partial dbeta
+constexpr uint32_t KO_BAR = KO_X + 2 * PARTS * 512;
 constexpr uint32_t SMEM_K = KO_BAR + 256 + 1024;
 constexpr uint32_t KCOL_DV = 0, KCOL_DPK = 128;
 static_assert(SMEM_Q <= 232448 && SMEM_K <= 232448, "shared memory budget");
@@ -72,6 +73,7 @@ struct BarsQ {
   int abort_flag;
 };
 struct BarsK {
+  uint64_t pair[4];  // the four warps of rows 32q .. 32q+31 (write gate: partial dbeta)
   uint64_t full;    // K (and the dS image at a unit's first tile) landed
   uint64_t full_v;  // V landed
   uint64_t rot;
@@ -93,14 +95,18 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
   return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
 }
 
-template <int DT, int DH>
+// RMS: RMSNorm before the output gate (SANA-Video 2.0, Eq. (1)); its gradient is formed from two
+// row sums, sum y^2 and sum y du gamma, which the four quarters of a row swap once, and dgamma's
+// column sums are kept per warp and written to dgamma_part[(CTA * 4 + lane quarter) * D + channel].
+template <int DT, int DH, bool RMS>
 __global__ void __launch_bounds__(THREADS, 1)
 bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
                const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmDQ,
                const __grid_constant__ CUtensorMap tmDG, const Plan p, const __grid_constant__ Rope rope,
                const uint8_t* __restrict__ simg, const float* __restrict__ zimg, const float2* __restrict__ tab,
                const float4* __restrict__ tab2, float* __restrict__ partial, __nv_bfloat16* __restrict__ dQg,
-               __nv_bfloat16* __restrict__ dGg) {
+               __nv_bfloat16* __restrict__ dGg, const float* __restrict__ gamma, float norm_eps,
+               float* __restrict__ dgamma_part) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   BarsQ* bars = reinterpret_cast<BarsQ*>(smem + QO_BAR);
@@ -254,6 +260,7 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int cpart = 32 * part;  // this warp's channels
     uint64_t* pr = &bars->pair[quarter];
     float dzacc = 0.f;  // dz of channel 32 part + lane over this warp's rows
+    float dgacc = 0.f;  // RMSNorm: dgamma of channel 32 part + lane over this warp's rows
     int zslot = 0;      // z slot of the current unit
     int64_t prev_unit = -1;
     for (int64_t g = g0; g < g1; ++g) {
@@ -327,6 +334,8 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!warp_wait(&bars->full_g, ph, abort_flag)) break;
       if (!warp_wait(&bars->full_do, ph, abort_flag)) break;
       tc_fence_after();
+      float dden;
+      if constexpr (!RMS) {
       // Channel pairs in packed fp32 (sigmoid(g) = 1/2 + tanh(g/2)/2, with g/2 exact in bf16):
       //   y = num / den, dy = dO s, dG = dy y (1 - s), dnum = dy / den, dy . y accumulated.
       const uint64_t rden2 = pk(rden, rden), half2 = pk(0.5f, 0.5f), mhalf2 = pk(-0.5f, -0.5f);
@@ -379,7 +388,111 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (lane == 0) mbar_arrive(pr);
       if (!warp_wait(pr, 1u, abort_flag)) break;
       const float* yx = xch + PARTS * 128;
-      const float dden = -((yx[row] + yx[128 + row]) + (yx[256 + row] + yx[384 + row])) * rden;
+      dden = -((yx[row] + yx[128 + row]) + (yx[256 + row] + yx[384 + row])) * rden;
+      } else {
+      // RMSNorm before the gate: with y = num / den, r = sqrt(mean(y^2) + norm_eps), yh = y / r,
+      // u = yh gamma, s = sigmoid(g), du = dO s:
+      //   dG = dO u s (1 - s),  dy = (du gamma - yh (yh . du gamma) / d) / r,  dnum = dy / den,
+      //   dy . y = (1/r) T (1 - SS / (d r^2)) with SS = sum y^2, T = sum y du gamma,
+      // so the row needs only SS and T from the other quarters (pass 1), then pass 2 forms every
+      // output.  dgamma += du yh per channel.
+      float ssp = 0.f, ttp = 0.f;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[16];
+        tmem_ld_x16(tmem + QCOL_NUM + lane_bits + static_cast<uint32_t>(cpart) + 16u * static_cast<uint32_t>(hh), r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int ck = 4 * part + 2 * hh + cc;
+          const uint4 gr = lds128(row_chunk(sbase + QO_G, row, ck));
+          const uint4 dr = lds128(row_chunk(sbase + QO_DO, row, ck));
+          const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w}, dw[4] = {dr.x, dr.y, dr.z, dr.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int e = 8 * cc + 2 * q;
+            const int ch = 8 * ck + 2 * q;
+            const uint32_t gh = half_bf16x2(gw[q]);
+            const float s0 = 0.5f + 0.5f * tanh_f(bf16lo(gh)), s1 = 0.5f + 0.5f * tanh_f(bf16hi(gh));
+            const float y0 = __uint_as_float(r[e]) * rden, y1 = __uint_as_float(r[e + 1]) * rden;
+            const float g0 = gamma ? __ldg(gamma + ch) : 1.f, g1 = gamma ? __ldg(gamma + ch + 1) : 1.f;
+            ssp = fmaf(y0, y0, fmaf(y1, y1, ssp));
+            ttp = fmaf(y0 * g0, bf16lo(dw[q]) * s0, fmaf(y1 * g1, bf16hi(dw[q]) * s1, ttp));
+          }
+        }
+      }
+      xch[PARTS * 128 + part * 128 + row] = ssp;
+      xch[2 * PARTS * 128 + part * 128 + row] = ttp;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pr);
+      if (!warp_wait(pr, 1u, abort_flag)) break;
+      const float* sx = xch + PARTS * 128;
+      const float* tx = xch + 2 * PARTS * 128;
+      const float SS = (sx[row] + sx[128 + row]) + (sx[256 + row] + sx[384 + row]);
+      const float TT = (tx[row] + tx[128 + row]) + (tx[256 + row] + tx[384 + row]);
+      const float rinv = rsqrtf(SS * (1.f / D) + norm_eps);
+      const float dotd = rinv * TT * (1.f / D);  // (yh . dyh) / d
+      dden = -(rinv * TT * (1.f - rinv * rinv * SS * (1.f / D))) * rden;
+      float gv[32];  // du yh of this quarter's 32 channels (dgamma)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[16];
+        tmem_ld_x16(tmem + QCOL_NUM + lane_bits + static_cast<uint32_t>(cpart) + 16u * static_cast<uint32_t>(hh), r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int ck = 4 * part + 2 * hh + cc;
+          const uint32_t ag = row_chunk(sbase + QO_G, row, ck);
+          const uint4 gr = lds128(ag);
+          const uint32_t ad = row_chunk(sbase + QO_DO, row, ck);
+          const uint4 dr = lds128(ad);
+          const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w}, dw[4] = {dr.x, dr.y, dr.z, dr.w};
+          uint32_t dgw[4], dnw[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int e = 8 * cc + 2 * q;
+            const int ch = 8 * ck + 2 * q;
+            const uint32_t gh = half_bf16x2(gw[q]);
+            float o_g[2], o_n[2];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const float sgm = 0.5f + 0.5f * tanh_f(h2 ? bf16hi(gh) : bf16lo(gh));
+              const float y = __uint_as_float(r[e + h2]) * rden;
+              const float yh = y * rinv;
+              const float gmv = gamma ? __ldg(gamma + ch + h2) : 1.f;
+              const float dov = h2 ? bf16hi(dw[q]) : bf16lo(dw[q]);
+              const float du = dov * sgm;
+              o_g[h2] = dov * yh * gmv * sgm * (1.f - sgm);
+              o_n[h2] = (du * gmv - yh * dotd) * rinv * rden;
+              gv[16 * hh + e + h2] = du * yh;
+            }
+            dgw[q] = pack_bf16(o_g[0], o_g[1]);
+            dnw[q] = pack_bf16(o_n[0], o_n[1]);
+          }
+          if (tma_out) sts128(ag, make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]));
+          else if (valid) *reinterpret_cast<uint4*>(dg_row + 8 * (2 * hh + cc)) = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
+          sts128(ad, make_uint4(dnw[0], dnw[1], dnw[2], dnw[3]));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->dn);
+      // dgamma over this warp's 32 rows for this quarter's 32 channels (rows past the unit's end
+      // have yh = 0): lane L ends with channel 32 part + L, as for dz below.
+#pragma unroll
+      for (int off = 16, size = 32; off >= 1; off >>= 1, size >>= 1) {
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int e = 0; e < size / 2; ++e) {
+          const float keep = up ? gv[e + size / 2] : gv[e];
+          const float send = up ? gv[e] : gv[e + size / 2];
+          const float other = __shfl_xor_sync(0xffffffffu, send, off);
+          gv[e] = up ? other + keep : keep + other;
+        }
+      }
+      dgacc += gv[0];
+      }
       // dz over this warp's 32 rows for this quarter's 32 channels: lane L ends with channel
       // 32 part + L (a butterfly that halves the range per step, each sum formed once, lower
       // lane first).
@@ -467,6 +580,8 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->out);
     }
+    // This warp's dgamma column sums (rows 32 quarter .. +31 of every tile of the CTA).
+    if (RMS && dgamma_part) dgamma_part[(c * 4 + quarter) * D + cpart + lane] = dgacc;
   }
 
   tc_fence_before();
@@ -475,13 +590,17 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (warp == CTRL_WARP) tmem_dealloc(tmem, 512);
 }
 
-template <int DT, int DH>
+// BETA: the write gate of SANA-Video 2.0, Eq. (1), which scales each key's term of S:
+// dV = beta phi(K) dS, dphi(k) = beta V dS^T, and dbeta = phi(k) . (V dS^T) per row (the four
+// quarters of a row add their shares through shared memory).
+template <int DT, int DH, bool BETA>
 __global__ void __launch_bounds__(THREADS, 1)
 bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV, const Plan p,
                const __grid_constant__ Rope rope, const uint8_t* __restrict__ dsimg, const float* __restrict__ dzimg,
                const float2* __restrict__ tab, const float4* __restrict__ tab2, __nv_bfloat16* __restrict__ dKg,
-               __nv_bfloat16* __restrict__ dVg) {
+               __nv_bfloat16* __restrict__ dVg, const __nv_bfloat16* __restrict__ beta,
+               __nv_bfloat16* __restrict__ dbeta) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   BarsK* bars = reinterpret_cast<BarsK*>(smem + KO_BAR);
@@ -501,6 +620,7 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     mbar_init(&bars->ready, 1);
     mbar_init(&bars->out, MATH_WARPS);
     mbar_init(&bars->final_, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], PARTS);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -630,6 +750,9 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       uint32_t pt = 0, ph_ = 0, pw = 0;
       if (static_cast<int64_t>(n) < p.N) token_pos(p, n, pt, ph_, pw);
       const int ipt = static_cast<int>(pt), iph = static_cast<int>(ph_), ipw = static_cast<int>(pw);
+      // The row's write gate (1 without one).
+      const float bt = (BETA && valid) ? __bfloat162float(beta[ti.bh * p.N + n]) : 1.f;
+      uint32_t kr[16];  // phi(k) of this quarter, kept for dbeta
       {
         uint32_t a[16];
 #pragma unroll
@@ -643,6 +766,8 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4)
           sts128(row_chunk(sbase + KO_K, row, 4 * part + c4), make_uint4(a[4 * c4], a[4 * c4 + 1], a[4 * c4 + 2], a[4 * c4 + 3]));
+#pragma unroll
+        for (int e = 0; e < 16; ++e) kr[e] = BETA ? a[e] : 0u;
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -655,7 +780,7 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         tmem_ld_x32(tmem + KCOL_DV + lane_bits + static_cast<uint32_t>(cpart), r);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]) * bt;
       }
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
@@ -665,6 +790,7 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
       if (!warp_wait(&bars->ready, ph, abort_flag)) break;
       tc_fence_after();
       const float* zg = reinterpret_cast<const float*>(smem + KO_Z) + zslot * D + cpart;
+      float dbp = 0.f;  // this quarter's share of phi(k) . (V dS^T)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         // 16 channels at a time (fewer live registers)
@@ -675,6 +801,14 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 16; ++e) y[e] = __uint_as_float(r[e]);
+        }
+        if constexpr (BETA) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint32_t w = kr[8 * hh + e / 2];
+            dbp = fmaf((e & 1) ? bf16hi(w) : bf16lo(w), y[e], dbp);
+            y[e] *= bt;
+          }
         }
         switch (2 * part + hh) {
           case 0: rotate_span_t<DT, DH, 0, 8>(y, tab, tab2, rope, p, ipt, iph, ipw); break;
@@ -702,6 +836,18 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
           if (tma_out) sts128(row_chunk(sbase + KO_DK, row, 4 * part + c4), pack8(o8));
           else if (valid) *reinterpret_cast<uint4*>(dk_row + 8 * c4) = pack8(o8);
         }
+      }
+      if constexpr (BETA) {
+        // dbeta of the row: the four quarters' shares added in a fixed order by quarter 0 (two
+        // slots by tile parity: a quarter reaching the next tile's write has met the others on
+        // this one, but quarter 0 may not have read yet).
+        float* xk = reinterpret_cast<float*>(smem + KO_X) + ph * (PARTS * 128);
+        xk[part * 128 + row] = dbp;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->pair[quarter]);
+        if (!warp_wait(&bars->pair[quarter], ph, abort_flag)) break;
+        if (part == 0 && valid)
+          dbeta[ti.bh * p.N + n] = __float2bfloat16_rn((xk[row] + xk[128 + row]) + (xk[256 + row] + xk[384 + row]));
       }
       fence_proxy_async_smem();
       tc_fence_before();

@@ -173,8 +173,8 @@ PlanSet make_plans(const la_problem& q, int sm_count) {
   off = align256(off + size_t(s.ps.grid) * size_t(D * D + D) * 4);
   s.off_states2 = off;  // gradients on the CUDA cores: per-unit dS, dz (suffix sums over blocks)
   off = align256(off + (s.tc ? 0 : size_t(s.units) * size_t(D * D + D) * 4));
-  s.off_dgamma = off;   // gradients: one dgamma row per CTA of the query side
-  off = align256(off + size_t(s.ps.grid) * size_t(D) * 4);
+  s.off_dgamma = off;   // gradients: the query side's dgamma rows (4 per CTA on the tensor cores)
+  off = align256(off + size_t(s.ps.grid) * size_t(D) * 4 * (s.tc ? 4 : 1));
   s.total = off;
   return s;
 }
@@ -653,8 +653,8 @@ int la_forward_tokencausal(const la_problem* p, const void* Q, const void* K, co
 }
 
 // Gradients of the operator in every form: bidirectional or block-causal (p->block_frames), with
-// the optional write gate and RMSNorm.  bf16 with d = 128 and neither gate on takes the
-// tensor-core kernels; everything else the CUDA-core kernels.
+// the optional write gate and RMSNorm.  bf16 with d = 128 takes the tensor-core kernels; fp32,
+// d = 32 / 64 and LA_FLAG_FORCE_SIMT the CUDA-core kernels.
 static int backward_common(const la_problem* p, const Gates& gt, const void* Q, const void* K, const void* V,
                            const void* G, const void* dO, void* dQ, void* dK, void* dV, void* dG, void* dbeta,
                            float* dgamma, void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -685,13 +685,13 @@ static int backward_common(const la_problem* p, const Gates& gt, const void* Q, 
   int nl = 0;
   uint8_t* w = static_cast<uint8_t*>(ws);
   const Rope rope = make_rope(*p);
-  const bool tc = s.tc && !gt.beta && !gt.rms;
-  if (tc) {
+  if (s.tc) {
     // Forward state (per unit: a head, or a block's inclusive prefix) and its operand image.
     if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
-    if ((rc = launch_state(s, *p, K, V, ws, stream, &nl))) return rc;
+    if ((rc = launch_state(s, *p, K, V, ws, stream, &nl, gt.beta))) return rc;
     if ((rc = launch_combine(s, *p, ws, nullptr, nullptr, nullptr, nullptr, true, stream, &nl))) return rc;
     const bool sb = standard_bands(*p);
+    float* dgp = reinterpret_cast<float*>(w + s.off_dgamma);
     CUtensorMap tq, tg, tdo, tdq, tdg, tk, tv, tdk, tdv;
     if (!make_tmap(&tq, Q, s.ps.BH, s.ps.N) || !make_tmap(&tg, G, s.ps.BH, s.ps.N) ||
         !make_tmap(&tdo, dO, s.ps.BH, s.ps.N) || !make_tmap(&tdq, dQ, s.ps.BH, s.ps.N) ||
@@ -700,14 +700,15 @@ static int backward_common(const la_problem* p, const Gates& gt, const void* Q, 
         !make_tmap(&tdv, dV, s.ps.BH, s.ps.N))
       return LA_ERR_CUDA;
     // Q side: dQ, dG and the partial sums of dS, dz.
-    auto kq = sb ? la::bw::bwdq_tc_kernel<32, 48> : la::bw::bwdq_tc_kernel<-1, -1>;
+    auto kq = sb ? (gt.rms ? la::bw::bwdq_tc_kernel<32, 48, true> : la::bw::bwdq_tc_kernel<32, 48, false>)
+                 : (gt.rms ? la::bw::bwdq_tc_kernel<-1, -1, true> : la::bw::bwdq_tc_kernel<-1, -1, false>);
     if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, la::bw::SMEM_Q) != cudaSuccess)
       return LA_ERR_CUDA;
     if (launch_k(kq, unsigned(s.ps.grid), la::bw::THREADS, la::bw::SMEM_Q, stream, true, tq, tg, tdo, tdq, tdg,
                  s.ps, rope, static_cast<const uint8_t*>(w + s.off_img), reinterpret_cast<const float*>(w + s.off_zimg),
                  reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2),
                  reinterpret_cast<float*>(w + s.off_partial), static_cast<__nv_bfloat16*>(dQ),
-                 static_cast<__nv_bfloat16*>(dG)))
+                 static_cast<__nv_bfloat16*>(dG), gt.gamma, gt.norm_eps, gt.rms ? dgp : nullptr))
       return LA_ERR_CUDA;
     ++nl;
     // dS, dz summed in fixed order into the operand image (reusing the state image's space); in
@@ -719,15 +720,23 @@ static int backward_common(const la_problem* p, const Gates& gt, const void* Q, 
                              /*reverse=*/true)))
       return rc;
     // K side: dK, dV.
-    auto kk = sb ? la::bw::bwdk_tc_kernel<32, 48> : la::bw::bwdk_tc_kernel<-1, -1>;
+    auto kk = sb ? (gt.beta ? la::bw::bwdk_tc_kernel<32, 48, true> : la::bw::bwdk_tc_kernel<32, 48, false>)
+                 : (gt.beta ? la::bw::bwdk_tc_kernel<-1, -1, true> : la::bw::bwdk_tc_kernel<-1, -1, false>);
     if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, la::bw::SMEM_K) != cudaSuccess)
       return LA_ERR_CUDA;
     if (launch_k(kk, unsigned(s.ps.grid), la::bw::THREADS, la::bw::SMEM_K, stream, true, tk, tv, tdk, tdv, s.ps,
                  rope, static_cast<const uint8_t*>(w + s.off_img), reinterpret_cast<const float*>(w + s.off_zimg),
                  reinterpret_cast<const float2*>(w + s.off_tab), reinterpret_cast<const float4*>(w + s.off_tab2),
-                 static_cast<__nv_bfloat16*>(dK), static_cast<__nv_bfloat16*>(dV)))
+                 static_cast<__nv_bfloat16*>(dK), static_cast<__nv_bfloat16*>(dV),
+                 static_cast<const __nv_bfloat16*>(gt.beta), static_cast<__nv_bfloat16*>(dbeta)))
       return LA_ERR_CUDA;
     ++nl;
+    if (gt.rms && gt.gamma) {  // dgamma: the query side's per-warp column sums, in a fixed order
+      la::simt::dgamma_sum_kernel<<<unsigned((p->d + la::simt::THREADS - 1) / la::simt::THREADS),
+                                    la::simt::THREADS, 0, stream>>>(s.ps.grid * 4, p->d, dgp, dgamma);
+      ++nl;
+      if ((rc = launched_ok())) return rc;
+    }
     g_last_launches = nl;
     return LA_OK;
   }

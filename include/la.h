@@ -204,8 +204,8 @@ int la_forward_gated(const la_problem* p, const la_gates* gates, const void* Q, 
  *   and with the suffix sums dS^c = sum_{b >= c} dS_b, dz^c likewise (a key of block c feeds
  *   the states of blocks c and later), for a key of block c:
  *   dV = beta phi(K) dS^c,  dK = [K > 0] (RoPE^T(beta V dS^cT) + dz^c),  dbeta = phi(K) . (dS^c V).
- * bf16 with d = 128 and neither beta nor RMSNorm runs on the tensor cores; every other case on
- * the CUDA cores.  The workspace is la_workspace_bytes() (which covers both). */
+ * bf16 with d = 128 runs on the tensor cores (every form); fp32, d = 32 / 64 and
+ * LA_FLAG_FORCE_SIMT on the CUDA cores.  The workspace is la_workspace_bytes(). */
 int la_backward(const la_problem* p, const la_gates* gates, const void* Q, const void* K, const void* V,
                 const void* G, const void* dO, void* dQ, void* dK, void* dV, void* dG, void* dbeta,
                 float* dgamma, void* workspace, size_t workspace_bytes, cudaStream_t stream);

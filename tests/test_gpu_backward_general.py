@@ -21,7 +21,7 @@ CASES = [
     (wl.custom("bwg_bc_sparse", B=1, H=2, T=5, Hh=4, W=33, block_frames=1, k_shift=-0.5, qkv_scale=1.0), False,
      False),
     (wl.custom("bwg_bc_long", B=1, H=3, T=12, Hh=9, W=40, block_frames=3), False, False),
-    # CUDA-core kernels: the gated forms, fp32 and small head dimensions
+    # the gated forms (tensor cores), fp32 and small head dimensions (CUDA cores)
     (wl.custom("bwg_beta", B=1, H=2, T=3, Hh=5, W=37), True, False),
     (wl.custom("bwg_rms", B=1, H=2, T=3, Hh=5, W=37), False, True),
     (wl.custom("bwg_bc_gated", B=1, H=2, T=5, Hh=6, W=10, block_frames=2), True, True),
@@ -73,10 +73,21 @@ def test_backward_forms_all_elements(w, use_beta, use_rms):
     _check(w, inputs, out, use_beta, use_rms)
 
 
-@pytest.mark.parametrize("w", [CASES[1][0], CASES[3][0]], ids=lambda w: w.name)
-def test_backward_blockcausal_cuda_core_path(w):
-    inputs, out = _run(w, False, False, simt=True)
-    _check(w, inputs, out, False, False)
+@pytest.mark.parametrize("w,use_beta,use_rms", [(CASES[1][0], False, False), (CASES[3][0], False, False),
+                                                 (CASES[6][0], True, True)], ids=["bc_ragged", "bc_long", "bc_gated"])
+def test_backward_cuda_core_path(w, use_beta, use_rms):
+    inputs, out = _run(w, use_beta, use_rms, simt=True)
+    _check(w, inputs, out, use_beta, use_rms)
+
+
+def test_backward_gated_forms_agree_across_paths():
+    # The tensor-core and CUDA-core kernels give the same gated gradients within the tolerance.
+    w = wl.custom("bwg_paths", B=2, H=3, T=5, Hh=5, W=37, block_frames=2)
+    _, a = _run(w, True, True)
+    _, b = _run(w, True, True, simt=True)
+    for i, (x, y) in enumerate(zip(a, b)):
+        scale = y.float().abs().max().item()
+        assert (x.float() - y.float()).abs().max().item() <= 2e-2 * scale, NAMES[i]
 
 
 def test_backward_bidirectional_forms_agree():
@@ -114,7 +125,7 @@ def test_backward_blockcausal_workload_sampled_heads():
 
 
 def test_backward_gated_720p_5s_sampled_heads():
-    # The full gated form at 720p/5s (CUDA-core kernels), two heads checked.
+    # The full gated form at 720p/5s, two heads checked.
     w = wl.WORKLOADS["720p_5s"]
     inputs, out = _run(w, True, True)
     Q, K, V, G, dO, beta, gamma = inputs
