@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--backward", action="store_true",
                     help="gradients (dQ, dK, dV, dG from dO; with --gated also dbeta, dgamma) of the "
                          "workload's form, bidirectional or block-causal")
+    ap.add_argument("--saved-state", action="store_true",
+                    help="with --backward: gradients from the states the forward pass returned "
+                         "(la_backward_saved), as a training step keeps them, instead of reducing them again")
     ap.add_argument("--stream", action="store_true",
                     help="block-causal workloads: one la_block_step call per block on a carried cache, "
                          "as a block-autoregressive generator runs")
@@ -279,6 +282,13 @@ def main():
             raise SystemExit("--backward takes no --causal or --stream")
         dO = wl.generate_grad(w, dev, seed=w.seed + 11 + 1000 * rank)
         grads = tuple(torch.empty_like(Q) for _ in range(4))
+        saved = {}
+        if args.saved_state:
+            # The states the forward pass computes (outside the timed region, as in a training step).
+            _, S_sv, z_sv = la.forward_gated(p, Q, K, V, G, ws=ws, return_states=True, **gates)
+            saved = dict(S=S_sv, z=z_sv)
+    elif args.saved_state:
+        raise SystemExit("--saved-state goes with --backward")
     if args.stream:
         # One block per call pair, on contiguous per-block tensors cut out before timing (a
         # generator produces each block's tensors as it goes).
@@ -306,7 +316,7 @@ def main():
         counter = {"launches": 0}
 
         def forward_plain():
-            la.backward(p, Q, K, V, G, dO, grads=grads, ws=ws, **gates)
+            la.backward(p, Q, K, V, G, dO, grads=grads, ws=ws, **gates, **saved)
             counter["launches"] = la.last_launch_count()
     elif args.causal:
         if w.block_frames > 0 or args.gated:
@@ -430,7 +440,8 @@ def main():
         config["gated"] = "write gate beta [B,H,N] + RMSNorm (gamma [d]) before the output gate"
     if args.backward:
         config["mode"] = ("backward: dQ, dK, dV, dG" + (", dbeta, dgamma" if args.gated else "") +
-                          " from dO (recomputes the forward state)")
+                          (" from dO and the forward's saved states (la_backward_saved)" if args.saved_state
+                           else " from dO (recomputes the forward state)"))
     if args.causal:
         config["mode"] = "token-causal (token n reads tokens 0..n; K and V are read by both passes)"
     if args.stream:
@@ -456,7 +467,8 @@ def main():
         line["e2e"] = e2e_stream(la, w, blocks, ws_s, S_c, z_c, dev, args, ldist, world)
     elif not args.no_e2e:
         line["e2e"] = e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates, causal=args.causal,
-                          dO=dO if args.backward else None, grads=grads if args.backward else None)
+                          dO=dO if args.backward else None, grads=grads if args.backward else None,
+                          saved=saved if args.backward else None)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         mode = "causal" if args.causal else ("backward" if args.backward else ("gated" if args.gated else "forward"))
         if args.backward and args.gated:
@@ -541,10 +553,12 @@ def e2e_stream(la, w, blocks, ws, S_c, z_c, dev, args, ldist, world):
             "pipelined": f"{nb} la_block_step calls per video; block j+1 copied in while block j computes"}
 
 
-def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None, causal=False, dO=None, grads=None):
+def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None, causal=False, dO=None, grads=None,
+        saved=None):
     """Same metric through the public API with the inputs in pinned host memory: every step
     copies the step's inputs host->device (Q, K, V, G, and the write gate when gated, or dO for
-    the backward pass), runs the operator and copies its outputs (O, or dQ, dK, dV, dG)
+    the backward pass, with the forward's states when it starts from them), runs the operator and
+    copies its outputs (O, or dQ, dK, dV, dG)
     device->host.  Steps are pipelined the way a caller streaming batches would run them: two
     device copies of the inputs and of the outputs, the host->device copies on one stream, the
     operator on the current stream and the device->host copies on a third, so step k+1's inputs
@@ -554,13 +568,14 @@ def e2e(la, p, w, Q, K, V, G, O, ws, dev, args, ldist, world, gates=None, causal
 
     gates = gates or {}
     if dO is not None:
-        srcs0 = [Q, K, V, G, dO] + ([gates["beta"]] if "beta" in gates else [])
+        saved = saved or {}
+        extra = ([("beta", gates["beta"])] if "beta" in gates else []) + sorted(saved.items())
+        srcs0 = [Q, K, V, G, dO] + [t for _, t in extra]
         outs0 = list(grads)
 
         def run(d, o):
             g = dict(gates)
-            if len(d) > 5:
-                g["beta"] = d[5]
+            g.update({name: d[5 + i] for i, (name, _) in enumerate(extra)})
             la.backward(p, d[0], d[1], d[2], d[3], d[4], grads=tuple(o), ws=ws, **g)
     else:
         srcs0 = [Q, K, V, G] + ([gates["beta"]] if "beta" in gates else [])

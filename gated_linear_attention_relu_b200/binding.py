@@ -28,7 +28,7 @@ EXPORTS = [
     "la_forward_bidir", "la_forward_blockcausal", "la_status_string", "la_device_error",
     "la_last_launch_count", "la_forward_marked", "la_selftest_host", "la_forward_bidir_static",
     "la_state_update", "la_forward_gated", "la_block_step", "la_forward_tokencausal", "la_backward_bidir",
-    "la_backward",
+    "la_backward", "la_backward_saved",
 ]
 
 
@@ -86,6 +86,8 @@ def load(path: Optional[str] = None):
         "la_backward_bidir": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_backward": (ctypes.c_int, [P, ctypes.POINTER(LaGates), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                        vp, sz, vp]),
+        "la_backward_saved": (ctypes.c_int, [P, ctypes.POINTER(LaGates), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                             vp, vp, vp, vp, sz, vp]),
         "la_forward_gated": (ctypes.c_int, [P, ctypes.POINTER(LaGates), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_apply": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "la_forward_bidir": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -378,11 +380,12 @@ def backward_bidir(p: Problem, Q, K, V, G, dO, grads=None, ws=None, stream=None)
 
 
 def backward(p: Problem, Q, K, V, G, dO, beta=None, gamma=None, rms_norm=False, norm_eps=1e-6, grads=None,
-             ws=None, stream=None):
+             ws=None, stream=None, S=None, z=None):
     """Gradients of the operator in any form (bidirectional or block-causal as ``p.block_frames``
     says; write gate ``beta`` and RMSNorm optional): returns (dQ, dK, dV, dG, dbeta, dgamma), with
     dbeta [B,H,N] when ``beta`` is given and dgamma [d] fp32 when RMSNorm has a weight ``gamma``
-    (else None)."""
+    (else None).  ``S``, ``z``: the states the forward pass returned (``forward_gated(...,
+    return_states=True)``); given, the state is not reduced again (la_backward_saved)."""
     import torch
 
     lib = load()
@@ -397,9 +400,15 @@ def backward(p: Problem, Q, K, V, G, dO, beta=None, gamma=None, rms_norm=False, 
         nbytes = ws.numel()
     cp = p.c()
     gates = LaGates(_ptr(beta), _ptr(gamma), float(norm_eps), 1 if rms_norm else 0)
-    _check(lib.la_backward(ctypes.byref(cp), ctypes.byref(gates), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(dO),
-                           _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dG), _ptr(dbeta), _ptr(dgamma), _ptr(ws), nbytes,
-                           _stream(stream)), "la_backward")
+    if S is not None or z is not None:
+        _check(lib.la_backward_saved(ctypes.byref(cp), ctypes.byref(gates), _ptr(S), _ptr(z), _ptr(Q), _ptr(K),
+                                     _ptr(V), _ptr(G), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dG),
+                                     _ptr(dbeta), _ptr(dgamma), _ptr(ws), nbytes, _stream(stream)),
+               "la_backward_saved")
+    else:
+        _check(lib.la_backward(ctypes.byref(cp), ctypes.byref(gates), _ptr(Q), _ptr(K), _ptr(V), _ptr(G), _ptr(dO),
+                               _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dG), _ptr(dbeta), _ptr(dgamma), _ptr(ws), nbytes,
+                               _stream(stream)), "la_backward")
     return dQ, dK, dV, dG, dbeta, dgamma
 
 

@@ -308,6 +308,24 @@ int launch_table(const PlanSet& s, const la_problem& q, void* ws, cudaStream_t s
   return launched_ok();
 }
 
+// The bf16 operand image (and z) of given fp32 unit states, with the cos/sin tables, in one launch:
+// what the tensor-core apply and query-side gradient kernels read when the states come from the
+// caller instead of the state kernel.
+int launch_pack(const PlanSet& s, const la_problem& q, const float* S, const float* z, void* ws, cudaStream_t st,
+                int* nl) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const int64_t threads = s.units * ((128 * 128 + 128) / 8);
+  const int64_t pblocks = (threads + la::cmb::THREADS - 1) / la::cmb::THREADS;
+  const int64_t tblocks = (s.tab_entries + la::cmb::THREADS - 1) / la::cmb::THREADS;
+  const Rope rope = make_rope(q);
+  la::cmb::pack_kernel<<<unsigned(pblocks + tblocks), la::cmb::THREADS, 0, st>>>(
+      s.units, 128, S, z, w + s.off_img, reinterpret_cast<float*>(w + s.off_zimg), s.pa, rope,
+      reinterpret_cast<float2*>(w + s.off_tab), standard_bands(q) ? reinterpret_cast<float2*>(w + s.off_tab2) : nullptr,
+      pblocks);
+  ++*nl;
+  return launched_ok();
+}
+
 int launch_state(const PlanSet& s, const la_problem& q, const void* K, const void* V, void* ws,
                  cudaStream_t st, int* nl, const void* beta = nullptr) {
   if (s.ps.total == 0) return LA_OK;
@@ -360,7 +378,9 @@ int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk
   uint8_t* im = img ? w + s.off_img : nullptr;
   float* zim = img ? reinterpret_cast<float*>(w + s.off_zimg) : nullptr;
   (void)q;
-  const int64_t cblocks = (threads + la::cmb::THREADS - 1) / la::cmb::THREADS;
+  const int64_t cblocks = (threads + la::cmb::THREADS - 1) / la::cmb::THREADS;       // prefix: one thread per group
+  const int64_t hblocks = s.ps.BH * la::cmb::blocks_per_unit(s.ps.d);               // combine: per head
+  const int64_t ublocks = s.units * la::cmb::blocks_per_unit(s.ps.d);               // blocksum: per unit
   // Block-causal, tensor-core path (several blocks, no accumulation): per-block sums of all units
   // in parallel, then the prefix over blocks.  The per-block states go to the caller's S_blk if it
   // wants them, else to the workspace's state area (on this path the inclusive states go only to
@@ -368,9 +388,8 @@ int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk
   if (s.tc && s.ps.nblk > 1 && !accumulate) {
     float* sb = S_blk ? S_blk : reinterpret_cast<float*>(w + s.off_states);
     float* zb = S_blk ? z_blk : reinterpret_cast<float*>(w + s.off_states) + s.units * q.d * q.d;
-    const int64_t t1 = s.units * groups;
-    if (launch_k(la::cmb::blocksum_kernel, unsigned((t1 + la::cmb::THREADS - 1) / la::cmb::THREADS),
-                 la::cmb::THREADS, 0, st, s.tc && s.ps.total > 0, s.ps, partial, sb, zb))
+    if (launch_k(la::cmb::blocksum_kernel, unsigned(ublocks), la::cmb::THREADS, 0, st, s.tc && s.ps.total > 0, s.ps,
+                 partial, sb, zb))
       return LA_ERR_CUDA;
     ++*nl;
     if (after) after(*nl);
@@ -386,7 +405,7 @@ int launch_combine(const PlanSet& s, const la_problem& q, void* ws, float* S_blk
   }
   // After the tensor-core state kernel (if it ran) the combine kernel may launch early; it waits
   // for that kernel before its first read.
-  if (launch_k(la::cmb::combine_kernel, unsigned(cblocks), la::cmb::THREADS, 0, st, s.tc && s.ps.total > 0,
+  if (launch_k(la::cmb::combine_kernel, unsigned(hblocks), la::cmb::THREADS, 0, st, s.tc && s.ps.total > 0,
                s.ps, partial, S_blk, z_blk, S_inc, z_inc, im, zim, accumulate ? 1 : 0))
     return LA_ERR_CUDA;
   ++*nl;
@@ -655,9 +674,12 @@ int la_forward_tokencausal(const la_problem* p, const void* Q, const void* K, co
 // Gradients of the operator in every form: bidirectional or block-causal (p->block_frames), with
 // the optional write gate and RMSNorm.  bf16 with d = 128 takes the tensor-core kernels; fp32,
 // d = 32 / 64 and LA_FLAG_FORCE_SIMT the CUDA-core kernels.
+// S_saved / z_saved (both or neither): the unit states token n reads, as the forward computed them
+// (the head's state, or each block's inclusive prefix); given, the forward state is not recomputed.
 static int backward_common(const la_problem* p, const Gates& gt, const void* Q, const void* K, const void* V,
                            const void* G, const void* dO, void* dQ, void* dK, void* dV, void* dG, void* dbeta,
-                           float* dgamma, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                           float* dgamma, void* ws, size_t ws_bytes, cudaStream_t stream,
+                           const float* S_saved = nullptr, const float* z_saved = nullptr) {
   static_assert(la::st::TILE == la::bw::TILE, "the backward kernels walk the state kernel's tile ranges");
   int rc;
   const bool has_tok = elems(*p) > 0;
@@ -671,6 +693,9 @@ static int backward_common(const la_problem* p, const Gates& gt, const void* Q, 
   if (gt.rms && gt.gamma && (rc = check_ptr(dgamma, true))) return rc;
   if (gt.beta && !aligned16(gt.beta)) return LA_ERR_ALIGN;
   if (gt.gamma && !aligned16(gt.gamma)) return LA_ERR_ALIGN;
+  if (S_saved || z_saved) {
+    if ((rc = check_ptr(S_saved, has_tok)) || (rc = check_ptr(z_saved, has_tok))) return rc;
+  }
   if (!has_tok) {
     g_last_launches = 0;
     if (gt.rms && gt.gamma) {  // no tokens: dgamma is zero
@@ -686,10 +711,15 @@ static int backward_common(const la_problem* p, const Gates& gt, const void* Q, 
   uint8_t* w = static_cast<uint8_t*>(ws);
   const Rope rope = make_rope(*p);
   if (s.tc) {
-    // Forward state (per unit: a head, or a block's inclusive prefix) and its operand image.
-    if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
-    if ((rc = launch_state(s, *p, K, V, ws, stream, &nl, gt.beta))) return rc;
-    if ((rc = launch_combine(s, *p, ws, nullptr, nullptr, nullptr, nullptr, true, stream, &nl))) return rc;
+    // Forward state (per unit: a head, or a block's inclusive prefix) and its operand image: from
+    // the caller's states, or reduced again from K and V.
+    if (S_saved) {
+      if ((rc = launch_pack(s, *p, S_saved, z_saved, ws, stream, &nl))) return rc;
+    } else {
+      if ((rc = launch_table(s, *p, ws, stream, &nl))) return rc;
+      if ((rc = launch_state(s, *p, K, V, ws, stream, &nl, gt.beta))) return rc;
+      if ((rc = launch_combine(s, *p, ws, nullptr, nullptr, nullptr, nullptr, true, stream, &nl))) return rc;
+    }
     const bool sb = standard_bands(*p);
     float* dgp = reinterpret_cast<float*>(w + s.off_dgamma);
     CUtensorMap tq, tg, tdo, tdq, tdg, tk, tv, tdk, tdv;
@@ -746,23 +776,27 @@ static int backward_common(const la_problem* p, const Gates& gt, const void* Q, 
   const PlanSet sp = make_plans(qs, sm);  // the CUDA-core kernels' tile ranges (32-token tiles)
   if ((rc = check_ws(sp, ws, ws_bytes))) return rc;
   float* partial = reinterpret_cast<float*>(w + sp.off_partial);
-  float* Sf = reinterpret_cast<float*>(w + sp.off_states);
-  float* zf = Sf + sp.units * p->d * p->d;
+  float* Sw = reinterpret_cast<float*>(w + sp.off_states);
+  float* zw = Sw + sp.units * p->d * p->d;
+  const float* Sf = S_saved ? S_saved : Sw;
+  const float* zf = S_saved ? z_saved : zw;
   float* dSf = reinterpret_cast<float*>(w + sp.off_states2);
   float* dzf = dSf + sp.units * p->d * p->d;
   float* dgp = reinterpret_cast<float*>(w + sp.off_dgamma);
   const int64_t groups = (int64_t(p->d) * p->d + p->d) / 8;
-  const unsigned ublocks = unsigned((sp.units * groups + la::cmb::THREADS - 1) / la::cmb::THREADS);
+  const unsigned ublocks = unsigned(sp.units * la::cmb::blocks_per_unit(p->d));
   const unsigned hblocks = unsigned((sp.ps.BH * groups + la::cmb::THREADS - 1) / la::cmb::THREADS);
-  // Forward states: per-unit sums, then (block-causal) the inclusive prefix over blocks.
-  if ((rc = launch_state(sp, qs, K, V, ws, stream, &nl, gt.beta))) return rc;
-  la::cmb::blocksum_kernel<<<ublocks, la::cmb::THREADS, 0, stream>>>(sp.ps, partial, Sf, zf);
-  ++nl;
-  if (sp.ps.nblk > 1) {
-    la::cmb::scan_kernel<<<hblocks, la::cmb::THREADS, 0, stream>>>(sp.ps.BH, sp.ps.nblk, p->d, Sf, zf, 0);
+  // Forward states (unless given): per-unit sums, then (block-causal) the inclusive prefix over blocks.
+  if (!S_saved) {
+    if ((rc = launch_state(sp, qs, K, V, ws, stream, &nl, gt.beta))) return rc;
+    la::cmb::blocksum_kernel<<<ublocks, la::cmb::THREADS, 0, stream>>>(sp.ps, partial, Sw, zw);
     ++nl;
+    if (sp.ps.nblk > 1) {
+      la::cmb::scan_kernel<<<hblocks, la::cmb::THREADS, 0, stream>>>(sp.ps.BH, sp.ps.nblk, p->d, Sw, zw, 0);
+      ++nl;
+    }
+    if ((rc = launched_ok())) return rc;
   }
-  if ((rc = launched_ok())) return rc;
   // Query side.
   const size_t smq = la::simt::bwdq_simt_smem(p->d);
   LA_SIMT_DISPATCH(*p, {
@@ -850,17 +884,7 @@ int la_apply(const la_problem* p, const void* Q, const void* G, const float* S, 
   int nl = 0;
   if (s.tc) {
     if ((rc = check_ws(s, ws, ws_bytes))) return rc;
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    const int64_t threads = s.units * ((128 * 128 + 128) / 8);
-    const int64_t pblocks = (threads + la::cmb::THREADS - 1) / la::cmb::THREADS;
-    const int64_t tblocks = (s.tab_entries + la::cmb::THREADS - 1) / la::cmb::THREADS;
-    const Rope rope = make_rope(*p);
-    la::cmb::pack_kernel<<<unsigned(pblocks + tblocks), la::cmb::THREADS, 0, stream>>>(
-        s.units, 128, S, z, w + s.off_img, reinterpret_cast<float*>(w + s.off_zimg), s.pa, rope,
-        reinterpret_cast<float2*>(w + s.off_tab),
-        standard_bands(*p) ? reinterpret_cast<float2*>(w + s.off_tab2) : nullptr, pblocks);
-    ++nl;
-    if ((rc = launched_ok())) return rc;
+    if ((rc = launch_pack(s, *p, S, z, ws, stream, &nl))) return rc;
   }
   if ((rc = launch_apply(s, *p, Q, G, S, z, O, ws, stream, &nl))) return rc;
   g_last_launches = nl;
@@ -950,7 +974,6 @@ int la_forward_gated(const la_problem* p, const la_gates* gates, const void* Q, 
                      cudaStream_t stream) {
   int rc = validate(p);
   if (rc) return rc;
-  if (p->block_frames == 0 && (S_incl || z_incl)) return LA_ERR_SHAPE;
   Gates gt;
   if ((rc = read_gates(gates, &gt))) return rc;
   return forward_common(p, Q, K, V, G, O, S_incl, z_incl, ws, ws_bytes, stream, nullptr, 0, gt);
@@ -966,13 +989,24 @@ int la_backward(const la_problem* p, const la_gates* gates, const void* Q, const
   return backward_common(p, gt, Q, K, V, G, dO, dQ, dK, dV, dG, dbeta, dgamma, ws, ws_bytes, stream);
 }
 
+int la_backward_saved(const la_problem* p, const la_gates* gates, const float* S, const float* z, const void* Q,
+                      const void* K, const void* V, const void* G, const void* dO, void* dQ, void* dK, void* dV,
+                      void* dG, void* dbeta, float* dgamma, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = validate(p);
+  if (rc) return rc;
+  if (!S || !z) return LA_ERR_NULL;
+  if (!aligned16(S) || !aligned16(z)) return LA_ERR_ALIGN;
+  Gates gt;
+  if ((rc = read_gates(gates, &gt))) return rc;
+  return backward_common(p, gt, Q, K, V, G, dO, dQ, dK, dV, dG, dbeta, dgamma, ws, ws_bytes, stream, S, z);
+}
+
 int la_forward_marked(const la_problem* p, const la_gates* gates, const void* Q, const void* K, const void* V,
                       const void* G, void* O, float* S_incl, float* z_incl, void* ws, size_t ws_bytes,
                       cudaStream_t stream, cudaEvent_t* marks, int nmarks) {
   int rc = validate(p);
   if (rc) return rc;
   if (nmarks < 0 || (nmarks > 0 && !marks)) return LA_ERR_NULL;
-  if (p->block_frames == 0 && (S_incl || z_incl)) return LA_ERR_SHAPE;
   if (p->flags & LA_FLAG_TOKEN_CAUSAL) {
     if (gates || S_incl || z_incl) return LA_ERR_UNSUPPORTED;
     return tokencausal_common(p, Q, K, V, G, O, ws, ws_bytes, stream, marks, nmarks);

@@ -299,23 +299,95 @@ rope_table_kernel(const Plan p, const __grid_constant__ Rope rope, float2* tab, 
   if (e < rope.tab_entries) rope_table_entry(p, rope, e, tab, tab2);
 }
 
+// Thread blocks per unit of the combine kernels: each block covers THREADS groups of 8 elements
+// of one unit's [S | z], so all of its threads read the same partial slots.
+__host__ __device__ constexpr int blocks_per_unit(int D) { return ((D * D + D) / 8 + THREADS - 1) / THREADS; }
+
+constexpr int MAXC = THREADS;  // slot offsets staged in shared memory per round
+
+// Shared per-block bookkeeping of the slots of unit u: thread 0 finds the unit's CTA range, then
+// the block's threads compute the float offsets of the slots of up to MAXC CTAs at a time (a
+// negative offset marks a slot that failed its bounds check).  `fn(j, m)` is called by every
+// thread for each round with the offsets of CTAs c0 + j .. c0 + j + m - 1 in `off`, in
+// increasing CTA order, between two block-wide barriers.
+template <typename Fn>
+__device__ __forceinline__ void for_unit_slots(const Plan& p, int64_t u, int64_t slot_floats, int64_t* off,
+                                               int64_t* rng, Fn&& fn) {
+  if (threadIdx.x == 0) {
+    int64_t first = 0, count = 0, c0 = 0, n = 0;
+    if (p.total > 0) unit_tiles(p, u, &first, &count);
+    if (count > 0) {
+      c0 = cta_of(p, first);
+      n = cta_of(p, first + count - 1) - c0 + 1;
+    }
+    rng[0] = c0;
+    rng[1] = n;
+  }
+  __syncthreads();
+  const int64_t c0 = rng[0], n = rng[1];
+  for (int64_t j = 0; j < n; j += MAXC) {
+    const int m = static_cast<int>(n - j < MAXC ? n - j : MAXC);
+    if (static_cast<int>(threadIdx.x) < m) {
+      const int64_t cc = c0 + j + threadIdx.x;
+      const int64_t k = u - unit_of_tile(p, cta_start(p, cc));
+      off[threadIdx.x] = in_bounds(k >= 0 && k < p.maxseg && cc < p.grid) ? (cc * p.maxseg + k) * slot_floats : -1;
+    }
+    __syncthreads();
+    fn(m);
+    __syncthreads();
+  }
+}
+
+// Adds 8 consecutive elements (from e0) of the given slots in order: S part, or the z rows of a
+// slot one after another.
+__device__ __forceinline__ void add_slots(const float* __restrict__ partial, const int64_t* off, int m, int D,
+                                          int zparts, int e0, float (&acc)[8]) {
+  if (e0 < D * D) {
+#pragma unroll 4
+    for (int j = 0; j < m; ++j) {
+      const int64_t o = off[j];
+      if (o < 0) continue;
+      const float4* s4 = reinterpret_cast<const float4*>(partial + o + e0);
+      const float4 a = s4[0], b = s4[1];
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+  } else {
+    for (int j = 0; j < m; ++j) {
+      const int64_t o = off[j];
+      if (o < 0) continue;
+      for (int zp = 0; zp < zparts; ++zp) {
+        const float4* s4 = reinterpret_cast<const float4*>(partial + o + D * D + zp * D + (e0 - D * D));
+        const float4 a = s4[0], b = s4[1];
+        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+      }
+    }
+  }
+}
+
+// Grid: BH * blocks_per_unit(d) blocks; block (bh, chunk) walks the units of head bh in order.
 __global__ void __launch_bounds__(THREADS)
 combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, float* z_blk, float* S_inc,
                float* z_inc, uint8_t* img, float* zimg, int accumulate) {
-  // Every thread reads the state kernel's partial sums: wait for that kernel first.
+  __shared__ int64_t off[MAXC];
+  __shared__ int64_t rng[2];
   pdl_trigger();
-  pdl_wait();
   const int D = p.d;
   const int groups = (D * D + D) / 8;
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
-  const int64_t bh = idx / groups;
-  if (bh >= p.BH) return;
-  const int e0 = static_cast<int>(idx - bh * groups) * 8;
+  const int bpu = blocks_per_unit(D);
+  const int64_t bh = blockIdx.x / static_cast<uint32_t>(bpu);
+  const int gi = static_cast<int>(blockIdx.x - bh * bpu) * THREADS + static_cast<int>(threadIdx.x);
+  if (bh >= p.BH) return;  // (whole blocks only)
+  const bool active = gi < groups;
+  const int e0 = 8 * (active ? gi : 0);
   const int64_t slot_floats = static_cast<int64_t>(D) * D + static_cast<int64_t>(p.zparts) * D;
+  // Every thread reads the state kernel's partial sums: wait for that kernel first.
+  pdl_wait();
   float run[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) run[e] = 0.f;
-  if (accumulate) {
+  if (accumulate && active) {
     // Cache update: the running sum starts from the carried state in S_inc / z_inc (one unit per
     // head), which is then overwritten with carried + this call's sum.
     const float* src = (e0 < D * D) ? S_inc + bh * D * D + e0 : z_inc + bh * D + (e0 - D * D);
@@ -328,31 +400,10 @@ combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, fl
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    int64_t first = 0, count = 0;
-    if (p.total > 0) unit_tiles(p, u, &first, &count);
-    if (count > 0) {
-      const int64_t c0 = cta_of(p, first), c1 = cta_of(p, first + count - 1);
-      // (unrolled so that the loads of several slots are in flight together)
-#pragma unroll 4
-      for (int64_t cc = c0; cc <= c1; ++cc) {
-        const int64_t k = u - unit_of_tile(p, cta_start(p, cc));
-        if (!in_bounds(k >= 0 && k < p.maxseg && cc < p.grid)) continue;
-        const float* src = partial + (cc * p.maxseg + k) * slot_floats;
-        if (e0 < D * D) {
-          const float4* s4 = reinterpret_cast<const float4*>(src + e0);
-          const float4 a = s4[0], b = s4[1];
-          acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-          acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-        } else {
-          for (int zp = 0; zp < p.zparts; ++zp) {
-            const float4* s4 = reinterpret_cast<const float4*>(src + D * D + zp * D + (e0 - D * D));
-            const float4 a = s4[0], b = s4[1];
-            acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-            acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-          }
-        }
-      }
-    }
+    for_unit_slots(p, u, slot_floats, off, rng, [&](int m) {
+      if (active) add_slots(partial, off, m, D, p.zparts, e0, acc);
+    });
+    if (!active) continue;
     if (S_blk) store8(S_blk, z_blk, u, D, e0, acc);
 #pragma unroll
     for (int e = 0; e < 8; ++e) run[e] += acc[e];
@@ -362,39 +413,30 @@ combine_kernel(const Plan p, const float* __restrict__ partial, float* S_blk, fl
 }
 
 // Block-causal combine, first pass: the state of every (head, block) unit alone, summed over its
-// CTAs' partial slots in increasing CTA order.  One thread per (unit, group of 8 consecutive
-// elements of [S | z]), so all units run in parallel.
+// CTAs' partial slots in increasing CTA order.  Grid: units * blocks_per_unit(d) blocks, so all
+// units run in parallel.
 __global__ void __launch_bounds__(THREADS)
 blocksum_kernel(const Plan p, const float* __restrict__ partial, float* __restrict__ S_blk, float* __restrict__ z_blk) {
+  __shared__ int64_t off[MAXC];
+  __shared__ int64_t rng[2];
   pdl_trigger();
-  pdl_wait();
   const int D = p.d;
   const int groups = (D * D + D) / 8;
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * THREADS + threadIdx.x;
-  const int64_t u = idx / groups;
-  if (u >= p.BH * p.nblk) return;
-  const int e0 = static_cast<int>(idx - u * groups) * 8;
+  const int bpu = blocks_per_unit(D);
+  const int64_t u = blockIdx.x / static_cast<uint32_t>(bpu);
+  const int gi = static_cast<int>(blockIdx.x - u * bpu) * THREADS + static_cast<int>(threadIdx.x);
+  if (u >= p.BH * p.nblk) return;  // (whole blocks only)
+  const bool active = gi < groups;
+  const int e0 = 8 * (active ? gi : 0);
   const int64_t slot_floats = static_cast<int64_t>(D) * D + static_cast<int64_t>(p.zparts) * D;
+  pdl_wait();
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  int64_t first = 0, count = 0;
-  if (p.total > 0) unit_tiles(p, u, &first, &count);
-  if (count > 0) {
-    const int64_t c0 = cta_of(p, first), c1 = cta_of(p, first + count - 1);
-    for (int64_t cc = c0; cc <= c1; ++cc) {
-      const int64_t k = u - unit_of_tile(p, cta_start(p, cc));
-      if (!in_bounds(k >= 0 && k < p.maxseg && cc < p.grid)) continue;
-      const float* src = partial + (cc * p.maxseg + k) * slot_floats;
-      for (int zp = 0; zp < (e0 < D * D ? 1 : p.zparts); ++zp) {
-        const float4* s4 = reinterpret_cast<const float4*>(e0 < D * D ? src + e0 : src + D * D + zp * D + (e0 - D * D));
-        const float4 a = s4[0], b = s4[1];
-        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-      }
-    }
-  }
-  store8(S_blk, z_blk, u, D, e0, acc);
+  for_unit_slots(p, u, slot_floats, off, rng, [&](int m) {
+    if (active) add_slots(partial, off, m, D, p.zparts, e0, acc);
+  });
+  if (active) store8(S_blk, z_blk, u, D, e0, acc);
 }
 
 // Block-causal combine, second pass: inclusive prefix over the blocks of every head, from the

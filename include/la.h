@@ -180,8 +180,10 @@ typedef struct {
 } la_gates;
 
 /* The whole operator with the optional terms of la_gates: bidirectional if p->block_frames
- * == 0 (then S_incl and z_incl must be NULL), else block-causal with the same arguments as
- * la_forward_blockcausal (S_incl / z_incl receive the gated inclusive states when non-NULL).
+ * == 0, else block-causal with the same arguments as la_forward_blockcausal.  S_incl / z_incl
+ * (both or neither; fp32, 16-byte aligned) receive, when non-NULL, the states the outputs read:
+ * [B,H,d,d] / [B,H,d] bidirectional (each head's state, beta included), [B,H,nblk,d,d] /
+ * [B,H,nblk,d] block-causal (each block's inclusive prefix) -- what la_backward_saved takes.
  * gates == NULL, or beta == NULL with rms_norm == 0, computes exactly what la_forward_bidir /
  * la_forward_blockcausal compute.  beta and gamma must be 16-byte aligned when given. */
 int la_forward_gated(const la_problem* p, const la_gates* gates, const void* Q, const void* K,
@@ -209,6 +211,19 @@ int la_forward_gated(const la_problem* p, const la_gates* gates, const void* Q, 
 int la_backward(const la_problem* p, const la_gates* gates, const void* Q, const void* K, const void* V,
                 const void* G, const void* dO, void* dQ, void* dK, void* dV, void* dG, void* dbeta,
                 float* dgamma, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* la_backward given the states the forward pass computed, so that the forward state is not
+ * reduced again from K and V (a training step keeps them from its forward: 64 KB per head and
+ * block at d = 128).  S [B,H,nblk,d,d] and z [B,H,nblk,d] fp32 (nblk = 1 bidirectional), 16-byte
+ * aligned, exactly as la_forward_gated returns them in S_incl / z_incl for the same problem and
+ * gates (with beta, the gated state; z is never gated).  Results are those of la_backward up to
+ * the rounding of the states the caller passes: with the forward's own states, bit for bit on
+ * the tensor cores.  Errors: LA_ERR_NULL if S or z is NULL, LA_ERR_ALIGN if either is not
+ * 16-byte aligned; otherwise as la_backward.  Nothing is written to S or z. */
+int la_backward_saved(const la_problem* p, const la_gates* gates, const float* S, const float* z,
+                      const void* Q, const void* K, const void* V, const void* G, const void* dO, void* dQ,
+                      void* dK, void* dV, void* dG, void* dbeta, float* dgamma, void* workspace,
+                      size_t workspace_bytes, cudaStream_t stream);
 
 /* The whole operator (bidirectional if p->block_frames == 0, else block-causal, with the
  * same arguments as la_forward_gated; gates may be NULL; token-causal, as la_forward_tokencausal,

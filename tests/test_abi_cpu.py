@@ -132,6 +132,16 @@ def test_backward_rejects_bad_arguments_before_cuda():
     assert lib.la_backward(ctypes.byref(cp), ctypes.byref(g), *([16] * 9), None, 24, 16, 1 << 30, None) == 4
     g = bnd.LaGates(None, None, 1e-6, 3)
     assert lib.la_backward(ctypes.byref(cp), ctypes.byref(g), *([16] * 9), None, None, 16, 1 << 30, None) == 5
+    # with saved states: both states are required and 16-byte aligned; then the same checks
+    g = bnd.LaGates(None, None, 1e-6, 0)
+    for S, z, status in ((None, 16, 1), (16, None, 1), (24, 16, 4), (16, 40, 4)):
+        assert lib.la_backward_saved(ctypes.byref(cp), ctypes.byref(g), S, z, *([16] * 9), None, None, 16, 1 << 30,
+                                     None) == status
+    assert lib.la_backward_saved(ctypes.byref(cp), ctypes.byref(g), 16, 16, None, *([16] * 8), None, None, 16,
+                                 1 << 30, None) == 1
+    g = bnd.LaGates(None, None, 1e-6, 3)
+    assert lib.la_backward_saved(ctypes.byref(cp), ctypes.byref(g), 16, 16, *([16] * 9), None, None, 16, 1 << 30,
+                                 None) == 5
 
 
 def test_static_entry_point_checks_pointers_before_cuda():

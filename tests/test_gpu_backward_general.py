@@ -138,3 +138,71 @@ def test_backward_gated_720p_5s_sampled_heads():
             e = rel_err(to64(out[i][0, flat]), refs[i])
             print(f"gated backward 720p_5s head {flat} {NAMES[i]}: {e:.2e}")
             assert e <= tol_for(w.dtype), (flat, NAMES[i], e)
+
+
+SAVED = [CASES[0], CASES[1], CASES[4], CASES[5], CASES[6]]
+
+
+@pytest.mark.parametrize("w,use_beta,use_rms", SAVED, ids=[c[0].name for c in SAVED])
+def test_backward_from_saved_states_equals_recompute(w, use_beta, use_rms):
+    # la_backward_saved with the states la_forward_gated returned gives la_backward's gradients bit
+    # for bit on the tensor cores (the same operand image, built from the same fp32 sums).
+    (Q, K, V, G, dO, beta, gamma), ref = _run(w, use_beta, use_rms)
+    p = la.Problem.from_workload(w)
+    _, S, z = la.forward_gated(p, Q, K, V, G, beta=beta, gamma=gamma, rms_norm=use_rms, norm_eps=1e-6,
+                               return_states=True)
+    out = la.backward(p, Q, K, V, G, dO, beta=beta, gamma=gamma, rms_norm=use_rms, norm_eps=1e-6, S=S, z=z)
+    torch.cuda.synchronize()
+    assert la.device_error() == 0
+    for i, (x, y) in enumerate(zip(out, ref)):
+        assert (x is None) == (y is None), NAMES[i]
+        if x is not None:
+            assert torch.equal(x, y), NAMES[i]
+
+
+def test_forward_states_bidirectional_match_oracle():
+    # la_forward_gated returns each head's state in bidirectional mode too (beta included, z not).
+    w = wl.custom("fwd_states", B=1, H=2, T=3, Hh=5, W=37)
+    Q, K, V, G = wl.generate(w, "cuda")
+    beta, _ = wl.generate_gates(w, "cuda")
+    p = la.Problem.from_workload(w)
+    _, S, z = la.forward_gated(p, Q, K, V, G, beta=beta, return_states=True)
+    torch.cuda.synchronize()
+    pos = orc.grid_positions(w.T, w.Hh, w.W)
+    for flat in range(w.B * w.H):
+        b, h = divmod(flat, w.H)
+        Sr, zr = orc.head_state(to64(K[b, h]), to64(V[b, h]), pos, w.bands, w.rope_base, beta=to64(beta[b, h]))
+        assert rel_err(to64(S[b, h, 0]), Sr) <= tol_for(w.dtype)
+        assert rel_err(to64(z[b, h, 0]), zr) <= tol_for(w.dtype)
+
+
+@pytest.mark.parametrize("w,use_beta,use_rms", [CASES[7], CASES[8]], ids=[CASES[7][0].name, CASES[8][0].name])
+def test_backward_from_saved_states_cuda_core_path(w, use_beta, use_rms):
+    # fp32 and small head dimensions: the saved-state gradients match the oracle.
+    Q, K, V, G = wl.generate(w, "cuda")
+    dO = wl.generate_grad(w, "cuda")
+    beta, gamma = wl.generate_gates(w, "cuda")
+    b = beta if use_beta else None
+    gm = gamma if use_rms else None
+    p = la.Problem.from_workload(w)
+    _, S, z = la.forward_gated(p, Q, K, V, G, beta=b, gamma=gm, rms_norm=use_rms, norm_eps=1e-6,
+                               return_states=True)
+    out = la.backward(p, Q, K, V, G, dO, beta=b, gamma=gm, rms_norm=use_rms, norm_eps=1e-6, S=S, z=z)
+    torch.cuda.synchronize()
+    assert la.device_error() == 0
+    _check(w, (Q, K, V, G, dO, b, gm), out, use_beta, use_rms)
+
+
+def test_backward_from_saved_states_blockcausal_workload_equals_recompute():
+    # The block-causal workload with the inclusive states of its forward pass.
+    w = wl.WORKLOADS["blockcausal"]
+    Q, K, V, G = wl.generate(w, "cuda")
+    dO = wl.generate_grad(w, "cuda")
+    p = la.Problem.from_workload(w)
+    _, S, z = la.forward_gated(p, Q, K, V, G, return_states=True)
+    out = la.backward(p, Q, K, V, G, dO, S=S, z=z)
+    ref = la.backward(p, Q, K, V, G, dO)
+    torch.cuda.synchronize()
+    assert la.device_error() == 0
+    for i in range(4):
+        assert torch.equal(out[i], ref[i]), NAMES[i]
