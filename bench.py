@@ -92,7 +92,7 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clocks"}
 
-    def __init__(self, index, period=0.005):
+    def __init__(self, index, period=0.001):
         self.samples, self.reasons, self.ok = [], set(), False
         self.period, self._stop = period, threading.Event()
         try:
@@ -462,6 +462,9 @@ def main():
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
+    if line["clocks"].get("sm_mhz"):
+        # Clock-normalised step time: ms per step x median SM MHz (compare runs at different clocks).
+        line["clocks"]["ms_per_step_x_sm_mhz"] = ms_per_step * line["clocks"]["sm_mhz"]
 
     if not args.no_e2e and args.stream:
         line["e2e"] = e2e_stream(la, w, blocks, ws_s, S_c, z_c, dev, args, ldist, world)
