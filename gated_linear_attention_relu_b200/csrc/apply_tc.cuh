@@ -241,15 +241,24 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (warp < 4) {
     regs_dec<REGS_CTRL>();
     if (warp == 0 && lane == 0) {
-      // ---------------------------------------------------------- TMA producer: state, Q
-      pdl_wait();
+      // ---------------------------------------------------------- TMA producer: Q, state
+      // A tile's Q is requested before its unit's state image, and only the image waits for the
+      // kernels before (the first Q tiles land while they finish).
       int64_t issued_q = 0, issued_s = 0;
       int64_t prev_unit = -1;
       for (int64_t g = g0; g < g1; ++g) {
         const int64_t i = g - g0;
         const TileInfo ti = tile_info(p, g);
         in_bounds(ti.unit < p.BH * p.nblk && ti.bh < p.BH && ti.n0 < ti.n_end && ti.n_end <= p.N);
+        const int qs = static_cast<int>(i % QST);
+        if (!mbar_wait(&bars->qempty[qs], static_cast<uint32_t>(((i / QST) & 1) ^ 1), abort_flag, LA_SLEEP_PROD)) break;
+        mbar_arrive_expect_tx(&bars->qfull[qs], BUF);
+        const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
+        tma_load_3d(smem + OFF_Q + qs * BUF, &tmQ, 0, n0, bh, &bars->qfull[qs]);
+        tma_load_3d(smem + OFF_Q + qs * BUF + HALF, &tmQ, 64, n0, bh, &bars->qfull[qs]);
+        ++issued_q;
         if (ti.unit != prev_unit) {
+          if (prev_unit < 0) pdl_wait();
           const int64_t ku = ti.unit - u_first;
           const int b = static_cast<int>(ku % NSB);
           if (!mbar_wait(&bars->sfree[b], static_cast<uint32_t>(((ku / NSB) & 1) ^ 1), abort_flag, LA_SLEEP_PROD)) break;
@@ -258,13 +267,6 @@ apply_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           prev_unit = ti.unit;
           ++issued_s;
         }
-        const int qs = static_cast<int>(i % QST);
-        if (!mbar_wait(&bars->qempty[qs], static_cast<uint32_t>(((i / QST) & 1) ^ 1), abort_flag, LA_SLEEP_PROD)) break;
-        mbar_arrive_expect_tx(&bars->qfull[qs], BUF);
-        const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
-        tma_load_3d(smem + OFF_Q + qs * BUF, &tmQ, 0, n0, bh, &bars->qfull[qs]);
-        tma_load_3d(smem + OFF_Q + qs * BUF + HALF, &tmQ, 64, n0, bh, &bars->qfull[qs]);
-        ++issued_q;
       }
       if (*abort_flag) {
         // Let every copy still in flight land before the CTA's shared memory goes away.
