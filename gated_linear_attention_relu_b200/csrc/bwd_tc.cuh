@@ -108,7 +108,7 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                __nv_bfloat16* __restrict__ dGg, const float* __restrict__ gamma, float norm_eps,
                float* __restrict__ dgamma_part) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   BarsQ* bars = reinterpret_cast<BarsQ*>(smem + QO_BAR);
   float* xch = reinterpret_cast<float*>(smem + QO_X);
   const uint32_t sbase = smem_u32(smem);
@@ -602,7 +602,7 @@ bwdk_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                __nv_bfloat16* __restrict__ dVg, const __nv_bfloat16* __restrict__ beta,
                __nv_bfloat16* __restrict__ dbeta) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   BarsK* bars = reinterpret_cast<BarsK*>(smem + KO_BAR);
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;

@@ -90,7 +90,7 @@ causal_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                  const float* __restrict__ start, const float2* __restrict__ tab,
                  const float4* __restrict__ tab2) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
   float* zs = reinterpret_cast<float*>(smem + OFF_Z);
   const uint32_t sbase = smem_u32(smem);

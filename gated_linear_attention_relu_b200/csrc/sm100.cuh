@@ -43,6 +43,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The kernel's dynamic shared memory rounded up to a 1024-byte boundary (the 128B-swizzled operand
+// layouts need it), derived from the shared array itself so that the compiler still knows the
+// pointer to be in shared memory: plain C++ accesses through it become shared-memory loads and
+// stores rather than generic ones.
+__device__ __forceinline__ uint8_t* align_smem_1k(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

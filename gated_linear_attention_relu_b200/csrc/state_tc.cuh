@@ -84,7 +84,7 @@ state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 const float4* __restrict__ tab2, const __nv_bfloat16* __restrict__ beta,
                 float* __restrict__ partial) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
   const uint32_t sbase = smem_u32(smem);
 
