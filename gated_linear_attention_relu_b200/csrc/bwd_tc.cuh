@@ -488,14 +488,13 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const float keep = up ? gv[e + size / 2] : gv[e];
           const float send = up ? gv[e] : gv[e + size / 2];
           const float other = __shfl_xor_sync(0xffffffffu, send, off);
-          gv[e] = up ? other + keep : keep + other;
+          gv[e] = keep + other;  // (IEEE addition commutes: both lanes form the same sum)
         }
       }
       dgacc += gv[0];
       }
       // dz over this warp's 32 rows for this quarter's 32 channels: lane L ends with channel
-      // 32 part + L (a butterfly that halves the range per step, each sum formed once, lower
-      // lane first).
+      // 32 part + L (a butterfly that halves the range per step, each sum formed once).
       {
         float v[32];
 #pragma unroll
@@ -511,7 +510,7 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             const float keep = up ? v[e + size / 2] : v[e];
             const float send = up ? v[e] : v[e + size / 2];
             const float other = __shfl_xor_sync(0xffffffffu, send, off);
-            v[e] = up ? other + keep : keep + other;
+            v[e] = keep + other;  // (IEEE addition commutes: both lanes form the same sum)
           }
         }
         dzacc += v[0];
