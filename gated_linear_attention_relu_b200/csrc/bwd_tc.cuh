@@ -190,6 +190,17 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // dS += phi(Q)^T dnum (frees Q first);  dphi(q) = dnum S^T
         if (!mbar_wait(&bars->dn, ph, abort_flag)) break;
         tc_fence_after();
+        // The gate pass has written this tile's dG over G: it goes out now (one bulk group), so
+        // that G's buffer can take the next tile's G while this tile's dq epilogue runs.  A tile
+        // that ends inside a head's block (block-causal units) is written out row by row by the
+        // math warps; its groups stay (empty) so the group accounting is the same.
+        const bool tma_out = (ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N);
+        const int32_t tn0 = static_cast<int32_t>(ti.n0), tbh = static_cast<int32_t>(ti.bh);
+        if (tma_out) {
+          tma_store_3d(&tmDG, smem + QO_G, 0, tn0, tbh);
+          tma_store_3d(&tmDG, smem + QO_G + HALF, 64, tn0, tbh);
+        }
+        bulk_commit_group();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + QCOL_DS, desc_mn(sbase + QO_Q, kk), desc_mn(sbase + QO_DO, kk), IDESC_TD,
@@ -198,11 +209,13 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + QCOL_DPQ, desc_k(sbase + QO_DO, kk), desc_k(sbase + QO_S, kk), IDESC_QST, kk > 0 ? 1u : 0u);
-        bulk_wait_group_read0();  // the previous tile's dQ has left the staging buffer the epilogue reuses
+        // The previous tile's dQ (the older of the two groups in flight) has left the staging
+        // buffer the dq epilogue reuses.
+        bulk_wait_group_read1();
         mma_commit(&bars->dpqready);
         // The next tile's Q once dS has read this one (and, at a new unit, the state image and z
-        // once dphi(q) has read the image); its dO once dphi(q) has read dnum.  (G holds this
-        // tile's dG until it is stored.)
+        // once dphi(q) has read the image); its dO once dphi(q) has read dnum; its G once this
+        // tile's dG has been read out.
         if (has_next) {
           if (!mbar_wait(next_new_unit ? &bars->dpqready : &bars->qfree, ph, abort_flag)) break;
           mbar_arrive_expect_tx(&bars->full, BUF + (next_new_unit ? BUF + 512u : 0u));
@@ -217,32 +230,18 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           mbar_arrive_expect_tx(&bars->full_do, BUF);
           load2(QO_DO, &tmDO, tn, &bars->full_do);
           ++issued_do;
-        }
-        // dG (over G) and dQ (staged) of this tile out, as two groups; the next tile's G once dG
-        // has been read out (dQ's read is waited for before the next dq epilogue may start).
-        if (!mbar_wait(&bars->out, ph, abort_flag)) break;
-        {
-          // A tile that ends inside a head's block (block-causal units) was written out row by row
-          // by the math warps; the groups stay (empty) so the group accounting is the same.
-          const bool tma_out = (ti.n0 + TILE <= ti.n_end) || (ti.n_end == p.N);
-          const int32_t n0 = static_cast<int32_t>(ti.n0), bh = static_cast<int32_t>(ti.bh);
-          if (tma_out) {
-            tma_store_3d(&tmDG, smem + QO_G, 0, n0, bh);
-            tma_store_3d(&tmDG, smem + QO_G + HALF, 64, n0, bh);
-          }
-          bulk_commit_group();
-          if (tma_out) {
-            tma_store_3d(&tmDQ, smem + QO_DQ, 0, n0, bh);
-            tma_store_3d(&tmDQ, smem + QO_DQ + HALF, 64, n0, bh);
-          }
-          bulk_commit_group();
-          bulk_wait_group_read1();
-        }
-        if (has_next) {
+          bulk_wait_group_read0();
           mbar_arrive_expect_tx(&bars->full_g, BUF);
           load2(QO_G, &tmG, tn, &bars->full_g);
           ++issued_g;
         }
+        // dQ (staged) of this tile out.
+        if (!mbar_wait(&bars->out, ph, abort_flag)) break;
+        if (tma_out) {
+          tma_store_3d(&tmDQ, smem + QO_DQ, 0, tn0, tbh);
+          tma_store_3d(&tmDQ, smem + QO_DQ + HALF, 64, tn0, tbh);
+        }
+        bulk_commit_group();
       }
       bulk_wait_group0();
       if (*abort_flag) {
