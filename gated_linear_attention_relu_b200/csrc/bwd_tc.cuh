@@ -65,8 +65,8 @@ struct BarsQ {
   uint64_t full_do;  // dO landed
   uint64_t full_g;   // G landed
   uint64_t rot, numready, dn;
-  uint64_t qfree;     // MMA: dS += phi(Q)^T dnum done (the last reader of Q)
-  uint64_t dpqready;  // MMA: dphi(q) = dnum S^T done too (the last reader of dnum, the state image)
+  uint64_t dpqready;  // MMA: dphi(q) = dnum S^T done (the last reader of the state image)
+  uint64_t qfree;     // MMA: dS += phi(Q)^T dnum done too (the last reader of Q and dnum)
   uint64_t out, final_;
   uint64_t pair[4];  // the four warps of rows 32q .. 32q+31: two meetings per tile (den, then dy.y)
   uint32_t tmem_base;
@@ -201,11 +201,8 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tma_store_3d(&tmDG, smem + QO_G + HALF, 64, tn0, tbh);
         }
         bulk_commit_group();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + QCOL_DS, desc_mn(sbase + QO_Q, kk), desc_mn(sbase + QO_DO, kk), IDESC_TD,
-                   (kk > 0 || !first) ? 1u : 0u);
-        mma_commit(&bars->qfree);
+        // dphi(q) first: the math warps wait for it (dq epilogue); dS is read only at the end of a
+        // unit, and its completion frees Q for the next tile.
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + QCOL_DPQ, desc_k(sbase + QO_DO, kk), desc_k(sbase + QO_S, kk), IDESC_QST, kk > 0 ? 1u : 0u);
@@ -213,11 +210,15 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // buffer the dq epilogue reuses.
         bulk_wait_group_read1();
         mma_commit(&bars->dpqready);
-        // The next tile's Q once dS has read this one (and, at a new unit, the state image and z
-        // once dphi(q) has read the image); its dO once dphi(q) has read dnum; its G once this
-        // tile's dG has been read out.
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + QCOL_DS, desc_mn(sbase + QO_Q, kk), desc_mn(sbase + QO_DO, kk), IDESC_TD,
+                   (kk > 0 || !first) ? 1u : 0u);
+        mma_commit(&bars->qfree);
+        // The next tile's Q and dO once dS, the last product, has read this tile's (and, at a new
+        // unit, the state image and z with them); its G once this tile's dG has been read out.
         if (has_next) {
-          if (!mbar_wait(next_new_unit ? &bars->dpqready : &bars->qfree, ph, abort_flag)) break;
+          if (!mbar_wait(&bars->qfree, ph, abort_flag)) break;
           mbar_arrive_expect_tx(&bars->full, BUF + (next_new_unit ? BUF + 512u : 0u));
           if (next_new_unit) {
             zslot ^= 1;
@@ -226,7 +227,6 @@ bwdq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           load2(QO_Q, &tmQ, tn, &bars->full);
           ++issued;
-          if (!mbar_wait(&bars->dpqready, ph, abort_flag)) break;
           mbar_arrive_expect_tx(&bars->full_do, BUF);
           load2(QO_DO, &tmDO, tn, &bars->full_do);
           ++issued_do;
