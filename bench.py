@@ -94,7 +94,7 @@ class ClockSampler:
 
     def __init__(self, index, period=0.001):
         self.samples, self.reasons, self.ok = [], set(), False
-        self.mem, self.power = [], []
+        self.mem = []
         self.period, self._stop = period, threading.Event()
         try:
             import pynvml
@@ -115,7 +115,6 @@ class ClockSampler:
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
                 self.mem.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_MEM))
-                self.power.append(nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0)
                 r = get_r(self.h)
                 for bit, name in self.REASONS.items():
                     if r & bit:
@@ -141,8 +140,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
                 "samples": len(self.samples),
-                "mem_mhz": statistics.median(self.mem) if self.mem else None,
-                "power_w": statistics.median(self.power) if self.power else None}
+                "mem_mhz": statistics.median(self.mem) if self.mem else None}
 
 
 def oracle_sample(w, seconds, steps=None, warmup=0, mode="forward"):
