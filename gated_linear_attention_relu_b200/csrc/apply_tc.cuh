@@ -23,9 +23,8 @@
 //                 sigmoid(g) and rounded to bf16 in place over the staged G tile.  The two halves
 //                 of a row swap their partial denominators through tensor memory.
 // TMEM: group m owns accumulator columns [256m, 256m+128), A columns [256m+128, 256m+192) and
-// partial-denominator columns [256m+192, 256m+196).  One state buffer: a CTA whose range crosses
-// a unit boundary loads the next unit's image once the last product of the previous unit has
-// been issued; the 32 KB a second buffer would take stay with L1, which holds the cos/sin table.
+// partial-denominator columns [256m+192, 256m+196).  (Shared memory stays within the 196 KB
+// configuration, so that L1 keeps room for the cos/sin table.)
 // The control warpgroup hands registers to the math groups (setmaxnreg); the host checks the
 // launch's register budget before launching.
 #pragma once
@@ -39,7 +38,7 @@
 #define LA_AP_GST 2
 #endif
 #ifndef LA_AP_NSB
-#define LA_AP_NSB 1
+#define LA_AP_NSB 2
 #endif
 
 namespace la {
@@ -49,8 +48,7 @@ constexpr int TILE = 128;
 constexpr int D = 128;
 constexpr int QST = LA_AP_QST;  // Q stages (freed once the math group has read them)
 constexpr int GST = LA_AP_GST;  // G / O stages (freed when the O tile has been stored)
-constexpr int NSB = LA_AP_NSB;  // state operand buffers (a buffer's parity is tested one unit
-                                // ahead at most: a group cannot pass a tile whose image is missing)
+constexpr int NSB = LA_AP_NSB;  // state operand buffers
 constexpr int NWG = 2;          // math groups (two warpgroups each, one per channel half)
 constexpr int MATH_WGS = 2 * NWG;
 constexpr int THREADS = 128 * (1 + MATH_WGS);
