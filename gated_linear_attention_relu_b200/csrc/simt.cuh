@@ -303,12 +303,12 @@ rope_table_kernel(const Plan p, const __grid_constant__ Rope rope, float2* tab, 
 // of one unit's [S | z], so all of its threads read the same partial slots.
 __host__ __device__ constexpr int blocks_per_unit(int D) { return ((D * D + D) / 8 + THREADS - 1) / THREADS; }
 
-constexpr int MAXC = THREADS;  // slot offsets staged in shared memory per round
+constexpr int MAXC = THREADS;  // slot offsets staged in shared memory per pass
 
 // Shared per-block bookkeeping of the slots of unit u: thread 0 finds the unit's CTA range, then
 // the block's threads compute the float offsets of the slots of up to MAXC CTAs at a time (a
 // negative offset marks a slot that failed its bounds check).  `fn(j, m)` is called by every
-// thread for each round with the offsets of CTAs c0 + j .. c0 + j + m - 1 in `off`, in
+// thread for each pass with the offsets of CTAs c0 + j .. c0 + j + m - 1 in `off`, in
 // increasing CTA order, between two block-wide barriers.
 template <typename Fn>
 __device__ __forceinline__ void for_unit_slots(const Plan& p, int64_t u, int64_t slot_floats, int64_t* off,
