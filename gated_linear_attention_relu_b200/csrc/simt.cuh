@@ -307,9 +307,9 @@ constexpr int MAXC = THREADS;  // slot offsets staged in shared memory per pass
 
 // Shared per-block bookkeeping of the slots of unit u: thread 0 finds the unit's CTA range, then
 // the block's threads compute the float offsets of the slots of up to MAXC CTAs at a time (a
-// negative offset marks a slot that failed its bounds check).  `fn(j, m)` is called by every
-// thread for each pass with the offsets of CTAs c0 + j .. c0 + j + m - 1 in `off`, in
-// increasing CTA order, between two block-wide barriers.
+// negative offset marks a slot that failed its bounds check).  `fn(m)` is called by every thread
+// for each pass, with the offsets of the pass's m CTAs in off[0 .. m), in increasing CTA order,
+// between two block-wide barriers.
 template <typename Fn>
 __device__ __forceinline__ void for_unit_slots(const Plan& p, int64_t u, int64_t slot_floats, int64_t* off,
                                                int64_t* rng, Fn&& fn) {
@@ -325,6 +325,7 @@ __device__ __forceinline__ void for_unit_slots(const Plan& p, int64_t u, int64_t
   }
   __syncthreads();
   const int64_t c0 = rng[0], n = rng[1];
+  __syncthreads();  // every thread holds the range before thread 0 may write the next unit's
   for (int64_t j = 0; j < n; j += MAXC) {
     const int m = static_cast<int>(n - j < MAXC ? n - j : MAXC);
     if (static_cast<int>(threadIdx.x) < m) {
