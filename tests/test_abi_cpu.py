@@ -154,3 +154,27 @@ def test_static_entry_point_checks_pointers_before_cuda():
         assert lib.la_forward_bidir_static(ctypes.byref(cp), 16, 16, 16, 16, 24, None) == 4
     cp = la.Problem(B=1, H=2, T=3, Hh=4, W=5, block_frames=1).c()
     assert lib.la_forward_bidir_static(ctypes.byref(cp), 16, 16, 16, 16, 16, None) == 2
+
+
+def test_binding_routes_saved_states_to_la_backward_saved():
+    # With S and z the binding calls la_backward_saved, without them la_backward; host tensors and
+    # no GPU stop both at their first CUDA call (or, for a misaligned state, at the argument check).
+    import torch
+
+    class _Stream:
+        cuda_stream = 0
+
+    p = la.Problem(B=1, H=2, T=1, Hh=2, W=8)
+    Q, K, V, G, dO = (torch.zeros((1, 2, 16, 128), dtype=torch.bfloat16) for _ in range(5))
+    grads = tuple(torch.zeros_like(Q) for _ in range(4))
+    ws = torch.zeros(256, dtype=torch.uint8)
+    S = torch.zeros((1, 2, 1, 128, 128), dtype=torch.float32)
+    z = torch.zeros((1, 2, 1, 128), dtype=torch.float32)
+    kw = dict(grads=grads, ws=ws, stream=_Stream())
+    with pytest.raises(bnd.LaError, match="la_backward_saved"):
+        la.backward(p, Q, K, V, G, dO, S=S, z=z, **kw)
+    with pytest.raises(bnd.LaError, match=r"la_backward:"):
+        la.backward(p, Q, K, V, G, dO, **kw)
+    flat = torch.zeros(2 * 128 * 128 + 1, dtype=torch.float32)
+    with pytest.raises(bnd.LaError, match="LA_ERR_ALIGN"):
+        la.backward(p, Q, K, V, G, dO, S=flat[1:], z=z, **kw)
